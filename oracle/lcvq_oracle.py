@@ -1,0 +1,278 @@
+"""fp64 reference oracle for the LC-VQ hot path.  TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The library and its Python binding
+never import it, and it imports nothing from them; the two share no code.
+
+What it computes, and where the method is stated
+------------------------------------------------
+Sources (cited below by these short names):
+
+* "LC-QAT page": the technical summary of *LC-QAT: Data-Efficient 2-Bit QAT
+  for LLMs via Linear-Constrained Vector Quantization* (gist.science,
+  paper 2606.10531; Chinese, Portuguese and French editions say the same).
+  - Methodology 1 "linear-constrained parameterization": codewords are
+    ``c = A z + B`` with ``z`` in ``{0,1,2,3}^d`` and ``A`` (d x d), ``B`` (d)
+    floating-point parameters shared within one weight matrix; index search
+    becomes rounding and clamping followed by a linear projection, and
+    gradients flow through the linear map.
+  - Methodology 3 "training pipeline": proxy weights ``W_p`` are rounded and
+    clamped to integers ``W_z`` and decoded as ``A W_z + B``; the forward is
+    recast onto INT2 x FP16 matmul operators; the backward uses a gradient
+    estimator through the rounding (DGE in the paper, STE in its ablation).
+* "decoupleQ page": *decoupleQ: 2-bit post-training uniform quantization by
+  decoupling parameters into integer and floating-point parts* (lryc.cn
+  translation).  Eq. (1) fixes the linear-layer convention ``Y = X W~`` with
+  ``W~`` of shape ``d_in x d_out``; eq. (3)/(4) are the scalar
+  round/clip/affine special case used as a pin.
+
+Readings where the pages are silent (each one is listed in the design doc):
+
+* rounding is round-half-to-even (numpy ``rint``); clamp to ``[0, 3]``;
+  NaN -> 0, +Inf -> 3, -Inf -> 0;
+* the STE clamp mask is ``0 <= W_p <= 3`` on the proxy weight itself;
+* vectors are ``d`` consecutive elements along ``d_in``; ``A`` acts on column
+  vectors (``c_i = sum_j A[i, j] z_j``);
+* weights are stored ``[d_out][d_in]`` (the transpose of the decoupleQ
+  ``W~``), so ``Y[m, n] = sum_k X[m, k] W~[n, k]``;
+* packed format V1: 4 codes per byte, LSB first along ``d_in``; the clamp
+  mask is 8 bits per byte, LSB first.
+
+All arithmetic is fp64 after exact widening of the fp32/bf16 inputs.  Every
+floating result comes with the per-element normaliser ``D`` = the sum of the
+absolute values of the terms that make that element; the parity metric is
+``|got - ref| / D``.
+
+Parity status: every function here is pinned by a CPU test against values
+that do not come from this module (brute force, closed forms, hand-worked
+golden files, finite differences, distribution statistics).  No function is
+"parity unpinned".
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+CODE_MAX = 3  # z in {0, 1, 2, 3}: 2 bits per weight
+
+
+# --------------------------------------------------------------------------
+# code assignment (LC-QAT page, Methodology 1 and 3: "rounding and clamping")
+# --------------------------------------------------------------------------
+def assign(Wp: np.ndarray):
+    """Round the proxy weights to the nearest integer (ties to even) and clamp
+    to ``[0, 3]``.  Returns ``(z uint8, mask bool)`` with ``mask`` the STE
+    pass-through region ``0 <= W_p <= 3`` (false for NaN)."""
+    w = np.asarray(Wp, dtype=np.float64)
+    r = np.rint(w)
+    r = np.where(np.isnan(w), 0.0, r)
+    z = np.clip(r, 0.0, float(CODE_MAX)).astype(np.uint8)
+    with np.errstate(invalid="ignore"):
+        mask = (w >= 0.0) & (w <= float(CODE_MAX))
+    return z, mask
+
+
+# --------------------------------------------------------------------------
+# 2-bit storage (format V1; the pages fix only "2 bits per weight")
+# --------------------------------------------------------------------------
+def pack_codes(z: np.ndarray) -> np.ndarray:
+    """``[d_out][d_in]`` codes -> ``[d_out][d_in/4]`` bytes; element ``k`` of a
+    row sits in byte ``k // 4`` at bits ``2 (k % 4)`` and ``2 (k % 4) + 1``."""
+    z = np.asarray(z, dtype=np.uint8)
+    n, k = z.shape
+    assert k % 4 == 0
+    out = np.zeros((n, k // 4), dtype=np.uint8)
+    for pos in range(4):
+        out |= (z[:, pos::4] & 3) << (2 * pos)
+    return out
+
+
+def unpack_codes(packed: np.ndarray, d_in: int) -> np.ndarray:
+    packed = np.asarray(packed, dtype=np.uint8)
+    n = packed.shape[0]
+    z = np.zeros((n, d_in), dtype=np.uint8)
+    for pos in range(4):
+        z[:, pos::4] = (packed >> (2 * pos)) & 3
+    return z
+
+
+def pack_mask(mask: np.ndarray) -> np.ndarray:
+    """``[d_out][d_in]`` bools -> ``[d_out][d_in/8]`` bytes, bit ``k % 8`` of
+    byte ``k // 8``."""
+    m = np.asarray(mask, dtype=np.uint8)
+    n, k = m.shape
+    assert k % 8 == 0
+    out = np.zeros((n, k // 8), dtype=np.uint8)
+    for pos in range(8):
+        out |= (m[:, pos::8] & 1) << pos
+    return out
+
+
+def unpack_mask(bits: np.ndarray, d_in: int) -> np.ndarray:
+    bits = np.asarray(bits, dtype=np.uint8)
+    m = np.zeros((bits.shape[0], d_in), dtype=bool)
+    for pos in range(8):
+        m[:, pos::8] = (bits >> pos) & 1
+    return m
+
+
+# --------------------------------------------------------------------------
+# decode (LC-QAT page, Methodology 1: c = A z + B; Methodology 3: A W_z + B)
+# --------------------------------------------------------------------------
+def decode(z: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """``W~[n, g d + i] = sum_j A[i, j] z[n, g d + j] + B[i]`` in fp64."""
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    d = A.shape[0]
+    n, k = z.shape
+    zg = np.asarray(z, dtype=np.float64).reshape(n, k // d, d)
+    w = np.einsum("ij,ngj->ngi", A, zg) + B
+    return w.reshape(n, k)
+
+
+def decode_abs(z: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """Normaliser of :func:`decode`: ``sum_j |A[i, j]| z_j + |B[i]|``."""
+    return decode(z, np.abs(np.asarray(A, np.float64)), np.abs(np.asarray(B, np.float64)))
+
+
+# --------------------------------------------------------------------------
+# forward  Y = X W~  (decoupleQ page eq. (1) convention; LC-QAT Methodology 3)
+# --------------------------------------------------------------------------
+def forward(X: np.ndarray, z: np.ndarray, A: np.ndarray, B: np.ndarray):
+    """Returns ``(Y, D_Y)`` with ``Y[m, n] = sum_k X[m, k] W~[n, k]`` and
+    ``D_Y[m, n] = sum_k |X[m, k]| |W~[n, k]|``."""
+    X = np.asarray(X, dtype=np.float64)
+    W = decode(z, A, B)
+    return X @ W.T, np.abs(X) @ np.abs(W).T
+
+
+def forward_sampled(X, z_rows: dict, A, B, pairs):
+    """Y and D_Y at the listed ``(m, n)`` pairs only.  ``z_rows`` maps ``n`` to
+    that row's codes (so a caller can unpack only the rows it samples)."""
+    X = np.asarray(X, dtype=np.float64)
+    y = np.empty(len(pairs))
+    dd = np.empty(len(pairs))
+    cache = {}
+    for t, (m, n) in enumerate(pairs):
+        if n not in cache:
+            cache[n] = decode(np.asarray(z_rows[n]).reshape(1, -1), A, B)[0]
+        w = cache[n]
+        y[t] = float(np.dot(X[m], w))
+        dd[t] = float(np.dot(np.abs(X[m]), np.abs(w)))
+    return y, dd
+
+
+def forward_algebraic(X, z, A, B):
+    """The same product regrouped as ``X' Z^T + s 1^T`` with
+    ``X'[m, g d + j] = sum_i X[m, g d + i] A[i, j]`` and
+    ``s[m] = sum_g sum_i X[m, g d + i] B[i]``: exact algebra on
+    ``sum_k x_k w~_k = sum_g x_g^T (A z_g + B)``.  Used only as an fp64
+    cross-check of :func:`forward`."""
+    X = np.asarray(X, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    d = A.shape[0]
+    m, k = X.shape
+    Xg = X.reshape(m, k // d, d)
+    Xp = np.einsum("mgi,ij->mgj", Xg, A).reshape(m, k)
+    s = np.einsum("mgi,i->m", Xg, B)
+    return Xp @ np.asarray(z, np.float64).T + s[:, None]
+
+
+# --------------------------------------------------------------------------
+# straight-through backward (LC-QAT page, Methodology 1 "gradients flow
+# through the linear map"; Methodology 3 and the gradient-estimation
+# ablation: STE).  Loss gradient dY = dL/dY is an input.
+# --------------------------------------------------------------------------
+def backward(X, dY, z, mask, A, B):
+    """Returns a dict with dX, dA, dB, dWp and their normalisers.
+
+    * ``dX = dY W~``                                        (input gradient)
+    * ``G[n, k] = sum_m dY[m, n] X[m, k]``                  (dL/dW~)
+    * ``dA[i, j] = sum_{n, g} G[n, g d + i] z[n, g d + j]`` (chain rule on
+      ``c = A z + B``)
+    * ``dB[i] = sum_{n, g} G[n, g d + i]``
+    * ``dWp[n, g d + j] = mask * sum_i A[i, j] G[n, g d + i]`` (STE: identity
+      through the rounding, zero where the clamp is active)
+    """
+    X = np.asarray(X, dtype=np.float64)
+    dY = np.asarray(dY, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    d = A.shape[0]
+    n, k = z.shape
+    W = decode(z, A, B)
+    Wabs = np.abs(W)
+    out = {}
+    out["dX"] = dY @ W
+    out["D_dX"] = np.abs(dY) @ Wabs
+    G = dY.T @ X
+    DG = np.abs(dY).T @ np.abs(X)
+    Gg = G.reshape(n, k // d, d)
+    DGg = DG.reshape(n, k // d, d)
+    zg = np.asarray(z, np.float64).reshape(n, k // d, d)
+    out["dA"] = np.einsum("ngi,ngj->ij", Gg, zg)
+    out["D_dA"] = np.einsum("ngi,ngj->ij", DGg, zg)
+    out["dB"] = Gg.sum(axis=(0, 1))
+    out["D_dB"] = DGg.sum(axis=(0, 1))
+    mg = np.asarray(mask, np.float64).reshape(n, k // d, d)
+    out["dWp"] = (mg * np.einsum("ij,ngi->ngj", A, Gg)).reshape(n, k)
+    out["D_dWp"] = (mg * np.einsum("ij,ngi->ngj", np.abs(A), DGg)).reshape(n, k)
+    return out
+
+
+def backward_dx_sampled(dY, z_cols_fn, A, B, pairs):
+    """dX and D_dX at ``(m, k)`` pairs; ``z_cols_fn(k)`` returns the codes of
+    column group ``k // d`` for all rows, shape ``[d_out, d]``."""
+    dY = np.asarray(dY, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    d = A.shape[0]
+    v = np.empty(len(pairs))
+    dd = np.empty(len(pairs))
+    for t, (m, kk) in enumerate(pairs):
+        zc = np.asarray(z_cols_fn(kk), dtype=np.float64)  # [d_out, d]
+        i = kk % d
+        wcol = zc @ A[i] + B[i]                          # W~[:, kk]
+        v[t] = float(np.dot(dY[m], wcol))
+        dd[t] = float(np.dot(np.abs(dY[m]), np.abs(wcol)))
+    return v, dd
+
+
+def backward_dwp_sampled(X, dY, mask_rows_fn, A, pairs):
+    """dWp and D_dWp at ``(n, k)`` pairs; ``mask_rows_fn(n)`` returns the clamp
+    mask of row ``n``."""
+    X = np.asarray(X, dtype=np.float64)
+    dY = np.asarray(dY, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    d = A.shape[0]
+    v = np.empty(len(pairs))
+    dd = np.empty(len(pairs))
+    for t, (n, kk) in enumerate(pairs):
+        g0 = (kk // d) * d
+        j = kk % d
+        Gv = dY[:, n] @ X[:, g0:g0 + d]                  # G[n, g d + i], i < d
+        DGv = np.abs(dY[:, n]) @ np.abs(X[:, g0:g0 + d])
+        mk = float(mask_rows_fn(n)[kk])
+        v[t] = mk * float(np.dot(A[:, j], Gv))
+        dd[t] = mk * float(np.dot(np.abs(A[:, j]), DGv))
+    return v, dd
+
+
+# --------------------------------------------------------------------------
+# parity metric
+# --------------------------------------------------------------------------
+def rel_err(got, ref, D) -> float:
+    """max over elements of ``|got - ref| / D``; where ``D == 0`` the element
+    must be exactly equal (returns inf otherwise)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    D = np.asarray(D, dtype=np.float64)
+    diff = np.abs(got - ref)
+    if not np.all(np.isfinite(got)):
+        return float("inf")
+    zero = D == 0
+    if np.any(diff[zero] != 0):
+        return float("inf")
+    if np.all(zero):
+        return 0.0
+    return float(np.max(diff[~zero] / D[~zero]))

@@ -1,0 +1,393 @@
+"""Pins for the fp64 oracle: every function is checked against something that
+does not come from the oracle itself (hand-worked golden files, brute force
+over all 4^d codes, closed forms, exact integer arithmetic, finite
+differences, distribution statistics)."""
+
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import lcvq_oracle as O
+from bit_weight_only_lcvq_b200 import synth
+
+
+# ---------------------------------------------------------------- helpers
+def _read(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return [ln.split("#")[0].strip() for ln in f if ln.split("#")[0].strip()]
+
+
+def _f32(tok):
+    return np.float32(float(tok))
+
+
+# ---------------------------------------------------------------- assign
+def test_round_clamp_golden(golden_dir):
+    rows = [ln.split() for ln in _read(golden_dir, "round_clamp_ties.txt")]
+    w = np.array([_f32(r[0]) for r in rows], dtype=np.float32)
+    z, mask = O.assign(w)
+    assert z.tolist() == [int(r[1]) for r in rows]
+    assert mask.astype(int).tolist() == [int(r[2]) for r in rows]
+
+
+@pytest.mark.parametrize("d", [1, 2, 4])
+def test_assign_is_nearest_code_brute_force(d):
+    """Round-and-clamp equals the exhaustive nearest-neighbour search over all
+    4^d codes (the box-constrained problem is separable)."""
+    g = np.random.Generator(np.random.PCG64(11 + d))
+    cand = np.array(list(itertools.product(range(4), repeat=d)), dtype=np.float64)
+    w = g.uniform(-1.5, 4.5, size=(400, d)).astype(np.float32)
+    frac = np.abs(w - np.floor(w) - 0.5)
+    w = w[np.all(frac > 1e-4, axis=1)]          # ties are pinned by the golden table
+    z, _ = O.assign(w)
+    dist = ((w[:, None, :].astype(np.float64) - cand[None]) ** 2).sum(-1)
+    best = cand[np.argmin(dist, axis=1)].astype(np.uint8)
+    assert np.array_equal(z, best)
+
+
+def test_assign_brute_force_d8():
+    g = np.random.Generator(np.random.PCG64(7))
+    cand = np.array(list(itertools.product(range(4), repeat=8)), dtype=np.float64)
+    for _ in range(3):
+        w = g.uniform(-1.0, 4.0, size=8).astype(np.float32)
+        if np.any(np.abs(w - np.floor(w) - 0.5) < 1e-4):
+            continue
+        z, _ = O.assign(w[None])
+        best = cand[np.argmin(((cand - w.astype(np.float64)) ** 2).sum(-1))]
+        assert np.array_equal(z[0], best.astype(np.uint8))
+
+
+def test_scalar_special_case_matches_uniform_quantizer():
+    """With A = s I and B = b 1 the linear-constrained codebook is a scalar
+    uniform grid: nearest codeword of w0 = clamp(round((w0 - b)/s), 0, 3) and
+    the decode is s z + b (decoupleQ page, eq. (3) and (4), with the integer
+    range [0, 3]).  Checked by exhaustive search over the 4^d codewords."""
+    d = 4
+    s, b = 0.37, -0.61
+    A = s * np.eye(d)
+    B = b * np.ones(d)
+    cand = np.array(list(itertools.product(range(4), repeat=d)), dtype=np.uint8)
+    cw = O.decode(cand, A, B)                         # [256, d] codewords
+    assert np.allclose(cw, s * cand + b, rtol=0, atol=1e-15)
+    g = np.random.Generator(np.random.PCG64(3))
+    w0 = g.uniform(b - 1.0, b + 4 * s, size=(300, d))
+    q = (w0 - b) / s
+    ok = np.all(np.abs(q - np.floor(q) - 0.5) > 1e-6, axis=1)
+    w0, q = w0[ok], q[ok]
+    nn = cand[np.argmin(((w0[:, None, :] - cw[None]) ** 2).sum(-1), axis=1)]
+    z, _ = O.assign(q)
+    assert np.array_equal(z, nn)
+
+
+def _phi(x):
+    return 0.5 * (1.0 + math.erf(x / math.sqrt(2.0)))
+
+
+def test_code_statistics_uniform_and_normal():
+    """U[-0.5, 3.5] gives uniform codes; N(1.5, 1) gives
+    Phi(-1), Phi(0)-Phi(-1), ... and a clamp fraction 2 (1 - Phi(1.5))."""
+    n = 1 << 20
+    g = np.random.Generator(np.random.PCG64(5))
+    z, _ = O.assign(g.uniform(-0.5, 3.5, size=n).astype(np.float32))
+    freq = np.bincount(z, minlength=4) / n
+    assert np.allclose(freq, 0.25, atol=3e-3)
+    z, mask = O.assign(g.normal(1.5, 1.0, size=n).astype(np.float32))
+    freq = np.bincount(z, minlength=4) / n
+    p0 = _phi(-1.0)
+    p1 = _phi(0.0) - _phi(-1.0)
+    assert np.allclose(freq, [p0, p1, p1, p0], atol=3e-3)
+    clamp_frac = 1.0 - mask.mean()
+    assert abs(clamp_frac - 2 * (1 - _phi(1.5))) < 3e-3
+    assert abs(2 * (1 - _phi(1.5)) - 0.1336) < 1e-4
+
+
+# ---------------------------------------------------------------- pack
+def test_pack_golden(golden_dir):
+    for ln in _read(golden_dir, "pack_v1.txt"):
+        codes, hexes = ln.split("|")
+        z = np.array([[int(t) for t in codes.split()]], dtype=np.uint8)
+        want = [int(h, 16) for h in hexes.split()]
+        got = O.pack_codes(z)
+        assert got[0].tolist() == want
+        assert np.array_equal(O.unpack_codes(got, z.shape[1]), z)
+
+
+def test_mask_golden(golden_dir):
+    for ln in _read(golden_dir, "mask_v1.txt"):
+        bits, hexes = ln.split("|")
+        m = np.array([[int(t) for t in bits.split()]], dtype=bool)
+        want = [int(h, 16) for h in hexes.split()]
+        got = O.pack_mask(m)
+        assert got[0].tolist() == want
+        assert np.array_equal(O.unpack_mask(got, m.shape[1]), m)
+
+
+def test_pack_is_bijection_on_bytes():
+    allb = np.arange(256, dtype=np.uint8)[None, :]
+    z = O.unpack_codes(allb, 1024)
+    assert np.array_equal(O.pack_codes(z), allb)
+    g = np.random.Generator(np.random.PCG64(9))
+    z = g.integers(0, 4, size=(37, 64), dtype=np.uint8)
+    assert np.array_equal(O.unpack_codes(O.pack_codes(z), 64), z)
+    m = g.integers(0, 2, size=(5, 64)).astype(bool)
+    assert np.array_equal(O.unpack_mask(O.pack_mask(m), 64), m)
+
+
+def test_packed_d8_vector_is_codebook_index():
+    g = np.random.Generator(np.random.PCG64(13))
+    z = g.integers(0, 4, size=(4, 32), dtype=np.uint8)
+    p = O.pack_codes(z)
+    for r in range(4):
+        for v in range(4):
+            idx = sum(int(z[r, 8 * v + j]) * 4 ** j for j in range(8))
+            assert int(p[r, 2 * v]) | (int(p[r, 2 * v + 1]) << 8) == idx
+
+
+# ---------------------------------------------------------------- decode
+def test_decode_golden(golden_dir):
+    lines = _read(golden_dir, "affine_hand.txt")
+    cases, cur = [], None
+    for ln in lines:
+        t = ln.split()
+        if t[0] == "case":
+            cur = dict(A=[], z=[], c=[])
+            cases.append(cur)
+        elif t[0] == "d":
+            cur["d"] = int(t[1])
+        elif t[0] == "A":
+            cur["A"].append([float(v) for v in t[1:]])
+        elif t[0] == "B":
+            cur["B"] = [float(v) for v in t[1:]]
+        elif t[0] == "z":
+            k = t.index("->")
+            cur["z"].append([int(v) for v in t[1:k]])
+            cur["c"].append([float(v) for v in t[k + 1:]])
+    assert len(cases) == 2
+    for c in cases:
+        z = np.array(c["z"], dtype=np.uint8)
+        W = O.decode(z, np.array(c["A"]), np.array(c["B"]))
+        assert np.array_equal(W, np.array(c["c"]))
+
+
+def test_decode_equals_codebook_lookup():
+    """Materialize the 4^d codebook and look each vector up by its packed
+    index: must equal the grouped affine decode."""
+    d = 4
+    A, B = synth.affine_single_layer(d, np.random.Generator(np.random.PCG64(1)))
+    book = {}
+    for zt in itertools.product(range(4), repeat=d):
+        idx = sum(v * 4 ** j for j, v in enumerate(zt))
+        book[idx] = [sum(float(A[i, j]) * zt[j] for j in range(d)) + float(B[i]) for i in range(d)]
+    g = np.random.Generator(np.random.PCG64(2))
+    z = g.integers(0, 4, size=(6, 32), dtype=np.uint8)
+    p = O.pack_codes(z)
+    W = O.decode(z, A, B)
+    for r in range(6):
+        for v in range(32 // d):
+            idx = int(p[r, v])           # d = 4: one byte per vector
+            assert np.allclose(W[r, v * d:(v + 1) * d], book[idx], rtol=0, atol=1e-15)
+
+
+def test_decode_scalar_case_is_cross_d_invariant():
+    g = np.random.Generator(np.random.PCG64(4))
+    z = g.integers(0, 4, size=(3, 64), dtype=np.uint8)
+    ref = 0.25 * z.astype(np.float64) - 0.375
+    for d in (1, 2, 4, 8):
+        W = O.decode(z, 0.25 * np.eye(d), -0.375 * np.ones(d))
+        assert np.array_equal(W, ref)
+
+
+# ---------------------------------------------------------------- forward
+def test_linear_layer_golden(golden_dir):
+    rec = {}
+    for ln in _read(golden_dir, "linear_layer_hand.txt"):
+        t = ln.split()
+        rec.setdefault(t[0], []).append([float(v) for v in t[1:]])
+    A = np.array(rec["A"])
+    B = np.array(rec["B"][0])
+    Wp = np.array(rec["Wp"][0], dtype=np.float32)[None]
+    z, mask = O.assign(Wp)
+    assert z[0].tolist() == [int(v) for v in rec["z"][0]]
+    assert mask[0].astype(int).tolist() == [int(v) for v in rec["mask"][0]]
+    assert np.array_equal(O.decode(z, A, B)[0], rec["W"][0])
+    X = np.array(rec["X"][0])[None]
+    Y, _ = O.forward(X, z, A, B)
+    assert Y[0, 0] == rec["Y"][0][0]
+    assert O.forward_algebraic(X, z, A, B)[0, 0] == rec["Y"][0][0]
+    dY = np.array(rec["dY"][0])[None]
+    bw = O.backward(X, dY, z, mask, A, B)
+    assert np.array_equal(bw["dX"][0], rec["dX"][0])
+    assert np.array_equal(bw["dA"], np.array(rec["dA"]))
+    assert np.array_equal(bw["dB"], rec["dB"][0])
+    assert np.array_equal(bw["dWp"][0], rec["dWp"][0])
+
+
+def test_forward_identity_is_integer_code_gemm():
+    """A = I, B = 0: Y = X Z^T exactly (checked in int64 arithmetic)."""
+    g = np.random.Generator(np.random.PCG64(21))
+    for d in (4, 8):
+        X = g.integers(-8, 9, size=(5, 64))
+        z = g.integers(0, 4, size=(7, 64), dtype=np.uint8)
+        Y, D = O.forward(X.astype(np.float64), z, np.eye(d), np.zeros(d))
+        Yi = X.astype(np.int64) @ z.astype(np.int64).T
+        assert np.array_equal(Y, Yi.astype(np.float64))
+        assert np.array_equal(D, (np.abs(X) @ z.astype(np.int64).T).astype(np.float64))
+
+
+def _rand_case(seed, M=3, N=5, K=32, d=8):
+    g = np.random.Generator(np.random.PCG64(seed))
+    X = g.standard_normal((M, K))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A = g.standard_normal((d, d))
+    B = g.standard_normal(d)
+    return X, z, A, B
+
+
+def test_forward_linearity_and_pow2_scaling():
+    X, z, A1, B1 = _rand_case(31)
+    _, _, A2, B2 = _rand_case(32)
+    Y1, D1 = O.forward(X, z, A1, B1)
+    Y2, _ = O.forward(X, z, A2, B2)
+    Y12, _ = O.forward(X, z, A1 + A2, B1 + B2)
+    assert np.max(np.abs(Y12 - Y1 - Y2)) <= 1e-12 * np.max(D1 + 1)
+    Y8, _ = O.forward(X, z, 8.0 * A1, 8.0 * B1)
+    assert np.array_equal(Y8, 8.0 * Y1)
+
+
+def test_forward_direct_equals_algebraic():
+    X, z, A, B = _rand_case(41, M=4, N=6, K=64)
+    Y, D = O.forward(X, z, A, B)
+    assert O.rel_err(O.forward_algebraic(X, z, A, B), Y, D) < 1e-13
+
+
+def test_forward_sampled_matches_full():
+    X, z, A, B = _rand_case(43, M=4, N=6, K=64)
+    Y, D = O.forward(X, z, A, B)
+    pairs = [(0, 0), (3, 5), (2, 1)]
+    y, dd = O.forward_sampled(X, {n: z[n] for n in range(6)}, A, B, pairs)
+    for t, (m, n) in enumerate(pairs):
+        assert abs(y[t] - Y[m, n]) <= 1e-13 * D[m, n] and abs(dd[t] - D[m, n]) <= 1e-13 * D[m, n]
+
+
+# ---------------------------------------------------------------- backward
+def _loss(X, dY, z, A, B):
+    Y, _ = O.forward(X, z, A, B)
+    return float(np.sum(dY * Y))
+
+
+def test_backward_finite_differences_exact():
+    """L = sum dY * Y is linear in X, in A and in B (codes fixed), so a
+    central difference with any step is exact up to fp64 rounding."""
+    X, z, A, B = _rand_case(51, M=3, N=4, K=16, d=4)
+    g = np.random.Generator(np.random.PCG64(52))
+    dY = g.standard_normal((3, 4))
+    mask = np.ones_like(z, dtype=bool)
+    bw = O.backward(X, dY, z, mask, A, B)
+    h = 0.5
+    for (m, k) in [(0, 0), (2, 15), (1, 7)]:
+        Xp, Xm = X.copy(), X.copy()
+        Xp[m, k] += h
+        Xm[m, k] -= h
+        fd = (_loss(Xp, dY, z, A, B) - _loss(Xm, dY, z, A, B)) / (2 * h)
+        assert abs(fd - bw["dX"][m, k]) < 1e-12 * (1 + abs(fd))
+    for (i, j) in [(0, 0), (3, 1), (2, 3)]:
+        Ap, Am = A.copy(), A.copy()
+        Ap[i, j] += h
+        Am[i, j] -= h
+        fd = (_loss(X, dY, z, Ap, B) - _loss(X, dY, z, Am, B)) / (2 * h)
+        assert abs(fd - bw["dA"][i, j]) < 1e-11 * (1 + abs(fd))
+    for i in range(4):
+        Bp, Bm = B.copy(), B.copy()
+        Bp[i] += h
+        Bm[i] -= h
+        fd = (_loss(X, dY, z, A, Bp) - _loss(X, dY, z, A, Bm)) / (2 * h)
+        assert abs(fd - bw["dB"][i]) < 1e-11 * (1 + abs(fd))
+
+
+def test_backward_dwp_ste_surrogate_finite_differences():
+    """STE: the rounding is treated as identity, the clamp is kept.  The
+    surrogate L(Wp) = sum dY * (X decode(clamp(Wp, 0, 3))^T) is piecewise
+    linear; at points >= 1e-3 away from 0 and 3 a step of 1e-4 is exact up to
+    rounding, and the gradient is zero wherever the clamp is active."""
+    M, N, K, d = 3, 4, 16, 4
+    g = np.random.Generator(np.random.PCG64(61))
+    X = g.standard_normal((M, K))
+    dY = g.standard_normal((M, N))
+    A = g.standard_normal((d, d))
+    B = g.standard_normal(d)
+    Wp = g.uniform(-1.0, 4.0, size=(N, K))
+    Wp[np.abs(Wp) < 1e-3] += 2e-3
+    Wp[np.abs(Wp - 3) < 1e-3] += 2e-3
+    z, mask = O.assign(Wp.astype(np.float32))
+    bw = O.backward(X, dY, z, mask, A, B)
+
+    def surrogate(W):
+        return _loss(X, dY, np.clip(W, 0.0, 3.0), A, B)
+
+    h = 1e-4
+    for n in range(N):
+        for k in range(K):
+            Wa, Wb = Wp.copy(), Wp.copy()
+            Wa[n, k] += h
+            Wb[n, k] -= h
+            fd = (surrogate(Wa) - surrogate(Wb)) / (2 * h)
+            assert abs(fd - bw["dWp"][n, k]) < 1e-7 * (1 + abs(fd)), (n, k)
+    assert np.all(bw["dWp"][~mask] == 0)
+
+
+def test_backward_sampled_matches_full():
+    M, N, K, d = 4, 6, 32, 8
+    g = np.random.Generator(np.random.PCG64(71))
+    X = g.standard_normal((M, K))
+    dY = g.standard_normal((M, N))
+    A = g.standard_normal((d, d))
+    B = g.standard_normal(d)
+    Wp = g.uniform(-1.0, 4.0, size=(N, K)).astype(np.float32)
+    z, mask = O.assign(Wp)
+    bw = O.backward(X, dY, z, mask, A, B)
+    pairs = [(0, 0), (3, 31), (1, 9)]
+    v, dd = O.backward_dx_sampled(dY, lambda k: z[:, (k // d) * d:(k // d + 1) * d], A, B, pairs)
+    for t, (m, k) in enumerate(pairs):
+        assert abs(v[t] - bw["dX"][m, k]) <= 1e-13 * bw["D_dX"][m, k]
+        assert abs(dd[t] - bw["D_dX"][m, k]) <= 1e-13 * bw["D_dX"][m, k]
+    pairs = [(0, 0), (5, 31), (2, 10)]
+    v, dd = O.backward_dwp_sampled(X, dY, lambda n: mask[n], A, pairs)
+    for t, (n, k) in enumerate(pairs):
+        assert abs(v[t] - bw["dWp"][n, k]) <= 1e-13 * (bw["D_dWp"][n, k] + 1e-300)
+        assert abs(dd[t] - bw["D_dWp"][n, k]) <= 1e-13 * (bw["D_dWp"][n, k] + 1e-300)
+
+
+def test_db_identity_at_any_size():
+    """dB[i] = sum_m rowsum(dY)[m] * sum_g X[m, g d + i]: an O(M (N + K))
+    identity the tests use to check dB at full size."""
+    M, N, K, d = 5, 7, 32, 8
+    g = np.random.Generator(np.random.PCG64(81))
+    X = g.standard_normal((M, K))
+    dY = g.standard_normal((M, N))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    bw = O.backward(X, dY, z, np.ones((N, K), bool), np.eye(d), np.zeros(d))
+    ident = dY.sum(1) @ X.reshape(M, K // d, d).sum(1)
+    assert np.allclose(bw["dB"], ident, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- metric
+def test_rel_err_semantics():
+    assert O.rel_err([1.0, 2.0], [1.0, 2.5], [1.0, 5.0]) == pytest.approx(0.1)
+    assert O.rel_err([0.0], [0.0], [0.0]) == 0.0
+    assert O.rel_err([1e-30], [0.0], [0.0]) == float("inf")
+    assert O.rel_err([float("nan")], [0.0], [1.0]) == float("inf")
+
+
+def test_planted_mistakes_are_caught(golden_dir):
+    """A transposed A, a dropped B, or a wrong tie rule in a copy of the
+    oracle's formulas each fail a pin above (checked here directly)."""
+    A = np.array([[1.0, 2.0], [3.0, 4.0]])
+    B = np.array([10.0, 20.0])
+    z = np.array([[1, 3]], dtype=np.uint8)
+    assert not np.array_equal(O.decode(z, A.T, B), [[17.0, 35.0]])
+    assert not np.array_equal(O.decode(z, A, 0 * B), [[17.0, 35.0]])
+    w = np.array([2.5], dtype=np.float32)
+    assert np.floor(w + 0.5)[0] != O.assign(w)[0][0]   # half-up would give 3

@@ -1,0 +1,564 @@
+#!/usr/bin/env python
+"""LC-VQ 2-bit hot-path benchmark (one JSON line on rank 0).
+
+Headline workload: decode-GEMV, d_in = d_out = 4096, d = 8, M in {1, 4, 16}
+bf16 tokens.  One step = one lcvq_gemm call per token count (the X-transform
+prologue plus the decode-GEMV kernel each), every call on the next of R
+rotated copies of the packed weights (R x 4 MiB > 4 x L2, so each call streams
+its codes from HBM).  value = packed-weight bytes of all calls on all ranks /
+max-over-ranks device time.
+
+The other hot-path rows (assign/pack, decode, prefill GEMM in both forms, the
+QAT step, the 7B-shaped stack) are measured after the headline and reported
+under "rows", each with its own metric and roofline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--rows all|none|name,...]
+Multi-GPU: launched by torch.distributed.run, one process per GPU; ranks run
+independent replicas (no collective in the data path) -> "scaling": "weak".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_weight_only_lcvq_b200 import lcvq, synth  # noqa: E402
+
+METRIC = "LC-VQ 2-bit GEMM: packed-weight GB/s (M≤16), TFLOP/s (prefill), % roofline"
+MIB = 1 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- setup
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--rows", default="all")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world > 1:
+            import datetime
+            torch.cuda.set_device(self.local)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        else:
+            torch.cuda.set_device(0)
+        self.dev = torch.device("cuda", torch.cuda.current_device())
+
+    def barrier(self):
+        if self.world > 1:
+            torch.distributed.barrier()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=self.dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            torch.distributed.destroy_process_group()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during a timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        # nvidia-smi numbers GPUs physically; address ours by UUID so a
+        # CUDA_VISIBLE_DEVICES remap cannot point the sampler at another GPU
+        try:
+            self.idx = "GPU-" + str(torch.cuda.get_device_properties(gpu_index).uuid)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            self.idx = vis.split(",")[gpu_index] if vis else str(gpu_index)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def ev_time(fn, n, stream=None):
+    """Average device time (ms) of fn() over n calls, CUDA events on the stream."""
+    s = stream or torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(n):
+        fn()
+    e1.record(s)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def capture(fn):
+    """CUDA graph of fn() (the library launches on torch's current stream, which
+    is the capture stream inside the context)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+class StepGraphs:
+    """K steps as graph replays: one graph holds `chunk` consecutive steps and a
+    second one the remainder, so exactly K steps run.  `step()` launches one
+    step and returns the number of library kernels it launched."""
+
+    def __init__(self, step, chunk: int, k: int):
+        self.step = step
+        self.chunk = max(1, min(chunk, k))
+        self.q, self.rem = divmod(k, self.chunk)
+        self.g_full, self.n_full = self._capture(self.chunk)
+        self.g_rem, self.n_rem = self._capture(self.rem) if self.rem else (None, 0)
+
+    def _capture(self, n):
+        box = [0]
+
+        def run():
+            box[0] = 0
+            for _ in range(n):
+                box[0] += self.step()
+        g = capture(run)
+        return g, box[0]
+
+    def replay(self) -> int:
+        for _ in range(self.q):
+            self.g_full.replay()
+        if self.g_rem is not None:
+            self.g_rem.replay()
+        return self.q * self.n_full + self.n_rem
+
+
+def timed_graphs(D, sg: StepGraphs, sampler=None):
+    """Barrier + sync on both sides; returns (max-over-ranks ms, launches, clocks)."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.start()
+    D.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    launches = sg.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    D.barrier()
+    ck = sampler.stop() if sampler else None
+    return D.max(e0.elapsed_time(e1)), launches, ck
+
+
+# ----------------------------------------------------------------------------- oracle leg
+def oracle_gemv_sample(Ms, seconds=10.0):
+    """The oracle (fp64) on the decode-GEMV workload's codes: Y for the three
+    token counts over as many full 4096 x 4096 passes as fit in ~`seconds`."""
+    from oracle import lcvq_oracle as O
+    w = synth.workload(2, M=max(Ms), with_dy=False)
+    z, _ = O.assign(w["Wp"])
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        for M in Ms:
+            O.forward(w["X"][:M], z, w["A"], w["B"])
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    packed_bytes = passes * len(Ms) * (4096 * 4096 // 4)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count() or 1
+    return dict(value=packed_bytes / dt / 1e9, unit="GB/s", cores=int(threads), kind="oracle",
+                sample=f"{passes} full passes of d_in=d_out=4096, d=8 at M={list(Ms)} "
+                       f"(fp64 decode + BLAS matmul incl. |x||w| normaliser), {dt:.1f} s")
+
+
+# ----------------------------------------------------------------------------- headline
+def headline(args, D: Dist, pk):
+    K = N = 4096
+    d = 8
+    Ms = (1, 4, 16)
+    dev = D.dev
+    w = synth.workload(2, M=max(Ms), with_dy=False)
+    Wp = torch.from_numpy(w["Wp"]).to(dev)
+    packed0, _ = lcvq.assign_pack(Wp, d, with_mask=False)
+    del Wp
+    L2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(8, math.ceil(4 * L2 / (N * K // 4)))
+    copies = [packed0.clone() for _ in range(R)]
+    A = torch.from_numpy(w["A"]).to(dev)
+    B = torch.from_numpy(w["B"]).to(dev)
+    X = {M: torch.from_numpy(w["X"][:M].copy()).to(torch.bfloat16).to(dev) for M in Ms}
+    Y = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in Ms}
+    ws = {M: lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, d), dev)
+          for M in Ms}
+
+    # parity before timing (oracle on rank 0, M = 16 full output)
+    parity = None
+    if D.rank == 0:
+        from oracle import lcvq_oracle as O
+        z, _ = O.assign(w["Wp"])
+        for M in Ms:
+            lcvq.gemm(X[M], copies[0], K, A, B, d, out=Y[M], workspace=ws[M])
+            ref, Dn = O.forward(w["X"][:M], z, w["A"], w["B"])
+            e = O.rel_err(Y[M].float().cpu().numpy(), ref, Dn)
+            parity = e if parity is None else max(parity, e)
+        assert parity <= 4e-3, f"parity failed before timing: {parity}"
+
+    ctr = [0]
+
+    def step():
+        n = 0
+        for M in Ms:
+            r = ctr[0] % R
+            ctr[0] += 1
+            lcvq.gemm(X[M], copies[r], K, A, B, d, out=Y[M], workspace=ws[M])
+            n += lcvq.last_launch_count()
+        return n
+
+    chunk = R  # one graph = R steps (every copy is visited 3 times)
+    warm = StepGraphs(step, chunk, max(args.warmup, 3))
+    warm.replay()
+    sg = StepGraphs(step, chunk, args.steps)
+    ms_total, launches, ck = timed_graphs(D, sg, ClockSampler(dev.index))
+    per_step_bytes = len(Ms) * (N * K // 4)
+    value = D.world * args.steps * per_step_bytes / (ms_total * 1e-3) / 1e9
+
+    # dominant kernel alone: decode-GEMV on a pre-transformed X'', per token count
+    xpp, corr = {}, {}
+    for M in Ms:
+        xpp[M], corr[M] = lcvq.xform(X[M], A, B, d)
+    per_m = {}
+    for M in Ms:
+        kc = [0]
+
+        def kstep(M=M, kc=kc):
+            lcvq.gemm_xformed(xpp[M], corr[M], copies[kc[0] % R], out=Y[M])
+            kc[0] += 1
+            return lcvq.last_launch_count()
+        n = 4 * R
+        g = StepGraphs(kstep, R, n)
+        g.replay()
+        t, _, _ = timed_graphs(D, g)
+        per_m[M] = t / n
+    kern_ms = sum(per_m.values())
+    achieved = per_step_bytes / (kern_ms * 1e-3) / 1e9
+    hbm = pk["hbm_gbs"]
+
+    # end to end through the public API with pinned host buffers
+    Xh = {M: X[M].cpu().pin_memory() for M in Ms}
+    Yh = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in Ms}
+    e2e_steps = max(8, min(args.steps, 4 * R))
+
+    def e2e_step():
+        n = 0
+        for M in Ms:
+            r = ctr[0] % R
+            ctr[0] += 1
+            X[M].copy_(Xh[M], non_blocking=True)
+            lcvq.gemm(X[M], copies[r], K, A, B, d, out=Y[M], workspace=ws[M])
+            n += lcvq.last_launch_count()
+            Yh[M].copy_(Y[M], non_blocking=True)
+        return n
+
+    ge = StepGraphs(e2e_step, R, e2e_steps)
+    ge.replay()
+    e2e_ms, _, _ = timed_graphs(D, ge)
+    e2e = dict(value=D.world * e2e_steps * per_step_bytes / (e2e_ms * 1e-3) / 1e9, unit="GB/s",
+               h2d_bytes_per_step=int(sum(M * K * 2 for M in Ms)),
+               d2h_bytes_per_step=int(sum(M * N * 2 for M in Ms)),
+               note="each step copies X in from pinned host memory and Y back, inside the timed graph")
+
+    res = dict(
+        metric=METRIC, value=value, unit="GB/s", n_gpus=D.world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=ms_total / args.steps, higher_is_better=True,
+        scaling="weak", vs_baseline=None, dtype="bf16",
+        data="synthetic (seeded: W_p ~ U[-0.5,3.5] -> uniform codes; X ~ N(0,1), 1% channels x20)",
+        config={"workload": "decode_gemv d_in=4096 d_out=4096 d=8 M={1,4,16} bf16",
+                "l2": f"inputs larger than L2: {R} rotated packed-weight copies ({R * 4} MiB)",
+                "parallelism": f"replicas x{D.world}" if D.world > 1 else "single GPU"},
+        roofline=dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
+                      traffic=None, kernel="gemv_kernel (decode-GEMV, M=1,4,16 summed)",
+                      per_m_us={str(M): per_m[M] * 1e3 for M in Ms},
+                      peak_source=f"{PEAK_SRC} hbm_gbs"),
+        e2e=e2e, clocks=ck, gpu_launches=int(launches), parity_max_rel_err=parity,
+    )
+    return res
+
+
+# ----------------------------------------------------------------------------- other rows
+def row_assign_pack(D, pk):
+    """Assign + pack (+ mask) on the QAT-step weights: 4096 x 14336 fp32."""
+    dev = D.dev
+    N, K = 4096, 14336
+    w = synth.workload(4, M=1, with_dy=False)
+    Wp = torch.from_numpy(w["Wp"]).to(dev)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    mask = torch.empty((N, K // 8), dtype=torch.uint8, device=dev)
+    from oracle import lcvq_oracle as O
+    z, m = O.assign(w["Wp"])
+    lcvq.assign_pack(Wp, 8, packed=packed, mask=mask)
+    exact = bool(np.array_equal(packed.cpu().numpy(), O.pack_codes(z)) and
+                 np.array_equal(mask.cpu().numpy(), O.pack_mask(m)))
+    ms = ev_time(lambda: lcvq.assign_pack(Wp, 8, packed=packed, mask=mask), 50)
+    nbytes = N * K * (4 + 0.25 + 0.125)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return dict(metric="assign+pack GB/s (fp32 in, codes+mask out)", value=gbs, unit="GB/s",
+                us=ms * 1e3, bit_exact=exact,
+                roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
+                              frac=gbs / pk["hbm_gbs"]))
+
+
+def row_decode(D, pk):
+    dev = D.dev
+    N, K = 4096, 14336
+    w = synth.workload(4, M=1, with_dy=False)
+    packed, _ = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev), 8, with_mask=False)
+    A = torch.from_numpy(w["A"]).to(dev)
+    B = torch.from_numpy(w["B"]).to(dev)
+    W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    ms = ev_time(lambda: lcvq.decode(packed, K, A, B, 8, out=W), 50)
+    nbytes = N * K * (0.25 + 2)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return dict(metric="decode GB/s (codes in, bf16 W~ out)", value=gbs, unit="GB/s", us=ms * 1e3,
+                roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
+                              frac=gbs / pk["hbm_gbs"]))
+
+
+def row_prefill(D, pk):
+    """Prefill GEMM, d_in=4096 -> d_out=11008, M=2048, both forward forms."""
+    dev = D.dev
+    M, K, N, d = 2048, 4096, 11008, 8
+    w = synth.workload(3, M=M, with_dy=False)
+    packed, _ = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev), d, with_mask=False)
+    A = torch.from_numpy(w["A"]).to(dev)
+    B = torch.from_numpy(w["B"]).to(dev)
+    X = torch.from_numpy(w["X"]).to(torch.bfloat16).to(dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, d), dev)
+    from oracle import lcvq_oracle as O
+    z, _ = O.assign(w["Wp"])
+    rng = np.random.Generator(np.random.PCG64(1))
+    pairs = [(int(a), int(b)) for a, b in zip(rng.integers(0, M, 256), rng.integers(0, N, 256))]
+    out = {}
+    flops = 2.0 * M * N * K
+    for form in ("algebraic", "decode"):
+        lcvq.gemm(X, packed, K, A, B, d, form=form, out=Y, workspace=ws)
+        Yc = Y.float().cpu().numpy()
+        y, dd = O.forward_sampled(w["X"], {n: z[n] for _, n in pairs}, w["A"], w["B"], pairs)
+        err = O.rel_err(np.array([Yc[m, n] for m, n in pairs]), y, dd)
+        ms = ev_time(lambda: lcvq.gemm(X, packed, K, A, B, d, form=form, out=Y, workspace=ws), 5)
+        tf = flops / (ms * 1e-3) / 1e12
+        out[form] = dict(value=tf, unit="TFLOP/s", us=ms * 1e3, sampled_rel_err=err,
+                         roofline=dict(bound="tensor", achieved=tf, peak=pk["bf16_tflops"],
+                                       unit="TFLOP/s", frac=tf / pk["bf16_tflops"]))
+    return dict(metric="prefill GEMM TFLOP/s (2MNK / time)", forms=out)
+
+
+def row_qat(D, pk):
+    """QAT step on d_in=14336, d_out=4096, M=8192: assign/pack, forward, backward."""
+    dev = D.dev
+    M, K, N, d = 8192, 14336, 4096, 8
+    w = synth.workload(4, M=M)
+    Wp = torch.from_numpy(w["Wp"]).to(dev)
+    A = torch.from_numpy(w["A"]).to(dev)
+    B = torch.from_numpy(w["B"]).to(dev)
+    X = torch.from_numpy(w["X"]).to(torch.bfloat16).to(dev)
+    dY = torch.from_numpy(w["dY"]).to(torch.bfloat16).to(dev)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    mask = torch.empty((N, K // 8), dtype=torch.uint8, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    wsf = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, d), dev)
+    wsb = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM_BACKWARD, torch.bfloat16, M, N, K, d), dev)
+    outs = dict(dX=torch.empty((M, K), dtype=torch.bfloat16, device=dev),
+                dWp=torch.empty((N, K), dtype=torch.float32, device=dev),
+                dA=torch.empty((d, d), dtype=torch.float32, device=dev),
+                dB=torch.empty((d,), dtype=torch.float32, device=dev))
+    t_ap = ev_time(lambda: lcvq.assign_pack(Wp, d, packed=packed, mask=mask), 3)
+    t_fw = ev_time(lambda: lcvq.gemm(X, packed, K, A, B, d, out=Y, workspace=wsf), 2)
+    t_bw = ev_time(lambda: lcvq.gemm_backward(X, dY, packed, mask, K, A, B, d, outs=outs,
+                                              workspace=wsb), 1)
+    gemm_flops = 2.0 * M * N * K
+    total = t_ap + t_fw + t_bw
+    tf = 3 * gemm_flops / (total * 1e-3) / 1e12
+    return dict(metric="QAT step TFLOP/s (3 x 2MNK / step time)", value=tf, unit="TFLOP/s",
+                step_us=total * 1e3, assign_pack_us=t_ap * 1e3, forward_us=t_fw * 1e3,
+                backward_us=t_bw * 1e3,
+                roofline=dict(bound="tensor", achieved=tf, peak=pk["bf16_tflops_sustained"],
+                              unit="TFLOP/s", frac=tf / pk["bf16_tflops_sustained"]))
+
+
+def row_stack(D, pk):
+    """7B-shaped stack: 224 matrices, M in {1, 8, 32}; packed GB/s over the stack."""
+    dev = D.dev
+    mats = []
+    for layer in range(32):
+        for p in range(len(synth.STACK_PROJS)):
+            m = synth.stack_matrix(layer, p, 32, with_x=(layer == 0))
+            mats.append(m)
+    total_bytes = sum(m["packed"].nbytes for m in mats)
+    dmats = []
+    xs = {}
+    for m in mats:
+        key = (m["proj"], m["d_in"])
+        if m["layer"] == 0:
+            xs[m["proj"]] = torch.from_numpy(m["X"]).to(torch.bfloat16).to(dev)
+        dmats.append(dict(packed=torch.from_numpy(m["packed"]).to(dev), A=torch.from_numpy(m["A"]).to(dev),
+                          B=torch.from_numpy(m["B"]).to(dev), proj=m["proj"], d_in=m["d_in"],
+                          d_out=m["d_out"]))
+    out = {}
+    for M in (1, 8, 32):
+        ys = {p: torch.empty((M, do), dtype=torch.bfloat16, device=dev) for p, _, do in synth.STACK_PROJS}
+        wss = {p: lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, do, di, 8), dev)
+               for p, di, do in synth.STACK_PROJS}
+
+        def run(M=M, ys=ys, wss=wss):
+            n = 0
+            for m in dmats:
+                lcvq.gemm(xs[m["proj"]][:M], m["packed"], m["d_in"], m["A"], m["B"], 8,
+                          out=ys[m["proj"]], workspace=wss[m["proj"]])
+                n += lcvq.last_launch_count()
+            return n
+        sg = StepGraphs(run, 1, 5)
+        sg.replay()
+        t, _, _ = timed_graphs(D, sg)
+        ms = t / 5
+        gbs = total_bytes / (ms * 1e-3) / 1e9
+        out[str(M)] = dict(value=gbs, unit="GB/s", us=ms * 1e3,
+                           roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
+                                         frac=gbs / pk["hbm_gbs"]))
+    return dict(metric="stack packed-weight GB/s (224 matrices, 1.62 GB of codes)", per_m=out,
+                packed_bytes=total_bytes)
+
+
+ROWS = {"assign_pack": row_assign_pack, "decode": row_decode, "prefill": row_prefill,
+        "qat": row_qat, "stack": row_stack}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    global PEAK_SRC
+    args = parse()
+    pk, PEAK_SRC = peaks()
+    if args.impl == "reference":
+        D_rank = int(os.environ.get("RANK", "0"))
+        if D_rank != 0:
+            return 0
+        cb = oracle_gemv_sample((1, 4, 16), seconds=10.0)
+        line = dict(impl="reference", metric=METRIC, value=cb["value"], unit="GB/s",
+                    n_gpus=int(os.environ.get("WORLD_SIZE", "1")), steps=args.steps,
+                    warmup=args.warmup, higher_is_better=True, scaling="weak", vs_baseline=None,
+                    dtype="f64", data="synthetic",
+                    config={"workload": "decode_gemv d_in=4096 d_out=4096 d=8 M={1,4,16} bf16"},
+                    cpu_baseline=cb,
+                    e2e=dict(value=cb["value"], unit="GB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+        print(json.dumps(line))
+        return 0
+
+    D = Dist()
+    res = headline(args, D, pk)
+    if D.rank == 0 and D.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = oracle_gemv_sample((1, 4, 16), seconds=10.0)
+    rows = {}
+    want = list(ROWS) if args.rows == "all" else ([] if args.rows == "none" else args.rows.split(","))
+    if D.rank == 0:
+        for name in want:
+            try:
+                rows[name] = ROWS[name](D, pk)
+            except Exception as ex:  # report, do not hide
+                rows[name] = {"error": f"{type(ex).__name__}: {ex}"}
+            torch.cuda.empty_cache()
+    res["rows"] = rows
+    if D.rank == 0:
+        print(json.dumps(res))
+    D.close()
+    return 0
+
+
+PEAK_SRC = "measured"
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,280 @@
+// C ABI of liblcvq: argument validation, workspace layout and dispatch.
+// Every entry point validates all of its arguments before it launches
+// anything, so a failing call has no side effect.
+#include <atomic>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace lcvq;
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, 2 other
+
+lcvq_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LCVQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LCVQ_ERR_UNSUPPORTED;
+  int v = g_dev_ok[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return LCVQ_ERR_CUDA;
+    v = (major == 10 && minor == 0) ? 1 : 2;
+    g_dev_ok[dev].store(v, std::memory_order_relaxed);
+  }
+  return v == 1 ? LCVQ_OK : LCVQ_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_d(int d) { return d == 1 || d == 2 || d == 4 || d == 8; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- workspace layouts ----
+struct GemmWs {
+  size_t xpp_off, corr_off, total;
+};
+GemmWs gemm_ws(lcvq_dtype dtype, int64_t M, int64_t d_in) {
+  GemmWs w{};
+  size_t off = kWsHeaderBytes;
+  if (dtype == LCVQ_BF16) {
+    w.xpp_off = off;
+    off = round_up(off + size_t(M) * size_t(d_in) * 2, 256);
+    w.corr_off = off;
+    off = round_up(off + size_t(M) * 4, 256);
+  }
+  w.total = off;
+  return w;
+}
+struct BwdWs {
+  size_t part_off, num_parts, total;
+};
+BwdWs bwd_ws(int64_t d_out, int64_t d_in, int d) {
+  BwdWs w{};
+  w.num_parts = size_t(simt_dw_num_tiles(d_out, d_in));
+  w.part_off = kWsHeaderBytes;
+  w.total = round_up(w.part_off + w.num_parts * size_t(d * d + d) * 4, 256);
+  return w;
+}
+
+lcvq_status finish(cudaError_t e, int launches) {
+  if (e != cudaSuccess) return LCVQ_ERR_CUDA;
+  g_last_launches = launches;
+  return LCVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lcvq_status_string(lcvq_status s) {
+  switch (s) {
+    case LCVQ_OK: return "LCVQ_OK";
+    case LCVQ_ERR_INVALID_ARG: return "LCVQ_ERR_INVALID_ARG";
+    case LCVQ_ERR_UNSUPPORTED: return "LCVQ_ERR_UNSUPPORTED";
+    case LCVQ_ERR_ALIGNMENT: return "LCVQ_ERR_ALIGNMENT";
+    case LCVQ_ERR_WORKSPACE: return "LCVQ_ERR_WORKSPACE";
+    case LCVQ_ERR_CUDA: return "LCVQ_ERR_CUDA";
+    case LCVQ_ERR_DEVICE_TIMEOUT: return "LCVQ_ERR_DEVICE_TIMEOUT";
+  }
+  return "LCVQ_ERR_UNKNOWN";
+}
+
+int lcvq_last_launch_count(void) { return g_last_launches; }
+
+lcvq_status lcvq_assign_pack(const float* Wp, int64_t d_out, int64_t d_in, int d,
+                             uint8_t* packed, uint8_t* mask_bits, void* stream) {
+  if (d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
+  if (d_in % 8 != 0 || d_in % d != 0) return LCVQ_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d_out == 0 || d_in == 0) return LCVQ_OK;
+  if (Wp == nullptr || packed == nullptr) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(Wp) || !aligned16(packed) || (mask_bits && !aligned16(mask_bits)))
+    return LCVQ_ERR_ALIGNMENT;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  cudaError_t e = launch_assign_pack(Wp, d_out * d_in, packed, mask_bits,
+                                     static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
+}
+
+lcvq_status lcvq_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
+                        const float* A, const float* B, void* W, lcvq_dtype w_dtype,
+                        void* stream) {
+  if (d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
+  if (d_in % 16 != 0) return LCVQ_ERR_INVALID_ARG;
+  if (w_dtype != LCVQ_F32 && w_dtype != LCVQ_BF16) return LCVQ_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d_out == 0 || d_in == 0) return LCVQ_OK;
+  if (!packed || !A || !B || !W) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(W) || !aligned16(A) || !aligned16(B))
+    return LCVQ_ERR_ALIGNMENT;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  cudaError_t e = launch_decode(packed, d_out, d_in, d, A, B, W, w_dtype == LCVQ_BF16,
+                                static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
+}
+
+size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_out, int64_t d_in,
+                           int d) {
+  if (M < 0 || d_out < 0 || d_in < 0 || !valid_d(d)) return 0;
+  if (dtype != LCVQ_F32 && dtype != LCVQ_BF16) return 0;
+  if (op == LCVQ_OP_GEMM) return gemm_ws(dtype, M, d_in).total;
+  if (op == LCVQ_OP_GEMM_BACKWARD) return bwd_ws(d_out, d_in, d).total;
+  return 0;
+}
+
+static lcvq_status validate_gemm_shapes(lcvq_dtype dtype, int64_t M, int64_t d_out, int64_t d_in,
+                                        int d) {
+  if (M < 0 || d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
+  if (dtype != LCVQ_F32 && dtype != LCVQ_BF16) return LCVQ_ERR_INVALID_ARG;
+  if (d_in % 64 != 0 || d_out % 8 != 0) return LCVQ_ERR_INVALID_ARG;
+  if (M > INT32_MAX) return LCVQ_ERR_INVALID_ARG;
+  return LCVQ_OK;
+}
+
+lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t* packed,
+                      int64_t d_out, int64_t d_in, int d, const float* A, const float* B,
+                      void* Y, lcvq_form form, void* workspace, size_t ws_bytes, void* stream) {
+  if (lcvq_status st = validate_gemm_shapes(dtype, M, d_out, d_in, d); st != LCVQ_OK) return st;
+  if (form != LCVQ_FORM_AUTO && form != LCVQ_FORM_DECODE && form != LCVQ_FORM_ALGEBRAIC)
+    return LCVQ_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (M == 0 || d_out == 0) return LCVQ_OK;
+  if (!Y) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(Y)) return LCVQ_ERR_ALIGNMENT;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t esz = dtype == LCVQ_BF16 ? 2 : 4;
+  if (d_in == 0) {
+    if (cudaMemsetAsync(Y, 0, size_t(M) * size_t(d_out) * esz, s) != cudaSuccess)
+      return LCVQ_ERR_CUDA;
+    return LCVQ_OK;
+  }
+  if (!X || !packed || !A || !B || !workspace) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(packed) || !aligned16(A) || !aligned16(B) ||
+      !aligned16(workspace))
+    return LCVQ_ERR_ALIGNMENT;
+  const GemmWs w = gemm_ws(dtype, M, d_in);
+  if (ws_bytes < w.total) return LCVQ_ERR_WORKSPACE;
+
+  int launches = 0;
+  cudaError_t e = cudaSuccess;
+  char* ws = static_cast<char*>(workspace);
+  if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
+    uint16_t* Xpp = reinterpret_cast<uint16_t*>(ws + w.xpp_off);
+    float* corr = reinterpret_cast<float*>(ws + w.corr_off);
+    e = launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr, s, &launches);
+    if (e == cudaSuccess)
+      e = launch_gemm_xformed(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), s,
+                              &launches);
+  } else {
+    e = launch_simt_forward(X, dtype == LCVQ_BF16, M, packed, d_out, d_in, d, A, B, Y, s,
+                            &launches);
+  }
+  return finish(e, launches);
+}
+
+lcvq_status lcvq_xform(const void* X, lcvq_dtype dtype, int64_t M, int64_t d_in, int d,
+                       const float* A, const float* B, void* Xpp, float* corr, void* stream) {
+  if (lcvq_status st = validate_gemm_shapes(dtype, M, 8, d_in, d); st != LCVQ_OK) return st;
+  if (dtype != LCVQ_BF16) return LCVQ_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (M == 0 || d_in == 0) return LCVQ_OK;
+  if (!X || !A || !B || !Xpp || !corr) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Xpp) || !aligned16(corr))
+    return LCVQ_ERR_ALIGNMENT;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  cudaError_t e = launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B,
+                               static_cast<uint16_t*>(Xpp), corr,
+                               static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
+}
+
+lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64_t M,
+                              const uint8_t* packed, int64_t d_out, int64_t d_in, void* Y,
+                              void* stream) {
+  if (lcvq_status st = validate_gemm_shapes(LCVQ_BF16, M, d_out, d_in, 8); st != LCVQ_OK) return st;
+  g_last_launches = 0;
+  if (M == 0 || d_out == 0) return LCVQ_OK;
+  if (!Xpp || !corr || !packed || !Y) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(Xpp) || !aligned16(corr) || !aligned16(packed) || !aligned16(Y))
+    return LCVQ_ERR_ALIGNMENT;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  cudaError_t e = launch_gemm_xformed(static_cast<const uint16_t*>(Xpp), corr, M, packed, d_out,
+                                      d_in, static_cast<uint16_t*>(Y),
+                                      static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
+}
+
+lcvq_status lcvq_gemm_backward(const void* X, const void* dY, lcvq_dtype dtype, int64_t M,
+                               const uint8_t* packed, const uint8_t* mask_bits, int64_t d_out,
+                               int64_t d_in, int d, const float* A, const float* B, void* dX,
+                               float* dA, float* dB, float* dWp, void* workspace,
+                               size_t ws_bytes, void* stream) {
+  if (lcvq_status st = validate_gemm_shapes(dtype, M, d_out, d_in, d); st != LCVQ_OK) return st;
+  g_last_launches = 0;
+  if (!dA || !dB) return LCVQ_ERR_INVALID_ARG;
+  if (dWp != nullptr && mask_bits == nullptr) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(dA) || !aligned16(dB) || (dWp && !aligned16(dWp)) || (dX && !aligned16(dX)) ||
+      (mask_bits && !aligned16(mask_bits)))
+    return LCVQ_ERR_ALIGNMENT;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t esz = dtype == LCVQ_BF16 ? 2 : 4;
+  if (M == 0 || d_out == 0 || d_in == 0) {
+    // no tokens / no weights: all gradients are empty sums
+    if (cudaMemsetAsync(dA, 0, size_t(d) * d * 4, s) != cudaSuccess) return LCVQ_ERR_CUDA;
+    if (cudaMemsetAsync(dB, 0, size_t(d) * 4, s) != cudaSuccess) return LCVQ_ERR_CUDA;
+    if (dWp && d_out > 0 && d_in > 0 &&
+        cudaMemsetAsync(dWp, 0, size_t(d_out) * size_t(d_in) * 4, s) != cudaSuccess)
+      return LCVQ_ERR_CUDA;
+    if (dX && M > 0 && d_in > 0 &&
+        cudaMemsetAsync(dX, 0, size_t(M) * size_t(d_in) * esz, s) != cudaSuccess)
+      return LCVQ_ERR_CUDA;
+    return LCVQ_OK;
+  }
+  if (!X || !dY || !packed || !A || !B || !workspace) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(packed) || !aligned16(A) || !aligned16(B) ||
+      !aligned16(workspace))
+    return LCVQ_ERR_ALIGNMENT;
+  const BwdWs w = bwd_ws(d_out, d_in, d);
+  if (ws_bytes < w.total) return LCVQ_ERR_WORKSPACE;
+  float* partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + w.part_off);
+  const bool bf = dtype == LCVQ_BF16;
+  int launches = 0;
+  cudaError_t e = cudaSuccess;
+  if (dX) e = launch_simt_backward_dx(dY, bf, M, packed, d_out, d_in, d, A, B, dX, s, &launches);
+  if (e == cudaSuccess)
+    e = launch_simt_backward_dw(X, dY, bf, M, packed, mask_bits, d_out, d_in, d, A, dWp, partials,
+                                s, &launches);
+  if (e == cudaSuccess)
+    e = launch_reduce_partials(partials, int64_t(w.num_parts), d, dA, dB, s, &launches);
+  return finish(e, launches);
+}
+
+lcvq_status lcvq_check_device_error(void* workspace, void* stream) {
+  if (!workspace) return LCVQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int h[2] = {0, 0};
+  if (cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return LCVQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LCVQ_ERR_CUDA;
+  if (h[0] != 0) {
+    const unsigned int zero[2] = {0, 0};
+    if (cudaMemcpy(workspace, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return LCVQ_ERR_CUDA;
+    return h[0] == LCVQ_ERR_DEVICE_TIMEOUT ? LCVQ_ERR_DEVICE_TIMEOUT : LCVQ_ERR_CUDA;
+  }
+  return LCVQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// Internal launchers behind the C ABI (host side).  Each returns the CUDA error
+// of its launch(es) and adds the number of kernels it launched to *launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lcvq {
+
+// ---- elementwise ----
+cudaError_t launch_assign_pack(const float* Wp, int64_t n_elems, uint8_t* packed,
+                               uint8_t* mask_bits, cudaStream_t s, int* launches);
+cudaError_t launch_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
+                          const float* A, const float* B, void* W, bool w_bf16,
+                          cudaStream_t s, int* launches);
+
+// ---- algebraic-form prologue (bf16 tensor-core paths) ----
+// Xpp[M][d_in] bf16: X' = group-wise X A, rounded to bf16, scaled by the
+// per-position power of two of the code decoder, in the decoder's K order.
+// corr[M] fp32: per-row constant that turns the tensor-core accumulator into Y.
+cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
+                         const float* B, uint16_t* Xpp, float* corr, cudaStream_t s,
+                         int* launches);
+
+// ---- decode-GEMV (bf16, M <= 32) ----
+cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
+                        int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s, int* launches);
+
+// integer-code GEMM on X'' (dispatches on M: decode-GEMV for M <= 32, else
+// the CUDA-core fallback until the tensor-core GEMM takes it)
+cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,
+                                const uint8_t* packed, int64_t d_out, int64_t d_in, uint16_t* Y,
+                                cudaStream_t s, int* launches);
+
+// ---- CUDA-core paths (any M; fp32 or bf16 activations) ----
+cudaError_t launch_simt_forward(const void* X, bool bf16, int64_t M, const uint8_t* packed,
+                                int64_t d_out, int64_t d_in, int d, const float* A,
+                                const float* B, void* Y, cudaStream_t s, int* launches);
+cudaError_t launch_simt_backward_dx(const void* dY, bool bf16, int64_t M, const uint8_t* packed,
+                                    int64_t d_out, int64_t d_in, int d, const float* A,
+                                    const float* B, void* dX, cudaStream_t s, int* launches);
+// G = dY^T X tiles with the fused epilogue: dWp (if non-null) and per-tile
+// partials of dA/dB into `partials` ([num_tiles][d*d + d] fp32).
+cudaError_t launch_simt_backward_dw(const void* X, const void* dY, bool bf16, int64_t M,
+                                    const uint8_t* packed, const uint8_t* mask_bits,
+                                    int64_t d_out, int64_t d_in, int d, const float* A,
+                                    float* dWp, float* partials, cudaStream_t s, int* launches);
+int64_t simt_dw_num_tiles(int64_t d_out, int64_t d_in);
+
+// fixed-order fp64 reduction of [num_parts][d*d + d] fp32 partials into dA, dB
+cudaError_t launch_reduce_partials(const float* partials, int64_t num_parts, int d, float* dA,
+                                   float* dB, cudaStream_t s, int* launches);
+
+}  // namespace lcvq

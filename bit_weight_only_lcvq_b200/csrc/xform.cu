@@ -1,0 +1,139 @@
+// Prologue of the algebraic form of the forward (LC-QAT technical summary,
+// Methodology 3: the forward is recast onto INT2 x FP16 matmul operators).
+//
+// For every activation row x and every d-vector g:
+//     sum_k x_k W~[n][k] = sum_g x_g^T (A z_g + B)
+//                        = sum_k X'_k z_k + sum_g x_g^T B
+// with X'[g d + j] = sum_i x[g d + i] A[i][j].  Centering the codes
+// (zc = z - 3/2, W~ = A zc + B', B' = B + 3/2 A 1) gives the same sum as
+// sum_k X'_k zc_k + s', s' = sum_g x_g^T B'.
+//
+// The tensor-core main loops multiply X'' (below) with codes that are decoded
+// by one LOP3 each into the bf16 value 128 + 4^p z, p = p(position) in {0,1,2}
+// (the code lands in mantissa bits 2p..2p+1 of a bf16 whose exponent says 128).
+// So the B operand is X'' = bf16(X') * 4^-p (exact power-of-two scaling) and
+//     acc = sum_k X''_k (128 + 4^p z_k) = sum_k X'r_k z_k + 128 sum_k X''_k,
+// where X'r = bf16(X').  The per-row constant
+//     corr = s' - 3/2 sum_k X'r_k - 128 sum_k X''_k
+// makes acc + corr = sum_k X'r_k zc_k + s': the centred form, whose only
+// rounding is that of X' to bf16 (relative 2^-9 per term, against codes of
+// magnitude <= 3/2).  The sums are formed in fp64.
+//
+// K order ("decoder order"): inside every block of 16 consecutive k, the decoder
+// turns one 32-bit word of codes into 8 bf16x2 pairs, pair c holding positions
+// c and c + 8 (the same bit offset in the two 16-bit halves).  X'' is stored in
+// that order: element 2c of the block is position c, element 2c+1 is c + 8;
+// p(c) = c mod 3.
+#include "common.cuh"
+#include "internal.h"
+
+namespace lcvq {
+
+constexpr int kXfThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __restrict__ X,
+                                                           int64_t d_in,
+                                                           const float* __restrict__ A,
+                                                           const float* __restrict__ B,
+                                                           uint16_t* __restrict__ Xpp,
+                                                           float* __restrict__ corr) {
+  __shared__ float sA[D * D];
+  __shared__ float sBp[D];
+  __shared__ double red[3][kXfThreads / 32];
+  if (threadIdx.x < D * D) sA[threadIdx.x] = A[threadIdx.x];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float rs = 0.f;
+    for (int j = 0; j < D; ++j) rs += sA[threadIdx.x * D + j];
+    sBp[threadIdx.x] = B[threadIdx.x] + 1.5f * rs;
+  }
+  __syncthreads();
+
+  const int64_t m = blockIdx.x;
+  const uint16_t* xr = X + m * d_in;
+  uint16_t* orow = Xpp + m * d_in;
+  double s_b = 0.0, s_xr = 0.0, s_xpp = 0.0;
+  const int64_t nblk = d_in / 16;
+  for (int64_t b = threadIdx.x; b < nblk; b += kXfThreads) {
+    const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
+    const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float x[16];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      x[2 * q] = bf16_lo(w[q]);
+      x[2 * q + 1] = bf16_hi(w[q]);
+    }
+    float xrd[16];  // bf16(X') as fp32
+    float sb = 0.f, sxr = 0.f;
+#pragma unroll
+    for (int v = 0; v < 16 / D; ++v) {
+#pragma unroll
+      for (int j = 0; j < D; ++j) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < D; ++i) acc = fmaf(x[v * D + i], sA[i * D + j], acc);
+        xrd[v * D + j] = bf16_to_f32(f32_to_bf16(acc));
+        sxr += xrd[v * D + j];
+      }
+#pragma unroll
+      for (int i = 0; i < D; ++i) sb = fmaf(x[v * D + i], sBp[i], sb);
+    }
+    uint32_t o[8];
+    float sxpp = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float scale = (c % 3 == 0) ? 1.0f : ((c % 3 == 1) ? 0.25f : 0.0625f);
+      const float lo = xrd[c] * scale;
+      const float hi = xrd[c + 8] * scale;
+      sxpp += lo + hi;
+      o[c] = pack_bf16x2(lo, hi);  // exact: power-of-two scaling of bf16 values
+    }
+    uint4* dst = reinterpret_cast<uint4*>(orow + 16 * b);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    s_b += sb;
+    s_xr += sxr;
+    s_xpp += sxpp;
+  }
+  // block reduction in a fixed order
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    s_b += __shfl_down_sync(0xffffffffu, s_b, off);
+    s_xr += __shfl_down_sync(0xffffffffu, s_xr, off);
+    s_xpp += __shfl_down_sync(0xffffffffu, s_xpp, off);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[0][warp] = s_b;
+    red[1][warp] = s_xr;
+    red[2][warp] = s_xpp;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0, b = 0.0, c = 0.0;
+    for (int w = 0; w < kXfThreads / 32; ++w) {
+      a += red[0][w];
+      b += red[1][w];
+      c += red[2][w];
+    }
+    corr[m] = static_cast<float>(a - 1.5 * b - 128.0 * c);
+  }
+}
+
+cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
+                         const float* B, uint16_t* Xpp, float* corr, cudaStream_t s,
+                         int* launches) {
+  const dim3 grid(static_cast<unsigned>(M));
+  switch (d) {
+    case 1: xform_kernel<1><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
+    case 2: xform_kernel<2><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
+    case 4: xform_kernel<4><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
+    default: xform_kernel<8><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
+  }
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace lcvq

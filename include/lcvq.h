@@ -1,0 +1,199 @@
+/*
+ * lcvq.h - C ABI of liblcvq: the data-parallel hot path of linear-constrained
+ * vector quantization (LC-VQ) at 2 bits per weight, for NVIDIA B200 (sm_100a).
+ *
+ * The method (LC-QAT: Data-Efficient 2-Bit QAT for LLMs via Linear-Constrained
+ * Vector Quantization; technical summary, Methodology 1 and 3):
+ *   - a weight matrix is cut into d-element vectors along its input dimension;
+ *   - each vector is the codeword c = A z + B of a 2-bit code z in {0,1,2,3}^d,
+ *     with A (d x d) and B (d) floating-point parameters shared by the whole
+ *     matrix (Methodology 1, "linear-constrained parameterization");
+ *   - in QAT the float proxy weights W_p are rounded and clamped to the codes
+ *     W_z, decoded as A W_z + B and used in the layer's matmul; gradients reach
+ *     A, B and (straight-through the rounding) W_p (Methodology 3, "training
+ *     pipeline", and the gradient-estimation ablation, which uses STE).
+ *
+ * Conventions (shared by every call):
+ *   - Storage order: weights [d_out][d_in] row-major (the transpose of the
+ *     d_in x d_out matrix W~ of decoupleQ eq. (1), Y = X W~); activations
+ *     [M][d_in] and [M][d_out] row-major.  So Y[m][n] = sum_k X[m][k] W~[n][k].
+ *   - Vectors are d consecutive elements along d_in: element k of row n belongs
+ *     to vector k / d, position k % d.  c_i = sum_j A[i*d + j] z_j + B[i]
+ *     (A row-major, acting on column vectors).
+ *   - Packed codes, format V1: [d_out][d_in/4] bytes; element k of a row sits in
+ *     byte k/4 at bits 2(k%4) and 2(k%4)+1 (LSB first).  For d = 8 the two bytes
+ *     of one vector read as a little-endian u16 equal its codebook index
+ *     sum_j z_j 4^j.
+ *   - Clamp mask bits: [d_out][d_in/8] bytes, bit k%8 of byte k/8, set where
+ *     0 <= W_p <= 3 (the straight-through pass region).
+ *   - Rounding is round-half-to-even; NaN -> 0, +inf -> 3, -inf -> 0; NaN is
+ *     outside the mask.
+ *
+ * Ownership and execution: every pointer is a DEVICE pointer owned by the
+ * caller (except where a parameter says "host").  The library allocates no
+ * device memory and never synchronizes the stream on the hot path; scratch goes
+ * in a caller-provided workspace sized by lcvq_workspace_size().  All calls are
+ * asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the legacy
+ * default stream).  Outputs are overwritten, never accumulated into.
+ *
+ * Errors: arguments are validated before anything is launched; a failing call
+ * launches nothing and returns a status.  Launch failures return
+ * LCVQ_ERR_CUDA.  Kernels that wait on mbarriers give up after a bounded number
+ * of polls and record LCVQ_ERR_DEVICE_TIMEOUT in the workspace's error word,
+ * read by lcvq_check_device_error().  Nothing aborts, throws or traps.
+ *
+ * Requirements: a compute capability 10.0 device (sm_100a); otherwise
+ * LCVQ_ERR_UNSUPPORTED.  Pointers 16-byte aligned (LCVQ_ERR_ALIGNMENT).
+ * d in {1, 2, 4, 8}.  Shape rules are listed per call.  Thread safety: calls
+ * hold no global state except a per-device cache of device properties and
+ * kernel attributes, guarded for concurrent first use.
+ */
+#ifndef LCVQ_H_
+#define LCVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LCVQ_FORMAT_V1 1
+
+#if defined(__GNUC__)
+#define LCVQ_API __attribute__((visibility("default")))
+#else
+#define LCVQ_API
+#endif
+
+typedef enum {
+  LCVQ_OK = 0,
+  LCVQ_ERR_INVALID_ARG = 1,    /* null pointer, bad shape, bad enum */
+  LCVQ_ERR_UNSUPPORTED = 2,    /* not an sm_100 device, or unsupported d/dtype combination */
+  LCVQ_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
+  LCVQ_ERR_WORKSPACE = 4,      /* workspace missing or smaller than lcvq_workspace_size() */
+  LCVQ_ERR_CUDA = 5,           /* a CUDA runtime call or kernel launch failed */
+  LCVQ_ERR_DEVICE_TIMEOUT = 6  /* a device-side bounded wait gave up (from lcvq_check_device_error) */
+} lcvq_status;
+
+typedef enum {
+  LCVQ_F32 = 0,   /* float */
+  LCVQ_BF16 = 1   /* bfloat16 bit patterns (uint16_t) */
+} lcvq_dtype;
+
+/* Forward formulation for lcvq_gemm (both compute the same Y = X W~):
+ *  DECODE:    codes are decoded to bf16 tiles of A z + B on chip and multiplied
+ *             with X directly.
+ *  ALGEBRAIC: X is first multiplied group-wise by A (X'[m][g d + j] =
+ *             sum_i X[m][g d + i] A[i][j]) and dotted with B; the main loop then
+ *             multiplies X' with the raw integer codes and adds the per-row
+ *             B term:  Y = X' Z^T + s 1^T.  Exact algebra on
+ *             sum_k x_k w~_k = sum_g x_g^T (A z_g + B).
+ *  AUTO:      the library's choice (ALGEBRAIC on the tensor-core paths). */
+typedef enum { LCVQ_FORM_AUTO = 0, LCVQ_FORM_DECODE = 1, LCVQ_FORM_ALGEBRAIC = 2 } lcvq_form;
+
+typedef enum { LCVQ_OP_GEMM = 0, LCVQ_OP_GEMM_BACKWARD = 1 } lcvq_op;
+
+/* Code assignment and 2-bit packing (LC-QAT technical summary, Methodology 1:
+ * index selection becomes rounding and clamping; Methodology 3: proxy weights
+ * are rounded and clamped to integer weights).
+ *   Wp        [d_out][d_in] fp32 proxy weights (read only).
+ *   packed    [d_out][d_in/4] out: codes z = clamp(rint(Wp), 0, 3), format V1.
+ *   mask_bits [d_out][d_in/8] out, may be NULL: bit set where 0 <= Wp <= 3.
+ *   d         vector length (only checked: d_in % d == 0).
+ * Shapes: d_in % 8 == 0; d_out, d_in >= 0 (an empty matrix is a no-op). */
+LCVQ_API lcvq_status lcvq_assign_pack(const float* Wp, int64_t d_out, int64_t d_in, int d,
+                             uint8_t* packed, uint8_t* mask_bits, void* stream);
+
+/* Decode: materialize W~[n][g d + i] = sum_j A[i][j] z[n][g d + j] + B[i]
+ * (Methodology 1, c = A z + B; Methodology 3, A W_z + B), computed in fp32 and
+ * stored as w_dtype (bf16 rounds to nearest even).
+ *   packed [d_out][d_in/4] codes; A [d*d] fp32 row-major; B [d] fp32;
+ *   W      [d_out][d_in] out.
+ * Shapes: d_in % 16 == 0. */
+LCVQ_API lcvq_status lcvq_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
+                        const float* A, const float* B, void* W, lcvq_dtype w_dtype,
+                        void* stream);
+
+/* Fused decode-and-GEMM  Y = X W~  (Methodology 3: the forward is recast onto
+ * INT2 x FP16 matmul operators; decoupleQ eq. (1) for the layer convention).
+ *   X [M][d_in] in `dtype`; Y [M][d_out] out in `dtype`.
+ *   dtype BF16: tensor-core paths (M <= 32: decode-GEMV; larger M: tcgen05
+ *   GEMM), fp32 accumulation.  dtype F32: an fp32 CUDA-core path.
+ *   form: see lcvq_form (F32 always uses DECODE).
+ *   workspace: >= lcvq_workspace_size(LCVQ_OP_GEMM, ...) bytes, 256-byte aligned.
+ * Shapes: d_in % 64 == 0, d_out % 8 == 0, M >= 0.  M == 0 or d_out == 0 is a
+ * no-op; d_in == 0 writes Y = 0. */
+LCVQ_API lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M,
+                      const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
+                      const float* A, const float* B, void* Y, lcvq_form form,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* The algebraic form in two calls (bf16 only).  lcvq_gemm with
+ * LCVQ_FORM_ALGEBRAIC is exactly lcvq_xform followed by lcvq_gemm_xformed; the
+ * split lets a caller time or reuse the halves.
+ *
+ * lcvq_xform: X'[m][g d + j] = sum_i X[m][g d + i] A[i][j] is rounded to bf16
+ * and stored in the "decoder order" the integer-code GEMM consumes: within each
+ * block of 16 consecutive k, element 2c holds position c and element 2c + 1
+ * position c + 8 (c = 0..7), each multiplied by 4^-(c mod 3).  corr[m] is the
+ * per-row constant  s'[m] - 3/2 sum_k bf16(X')[m][k] - 128 sum_k X''[m][k]
+ * with s'[m] = sum_g x_g . (B + 3/2 A 1), formed in fp64 and stored as fp32.
+ *   X [M][d_in] bf16;  Xpp [M][d_in] bf16 out;  corr [M] fp32 out.
+ * lcvq_gemm_xformed: Y[m][n] = sum_k X''[m][k] v[n][k] + corr[m], where
+ * v = 128 + 4^(c mod 3) z is the bf16 value the kernel's one-instruction code
+ * decoder produces; this equals sum_k bf16(X')[m][k] (z[n][k] - 3/2) + s'[m],
+ * the centred algebraic form of Y = X W~.
+ *   Y [M][d_out] bf16 out.
+ * Shapes as lcvq_gemm (M >= 1). */
+LCVQ_API lcvq_status lcvq_xform(const void* X, lcvq_dtype dtype, int64_t M, int64_t d_in, int d,
+                                const float* A, const float* B, void* Xpp, float* corr,
+                                void* stream);
+LCVQ_API lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64_t M,
+                                       const uint8_t* packed, int64_t d_out, int64_t d_in,
+                                       void* Y, void* stream);
+
+/* Straight-through QAT backward of Y = X W~ with W~ = decode(clamp(rint(Wp))).
+ * (Methodology 1: gradients flow through the linear map c = A z + B;
+ * Methodology 3 and the gradient-estimation ablation: STE through the
+ * rounding, zero where the clamp is active.)  Given dY = dL/dY:
+ *   dX [M][d_in]  = dY W~                               (may be NULL)
+ *   G[n][k]       = sum_m dY[m][n] X[m][k]               (never stored)
+ *   dA [d*d]      = sum_{n,g} G[n][g d + i] z[n][g d + j]   (fp32, overwritten)
+ *   dB [d]        = sum_{n,g} G[n][g d + i]                 (fp32, overwritten)
+ *   dWp [d_out][d_in] = mask * sum_i A[i][j] G[n][g d + i]   (fp32, may be NULL)
+ * X, dY, dX in `dtype`.  mask_bits is required when dWp is non-NULL.
+ * dA and dB are reduced in a fixed order (bitwise reproducible run to run).
+ * Shapes as lcvq_gemm.  M == 0 writes dA = dB = dWp = 0. */
+LCVQ_API lcvq_status lcvq_gemm_backward(const void* X, const void* dY, lcvq_dtype dtype, int64_t M,
+                               const uint8_t* packed, const uint8_t* mask_bits,
+                               int64_t d_out, int64_t d_in, int d,
+                               const float* A, const float* B,
+                               void* dX, float* dA, float* dB, float* dWp,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes a call with these arguments needs (0 on invalid input).
+ * The workspace holds the device error word (its first 256 bytes, which the
+ * caller zeroes once before first use), the transformed activations of the
+ * algebraic form and the per-block partial sums of dA/dB.  A workspace may be
+ * reused by calls that are ordered on one stream; calls that may overlap on the
+ * GPU need separate workspaces. */
+LCVQ_API size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_out,
+                           int64_t d_in, int d);
+
+/* Synchronizes `stream`, reads and clears the workspace's device error word.
+ * Returns LCVQ_OK, LCVQ_ERR_DEVICE_TIMEOUT, or LCVQ_ERR_CUDA. */
+LCVQ_API lcvq_status lcvq_check_device_error(void* workspace, void* stream);
+
+/* Static string naming a status. */
+LCVQ_API const char* lcvq_status_string(lcvq_status s);
+
+/* Number of kernels the last successful call on this host thread launched
+ * (for launch accounting by benchmarks). */
+LCVQ_API int lcvq_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCVQ_H_ */

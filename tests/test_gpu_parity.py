@@ -1,0 +1,264 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Codes, packed bytes and mask bits must match bit for bit; floating outputs
+must meet max |y - y_ref| / sum|x||w~| <= 4e-3 (bf16 activations) or 1e-5
+(fp32).  Shapes span several tiles and ragged tails; the full workload sizes
+are covered in test_gpu_fullsize.py.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from bit_weight_only_lcvq_b200 import lcvq, synth
+from oracle import lcvq_oracle as O
+from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, dev, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+# --------------------------------------------------------------- assign/pack
+def _adversarial_wp(n_rows, n_cols, seed):
+    g = np.random.Generator(np.random.PCG64(seed))
+    w = g.uniform(-1.0, 4.0, size=(n_rows, n_cols)).astype(np.float32)
+    special = np.array([0.5, 1.5, 2.5, 3.5, -0.5, -0.0, 0.0, 3.0, 3.0000002, -1e-45, 1e-45,
+                        np.inf, -np.inf, np.nan, 1e30, -1e30, 0.49999997, 2.4999998,
+                        np.float32(1.17549435e-38), 7.25], dtype=np.float32)
+    flat = w.reshape(-1)
+    idx = g.choice(flat.size, size=min(flat.size, 4 * special.size), replace=False)
+    flat[idx] = np.resize(special, idx.size)
+    return w
+
+
+@pytest.mark.parametrize("shape", [(1, 8), (3, 40), (7, 64), (33, 520), (128, 4096), (5, 1032)])
+def test_assign_pack_bit_exact(shape):
+    Wp = _adversarial_wp(*shape, seed=shape[0] * 7 + shape[1])
+    z, mask = O.assign(Wp)
+    packed, mbits = lcvq.assign_pack(torch.from_numpy(Wp).to(dev()), d=8 if shape[1] % 8 == 0 else 4)
+    assert np.array_equal(packed.cpu().numpy(), O.pack_codes(z))
+    assert np.array_equal(mbits.cpu().numpy(), O.pack_mask(mask))
+
+
+def test_assign_pack_workload_distributions():
+    for wid in (2, 4):
+        w = synth.workload(wid, M=1, d_in=1024, d_out=256, with_dy=False)
+        z, mask = O.assign(w["Wp"])
+        packed, mbits = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev()), d=8)
+        assert np.array_equal(packed.cpu().numpy(), O.pack_codes(z))
+        assert np.array_equal(mbits.cpu().numpy(), O.pack_mask(mask))
+
+
+def test_assign_pack_without_mask():
+    Wp = _adversarial_wp(16, 256, 3)
+    z, _ = O.assign(Wp)
+    packed, m = lcvq.assign_pack(torch.from_numpy(Wp).to(dev()), d=8, with_mask=False)
+    assert m is None
+    assert np.array_equal(packed.cpu().numpy(), O.pack_codes(z))
+
+
+# --------------------------------------------------------------- decode
+@pytest.mark.parametrize("d", [1, 2, 4, 8])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode(d, dtype):
+    g = np.random.Generator(np.random.PCG64(100 + d))
+    N, K = 40, 256
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A, B = synth.affine_diag_dominant(d, g)
+    W = lcvq.decode(torch.from_numpy(O.pack_codes(z)).to(dev()), K, torch.from_numpy(A).to(dev()),
+                    torch.from_numpy(B).to(dev()), d, dtype=dtype)
+    ref = O.decode(z, A, B)
+    D = O.decode_abs(z, A, B)
+    tol = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-6
+    assert_close("decode", to_np(W), ref, D, tol)
+
+
+# --------------------------------------------------------------- forward
+def _fwd_case(wid, M, d_in, d_out, d=None, seed_shift=0):
+    w = synth.workload(wid, M=M, d_in=d_in, d_out=d_out, d=d, with_dy=False)
+    z, _ = O.assign(w["Wp"])
+    return w, z
+
+
+def _run_fwd(w, z, dtype, form="auto"):
+    packed = torch.from_numpy(O.pack_codes(z)).to(dev())
+    X = to_dev(w["X"], dtype)
+    A = torch.from_numpy(w["A"]).to(dev())
+    B = torch.from_numpy(w["B"]).to(dev())
+    return lcvq.gemm(X, packed, w["d_in"], A, B, w["d"], form=form)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 5, 8, 13, 16, 27, 32])
+def test_gemv_bf16_ragged(M):
+    w, z = _fwd_case(2, M, d_in=1088, d_out=520)   # K = 17 x 64, N not a multiple of 128
+    Y = _run_fwd(w, z, torch.bfloat16)
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close(f"gemv M={M}", to_np(Y), ref, D, TOL_BF16)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_gemv_bf16_decode_workload(M):
+    """Decode-GEMV workload shape: d_in = d_out = 4096, d = 8."""
+    w, z = _fwd_case(2, M, d_in=4096, d_out=4096)
+    Y = _run_fwd(w, z, torch.bfloat16)
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close(f"gemv 4096 M={M}", to_np(Y), ref, D, TOL_BF16)
+
+
+@pytest.mark.parametrize("d", [1, 2, 4])
+def test_gemv_bf16_small_d(d):
+    w, z = _fwd_case(2, 8, d_in=512, d_out=256, d=d)
+    Y = _run_fwd(w, z, torch.bfloat16)
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close(f"gemv d={d}", to_np(Y), ref, D, TOL_BF16)
+
+
+@pytest.mark.parametrize("M", [33, 200])
+def test_gemm_bf16_larger_m(M):
+    w, z = _fwd_case(3, M, d_in=512, d_out=264)
+    for form in ("auto", "decode", "algebraic"):
+        Y = _run_fwd(w, z, torch.bfloat16, form)
+        ref, D = O.forward(w["X"], z, w["A"], w["B"])
+        assert_close(f"gemm M={M} {form}", to_np(Y), ref, D, TOL_BF16)
+
+
+def test_gemm_f32_single_layer():
+    """fp32 single-layer workload (d_in = d_out = 512, d = 4, M = 16)."""
+    w, z = _fwd_case(1, 16, d_in=512, d_out=512)
+    Y = _run_fwd(w, z, torch.float32)
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close("gemm f32", to_np(Y), ref, D, TOL_F32)
+
+
+def test_gemm_f32_identity_is_exact():
+    """A = I, B = 0, small-integer X: Y = X Z^T is exact in fp32."""
+    g = np.random.Generator(np.random.PCG64(5))
+    M, N, K, d = 37, 72, 256, 8
+    X = g.integers(-8, 9, size=(M, K)).astype(np.float32)
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    Y = lcvq.gemm(torch.from_numpy(X).to(dev()), torch.from_numpy(O.pack_codes(z)).to(dev()), K,
+                  torch.eye(d, device=dev()), torch.zeros(d, device=dev()), d)
+    assert np.array_equal(Y.cpu().numpy(), (X.astype(np.int64) @ z.astype(np.int64).T).astype(np.float32))
+
+
+@pytest.mark.parametrize("M,dtype", [(4, torch.bfloat16), (16, torch.float32), (64, torch.bfloat16)])
+def test_gemm_pow2_scaling_bit_exact(M, dtype):
+    """Y(2^k A, 2^k B) = 2^k Y(A, B) bit for bit."""
+    w, z = _fwd_case(2, M, d_in=512, d_out=256)
+    packed = torch.from_numpy(O.pack_codes(z)).to(dev())
+    X = to_dev(w["X"], dtype)
+    A = torch.from_numpy(w["A"]).to(dev())
+    B = torch.from_numpy(w["B"]).to(dev())
+    Y1 = lcvq.gemm(X, packed, 512, A, B, 8)
+    Y8 = lcvq.gemm(X, packed, 512, 8 * A, 8 * B, 8)
+    assert torch.equal(Y8, 8 * Y1)
+
+
+def test_gemm_linearity():
+    w, z = _fwd_case(2, 16, d_in=512, d_out=256)
+    packed = torch.from_numpy(O.pack_codes(z)).to(dev())
+    X = to_dev(w["X"], torch.float32)
+    g = np.random.Generator(np.random.PCG64(9))
+    A2, B2 = synth.affine_diag_dominant(8, g)
+    A1 = torch.from_numpy(w["A"]).to(dev())
+    B1 = torch.from_numpy(w["B"]).to(dev())
+    A2t, B2t = torch.from_numpy(A2).to(dev()), torch.from_numpy(B2).to(dev())
+    Y1 = lcvq.gemm(X, packed, 512, A1, B1, 8).double()
+    Y2 = lcvq.gemm(X, packed, 512, A2t, B2t, 8).double()
+    Y12 = lcvq.gemm(X, packed, 512, A1 + A2t, B1 + B2t, 8).double()
+    _, D = O.forward(w["X"], z, np.abs(w["A"]) + np.abs(A2), np.abs(w["B"]) + np.abs(B2))
+    assert O.rel_err(to_np(Y12), to_np(Y1 + Y2), D) < 1e-5
+
+
+def test_gemm_empty_and_zero_k():
+    A = torch.eye(8, device=dev())
+    B = torch.zeros(8, device=dev())
+    X = torch.zeros((0, 64), dtype=torch.bfloat16, device=dev())
+    packed = torch.zeros((16, 16), dtype=torch.uint8, device=dev())
+    Y = lcvq.gemm(X, packed, 64, A, B, 8)
+    assert Y.shape == (0, 16)
+    X = torch.ones((3, 0), dtype=torch.bfloat16, device=dev())
+    packed = torch.zeros((16, 0), dtype=torch.uint8, device=dev())
+    Y = torch.full((3, 16), 7.0, dtype=torch.bfloat16, device=dev())
+    lcvq.gemm(X, packed, 0, A, B, 8, out=Y)
+    assert torch.count_nonzero(Y) == 0
+
+
+def test_gemm_deterministic():
+    w, z = _fwd_case(2, 16, d_in=4096, d_out=1024)
+    Y1 = _run_fwd(w, z, torch.bfloat16)
+    Y2 = _run_fwd(w, z, torch.bfloat16)
+    assert torch.equal(Y1, Y2)
+
+
+# --------------------------------------------------------------- backward
+def _bwd_case(wid, M, d_in, d_out, dtype, d=None):
+    w = synth.workload(wid, M=M, d_in=d_in, d_out=d_out, d=d)
+    z, mask = O.assign(w["Wp"])
+    packed, mbits = O.pack_codes(z), O.pack_mask(mask)
+    args = dict(X=to_dev(w["X"], dtype), dY=to_dev(w["dY"], dtype),
+                packed=torch.from_numpy(packed).to(dev()), mask=torch.from_numpy(mbits).to(dev()),
+                A=torch.from_numpy(w["A"]).to(dev()), B=torch.from_numpy(w["B"]).to(dev()))
+    return w, z, mask, args
+
+
+def _check_bwd(w, z, mask, out, tol, tag):
+    ref = O.backward(w["X"], w["dY"], z, mask, w["A"], w["B"])
+    assert_close(f"{tag} dX", to_np(out["dX"]), ref["dX"], ref["D_dX"], tol)
+    assert_close(f"{tag} dA", to_np(out["dA"]), ref["dA"], ref["D_dA"], tol)
+    assert_close(f"{tag} dB", to_np(out["dB"]), ref["dB"], ref["D_dB"], tol)
+    assert_close(f"{tag} dWp", to_np(out["dWp"]), ref["dWp"], ref["D_dWp"], tol)
+
+
+def test_backward_f32_single_layer():
+    w, z, mask, a = _bwd_case(1, 16, 512, 512, torch.float32)
+    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 512, a["A"], a["B"], 4)
+    _check_bwd(w, z, mask, out, TOL_F32, "f32")
+
+
+@pytest.mark.parametrize("M,d_in,d_out", [(37, 576, 264), (200, 1024, 512)])
+def test_backward_bf16(M, d_in, d_out):
+    w, z, mask, a = _bwd_case(4, M, d_in, d_out, torch.bfloat16)
+    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], d_in, a["A"], a["B"], 8)
+    _check_bwd(w, z, mask, out, TOL_BF16, f"bf16 M={M}")
+
+
+@pytest.mark.parametrize("d", [1, 2, 4])
+def test_backward_small_d(d):
+    w, z, mask, a = _bwd_case(4, 24, 256, 128, torch.float32, d=d)
+    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 256, a["A"], a["B"], d)
+    _check_bwd(w, z, mask, out, TOL_F32, f"d={d}")
+
+
+def test_backward_optional_outputs_and_determinism():
+    w, z, mask, a = _bwd_case(4, 64, 512, 256, torch.bfloat16)
+    o1 = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 512, a["A"], a["B"], 8,
+                            want_dx=False, want_dwp=False)
+    o2 = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 512, a["A"], a["B"], 8)
+    o3 = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 512, a["A"], a["B"], 8)
+    assert o1["dX"] is None and o1["dWp"] is None
+    assert torch.equal(o1["dA"], o2["dA"]) and torch.equal(o1["dB"], o2["dB"])
+    for k in ("dX", "dA", "dB", "dWp"):
+        assert torch.equal(o2[k], o3[k]), k
+
+
+def test_backward_empty_tokens():
+    a = dict(X=torch.zeros((0, 64), dtype=torch.bfloat16, device=dev()),
+             dY=torch.zeros((0, 16), dtype=torch.bfloat16, device=dev()),
+             packed=torch.zeros((16, 16), dtype=torch.uint8, device=dev()),
+             mask=torch.zeros((16, 8), dtype=torch.uint8, device=dev()))
+    A, B = torch.eye(8, device=dev()), torch.zeros(8, device=dev())
+    outs = dict(dA=torch.ones((8, 8), device=dev()), dB=torch.ones(8, device=dev()),
+                dWp=torch.ones((16, 64), device=dev()))
+    o = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 64, A, B, 8, outs=outs)
+    assert torch.count_nonzero(o["dA"]) == 0 and torch.count_nonzero(o["dB"]) == 0
+    assert torch.count_nonzero(o["dWp"]) == 0
+
+
+def test_launch_count_and_error_word():
+    w, z = _fwd_case(2, 4, d_in=512, d_out=256)
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, 4, 256, 512, 8))
+    packed = torch.from_numpy(O.pack_codes(z)).to(dev())
+    lcvq.gemm(to_dev(w["X"], torch.bfloat16), packed, 512, torch.from_numpy(w["A"]).to(dev()),
+              torch.from_numpy(w["B"]).to(dev()), 8, workspace=ws)
+    assert lcvq.last_launch_count() >= 1
+    assert lcvq.check_device_error(ws) == 0

@@ -52,12 +52,15 @@ GemmWs gemm_ws(lcvq_dtype dtype, int64_t M, int64_t d_in) {
   return w;
 }
 struct BwdWs {
-  size_t part_off, num_parts, total;
+  size_t rsum_off, part_off, num_parts, total;
 };
-BwdWs bwd_ws(int64_t d_out, int64_t d_in, int d) {
+BwdWs bwd_ws(int64_t M, int64_t d_out, int64_t d_in, int d) {
   BwdWs w{};
-  w.num_parts = size_t(simt_dw_num_tiles(d_out, d_in));
-  w.part_off = kWsHeaderBytes;
+  const int64_t simt_parts = simt_dw_num_tiles(d_out, d_in);
+  const int64_t tc_parts = kNumSMsB200 * 2;  // >= any persistent grid on one device
+  w.num_parts = size_t(simt_parts > tc_parts ? simt_parts : tc_parts);
+  w.rsum_off = kWsHeaderBytes;
+  w.part_off = round_up(w.rsum_off + size_t(M) * 4, 256);
   w.total = round_up(w.part_off + w.num_parts * size_t(d * d + d) * 4, 256);
   return w;
 }
@@ -126,7 +129,7 @@ size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_ou
   if (M < 0 || d_out < 0 || d_in < 0 || !valid_d(d)) return 0;
   if (dtype != LCVQ_F32 && dtype != LCVQ_BF16) return 0;
   if (op == LCVQ_OP_GEMM) return gemm_ws(dtype, M, d_in).total;
-  if (op == LCVQ_OP_GEMM_BACKWARD) return bwd_ws(d_out, d_in, d).total;
+  if (op == LCVQ_OP_GEMM_BACKWARD) return bwd_ws(M, d_out, d_in, d).total;
   return 0;
 }
 
@@ -167,13 +170,17 @@ lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t*
   int launches = 0;
   cudaError_t e = cudaSuccess;
   char* ws = static_cast<char*>(workspace);
+  unsigned int* err = reinterpret_cast<unsigned int*>(ws);
   if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
     uint16_t* Xpp = reinterpret_cast<uint16_t*>(ws + w.xpp_off);
     float* corr = reinterpret_cast<float*>(ws + w.corr_off);
     e = launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr, s, &launches);
     if (e == cudaSuccess)
-      e = launch_gemm_xformed(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), s,
-                              &launches);
+      e = launch_gemm_xformed(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), err,
+                              s, &launches);
+  } else if (dtype == LCVQ_BF16) {  // decode form on the tensor cores
+    e = launch_tc_forward(static_cast<const uint16_t*>(X), false, nullptr, M, packed, d_out, d_in,
+                          d, A, B, static_cast<uint16_t*>(Y), err, s, &launches);
   } else {
     e = launch_simt_forward(X, dtype == LCVQ_BF16, M, packed, d_out, d_in, d, A, B, Y, s,
                             &launches);
@@ -210,7 +217,7 @@ lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64_t M,
   if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
   int launches = 0;
   cudaError_t e = launch_gemm_xformed(static_cast<const uint16_t*>(Xpp), corr, M, packed, d_out,
-                                      d_in, static_cast<uint16_t*>(Y),
+                                      d_in, static_cast<uint16_t*>(Y), nullptr,
                                       static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches);
 }
@@ -246,18 +253,36 @@ lcvq_status lcvq_gemm_backward(const void* X, const void* dY, lcvq_dtype dtype, 
   if (!aligned16(X) || !aligned16(dY) || !aligned16(packed) || !aligned16(A) || !aligned16(B) ||
       !aligned16(workspace))
     return LCVQ_ERR_ALIGNMENT;
-  const BwdWs w = bwd_ws(d_out, d_in, d);
+  const BwdWs w = bwd_ws(M, d_out, d_in, d);
   if (ws_bytes < w.total) return LCVQ_ERR_WORKSPACE;
-  float* partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + w.part_off);
-  const bool bf = dtype == LCVQ_BF16;
+  char* ws = static_cast<char*>(workspace);
+  unsigned int* err = reinterpret_cast<unsigned int*>(ws);
+  float* partials = reinterpret_cast<float*>(ws + w.part_off);
   int launches = 0;
   cudaError_t e = cudaSuccess;
-  if (dX) e = launch_simt_backward_dx(dY, bf, M, packed, d_out, d_in, d, A, B, dX, s, &launches);
-  if (e == cudaSuccess)
-    e = launch_simt_backward_dw(X, dY, bf, M, packed, mask_bits, d_out, d_in, d, A, dWp, partials,
-                                s, &launches);
-  if (e == cudaSuccess)
-    e = launch_reduce_partials(partials, int64_t(w.num_parts), d, dA, dB, s, &launches);
+  int64_t parts = 0;
+  if (dtype == LCVQ_BF16) {
+    float* rsum = reinterpret_cast<float*>(ws + w.rsum_off);
+    const uint16_t* dYb = static_cast<const uint16_t*>(dY);
+    if (dX) {
+      e = launch_rowsum(dYb, M, d_out, rsum, s, &launches);
+      if (e == cudaSuccess)
+        e = launch_tc_backward_dx(dYb, rsum, M, packed, d_out, d_in, d, A, B,
+                                  static_cast<uint16_t*>(dX), err, s, &launches);
+    }
+    int grid = 0;
+    if (e == cudaSuccess)
+      e = launch_tc_backward_dw(static_cast<const uint16_t*>(X), dYb, M, packed, mask_bits, d_out,
+                                d_in, d, A, dWp, partials, &grid, err, s, &launches);
+    parts = grid;
+  } else {
+    if (dX) e = launch_simt_backward_dx(dY, false, M, packed, d_out, d_in, d, A, B, dX, s, &launches);
+    if (e == cudaSuccess)
+      e = launch_simt_backward_dw(X, dY, false, M, packed, mask_bits, d_out, d_in, d, A, dWp,
+                                  partials, s, &launches);
+    parts = simt_dw_num_tiles(d_out, d_in);
+  }
+  if (e == cudaSuccess) e = launch_reduce_partials(partials, parts, d, dA, dB, s, &launches);
   return finish(e, launches);
 }
 

@@ -251,9 +251,10 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
 
 cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,
                                 const uint8_t* packed, int64_t d_out, int64_t d_in, uint16_t* Y,
-                                cudaStream_t s, int* launches) {
-  // M > 32: the same kernel walks 32-token chunks along grid z
-  return launch_gemv(Xpp, corr, M, packed, d_out, d_in, Y, s, launches);
+                                unsigned int* err, cudaStream_t s, int* launches) {
+  if (M <= 32) return launch_gemv(Xpp, corr, M, packed, d_out, d_in, Y, s, launches);
+  return launch_tc_forward(Xpp, true, corr, M, packed, d_out, d_in, 8, nullptr, nullptr, Y, err, s,
+                           launches);
 }
 
 }  // namespace lcvq

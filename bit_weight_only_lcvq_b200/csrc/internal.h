@@ -28,10 +28,31 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
                         int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s, int* launches);
 
 // integer-code GEMM on X'' (dispatches on M: decode-GEMV for M <= 32, else
-// the CUDA-core fallback until the tensor-core GEMM takes it)
+// the tcgen05 GEMM); err may be null (no device error word)
 cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,
                                 const uint8_t* packed, int64_t d_out, int64_t d_in, uint16_t* Y,
-                                cudaStream_t s, int* launches);
+                                unsigned int* err, cudaStream_t s, int* launches);
+
+// ---- tcgen05 GEMMs (bf16, persistent, one CTA per SM) ----
+int tc_max_grid();
+// Xa is X'' (algebraic, with corr) or X (decode form, A z + B decoded on chip)
+cudaError_t launch_tc_forward(const uint16_t* Xa, bool algebraic, const float* corr, int64_t M,
+                              const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
+                              const float* A, const float* B, uint16_t* Y, unsigned int* err,
+                              cudaStream_t s, int* launches);
+cudaError_t launch_tc_backward_dx(const uint16_t* dY, const float* rsum, int64_t M,
+                                  const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
+                                  const float* A, const float* B, uint16_t* dX, unsigned int* err,
+                                  cudaStream_t s, int* launches);
+// *num_parts receives the number of per-CTA partial rows written
+cudaError_t launch_tc_backward_dw(const uint16_t* X, const uint16_t* dY, int64_t M,
+                                  const uint8_t* packed, const uint8_t* mask, int64_t d_out,
+                                  int64_t d_in, int d, const float* A, float* dWp,
+                                  float* partials, int* num_parts, unsigned int* err,
+                                  cudaStream_t s, int* launches);
+// r[m] = sum_n dY[m][n] (fp64 accumulation), bf16 dY
+cudaError_t launch_rowsum(const uint16_t* dY, int64_t M, int64_t n, float* r, cudaStream_t s,
+                          int* launches);
 
 // ---- CUDA-core paths (any M; fp32 or bf16 activations) ----
 cudaError_t launch_simt_forward(const void* X, bool bf16, int64_t M, const uint8_t* packed,

@@ -136,4 +136,34 @@ cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, cons
   return cudaGetLastError();
 }
 
+// r[m] = sum_n dY[m][n]: the rank-1 term of the dX epilogue (the B part of
+// W~ = A z + B contributes B_i r[m] to dX[m][g d + i]).
+__global__ void __launch_bounds__(256) rowsum_kernel(const uint16_t* __restrict__ dY, int64_t n,
+                                                     float* __restrict__ r) {
+  __shared__ double red[8];
+  const uint16_t* row = dY + int64_t(blockIdx.x) * n;
+  double s = 0.0;
+  for (int64_t j = threadIdx.x * 8; j < n; j += 256 * 8) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + j));
+    s += double(bf16_lo(u.x)) + double(bf16_hi(u.x)) + double(bf16_lo(u.y)) + double(bf16_hi(u.y)) +
+         double(bf16_lo(u.z)) + double(bf16_hi(u.z)) + double(bf16_lo(u.w)) + double(bf16_hi(u.w));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_down_sync(0xffffffffu, s, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < 8; ++w) t += red[w];
+    r[blockIdx.x] = static_cast<float>(t);
+  }
+}
+
+cudaError_t launch_rowsum(const uint16_t* dY, int64_t M, int64_t n, float* r, cudaStream_t s,
+                          int* launches) {
+  rowsum_kernel<<<static_cast<unsigned>(M), 256, 0, s>>>(dY, n, r);
+  ++*launches;
+  return cudaGetLastError();
+}
+
 }  // namespace lcvq

@@ -1,0 +1,117 @@
+"""Parity at the full workload sizes, in the launch configuration the
+benchmark times: bit-exact codes/masks over whole matrices, floating outputs
+on sampled elements the oracle computes one by one, and dB through an exact
+O(M (N + K)) identity.  dA is computed in full in fp64 (chunked)."""
+
+import numpy as np
+import pytest
+import torch
+
+from bit_weight_only_lcvq_b200 import lcvq, synth
+from oracle import lcvq_oracle as O
+from tests.gpu_util import TOL_BF16, assert_close, dev
+
+pytestmark = pytest.mark.gpu
+
+N_SAMPLES = 384
+
+
+def _pairs(seed, a, b, n=N_SAMPLES):
+    g = np.random.Generator(np.random.PCG64(seed))
+    return [(int(x), int(y)) for x, y in zip(g.integers(0, a, n), g.integers(0, b, n))]
+
+
+def _check_sampled_forward(Y, Xnp, z, A, B, pairs, tag):
+    y, dd = O.forward_sampled(Xnp, {n: z[n] for _, n in pairs}, A, B, pairs)
+    Yc = Y.float().cpu().numpy()
+    got = np.array([Yc[m, n] for m, n in pairs])
+    assert_close(tag, got, y, dd, TOL_BF16)
+
+
+@pytest.mark.parametrize("form", ["algebraic", "decode"])
+def test_prefill_full(form):
+    """Prefill GEMM: d_in=4096, d_out=11008, d=8, M=2048 bf16."""
+    w = synth.workload(3, with_dy=False)
+    z, _ = O.assign(w["Wp"])
+    packed, _ = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev()), 8, with_mask=False)
+    assert np.array_equal(packed.cpu().numpy(), O.pack_codes(z))
+    X = torch.from_numpy(w["X"]).to(torch.bfloat16).to(dev())
+    Y = lcvq.gemm(X, packed, 4096, torch.from_numpy(w["A"]).to(dev()),
+                  torch.from_numpy(w["B"]).to(dev()), 8, form=form)
+    _check_sampled_forward(Y, w["X"], z, w["A"], w["B"], _pairs(3, 2048, 11008), f"prefill {form}")
+
+
+@pytest.fixture(scope="module")
+def qat():
+    w = synth.workload(4)
+    z, mask = O.assign(w["Wp"])
+    return w, z, mask
+
+
+def test_qat_assign_pack_full(qat):
+    w, z, mask = qat
+    packed, mbits = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev()), 8)
+    assert np.array_equal(packed.cpu().numpy(), O.pack_codes(z))
+    assert np.array_equal(mbits.cpu().numpy(), O.pack_mask(mask))
+    frac = 1.0 - mask.mean()
+    assert abs(frac - 0.1336) < 2e-3   # N(1.5, 1): 2 (1 - Phi(1.5)) outside [0, 3]
+
+
+def test_qat_forward_and_backward_full(qat):
+    """QAT step on d_in=14336, d_out=4096, M=8192: forward, then dX, dA, dB,
+    dWp of the straight-through backward."""
+    w, z, mask = qat
+    M, K, N, d = 8192, 14336, 4096, 8
+    Wp = torch.from_numpy(w["Wp"]).to(dev())
+    packed, mbits = lcvq.assign_pack(Wp, d)
+    A = torch.from_numpy(w["A"]).to(dev())
+    B = torch.from_numpy(w["B"]).to(dev())
+    X = torch.from_numpy(w["X"]).to(torch.bfloat16).to(dev())
+    dY = torch.from_numpy(w["dY"]).to(torch.bfloat16).to(dev())
+    Y = lcvq.gemm(X, packed, K, A, B, d)
+    _check_sampled_forward(Y, w["X"], z, w["A"], w["B"], _pairs(4, M, N), "qat forward")
+    del Y
+    out = lcvq.gemm_backward(X, dY, packed, mbits, K, A, B, d)
+    dX = out["dX"].float().cpu().numpy()
+    pairs = _pairs(5, M, K)
+    v, dd = O.backward_dx_sampled(w["dY"], lambda k: z[:, (k // d) * d:(k // d + 1) * d],
+                                  w["A"], w["B"], pairs)
+    assert_close("qat dX", np.array([dX[m, k] for m, k in pairs]), v, dd, TOL_BF16)
+    del dX
+    dWp = out["dWp"].cpu().numpy()
+    pairs = _pairs(6, N, K)
+    v, dd = O.backward_dwp_sampled(w["X"], w["dY"], lambda n: mask[n], w["A"], pairs)
+    assert_close("qat dWp", np.array([dWp[n, k] for n, k in pairs]), v, dd, TOL_BF16)
+    assert np.all(dWp[~mask] == 0)
+    del dWp
+    # dB through sum_m rowsum(dY)[m] * sum_g X[m, g d + i]  (exact identity)
+    X64 = w["X"].astype(np.float64)
+    dY64 = w["dY"].astype(np.float64)
+    xs = X64.reshape(M, K // d, d).sum(1)
+    ref_dB = dY64.sum(1) @ xs
+    D_dB = np.abs(dY64).sum(1) @ np.abs(X64).reshape(M, K // d, d).sum(1)
+    assert_close("qat dB", out["dB"].cpu().numpy(), ref_dB, D_dB, TOL_BF16)
+    # dA in full: dA[i][j] = sum_m sum_g X[m, g d + i] P[m, g d + j], P = dY Z
+    Z = z.astype(np.float64)
+    ref_dA = np.zeros((d, d))
+    D_dA = np.zeros((d, d))
+    for c0 in range(0, M, 1024):
+        P = dY64[c0:c0 + 1024] @ Z
+        Pa = np.abs(dY64[c0:c0 + 1024]) @ Z
+        Xc = X64[c0:c0 + 1024].reshape(-1, K // d, d)
+        ref_dA += np.einsum("mgi,mgj->ij", Xc, P.reshape(-1, K // d, d))
+        D_dA += np.einsum("mgi,mgj->ij", np.abs(Xc), Pa.reshape(-1, K // d, d))
+    assert_close("qat dA", out["dA"].cpu().numpy(), ref_dA, D_dA, TOL_BF16)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_stack_matrices(M):
+    """One matrix of each projection shape of the 7B-shaped stack."""
+    for proj in range(len(synth.STACK_PROJS)):
+        m = synth.stack_matrix(proj, proj, M)
+        z = O.unpack_codes(m["packed"], m["d_in"])
+        X = torch.from_numpy(m["X"]).to(torch.bfloat16).to(dev())
+        Y = lcvq.gemm(X, torch.from_numpy(m["packed"]).to(dev()), m["d_in"],
+                      torch.from_numpy(m["A"]).to(dev()), torch.from_numpy(m["B"]).to(dev()), 8)
+        pairs = _pairs(7 + proj, M, m["d_out"], 128)
+        _check_sampled_forward(Y, m["X"], z, m["A"], m["B"], pairs, f"stack {m['proj']} M={M}")

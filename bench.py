@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from bit_weight_only_lcvq_b200 import lcvq, synth  # noqa: E402
+from bit_weight_only_lcvq_b200.replicas import Replicas as Dist  # noqa: E402
 
 METRIC = "LC-VQ 2-bit GEMM: packed-weight GB/s (M≤16), TFLOP/s (prefill), % roofline"
 MIB = 1 << 20
@@ -52,35 +53,6 @@ def parse():
     p.add_argument("--rows", default="all")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
-
-
-class Dist:
-    def __init__(self):
-        self.world = int(os.environ.get("WORLD_SIZE", "1"))
-        self.rank = int(os.environ.get("RANK", "0"))
-        self.local = int(os.environ.get("LOCAL_RANK", "0"))
-        if self.world > 1:
-            import datetime
-            torch.cuda.set_device(self.local)
-            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        else:
-            torch.cuda.set_device(0)
-        self.dev = torch.device("cuda", torch.cuda.current_device())
-
-    def barrier(self):
-        if self.world > 1:
-            torch.distributed.barrier()
-
-    def max(self, x: float) -> float:
-        if self.world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=self.dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
-
-    def close(self):
-        if self.world > 1:
-            torch.distributed.destroy_process_group()
 
 
 def peaks():

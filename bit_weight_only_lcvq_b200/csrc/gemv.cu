@@ -29,15 +29,6 @@ namespace lcvq {
 namespace {
 
 constexpr int kGemvRows = 128;   // weight rows per CTA
-constexpr int kGemvIterK = 256;  // codes per row per main-loop iteration (64 B)
-
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
@@ -62,78 +53,112 @@ __device__ __forceinline__ uint32_t dec_pair(uint32_t w0, uint32_t w6, uint32_t 
   return r;
 }
 
+// same as dec_pair<C> for a C that is a compile-time constant after unrolling
+__device__ __forceinline__ uint32_t dec_pair_rt(int c, uint32_t w0, uint32_t w6, uint32_t w12) {
+  switch (c) {
+    case 0: return dec_pair<0>(w0, w6, w12);
+    case 1: return dec_pair<1>(w0, w6, w12);
+    case 2: return dec_pair<2>(w0, w6, w12);
+    case 3: return dec_pair<3>(w0, w6, w12);
+    case 4: return dec_pair<4>(w0, w6, w12);
+    case 5: return dec_pair<5>(w0, w6, w12);
+    case 6: return dec_pair<6>(w0, w6, w12);
+    default: return dec_pair<7>(w0, w6, w12);
+  }
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
   return q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
 }
 
-template <int NT, int R, int W>
-__global__ void __launch_bounds__(W * 32) gemv_kernel(const uint16_t* __restrict__ Xpp,
-                                                      const float* __restrict__ corr, int M,
-                                                      const uint8_t* __restrict__ packed,
-                                                      int64_t N, int64_t K,
-                                                      uint16_t* __restrict__ Y) {
-  static_assert(W * R * 16 == kGemvRows, "tile rows");
+// CTA: 8 warps on a 128-row weight tile; warp w takes row half (w & 1) (4 row
+// blocks of 16) and K slice (w >> 1) of the CTA's 4; the cluster (grid y)
+// splits K S ways more.  A "unit" is 128 codes of each of the warp's 64 rows:
+// lane (g, t) holds 2 words of rows g and g + 8 of every row block (8 B each),
+// so one unit is 16 x 64-bit loads per lane, issued one unit ahead.
+constexpr int kUnit = 128;  // codes per row per unit (32 B)
+constexpr int kWarps = 8;
+constexpr int kRB = 4;      // row blocks of 16 per warp
+
+__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];\n"
+               : "=r"(v.x), "=r"(v.y)
+               : "l"(p));
+  return v;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(const uint16_t* __restrict__ Xpp,
+                                                           const float* __restrict__ corr, int M,
+                                                           const uint8_t* __restrict__ packed,
+                                                           int64_t N, int64_t K,
+                                                           uint16_t* __restrict__ Y) {
   constexpr int MP = NT * 8;
   __shared__ float part[kGemvRows][MP + 1];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int S = static_cast<int>(cluster.dim_blocks().y);
-  const int split = static_cast<int>(cluster.block_index().y);
+  const int rank = static_cast<int>(cluster.block_index().y);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
+  const int rh = warp & 1, ks = warp >> 1;
   const int64_t tile_row0 = int64_t(blockIdx.x) * kGemvRows;
-  const int64_t row0 = tile_row0 + warp * (R * 16);
-  const int64_t Kb = K / 4;  // bytes of codes per row
-  const int64_t niter = ceil_div(K, kGemvIterK);
-  const int64_t it0 = niter * split / S;
-  const int64_t it1 = niter * (split + 1) / S;
+  const int64_t Kb = K / 4;
+  const int64_t nunits = ceil_div(K, kUnit);
+  const int nslices = 4 * S;
+  const int gs = rank * 4 + ks;
+  const int64_t u0 = nunits * gs / nslices, u1 = nunits * (gs + 1) / nslices;
 
-  float acc[R][NT][4];
+  const uint8_t* rowp[kRB][2];
+  bool rowok[kRB][2];
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+  for (int r = 0; r < kRB; ++r)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t row = tile_row0 + rh * 64 + r * 16 + g + 8 * h;
+      rowok[r][h] = row < N;
+      rowp[r][h] = packed + (rowok[r][h] ? row : 0) * Kb + 8 * t;
+    }
+  const uint16_t* xrow[NT];
+  bool tokok[NT];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    const int tok = n * 8 + g;
+    tokok[n] = tok < M;
+    xrow[n] = Xpp + int64_t(tokok[n] ? tok : 0) * K + 32 * t;
+  }
+
+  float acc[kRB][NT][4];
+#pragma unroll
+  for (int r = 0; r < kRB; ++r)
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[r][n][e] = 0.f;
 
-  const uint8_t* rowp[R][2];
-  bool rowok[R][2];
+  auto load_codes = [&](int64_t u, uint2 (&cw)[kRB][2]) {
+    const bool kok = u * kUnit + 32 * t < K;  // K % 64 == 0: whole 32-code lane chunks
 #pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t row = row0 + r * 16 + g + 8 * h;
-      rowok[r][h] = row < N;
-      rowp[r][h] = packed + (rowok[r][h] ? row : 0) * Kb;
-    }
-  const int tok0 = static_cast<int>(blockIdx.z) * MP;  // token chunk of this CTA
-  const uint16_t* xrow[NT];
-  bool tokok[NT];
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const int tok = tok0 + n * 8 + g;
-    tokok[n] = tok < M;
-    xrow[n] = Xpp + int64_t(tokok[n] ? tok : 0) * K;
-  }
-
-  for (int64_t it = it0; it < it1; ++it) {
-    const int64_t kbyte = it * 64 + 16 * t;
-    const bool kok = kbyte < Kb;  // K % 64 == 0: a lane's 16 B are all in or all out
-    uint4 cw[R][2];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
+    for (int r = 0; r < kRB; ++r)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        cw[r][h] = (kok && rowok[r][h]) ? ld_stream_v4(rowp[r][h] + kbyte) : make_uint4(0, 0, 0, 0);
-    const int64_t kel = it * kGemvIterK + 64 * t;  // first X'' element of this lane
+        cw[r][h] = (kok && rowok[r][h]) ? ld_stream_v2(rowp[r][h] + u * 32) : make_uint2(0, 0);
+  };
+
+  uint2 cur[kRB][2], nxt[kRB][2];
+  if (u0 < u1) load_codes(u0, cur);
+  for (int64_t u = u0; u < u1; ++u) {
+    if (u + 1 < u1) load_codes(u + 1, nxt);
+    const bool kok = u * kUnit + 32 * t < K;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {  // word q of each row: 16 codes, 4 k16 tiles
       uint4 xb[NT][2];
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         if (kok && tokok[n]) {
-          const uint4* src = reinterpret_cast<const uint4*>(xrow[n] + kel + 16 * q);
+          const uint4* src = reinterpret_cast<const uint4*>(xrow[n] + u * kUnit + 16 * q);
           xb[n][0] = __ldg(src);
           xb[n][1] = __ldg(src + 1);
         } else {
@@ -141,84 +166,101 @@ __global__ void __launch_bounds__(W * 32) gemv_kernel(const uint16_t* __restrict
           xb[n][1] = make_uint4(0, 0, 0, 0);
         }
       }
-      uint32_t a[R][2][8];
+      uint32_t w0[kRB][2], w6[kRB][2], w12[kRB][2];
 #pragma unroll
-      for (int r = 0; r < R; ++r)
+      for (int r = 0; r < kRB; ++r)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint32_t w0 = word_of(cw[r][h], q);
-          const uint32_t w6 = w0 >> 6, w12 = w0 >> 12;
-          a[r][h][0] = dec_pair<0>(w0, w6, w12);
-          a[r][h][1] = dec_pair<1>(w0, w6, w12);
-          a[r][h][2] = dec_pair<2>(w0, w6, w12);
-          a[r][h][3] = dec_pair<3>(w0, w6, w12);
-          a[r][h][4] = dec_pair<4>(w0, w6, w12);
-          a[r][h][5] = dec_pair<5>(w0, w6, w12);
-          a[r][h][6] = dec_pair<6>(w0, w6, w12);
-          a[r][h][7] = dec_pair<7>(w0, w6, w12);
+          w0[r][h] = q == 0 ? cur[r][h].x : cur[r][h].y;
+          w6[r][h] = w0[r][h] >> 6;
+          w12[r][h] = w0[r][h] >> 12;
         }
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {  // k16 tile: pairs 2jj, 2jj+1 of word q
+        uint32_t a[kRB][2][2];
+#pragma unroll
+        for (int r = 0; r < kRB; ++r)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            a[r][h][0] = dec_pair_rt(2 * jj, w0[r][h], w6[r][h], w12[r][h]);
+            a[r][h][1] = dec_pair_rt(2 * jj + 1, w0[r][h], w6[r][h], w12[r][h]);
+          }
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           const uint32_t b0 = word_of(xb[n][jj >> 1], (2 * jj) & 3);
           const uint32_t b1 = word_of(xb[n][jj >> 1], (2 * jj + 1) & 3);
 #pragma unroll
-          for (int r = 0; r < R; ++r)
-            mma_bf16_16816(acc[r][n], a[r][0][2 * jj], a[r][1][2 * jj], a[r][0][2 * jj + 1],
-                           a[r][1][2 * jj + 1], b0, b1);
+          for (int r = 0; r < kRB; ++r)
+            mma_bf16_16816(acc[r][n], a[r][0][0], a[r][1][0], a[r][0][1], a[r][1][1], b0, b1);
         }
       }
     }
+    if (u + 1 < u1) {
+#pragma unroll
+      for (int r = 0; r < kRB; ++r)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) cur[r][h] = nxt[r][h];
+    }
   }
 
-  // partial tile -> shared memory
+  // the CTA's 4 K slices, summed into shared memory in slice order
+  for (int round = 0; round < 4; ++round) {
+    if (ks == round) {
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+      for (int r = 0; r < kRB; ++r)
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int lr = warp * R * 16 + r * 16 + g;
-      const int tk = n * 8 + 2 * t;
-      part[lr][tk] = acc[r][n][0];
-      part[lr][tk + 1] = acc[r][n][1];
-      part[lr + 8][tk] = acc[r][n][2];
-      part[lr + 8][tk + 1] = acc[r][n][3];
+        for (int n = 0; n < NT; ++n) {
+          const int lr = rh * 64 + r * 16 + g;
+          const int tk = n * 8 + 2 * t;
+          if (round == 0) {
+            part[lr][tk] = acc[r][n][0];
+            part[lr][tk + 1] = acc[r][n][1];
+            part[lr + 8][tk] = acc[r][n][2];
+            part[lr + 8][tk + 1] = acc[r][n][3];
+          } else {
+            part[lr][tk] += acc[r][n][0];
+            part[lr][tk + 1] += acc[r][n][1];
+            part[lr + 8][tk] += acc[r][n][2];
+            part[lr + 8][tk + 1] += acc[r][n][3];
+          }
+        }
     }
+    __syncthreads();
+  }
   cluster.sync();
 
-  // CTA `split` of the cluster reduces rows [r0, r1) of the tile over all ranks.
-  const int r0 = kGemvRows * split / S, r1 = kGemvRows * (split + 1) / S;
+  // rank r of the cluster finishes rows [r0, r1) of the tile over all ranks
+  const int r0 = kGemvRows * rank / S, r1 = kGemvRows * (rank + 1) / S;
   const int nrows = r1 - r0;
-  const int mtok = min(MP, M - tok0);
-  const int total = nrows * mtok;
-  for (int e = threadIdx.x; e < total; e += W * 32) {
+  const int total = nrows * M;
+  for (int e = threadIdx.x; e < total; e += kWarps * 32) {
     const int lr = r0 + e % nrows;
     const int tok = e / nrows;
     const int64_t grow = tile_row0 + lr;
     float sum = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float* rp = cluster.map_shared_rank(&part[0][0], s);
+    for (int s2 = 0; s2 < S; ++s2) {
+      const float* rp = cluster.map_shared_rank(&part[0][0], s2);
       sum += rp[lr * (MP + 1) + tok];
     }
-    if (grow < N) Y[int64_t(tok0 + tok) * N + grow] = f32_to_bf16(sum + corr[tok0 + tok]);
+    if (grow < N) Y[int64_t(tok) * N + grow] = f32_to_bf16(sum + corr[tok]);
   }
   cluster.sync();  // keep every CTA's shared memory alive until all reads are done
 }
 
-template <int NT, int R, int W>
+template <int NT>
 cudaError_t launch_gemv_t(const uint16_t* Xpp, const float* corr, int M, const uint8_t* packed,
                           int64_t N, int64_t K, uint16_t* Y, cudaStream_t s) {
   const int64_t tiles = ceil_div(N, kGemvRows);
-  const int64_t niter = ceil_div(K, kGemvIterK);
-  const int64_t chunks = ceil_div(M, NT * 8);
-  int S = static_cast<int>(ceil_div(2 * kNumSMsB200, tiles * chunks));
+  const int64_t nunits = ceil_div(K, kUnit);
+  int S = static_cast<int>(ceil_div(2 * kNumSMsB200, tiles));
   if (S > 8) S = 8;
-  if (S > niter) S = static_cast<int>(niter);
-  if (S < 1) S = 1;
+  int p2 = 1;
+  while (p2 * 2 <= S) p2 *= 2;
+  S = p2;
+  while (S > 1 && 4 * S > nunits) S /= 2;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(S),
-                     static_cast<unsigned>(chunks));
-  cfg.blockDim = dim3(W * 32, 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(S), 1);
+  cfg.blockDim = dim3(kWarps * 32, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -228,7 +270,7 @@ cudaError_t launch_gemv_t(const uint16_t* Xpp, const float* corr, int M, const u
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, R, W>, Xpp, corr, M, packed, N, K, Y);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT>, Xpp, corr, M, packed, N, K, Y);
 }
 
 }  // namespace
@@ -239,11 +281,11 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
   cudaError_t e;
   const int m = static_cast<int>(M);
   if (M <= 8)
-    e = launch_gemv_t<1, 4, 2>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<1>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else if (M <= 16)
-    e = launch_gemv_t<2, 4, 2>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<2>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else
-    e = launch_gemv_t<4, 2, 4>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<4>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   ++*launches;
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -41,6 +41,11 @@ __global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __res
   __shared__ float sA[D * D];
   __shared__ float sBp[D];
   __shared__ double red[3][kXfThreads / 32];
+  // Programmatic dependent launch: wait for every earlier kernel in the stream
+  // (X may be the previous layer's output), then let the decode-GEMV launch so
+  // its code loads overlap this kernel.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   if (threadIdx.x < D * D) sA[threadIdx.x] = A[threadIdx.x];
   __syncthreads();
   if (threadIdx.x < D) {
@@ -125,14 +130,24 @@ __global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __res
 cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
                          const float* B, uint16_t* Xpp, float* corr, cudaStream_t s,
                          int* launches) {
-  const dim3 grid(static_cast<unsigned>(M));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(M), 1, 1);
+  cfg.blockDim = dim3(kXfThreads, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   switch (d) {
-    case 1: xform_kernel<1><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
-    case 2: xform_kernel<2><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
-    case 4: xform_kernel<4><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
-    default: xform_kernel<8><<<grid, kXfThreads, 0, s>>>(X, d_in, A, B, Xpp, corr); break;
+    case 1: e = cudaLaunchKernelEx(&cfg, xform_kernel<1>, X, d_in, A, B, Xpp, corr); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, xform_kernel<2>, X, d_in, A, B, Xpp, corr); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, xform_kernel<4>, X, d_in, A, B, Xpp, corr); break;
+    default: e = cudaLaunchKernelEx(&cfg, xform_kernel<8>, X, d_in, A, B, Xpp, corr); break;
   }
   ++*launches;
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -37,6 +37,7 @@ EXPORTS = (
     "lcvq_gemm_backward",
     "lcvq_xform",
     "lcvq_gemm_xformed",
+    "lcvq_gemv_static",
     "lcvq_workspace_size",
     "lcvq_check_device_error",
     "lcvq_status_string",
@@ -71,6 +72,7 @@ def lib() -> ctypes.CDLL:
                                          _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
         L.lcvq_xform.argtypes = [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp]
         L.lcvq_gemm_xformed.argtypes = [_vp, _vp, _i64, _vp, _i64, _i64, _vp, _vp]
+        L.lcvq_gemv_static.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp]
         L.lcvq_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i64, _i32]
         L.lcvq_workspace_size.restype = _sz
         L.lcvq_check_device_error.argtypes = [_vp, _vp]
@@ -78,7 +80,7 @@ def lib() -> ctypes.CDLL:
         L.lcvq_status_string.restype = ctypes.c_char_p
         L.lcvq_last_launch_count.argtypes = []
         for fn in ("lcvq_assign_pack", "lcvq_decode", "lcvq_gemm", "lcvq_gemm_backward",
-                   "lcvq_xform", "lcvq_gemm_xformed", "lcvq_check_device_error",
+                   "lcvq_xform", "lcvq_gemm_xformed", "lcvq_gemv_static", "lcvq_check_device_error",
                    "lcvq_last_launch_count"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -212,6 +214,20 @@ def gemm_xformed(xpp: torch.Tensor, corr: torch.Tensor, packed: torch.Tensor, *,
         out = torch.empty((M, d_out), dtype=torch.bfloat16, device=xpp.device)
     _check("lcvq_gemm_xformed", lib().lcvq_gemm_xformed(
         _ptr(xpp), _ptr(corr), M, _ptr(packed), d_out, d_in, _ptr(out), _stream(stream)))
+    return out
+
+
+def gemv_static(X: torch.Tensor, packed: torch.Tensor, d_in: int, A: torch.Tensor,
+                B: torch.Tensor, d: int, *, out=None, stream=None) -> torch.Tensor:
+    """Decode-GEMV (bf16, M <= 32) that takes no workspace: its scratch lives in a
+    fixed array inside the library, for callers that cannot allocate device
+    memory (see lcvq_gemv_static in include/lcvq.h)."""
+    M = X.shape[0]
+    d_out = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, d_out), dtype=torch.bfloat16, device=X.device)
+    _check("lcvq_gemv_static", lib().lcvq_gemv_static(
+        _ptr(X), M, _ptr(packed), d_out, d_in, d, _ptr(A), _ptr(B), _ptr(out), _stream(stream)))
     return out
 
 

@@ -153,6 +153,30 @@ LCVQ_API lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64
                                        const uint8_t* packed, int64_t d_out, int64_t d_in,
                                        void* Y, void* stream);
 
+/* Decode-GEMV without a workspace.  The pages have no counterpart: this is a
+ * convenience of this library.  It computes exactly what lcvq_gemm computes for
+ * bf16 activations and M <= 32 (same kernels, same results), but takes no
+ * workspace, because some callers cannot provide one: code running while a
+ * CUDA graph is being captured (device allocation is not allowed there),
+ * runtimes that reserve all device memory at start-up and forbid later
+ * allocations, and extensions whose host framework owns the allocator and
+ * offers them no scratch space.
+ *   X [M][d_in] bf16, Y [M][d_out] bf16; packed, A, B as lcvq_gemm.
+ * Scratch: a fixed 2 MiB + 256 B array inside the library's device memory,
+ * held by every GPU that loads the library until the process exits.  Limits:
+ * M <= 32 and d_in <= 32768; larger sizes return LCVQ_ERR_WORKSPACE and
+ * launch nothing.  Other shape rules as lcvq_gemm.
+ * The first call on each device (made with that device current) looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it; make that first
+ * call before any stream capture begins.  The call allocates no memory.
+ * All calls share the one array and it keeps the last call's contents: two
+ * calls that may run at the same time on the GPU (different streams, or
+ * different host threads on the same device) race on it and must be ordered
+ * by the caller. */
+LCVQ_API lcvq_status lcvq_gemv_static(const void* X, int64_t M, const uint8_t* packed,
+                                      int64_t d_out, int64_t d_in, int d, const float* A,
+                                      const float* B, void* Y, void* stream);
+
 /* Straight-through QAT backward of Y = X W~ with W~ = decode(clamp(rint(Wp))).
  * (Methodology 1: gradients flow through the linear map c = A z + B;
  * Methodology 3 and the gradient-estimation ablation: STE through the

@@ -71,15 +71,14 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
   return q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
 }
 
-// CTA: 8 warps on 16 R weight rows over the whole K, so no partial sum leaves
-// the CTA.  Warp w takes K slice w of 8.  A "unit" is 128 codes of each of the
+// CTA: kWarps warps on 16 R weight rows over the whole K, so no partial sum
+// leaves the CTA.  Warp w takes K slice w.  A "unit" is 128 codes of each of the
 // CTA's rows: lane (g, t) holds 2 words of rows g and g + 8 of every row
 // block (8 B each); a warp keeps up to kAhead units of loads in flight.
 // Launch order with the X-transform (programmatic dependent launch): the code
 // loads are issued before griddepcontrol.wait, so they overlap the prologue;
 // X'' and corr are read only after it.
 constexpr int kUnit = 128;  // codes per row per unit (32 B)
-constexpr int kWarps = 8;
 constexpr int kAhead = 4;
 
 __device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
@@ -96,15 +95,14 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
 
-template <int NT, int R>
-__global__ void __launch_bounds__(kWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(const uint16_t* __restrict__ Xpp,
-                                                              const float* __restrict__ corr,
-                                                              int M,
-                                                              const uint8_t* __restrict__ packed,
-                                                              int64_t N, int64_t K,
-                                                              uint16_t* __restrict__ Y) {
+template <int NT, int R, int kWarps>
+__global__ void __launch_bounds__(kWarps * 32, (kWarps == 16 ? 1 : (NT <= 2 ? 2 : 1)))
+    gemv_kernel(const uint16_t* __restrict__ Xpp, const float* __restrict__ corr, int M,
+                const uint8_t* __restrict__ packed, int64_t N, int64_t K,
+                uint16_t* __restrict__ Y) {
   constexpr int MP = NT * 8;
   constexpr int ROWS = 16 * R;
+  constexpr bool kPrefX = NT == 1;  // keep the next unit's X'' fragments in flight
   __shared__ float part[kWarps][ROWS][MP + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -157,26 +155,34 @@ __global__ void __launch_bounds__(kWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(co
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[r][n][e] = 0.f;
 
+  // X'' fragments of one unit: word q, token tile n -> two 16-byte halves
+  auto load_x = [&](int64_t u, uint4 (&xb)[2][NT][2]) {
+    const bool kok = u < u1 && u * kUnit + 32 * t < K;
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        if (kok && tokok[n]) {
+          const uint4* src = reinterpret_cast<const uint4*>(xrow[n] + u * kUnit + 16 * q);
+          xb[q][n][0] = __ldg(src);
+          xb[q][n][1] = __ldg(src + 1);
+        } else {
+          xb[q][n][0] = make_uint4(0, 0, 0, 0);
+          xb[q][n][1] = make_uint4(0, 0, 0, 0);
+        }
+      }
+  };
+  uint4 xcur[2][NT][2], xnxt[2][NT][2];
+  load_x(u0, xcur);
+
   for (int64_t base = u0; base < u1; base += kAhead) {
 #pragma unroll
     for (int j = 0; j < kAhead; ++j) {
       const int64_t u = base + j;
       if (u >= u1) break;
-      const bool kok = u * kUnit + 32 * t < K;
+      if constexpr (kPrefX) load_x(u + 1, xnxt);
 #pragma unroll
       for (int q = 0; q < 2; ++q) {  // word q of each row: 16 codes, 4 k16 tiles
-        uint4 xb[NT][2];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          if (kok && tokok[n]) {
-            const uint4* src = reinterpret_cast<const uint4*>(xrow[n] + u * kUnit + 16 * q);
-            xb[n][0] = __ldg(src);
-            xb[n][1] = __ldg(src + 1);
-          } else {
-            xb[n][0] = make_uint4(0, 0, 0, 0);
-            xb[n][1] = make_uint4(0, 0, 0, 0);
-          }
-        }
         uint32_t w0[R][2], w6[R][2], w12[R][2];
 #pragma unroll
         for (int r = 0; r < R; ++r)
@@ -198,8 +204,8 @@ __global__ void __launch_bounds__(kWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(co
             }
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            const uint32_t b0 = word_of(xb[n][jj >> 1], (2 * jj) & 3);
-            const uint32_t b1 = word_of(xb[n][jj >> 1], (2 * jj + 1) & 3);
+            const uint32_t b0 = word_of(xcur[q][n][jj >> 1], (2 * jj) & 3);
+            const uint32_t b1 = word_of(xcur[q][n][jj >> 1], (2 * jj + 1) & 3);
 #pragma unroll
             for (int r = 0; r < R; ++r)
               mma_bf16_16816(acc[r][n], a[r][0][0], a[r][1][0], a[r][0][1], a[r][1][1], b0, b1);
@@ -207,6 +213,17 @@ __global__ void __launch_bounds__(kWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(co
         }
       }
       load_unit(u + kAhead, ring[j]);  // refill the slot just consumed
+      if constexpr (kPrefX) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            xcur[q][n][0] = xnxt[q][n][0];
+            xcur[q][n][1] = xnxt[q][n][1];
+          }
+      } else {
+        load_x(u + 1, xcur);
+      }
     }
   }
 
@@ -236,7 +253,7 @@ __global__ void __launch_bounds__(kWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(co
   }
 }
 
-template <int NT, int R>
+template <int NT, int R, int kWarps>
 cudaError_t launch_gemv_t(const uint16_t* Xpp, const float* corr, int M, const uint8_t* packed,
                           int64_t N, int64_t K, uint16_t* Y, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
@@ -249,7 +266,7 @@ cudaError_t launch_gemv_t(const uint16_t* Xpp, const float* corr, int M, const u
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, R>, Xpp, corr, M, packed, N, K, Y);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, R, kWarps>, Xpp, corr, M, packed, N, K, Y);
 }
 
 }  // namespace
@@ -260,11 +277,11 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
   cudaError_t e;
   const int m = static_cast<int>(M);
   if (M <= 8)
-    e = launch_gemv_t<1, 1>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<1, 1, 16>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else if (M <= 16)
-    e = launch_gemv_t<2, 2>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<2, 2, 8>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else
-    e = launch_gemv_t<4, 2>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<4, 2, 8>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   ++*launches;
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -41,11 +41,15 @@ __global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __res
   __shared__ float sA[D * D];
   __shared__ float sBp[D];
   __shared__ double red[3][kXfThreads / 32];
-  // Programmatic dependent launch: wait for every earlier kernel in the stream
-  // (X may be the previous layer's output), then let the decode-GEMV launch so
-  // its code loads overlap this kernel.
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // Programmatic dependent launch.  The decode-GEMV that follows may launch at
+  // once: before its own wait it only reads packed codes, and the only kernels
+  // that can still be running at that point are this one (waiting below) and
+  // the previous decode-GEMV in its epilogue, neither of which writes codes
+  // (every earlier kernel finished before the previous GEMV passed its wait).
+  // This kernel itself waits for every earlier kernel before it touches
+  // anything (X may be the previous layer's output).
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   if (threadIdx.x < D * D) sA[threadIdx.x] = A[threadIdx.x];
   __syncthreads();
   if (threadIdx.x < D) {

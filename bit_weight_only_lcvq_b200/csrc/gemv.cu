@@ -277,7 +277,7 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
   cudaError_t e;
   const int m = static_cast<int>(M);
   if (M <= 8)
-    e = launch_gemv_t<1, 1, 16>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<1, 1, 8>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else if (M <= 16)
     e = launch_gemv_t<2, 2, 8>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else

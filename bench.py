@@ -55,6 +55,29 @@ def parse():
     return p.parse_args()
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel, from one ncu capture (profiles/), valid only for the kernel
+# source that was captured: keyed by the SHA-1 of the source file.
+NCU_TRAFFIC = {
+    # source file -> (sha1 of the file when captured, {token count: bytes per launch})
+}
+
+
+def traffic_for(src_rel: str, key):
+    import hashlib
+    entry = NCU_TRAFFIC.get(src_rel)
+    if entry is None:
+        return None
+    path = os.path.join(ROOT, src_rel)
+    try:
+        h = hashlib.sha1(open(path, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if h != entry[0]:
+        return None  # the kernel changed since the counters were taken
+    return entry[1].get(key)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -229,6 +252,10 @@ def oracle_gemv_sample(Ms, seconds=10.0):
 
 
 # ----------------------------------------------------------------------------- headline
+def _sum_or_none(xs):
+    return None if any(x is None for x in xs) else float(sum(xs))
+
+
 def headline(args, D: Dist, pk):
     K = N = 4096
     d = 8
@@ -333,7 +360,10 @@ def headline(args, D: Dist, pk):
                 "l2": f"inputs larger than L2: {R} rotated packed-weight copies ({R * 4} MiB)",
                 "parallelism": f"replicas x{D.world}" if D.world > 1 else "single GPU"},
         roofline=dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
-                      traffic=None, kernel="gemv_kernel (decode-GEMV, M=1,4,16 summed)",
+                      traffic=_sum_or_none([traffic_for("bit_weight_only_lcvq_b200/csrc/gemv.cu", M)
+                                            for M in Ms]),
+                      traffic_unit="bytes per step (3 launches)",
+                      kernel="gemv_kernel (decode-GEMV, M=1,4,16 summed)",
                       per_m_us={str(M): per_m[M] * 1e3 for M in Ms},
                       peak_source=f"{PEAK_SRC} hbm_gbs"),
         e2e=e2e, clocks=ck, gpu_launches=int(launches), parity_max_rel_err=parity,

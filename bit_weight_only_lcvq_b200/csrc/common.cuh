@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/lcvq.h"
+#include "lcvq.h"
 
 namespace lcvq {
 

@@ -10,7 +10,7 @@
 //
 // D tiles are 128 x 256 fp32 in TMEM, double buffered (512 columns), so the
 // epilogue of one tile overlaps the main loop of the next.  Shared memory holds
-// two rings (TMA-filled A + codes, decoded B); mbarriers hand them between the roles.  Every
+// STAGES (A, B, codes) stages; mbarriers hand them between the roles.  Every
 // wait is bounded: a wait that gives up records LCVQ_ERR_DEVICE_TIMEOUT in the
 // workspace error word and the kernel winds down without trapping.
 //
@@ -45,9 +45,10 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
+constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int C_BYTES = 4096;         // packed codes of one k block
+constexpr int C_BYTES = 4096;         // packed codes of one stage
 constexpr int kTmemCols = 512;
 constexpr long long kWaitLimit = 1LL << 32;  // clock cycles (~2 s)
 
@@ -67,24 +68,19 @@ struct Params {
   unsigned int* err;
 };
 
-// Two shared-memory rings.  Ring A holds what TMA brings in: the A tile plus
-// either the packed codes of the B tile (kinds with decoders) or the B tile
-// itself (Dw).  Ring B holds decoded bf16 B tiles.  Ring A is deeper because a
-// slot is held from the TMA issue through decode and MMA.
 template <int KIND, int DW>
 struct Cfg {
   static constexpr int kThreads = 32 * (2 + DW + 4);
   static constexpr bool kHasCodes = KIND != kDw;
   static constexpr bool kAmn = KIND == kDw;
   static constexpr bool kBmn = KIND == kDx || KIND == kDw;
-  static constexpr int kSA = kHasCodes ? 6 : 4;
-  static constexpr int kSB = kHasCodes ? 3 : 0;
-  static constexpr int kStageA = A_BYTES + (kHasCodes ? C_BYTES : B_BYTES);
-  static constexpr uint32_t kStageTx = kStageA;
-  // 1024 B of alignment slack, the rings, then barriers, TMEM address, abort
-  // flag, A/B (<= 72 floats) and the dA/dB reduction scratch (4 x 72 floats)
-  static constexpr size_t kSmem = 1024 + size_t(kSA) * kStageA + size_t(kSB) * B_BYTES + 4096;
+  static constexpr uint32_t kStageTx = A_BYTES + (kHasCodes ? C_BYTES : B_BYTES);
 };
+
+// 1024 B of alignment slack, the stages, then barriers, TMEM address, abort
+// flag, A/B (<= 72 floats) and the dA/dB reduction scratch (4 x 72 floats)
+constexpr size_t kTailBytes = 4096;
+constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * (A_BYTES + B_BYTES + C_BYTES) + kTailBytes;
 
 __device__ __forceinline__ void fail(const Params& p, volatile int* abort_flag, unsigned site) {
   record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, site);
@@ -120,17 +116,16 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const Params p) {
   using C = Cfg<KIND, DW>;
-  constexpr int SA = C::kSA, SB = C::kSB > 0 ? C::kSB : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ringA = smem;                                // SA x (A tile, then codes or B tile)
-  uint8_t* ringB = ringA + size_t(SA) * C::kStageA;     // kSB x decoded B tile
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ringB + size_t(C::kSB) * B_BYTES);
-  uint64_t* fullA = bars;
-  uint64_t* emptyA = bars + SA;
-  uint64_t* decd = bars + 2 * SA;
-  uint64_t* emptyB = decd + SB;
-  uint64_t* tfull = emptyB + SB;
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sC = sB + STAGES * B_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + STAGES * C_BYTES);
+  uint64_t* full = bars;
+  uint64_t* decd = bars + STAGES;
+  uint64_t* empty = bars + 2 * STAGES;
+  uint64_t* tfull = bars + 3 * STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -144,17 +139,14 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
   const int64_t kblocks = ceil_div(p.K, BK);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) {
-      mbar_init(&fullA[s], 1);                 // producer's expect-tx arrive
-      mbar_init(&emptyA[s], 1 + DW);           // MMA commit + one arrive per decoder warp
-    }
-    for (int s = 0; s < SB; ++s) {
-      mbar_init(&decd[s], DW > 0 ? DW : 1);    // one arrive per decoder warp
-      mbar_init(&emptyB[s], 1);                // MMA commit
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&decd[s], DW > 0 ? DW : 1);     // one arrive per decoder warp
+      mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);                // one arrive per epilogue warp
+      mbar_init(&tempty[b], 4);                 // one arrive per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -186,26 +178,24 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
       for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
         const int mt = static_cast<int>(tile / n_tiles), nt = static_cast<int>(tile % n_tiles);
         for (int64_t kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&emptyA[s], ph ^ 1, kWaitLimit)) { fail(p, abort_flag, 1); break; }
+          if (!mbar_wait(&empty[s], ph ^ 1, kWaitLimit)) { fail(p, abort_flag, 1); break; }
           if (*abort_flag) break;
-          mbar_arrive_expect_tx(&fullA[s], C::kStageTx);
+          mbar_arrive_expect_tx(&full[s], C::kStageTx);
           const int kx = static_cast<int>(kb);
-          uint8_t* sa = ringA + size_t(s) * C::kStageA;
-          uint8_t* sx = sa + A_BYTES;  // codes, or the B tile for Dw
           if constexpr (KIND == kFwdAlg || KIND == kFwdDec) {
-            tma_load_2d(&tmA, &fullA[s], sa, kx * BK, mt * BM);
-            tma_load_2d(&tmB, &fullA[s], sx, kx * (BK / 4), nt * BN);
+            tma_load_2d(&tmA, &full[s], sA + s * A_BYTES, kx * BK, mt * BM);
+            tma_load_2d(&tmB, &full[s], sC + s * C_BYTES, kx * (BK / 4), nt * BN);
           } else if constexpr (KIND == kDx) {
-            tma_load_2d(&tmA, &fullA[s], sa, kx * BK, mt * BM);
-            tma_load_2d(&tmB, &fullA[s], sx, nt * (BN / 4), kx * BK);
+            tma_load_2d(&tmA, &full[s], sA + s * A_BYTES, kx * BK, mt * BM);
+            tma_load_2d(&tmB, &full[s], sC + s * C_BYTES, nt * (BN / 4), kx * BK);
           } else {
-            tma_load_2d(&tmA, &fullA[s], sa, mt * BM, kx * BK);
-            tma_load_2d(&tmA, &fullA[s], sa + 8192, mt * BM + 64, kx * BK);
+            tma_load_2d(&tmA, &full[s], sA + s * A_BYTES, mt * BM, kx * BK);
+            tma_load_2d(&tmA, &full[s], sA + s * A_BYTES + 8192, mt * BM + 64, kx * BK);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              tma_load_2d(&tmB, &fullA[s], sx + q * 8192, nt * BN + q * 64, kx * BK);
+              tma_load_2d(&tmB, &full[s], sB + s * B_BYTES + q * 8192, nt * BN + q * 64, kx * BK);
           }
-          if (++s == SA) { s = 0; ph ^= 1; }
+          if (++s == STAGES) { s = 0; ph ^= 1; }
         }
       }
     }
@@ -213,8 +203,8 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, C::kAmn, C::kBmn);
-      int sa = 0, sb = 0;
-      uint32_t pha = 0, phb = 0;
+      int s = 0;
+      uint32_t ph = 0;
       int64_t local = 0;
       bool issued = false;
       for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++local) {
@@ -225,13 +215,11 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
         const uint32_t dt = tmem + buf * BN;
         bool ok = true;
         for (int64_t kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&fullA[sa], pha, kWaitLimit)) { fail(p, abort_flag, 3); ok = false; break; }
-          if constexpr (C::kHasCodes) {
-            if (!mbar_wait(&decd[sb], phb, kWaitLimit)) { fail(p, abort_flag, 7); ok = false; break; }
-          }
+          uint64_t* ready = (DW > 0) ? &decd[s] : &full[s];
+          if (!mbar_wait(ready, ph, kWaitLimit)) { fail(p, abort_flag, 3); ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(ringA + size_t(sa) * C::kStageA);
-          const uint32_t b0 = C::kHasCodes ? smem_u32(ringB + size_t(sb) * B_BYTES) : a0 + A_BYTES;
+          const uint32_t a0 = smem_u32(sA + s * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + s * B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = C::kAmn ? sdesc_sw128(a0 + k * 2048, 8192, 1024)
@@ -241,12 +229,8 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
             mma_ss(dt, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           issued = true;
-          mma_commit(&emptyA[sa]);
-          if constexpr (C::kHasCodes) mma_commit(&emptyB[sb]);
-          if (++sa == SA) { sa = 0; pha ^= 1; }
-          if constexpr (C::kHasCodes) {
-            if (++sb == SB) { sb = 0; phb ^= 1; }
-          }
+          mma_commit(&empty[s]);
+          if (++s == STAGES) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
         mma_commit(&tfull[buf]);
@@ -259,14 +243,13 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
   } else if (warp < 2 + DW) {
     // ------------------------------------------------------------ decoders
     const int dt = threadIdx.x - 64;  // 0 .. 32*DW-1
-    int sa = 0, sb = 0;
-    uint32_t pha = 0, phb = 0;
+    int s = 0;
+    uint32_t ph = 0;
     for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
       for (int64_t kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&fullA[sa], pha, kWaitLimit)) { fail(p, abort_flag, 5); break; }
-        if (!mbar_wait(&emptyB[sb], phb ^ 1, kWaitLimit)) { fail(p, abort_flag, 8); break; }
-        const uint8_t* cs = ringA + size_t(sa) * C::kStageA + A_BYTES;
-        const uint32_t bs = smem_u32(ringB + size_t(sb) * B_BYTES);
+        if (!mbar_wait(&full[s], ph, kWaitLimit)) { fail(p, abort_flag, 5); break; }
+        const uint8_t* cs = sC + s * C_BYTES;
+        const uint32_t bs = smem_u32(sB + s * B_BYTES);
         if constexpr (KIND == kFwdAlg) {
 #pragma unroll
           for (int rr = 0; rr < BN / (32 * DW); ++rr) {
@@ -334,12 +317,8 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
         }
         fence_async_smem();  // this lane's B tile stores -> visible to the MMA
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&decd[sb]);   // B tile complete (this warp's rows)
-          mbar_arrive(&emptyA[sa]); // this warp is done reading the codes
-        }
-        if (++sa == SA) { sa = 0; pha ^= 1; }
-        if (++sb == SB) { sb = 0; phb ^= 1; }
+        if (lane == 0) mbar_arrive(&decd[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1; }
       }
     }
   } else {
@@ -538,7 +517,7 @@ cudaError_t launch_kind(const CUtensorMap& a, const CUtensorMap& b, const Params
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(C::kSmem));
+                                    static_cast<int>(kSmemBytes));
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int64_t tiles = ceil_div(p.M, BM) * ceil_div(p.N, BN);
@@ -546,7 +525,7 @@ cudaError_t launch_kind(const CUtensorMap& a, const CUtensorMap& b, const Params
   if (tiles < grid) grid = static_cast<int>(tiles);
   if (grid < 1) grid = 1;
   if (grid_out) *grid_out = grid;
-  kern<<<grid, C::kThreads, C::kSmem, s>>>(a, b, p);
+  kern<<<grid, C::kThreads, kSmemBytes, s>>>(a, b, p);
   return cudaGetLastError();
 }
 

@@ -82,6 +82,18 @@ struct Cfg {
 constexpr size_t kTailBytes = 4096;
 constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * (A_BYTES + B_BYTES + C_BYTES) + kTailBytes;
 
+// Tile order: bands of kBand D-row tiles, column-major inside a band, so the
+// CTAs that run at the same time share a few row blocks and a few column
+// blocks of the operands (both stay in L2 while the contraction sweeps).
+__device__ __forceinline__ void tile_coords(int64_t tile, int64_t m_tiles, int64_t n_tiles,
+                                            int band, int& mt, int& nt) {
+  const int64_t per_band = int64_t(band) * n_tiles;
+  const int64_t b = tile / per_band, r = tile % per_band;
+  const int64_t rows = (b + 1) * band <= m_tiles ? band : m_tiles - b * band;
+  mt = static_cast<int>(b * band + r % rows);
+  nt = static_cast<int>(r / rows);
+}
+
 __device__ __forceinline__ void fail(const Params& p, volatile int* abort_flag, unsigned site) {
   record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, site);
   *abort_flag = 1;
@@ -134,6 +146,7 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
   float* sRed = sAm + 80;                                 // 4 x (D*D + D) floats
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kBand = 16;
   const int64_t m_tiles = ceil_div(p.M, BM), n_tiles = ceil_div(p.N, BN);
   const int64_t tiles = m_tiles * n_tiles;
   const int64_t kblocks = ceil_div(p.K, BK);
@@ -176,7 +189,8 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
-        const int mt = static_cast<int>(tile / n_tiles), nt = static_cast<int>(tile % n_tiles);
+        int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
         for (int64_t kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, kWaitLimit)) { fail(p, abort_flag, 1); break; }
           if (*abort_flag) break;
@@ -301,8 +315,8 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
           // MN-major: 4 blocks of 64 k (8 KB), each [64 n lines][128 B]
 #pragma unroll
           for (int it = 0; it < (64 * 4) / (32 * DW); ++it) {
-            const int u = dt + it * 32 * DW;  // (row n_l, block q)
-            const int nl = u >> 2, q = u & 3;
+            const int u = dt + it * 32 * DW;  // (row n_l, block q): a warp = 32 rows of one block
+            const int nl = u & 63, q = u >> 6;
             const uint4 cw = *reinterpret_cast<const uint4*>(cs + nl * 64 + q * 16);
             const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
             const uint32_t line = bs + q * 8192 + nl * 128;
@@ -334,7 +348,8 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
     }
     int64_t local = 0;
     for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++local) {
-      const int mt = static_cast<int>(tile / n_tiles), nt = static_cast<int>(tile % n_tiles);
+      int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
       const int buf = static_cast<int>(local & 1);
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       if (!mbar_wait(&tfull[buf], use & 1, kWaitLimit)) { fail(p, abort_flag, 6); break; }

@@ -123,6 +123,118 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
+// One 32-column chunk of a D row (registers r[] from TMEM): the fused
+// epilogue of each kind.  gm is the D row, gn0 the first D column.
+template <int KIND, int D>
+__device__ __forceinline__ void epilogue_chunk(const Params& p, const float* sAm,
+                                               const uint32_t (&r)[32], int64_t gm, int64_t gn0,
+                                               float addc, float rs, float (&pa)[D * D],
+                                               float (&pb)[D]) {
+  if constexpr (KIND == kFwdAlg || KIND == kFwdDec) {
+    uint16_t* Y = static_cast<uint16_t*>(p.out) + gm * p.N + gn0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (gn0 + 8 * q >= p.N) break;
+      uint4 v;
+      v.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) + addc, __uint_as_float(r[8 * q + 1]) + addc);
+      v.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) + addc, __uint_as_float(r[8 * q + 3]) + addc);
+      v.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) + addc, __uint_as_float(r[8 * q + 5]) + addc);
+      v.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) + addc, __uint_as_float(r[8 * q + 7]) + addc);
+      *reinterpret_cast<uint4*>(Y + 8 * q) = v;
+    }
+  } else if constexpr (KIND == kDx) {
+    uint16_t* dX = static_cast<uint16_t*>(p.out) + gm * p.N + gn0;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {  // two 16-blocks of output k
+      float pz[16];
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const float inv = (cc % 3 == 0) ? 1.0f : ((cc % 3 == 1) ? 0.25f : 0.0625f);
+        pz[cc] = (__uint_as_float(r[16 * b + 2 * cc]) - 128.0f * rs) * inv;
+        pz[cc + 8] = (__uint_as_float(r[16 * b + 2 * cc + 1]) - 128.0f * rs) * inv;
+      }
+      float o[16];
+#pragma unroll
+      for (int v = 0; v < 16 / D; ++v)
+#pragma unroll
+        for (int i = 0; i < D; ++i) {
+          float a = sAm[D * D + i] * rs;
+#pragma unroll
+          for (int j = 0; j < D; ++j) a = fmaf(sAm[i * D + j], pz[v * D + j], a);
+          o[v * D + i] = a;
+        }
+      uint4 v0, v1;
+      v0.x = pack_bf16x2(o[0], o[1]); v0.y = pack_bf16x2(o[2], o[3]);
+      v0.z = pack_bf16x2(o[4], o[5]); v0.w = pack_bf16x2(o[6], o[7]);
+      v1.x = pack_bf16x2(o[8], o[9]); v1.y = pack_bf16x2(o[10], o[11]);
+      v1.z = pack_bf16x2(o[12], o[13]); v1.w = pack_bf16x2(o[14], o[15]);
+      reinterpret_cast<uint4*>(dX + 16 * b)[0] = v0;
+      reinterpret_cast<uint4*>(dX + 16 * b)[1] = v1;
+    }
+  } else {  // kDw: D row = n (d_out), D column = k (d_in)
+    const int64_t n = gm, k0 = gn0;
+    const uint2 zc = *reinterpret_cast<const uint2*>(p.codes + n * (p.d_in / 4) + k0 / 4);
+    const uint32_t mb = p.mask != nullptr
+                            ? *reinterpret_cast<const uint32_t*>(p.mask + n * (p.d_in / 8) + k0 / 8)
+                            : 0xFFFFFFFFu;
+    float* dWp = static_cast<float*>(p.out);
+    float o[32];
+#pragma unroll
+    for (int v = 0; v < 32 / D; ++v) {
+      float G[D], z[D];
+#pragma unroll
+      for (int i = 0; i < D; ++i) G[i] = __uint_as_float(r[v * D + i]);
+#pragma unroll
+      for (int j = 0; j < D; ++j) {
+        const int e = v * D + j;
+        const uint32_t word = e < 16 ? zc.x : zc.y;
+        z[j] = static_cast<float>((word >> (2 * (e & 15))) & 3u);
+      }
+#pragma unroll
+      for (int i = 0; i < D; ++i) {
+        pb[i] += G[i];
+#pragma unroll
+        for (int j = 0; j < D; ++j) pa[i * D + j] = fmaf(G[i], z[j], pa[i * D + j]);
+      }
+#pragma unroll
+      for (int j = 0; j < D; ++j) {
+        float sacc = 0.f;
+#pragma unroll
+        for (int i = 0; i < D; ++i) sacc = fmaf(sAm[i * D + j], G[i], sacc);
+        o[v * D + j] = ((mb >> (v * D + j)) & 1u) ? sacc : 0.f;
+      }
+    }
+    if (dWp != nullptr) {
+      float4* dst = reinterpret_cast<float4*>(dWp + n * p.d_in + k0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+  }
+}
+
+// Per-CTA partials of dA and dB: warp tree, then the 4 epilogue warps in a
+// fixed order; one row of p.partials per CTA.
+template <int D>
+__device__ __forceinline__ void dw_block_partials(const Params& p, float (&pa)[D * D],
+                                                  float (&pb)[D], float* sRed, int quarter,
+                                                  int lane) {
+  // per-CTA partials of dA, dB: warp tree, then the 4 warps in order
+  constexpr int NP = D * D + D;
+#pragma unroll
+  for (int e = 0; e < NP; ++e) {
+    float x = e < D * D ? pa[e] : pb[e - D * D];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xffffffffu, x, off);
+    if (lane == 0) sRed[quarter * NP + e] = x;
+  }
+  asm volatile("bar.sync 1, 128;\n" ::: "memory");  // the 4 epilogue warps only
+  if (quarter == 0 && lane < 1) {
+    for (int e = 0; e < NP; ++e)
+      p.partials[int64_t(blockIdx.x) * NP + e] =
+          ((sRed[e] + sRed[NP + e]) + sRed[2 * NP + e]) + sRed[3 * NP + e];
+  }
+}
+
 template <int KIND, int D, int DW>
 __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -367,108 +479,13 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
         tmem_ld_wait();
         const int64_t gn0 = int64_t(nt) * BN + c * 32;  // first D column of the chunk
         if (gm >= p.M || gn0 >= p.N) continue;
-        if constexpr (KIND == kFwdAlg || KIND == kFwdDec) {
-          uint16_t* Y = static_cast<uint16_t*>(p.out) + gm * p.N + gn0;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (gn0 + 8 * q >= p.N) break;
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) + addc, __uint_as_float(r[8 * q + 1]) + addc);
-            v.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) + addc, __uint_as_float(r[8 * q + 3]) + addc);
-            v.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) + addc, __uint_as_float(r[8 * q + 5]) + addc);
-            v.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) + addc, __uint_as_float(r[8 * q + 7]) + addc);
-            *reinterpret_cast<uint4*>(Y + 8 * q) = v;
-          }
-        } else if constexpr (KIND == kDx) {
-          uint16_t* dX = static_cast<uint16_t*>(p.out) + gm * p.N + gn0;
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {  // two 16-blocks of output k
-            float pz[16];
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              const float inv = (cc % 3 == 0) ? 1.0f : ((cc % 3 == 1) ? 0.25f : 0.0625f);
-              pz[cc] = (__uint_as_float(r[16 * b + 2 * cc]) - 128.0f * rs) * inv;
-              pz[cc + 8] = (__uint_as_float(r[16 * b + 2 * cc + 1]) - 128.0f * rs) * inv;
-            }
-            float o[16];
-#pragma unroll
-            for (int v = 0; v < 16 / D; ++v)
-#pragma unroll
-              for (int i = 0; i < D; ++i) {
-                float a = sAm[D * D + i] * rs;
-#pragma unroll
-                for (int j = 0; j < D; ++j) a = fmaf(sAm[i * D + j], pz[v * D + j], a);
-                o[v * D + i] = a;
-              }
-            uint4 v0, v1;
-            v0.x = pack_bf16x2(o[0], o[1]); v0.y = pack_bf16x2(o[2], o[3]);
-            v0.z = pack_bf16x2(o[4], o[5]); v0.w = pack_bf16x2(o[6], o[7]);
-            v1.x = pack_bf16x2(o[8], o[9]); v1.y = pack_bf16x2(o[10], o[11]);
-            v1.z = pack_bf16x2(o[12], o[13]); v1.w = pack_bf16x2(o[14], o[15]);
-            reinterpret_cast<uint4*>(dX + 16 * b)[0] = v0;
-            reinterpret_cast<uint4*>(dX + 16 * b)[1] = v1;
-          }
-        } else {  // kDw: D row = n (d_out), D column = k (d_in)
-          const int64_t n = gm, k0 = gn0;
-          const uint2 zc = *reinterpret_cast<const uint2*>(p.codes + n * (p.d_in / 4) + k0 / 4);
-          const uint32_t mb = p.mask != nullptr
-                                  ? *reinterpret_cast<const uint32_t*>(p.mask + n * (p.d_in / 8) + k0 / 8)
-                                  : 0xFFFFFFFFu;
-          float* dWp = static_cast<float*>(p.out);
-          float o[32];
-#pragma unroll
-          for (int v = 0; v < 32 / D; ++v) {
-            float G[D], z[D];
-#pragma unroll
-            for (int i = 0; i < D; ++i) G[i] = __uint_as_float(r[v * D + i]);
-#pragma unroll
-            for (int j = 0; j < D; ++j) {
-              const int e = v * D + j;
-              const uint32_t word = e < 16 ? zc.x : zc.y;
-              z[j] = static_cast<float>((word >> (2 * (e & 15))) & 3u);
-            }
-#pragma unroll
-            for (int i = 0; i < D; ++i) {
-              pb[i] += G[i];
-#pragma unroll
-              for (int j = 0; j < D; ++j) pa[i * D + j] = fmaf(G[i], z[j], pa[i * D + j]);
-            }
-#pragma unroll
-            for (int j = 0; j < D; ++j) {
-              float sacc = 0.f;
-#pragma unroll
-              for (int i = 0; i < D; ++i) sacc = fmaf(sAm[i * D + j], G[i], sacc);
-              o[v * D + j] = ((mb >> (v * D + j)) & 1u) ? sacc : 0.f;
-            }
-          }
-          if (dWp != nullptr) {
-            float4* dst = reinterpret_cast<float4*>(dWp + n * p.d_in + k0);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-          }
-        }
+        epilogue_chunk<KIND, D>(p, sAm, r, gm, gn0, addc, rs, pa, pb);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
     }
-    if constexpr (KIND == kDw) {
-      // per-CTA partials of dA, dB: warp tree, then the 4 warps in order
-      constexpr int NP = D * D + D;
-#pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        float x = e < D * D ? pa[e] : pb[e - D * D];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xffffffffu, x, off);
-        if (lane == 0) sRed[quarter * NP + e] = x;
-      }
-      asm volatile("bar.sync 1, 128;\n" ::: "memory");  // the 4 epilogue warps only
-      if (quarter == 0 && lane < 1) {
-        for (int e = 0; e < NP; ++e)
-          p.partials[int64_t(blockIdx.x) * NP + e] =
-              ((sRed[e] + sRed[NP + e]) + sRed[2 * NP + e]) + sRed[3 * NP + e];
-      }
-    }
+    if constexpr (KIND == kDw) dw_block_partials<D>(p, pa, pb, sRed, quarter, lane);
   }
 
   tc_fence_before();
@@ -476,6 +493,291 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- CTA pairs
+// The same GEMMs on CTA pairs (cta_group::2): a pair computes a 256 x 256 tile;
+// each CTA holds 128 rows of A and 128 rows (N) of B, the even CTA issues the
+// 256 x 256 x 16 MMAs for both and each CTA's TMEM receives its 128 rows of D.
+// Per SM this halves the B tile the tensor core reads and the codes each CTA
+// decodes.  Barriers: fullA/decd/tempty/drain live in the even CTA (the
+// odd CTA's TMA loads and arrivals are counted there); fullC, empty and tfull
+// are per CTA (the MMA commits arrive on both CTAs' copies).
+template <int KIND, int DW>
+struct Cfg2 {
+  static constexpr int kThreads = 32 * (2 + DW + 4);
+  static constexpr bool kHasCodes = KIND != kDw;
+  static constexpr bool kAmn = KIND == kDw;
+  static constexpr bool kBmn = KIND == kDx || KIND == kDw;
+  static constexpr int kStages = 6;
+  static constexpr int kA = 16384;                      // 128 rows x 64 bf16
+  static constexpr int kB = 16384;                      // this CTA's 128 rows of B
+  static constexpr int kC = kHasCodes ? 2048 : 0;       // codes of those 128 rows
+  static constexpr int kStage = kA + kB + kC;
+  static constexpr uint32_t kOperandTx = kHasCodes ? kA : kA + kB;  // per CTA, to fullA
+  static constexpr size_t kSmem = 1024 + size_t(kStages) * kStage + 4096;
+};
+
+template <int KIND, int D, int DW>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThreads, 1)
+    tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Params p) {
+  using C = Cfg2<KIND, DW>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * C::kStage);
+  uint64_t* fullA = bars;            // [S]  even CTA: A (+B) of both CTAs landed
+  uint64_t* fullC = bars + S;        // [S]  per CTA: its codes landed
+  uint64_t* decd = bars + 2 * S;     // [S]  even CTA: both CTAs' B halves decoded
+  uint64_t* empty = bars + 3 * S;    // [S]  per CTA: the MMA is done with stage s
+  uint64_t* tfull = bars + 4 * S;    // [2]  per CTA: accumulator buffer ready
+  uint64_t* tempty = tfull + 2;      // [2]  even CTA: both epilogues drained the buffer
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* sAm = reinterpret_cast<float*>(tmem_holder + 4);
+  float* sRed = sAm + 80;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  constexpr int kBand = 8;
+  const int64_t m_tiles = ceil_div(p.M, 2 * BM), n_tiles = ceil_div(p.N, BN);
+  const int64_t tiles = m_tiles * n_tiles;
+  const int64_t kblocks = ceil_div(p.K, BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&fullA[s], 1);
+      mbar_init(&fullC[s], 1);
+      mbar_init(&decd[s], DW > 0 ? 2 * DW : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if constexpr (KIND != kFwdAlg) {
+    if (threadIdx.x < D * D) sAm[threadIdx.x] = p.Amat[threadIdx.x];
+    if (KIND != kDw && threadIdx.x >= 64 && threadIdx.x < 64 + D)
+      sAm[D * D + threadIdx.x - 64] = p.Bvec[threadIdx.x - 64];
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmA);
+    tma_prefetch_map(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA use
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
+        int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
+        const int row0 = mt * 2 * BM + static_cast<int>(rank) * BM;  // this CTA's A rows
+        const int col0 = nt * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B rows
+        for (int64_t kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, kWaitLimit)) { fail(p, abort_flag, 11); break; }
+          if (*abort_flag) break;
+          uint8_t* st = smem + size_t(s) * C::kStage;
+          const uint32_t fa0 = mapa_shared(smem_u32(&fullA[s]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&fullA[s], 2 * C::kOperandTx);
+          const int kx = static_cast<int>(kb);
+          if constexpr (KIND == kFwdAlg || KIND == kFwdDec) {
+            mbar_arrive_expect_tx(&fullC[s], C::kC);
+            tma_load_2d(&tmB, &fullC[s], st + C::kA + C::kB, kx * (BK / 4), col0);
+            tma_load_2d_pair(&tmA, fa0, st, kx * BK, row0);
+          } else if constexpr (KIND == kDx) {
+            mbar_arrive_expect_tx(&fullC[s], C::kC);
+            tma_load_2d(&tmB, &fullC[s], st + C::kA + C::kB, col0 / 4, kx * BK);
+            tma_load_2d_pair(&tmA, fa0, st, kx * BK, row0);
+          } else {
+            tma_load_2d_pair(&tmA, fa0, st, row0, kx * BK);
+            tma_load_2d_pair(&tmA, fa0, st + 8192, row0 + 64, kx * BK);
+            tma_load_2d_pair(&tmB, fa0, st + C::kA, col0, kx * BK);
+            tma_load_2d_pair(&tmB, fa0, st + C::kA + 8192, col0 + 64, kx * BK);
+          }
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, C::kAmn, C::kBmn);
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t local = 0;
+      bool issued = false;
+      for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs, ++local) {
+        const int buf = static_cast<int>(local & 1);
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, kWaitLimit)) { fail(p, abort_flag, 12); break; }
+        tc_fence_after();
+        const uint32_t dt = tmem + buf * BN;
+        bool ok = true;
+        for (int64_t kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&fullA[s], ph, kWaitLimit)) { fail(p, abort_flag, 13); ok = false; break; }
+          if constexpr (C::kHasCodes) {
+            if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 14); ok = false; break; }
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + size_t(s) * C::kStage);
+          const uint32_t b0 = a0 + C::kA;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = C::kAmn ? sdesc_sw128(a0 + k * 2048, 8192, 1024)
+                                        : sdesc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = C::kBmn ? sdesc_sw128(b0 + k * 2048, 8192, 1024)
+                                        : sdesc_sw128(b0 + k * 32, 16, 1024);
+            mma_ss_pair(dt, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit_pair(&empty[s]);
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[buf]);
+      }
+      if (issued) {
+        mma_commit_pair(drain);
+        if (!mbar_wait(drain, 0, kWaitLimit)) fail(p, abort_flag, 15);
+      }
+    }
+  } else if (warp < 2 + DW) {
+    // ------------------------------------------------------------ decoders (both CTAs)
+    const int dt = threadIdx.x - 64;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
+      for (int64_t kb = 0; kb < kblocks; ++kb) {
+        if (!mbar_wait(&fullC[s], ph, kWaitLimit)) { fail(p, abort_flag, 16); break; }
+        uint8_t* st = smem + size_t(s) * C::kStage;
+        const uint8_t* cs = st + C::kA + C::kB;
+        const uint32_t bs = smem_u32(st + C::kA);
+        if constexpr (KIND == kFwdAlg) {  // 128 rows, one per thread
+          const int r = dt;
+          const uint4 cw = *reinterpret_cast<const uint4*>(cs + r * 16);
+          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+          const uint32_t row = bs + r * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 c0, c1;
+            dec_word(w[q], c0, c1);
+            st_shared_v4(row + (((2 * q) ^ (r & 7)) << 4), c0);
+            st_shared_v4(row + (((2 * q + 1) ^ (r & 7)) << 4), c1);
+          }
+        } else if constexpr (KIND == kFwdDec) {  // 128 rows, two threads per row
+          const int r = dt >> 1, h = dt & 1;
+          const uint2 cw = *reinterpret_cast<const uint2*>(cs + r * 16 + h * 8);
+          const uint32_t w[2] = {cw.x, cw.y};
+          const uint32_t row = bs + r * 128;
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const int q = 2 * h + qq;
+            float o[16];
+#pragma unroll
+            for (int v = 0; v < 16 / D; ++v) {
+              float z[D];
+#pragma unroll
+              for (int j = 0; j < D; ++j) z[j] = static_cast<float>((w[qq] >> (2 * (v * D + j))) & 3u);
+#pragma unroll
+              for (int i = 0; i < D; ++i) {
+                float a = sAm[D * D + i];
+#pragma unroll
+                for (int j = 0; j < D; ++j) a = fmaf(sAm[i * D + j], z[j], a);
+                o[v * D + i] = a;
+              }
+            }
+            const uint4 c0 = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                        pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+            const uint4 c1 = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
+                                        pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
+            st_shared_v4(row + (((2 * q) ^ (r & 7)) << 4), c0);
+            st_shared_v4(row + (((2 * q + 1) ^ (r & 7)) << 4), c1);
+          }
+        } else if constexpr (KIND == kDx) {  // [64 contraction rows][2 MN blocks of 64]
+          const int nl = dt & 63, q = dt >> 6;
+          const uint4 cw = *reinterpret_cast<const uint4*>(cs + nl * 32 + q * 16);
+          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+          const uint32_t line = bs + q * 8192 + nl * 128;
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            uint4 c0, c1;
+            dec_word(w[qq], c0, c1);
+            st_shared_v4(line + (((2 * qq) ^ (nl & 7)) << 4), c0);
+            st_shared_v4(line + (((2 * qq + 1) ^ (nl & 7)) << 4), c1);
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&decd[s]), 0));
+        if (++s == S) { s = 0; ph ^= 1; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    float pa[D * D], pb[D];
+    if constexpr (KIND == kDw) {
+#pragma unroll
+      for (int i = 0; i < D * D; ++i) pa[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < D; ++i) pb[i] = 0.f;
+    }
+    int64_t local = 0;
+    for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs, ++local) {
+      int mt, nt;
+      tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
+      const int buf = static_cast<int>(local & 1);
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      if (!mbar_wait(&tfull[buf], use & 1, kWaitLimit)) { fail(p, abort_flag, 17); break; }
+      tc_fence_after();
+      const int64_t gm = int64_t(mt) * 2 * BM + int64_t(rank) * BM + row;
+      const uint32_t tbase = tmem + buf * BN + (static_cast<uint32_t>(quarter * 32) << 16);
+      float addc = 0.f;
+      if constexpr (KIND == kFwdAlg) addc = gm < p.M ? p.corr[gm] : 0.f;
+      float rs = 0.f;
+      if constexpr (KIND == kDx) rs = gm < p.M ? p.rsum[gm] : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c * 32, r);
+        tmem_ld_wait();
+        const int64_t gn0 = int64_t(nt) * BN + c * 32;
+        if (gm >= p.M || gn0 >= p.N) continue;
+        epilogue_chunk<KIND, D>(p, sAm, r, gm, gn0, addc, rs, pa, pb);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+    }
+    if constexpr (KIND == kDw) dw_block_partials<D>(p, pa, pb, sRed, quarter, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its peer may still use its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -555,6 +857,38 @@ cudaError_t launch_kind_d(int d, const CUtensorMap& a, const CUtensorMap& b, con
   }
 }
 
+template <int KIND, int D, int DW>
+cudaError_t launch_kind2(const CUtensorMap& a, const CUtensorMap& b, const Params& p,
+                         cudaStream_t s, int* grid_out) {
+  using C = Cfg2<KIND, DW>;
+  auto kern = tc2_gemm_kernel<KIND, D, DW>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(C::kSmem));
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int64_t tiles = ceil_div(p.M, 2 * BM) * ceil_div(p.N, BN);
+  int pairs = num_sms() / 2;
+  if (tiles < pairs) pairs = static_cast<int>(tiles);
+  if (pairs < 1) pairs = 1;
+  if (grid_out) *grid_out = 2 * pairs;
+  kern<<<2 * pairs, C::kThreads, C::kSmem, s>>>(a, b, p);
+  return cudaGetLastError();
+}
+
+template <int KIND, int DW>
+cudaError_t launch_kind2_d(int d, const CUtensorMap& a, const CUtensorMap& b, const Params& p,
+                           cudaStream_t s, int* grid_out) {
+  switch (d) {
+    case 1: return launch_kind2<KIND, 1, DW>(a, b, p, s, grid_out);
+    case 2: return launch_kind2<KIND, 2, DW>(a, b, p, s, grid_out);
+    case 4: return launch_kind2<KIND, 4, DW>(a, b, p, s, grid_out);
+    default: return launch_kind2<KIND, 8, DW>(a, b, p, s, grid_out);
+  }
+}
+
 }  // namespace
 
 int tc_max_grid() { return num_sms(); }
@@ -565,14 +899,14 @@ cudaError_t launch_tc_forward(const uint16_t* Xa, bool algebraic, const float* c
                               cudaStream_t s, int* launches) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Xa, d_in, M, d_in * 2, BK, BM, true) ||
-      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d_in / 4, d_out, d_in / 4, BK / 4, BN,
-                false))
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d_in / 4, d_out, d_in / 4, BK / 4,
+                BN / 2, false))
     return cudaErrorInvalidValue;
   Params p{};
   p.M = M; p.N = d_out; p.K = d_in; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.corr = corr; p.Amat = A; p.Bvec = B; p.out = Y; p.err = err;
-  cudaError_t e = algebraic ? launch_kind<kFwdAlg, 8, 4>(ta, tb, p, s, nullptr)
-                            : launch_kind_d<kFwdDec, 8>(d, ta, tb, p, s, nullptr);
+  cudaError_t e = algebraic ? launch_kind2<kFwdAlg, 8, 4>(ta, tb, p, s, nullptr)
+                            : launch_kind2_d<kFwdDec, 8>(d, ta, tb, p, s, nullptr);
   ++*launches;
   return e;
 }
@@ -583,13 +917,13 @@ cudaError_t launch_tc_backward_dx(const uint16_t* dY, const float* rsum, int64_t
                                   cudaStream_t s, int* launches) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, d_out, M, d_out * 2, BK, BM, true) ||
-      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d_in / 4, d_out, d_in / 4, BN / 4, BK,
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d_in / 4, d_out, d_in / 4, BN / 8, BK,
                 false))
     return cudaErrorInvalidValue;
   Params p{};
   p.M = M; p.N = d_in; p.K = d_out; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.rsum = rsum; p.Amat = A; p.Bvec = B; p.out = dX; p.err = err;
-  cudaError_t e = launch_kind_d<kDx, 4>(d, ta, tb, p, s, nullptr);
+  cudaError_t e = launch_kind2_d<kDx, 4>(d, ta, tb, p, s, nullptr);
   ++*launches;
   return e;
 }
@@ -607,7 +941,7 @@ cudaError_t launch_tc_backward_dw(const uint16_t* X, const uint16_t* dY, int64_t
   p.M = d_out; p.N = d_in; p.K = M; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.mask = mask; p.Amat = A; p.Bvec = A; p.out = dWp; p.partials = partials;
   p.err = err;
-  cudaError_t e = launch_kind_d<kDw, 0>(d, ta, tb, p, s, num_parts);
+  cudaError_t e = launch_kind2_d<kDw, 0>(d, ta, tb, p, s, num_parts);
   ++*launches;
   return e;
 }

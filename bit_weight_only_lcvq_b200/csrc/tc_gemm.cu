@@ -530,9 +530,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * C::kStage);
   uint64_t* fullA = bars;            // [S]  even CTA: A (+B) of both CTAs landed
   uint64_t* fullC = bars + S;        // [S]  per CTA: its codes landed
-  uint64_t* decd = bars + 2 * S;     // [S]  even CTA: both CTAs' B halves decoded
+  uint64_t* decd = bars + 2 * S;     // [S]  per CTA: its own B half decoded
   uint64_t* empty = bars + 3 * S;    // [S]  per CTA: the MMA is done with stage s
-  uint64_t* tfull = bars + 4 * S;    // [2]  per CTA: accumulator buffer ready
+  uint64_t* decd_peer = bars + 4 * S; // [S] even CTA: the odd CTA's B half decoded
+  uint64_t* tfull = bars + 5 * S;    // [2]  per CTA: accumulator buffer ready
   uint64_t* tempty = tfull + 2;      // [2]  even CTA: both epilogues drained the buffer
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -552,8 +553,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
     for (int s = 0; s < S; ++s) {
       mbar_init(&fullA[s], 1);
       mbar_init(&fullC[s], 1);
-      mbar_init(&decd[s], DW > 0 ? 2 * DW : 1);
+      mbar_init(&decd[s], DW > 0 ? DW : 1);   // this CTA's decoder warps
       mbar_init(&empty[s], 1);
+      mbar_init(&decd_peer[s], 1);            // one forwarded arrive from the odd CTA
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -628,7 +630,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs, ++local) {
         const int buf = static_cast<int>(local & 1);
         const uint32_t use = static_cast<uint32_t>(local >> 1);
-        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, kWaitLimit)) { fail(p, abort_flag, 12); break; }
+        // the odd CTA's epilogue arrives from the other SM: acquire at cluster scope
+        if (!mbar_wait_cluster(&tempty[buf], (use & 1) ^ 1, kWaitLimit)) { fail(p, abort_flag, 12); break; }
         tc_fence_after();
         const uint32_t dt = tmem + buf * BN;
         bool ok = true;
@@ -636,6 +639,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
           if (!mbar_wait(&fullA[s], ph, kWaitLimit)) { fail(p, abort_flag, 13); ok = false; break; }
           if constexpr (C::kHasCodes) {
             if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 14); ok = false; break; }
+            if (!mbar_wait_cluster(&decd_peer[s], ph, kWaitLimit)) {
+              fail(p, abort_flag, 18);
+              ok = false;
+              break;
+            }
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + size_t(s) * C::kStage);
@@ -658,6 +666,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       if (issued) {
         mma_commit_pair(drain);
         if (!mbar_wait(drain, 0, kWaitLimit)) fail(p, abort_flag, 15);
+      }
+    } else if (lane == 0 && C::kHasCodes) {
+      // odd CTA: forward "B half decoded" to the even CTA, one cluster-scope
+      // arrive per k block, so the decoder warps only ever arrive locally
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
+        for (int64_t kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 19); break; }
+          mbar_arrive_cluster(mapa_shared(smem_u32(&decd_peer[s]), 0));
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
       }
     }
   } else if (warp < 2 + DW) {
@@ -727,7 +747,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
         }
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&decd[s]), 0));
+        if (lane == 0) mbar_arrive(&decd[s]);
         if (++s == S) { s = 0; ph ^= 1; }
       }
     }

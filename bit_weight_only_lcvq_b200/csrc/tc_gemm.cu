@@ -553,7 +553,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
     for (int s = 0; s < S; ++s) {
       mbar_init(&fullA[s], 1);
       mbar_init(&fullC[s], 1);
-      mbar_init(&decd[s], DW > 0 ? DW : 1);   // this CTA's decoder warps
+      // this CTA's decoder warps of the group that owns stage s's k block
+      mbar_init(&decd[s], DW > 0 ? ((KIND == kFwdDec || DW < 8) ? DW : 4) : 1);
       mbar_init(&empty[s], 1);
       mbar_init(&decd_peer[s], 1);            // one forwarded arrive from the odd CTA
     }
@@ -682,11 +683,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
     }
   } else if (warp < 2 + DW) {
     // ------------------------------------------------------------ decoders (both CTAs)
-    const int dt = threadIdx.x - 64;
+    // kGroups groups of decoder warps take alternate k blocks, so each group has
+    // kGroups MMA k-block times to decode and publish one stage.
+    constexpr int kGroups = (KIND == kFwdDec || DW < 8) ? 1 : DW / 4;
+    constexpr int kGroupWarps = DW / kGroups > 0 ? DW / kGroups : 1;
+    const int grp = (warp - 2) / kGroupWarps;
+    const int dt = (threadIdx.x - 64) % (32 * kGroupWarps);
     int s = 0;
     uint32_t ph = 0;
+    int64_t it = 0;
     for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
-      for (int64_t kb = 0; kb < kblocks; ++kb) {
+      for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
+        if (it % kGroups != grp) {
+          if (++s == S) { s = 0; ph ^= 1; }
+          continue;
+        }
         if (!mbar_wait(&fullC[s], ph, kWaitLimit)) { fail(p, abort_flag, 16); break; }
         uint8_t* st = smem + size_t(s) * C::kStage;
         const uint8_t* cs = st + C::kA + C::kB;
@@ -925,7 +936,7 @@ cudaError_t launch_tc_forward(const uint16_t* Xa, bool algebraic, const float* c
   Params p{};
   p.M = M; p.N = d_out; p.K = d_in; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.corr = corr; p.Amat = A; p.Bvec = B; p.out = Y; p.err = err;
-  cudaError_t e = algebraic ? launch_kind2<kFwdAlg, 8, 4>(ta, tb, p, s, nullptr)
+  cudaError_t e = algebraic ? launch_kind2<kFwdAlg, 8, 8>(ta, tb, p, s, nullptr)
                             : launch_kind2_d<kFwdDec, 8>(d, ta, tb, p, s, nullptr);
   ++*launches;
   return e;
@@ -943,7 +954,7 @@ cudaError_t launch_tc_backward_dx(const uint16_t* dY, const float* rsum, int64_t
   Params p{};
   p.M = M; p.N = d_in; p.K = d_out; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.rsum = rsum; p.Amat = A; p.Bvec = B; p.out = dX; p.err = err;
-  cudaError_t e = launch_kind2_d<kDx, 4>(d, ta, tb, p, s, nullptr);
+  cudaError_t e = launch_kind2_d<kDx, 8>(d, ta, tb, p, s, nullptr);
   ++*launches;
   return e;
 }

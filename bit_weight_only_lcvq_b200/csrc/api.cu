@@ -171,7 +171,11 @@ lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t*
   cudaError_t e = cudaSuccess;
   char* ws = static_cast<char*>(workspace);
   unsigned int* err = reinterpret_cast<unsigned int*>(ws);
-  if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
+  if (dtype == LCVQ_BF16 && M <= 32 &&
+      launch_gemv_fused(static_cast<const uint16_t*>(X), M, packed, d_out, d_in, d, A, B,
+                        static_cast<uint16_t*>(Y), s, &launches, &e)) {
+    // decode-GEMV with the X-transform fused: one launch
+  } else if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
     uint16_t* Xpp = reinterpret_cast<uint16_t*>(ws + w.xpp_off);
     float* corr = reinterpret_cast<float*>(ws + w.corr_off);
     e = launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr, s, &launches);

@@ -27,6 +27,12 @@ cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, cons
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
                         int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s, int* launches);
 
+// single-kernel decode-GEMV with the X-transform fused (bf16, M <= 32).
+// Returns false (launching nothing) when the shape needs the two-kernel path.
+bool launch_gemv_fused(const uint16_t* X, int64_t M, const uint8_t* packed, int64_t d_out,
+                       int64_t d_in, int d, const float* A, const float* B, uint16_t* Y,
+                       cudaStream_t s, int* launches, cudaError_t* err);
+
 // integer-code GEMM on X'' (dispatches on M: decode-GEMV for M <= 32, else
 // the tcgen05 GEMM); err may be null (no device error word)
 cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,

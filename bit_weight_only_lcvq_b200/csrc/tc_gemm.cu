@@ -668,16 +668,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
         mma_commit_pair(drain);
         if (!mbar_wait(drain, 0, kWaitLimit)) fail(p, abort_flag, 15);
       }
-    } else if (lane == 0 && C::kHasCodes) {
-      // odd CTA: forward "B half decoded" to the even CTA, one cluster-scope
-      // arrive per k block, so the decoder warps only ever arrive locally
-      int s = 0;
+    } else if (rank == 1 && lane < S && C::kHasCodes) {
+      // odd CTA: forward "B half decoded" to the even CTA.  Lane s owns stage s,
+      // so up to S cross-CTA arrives are in flight at once and the decoder warps
+      // only ever arrive locally.
+      const int s = lane;
       uint32_t ph = 0;
+      int64_t it = 0;
       for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
-        for (int64_t kb = 0; kb < kblocks; ++kb) {
+        for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
+          if (it % S != s) continue;
           if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 19); break; }
           mbar_arrive_cluster(mapa_shared(smem_u32(&decd_peer[s]), 0));
-          if (++s == S) { s = 0; ph ^= 1; }
+          ph ^= 1;
         }
       }
     }

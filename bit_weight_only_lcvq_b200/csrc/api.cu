@@ -2,11 +2,41 @@
 // Every entry point validates all of its arguments before it launches
 // anything, so a failing call has no side effect.
 #include <atomic>
+#include <mutex>
+#include <set>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
 
 using namespace lcvq;
+
+namespace lcvq {
+
+cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;  // (function, device) already raised
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({func, dev})) return cudaSuccess;
+  // raise to the device maximum once, so any size up to it needs no further call
+  int max_optin = 0;
+  if (cudaError_t e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+      e != cudaSuccess)
+    return e;
+  if (bytes > size_t(max_optin)) return cudaErrorInvalidValue;
+  cudaFuncAttributes fa{};
+  if (cudaError_t e = cudaFuncGetAttributes(&fa, func); e != cudaSuccess) return e;
+  const int dyn_max = max_optin - static_cast<int>(fa.sharedSizeBytes);
+  if (cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max);
+      e != cudaSuccess)
+    return e;
+  done.insert({func, dev});
+  return cudaSuccess;
+}
+
+}  // namespace lcvq
 
 namespace {
 
@@ -171,11 +201,7 @@ lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t*
   cudaError_t e = cudaSuccess;
   char* ws = static_cast<char*>(workspace);
   unsigned int* err = reinterpret_cast<unsigned int*>(ws);
-  if (dtype == LCVQ_BF16 && M <= 32 &&
-      launch_gemv_fused(static_cast<const uint16_t*>(X), M, packed, d_out, d_in, d, A, B,
-                        static_cast<uint16_t*>(Y), s, &launches, &e)) {
-    // decode-GEMV with the X-transform fused: one launch
-  } else if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
+  if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
     uint16_t* Xpp = reinterpret_cast<uint16_t*>(ws + w.xpp_off);
     float* corr = reinterpret_cast<float*>(ws + w.corr_off);
     e = launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr, s, &launches);

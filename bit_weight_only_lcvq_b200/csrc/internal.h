@@ -8,6 +8,10 @@
 
 namespace lcvq {
 
+// cudaFuncAttributeMaxDynamicSharedMemorySize for `func` on the current device,
+// set once per (function, device)
+cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
+
 // ---- elementwise ----
 cudaError_t launch_assign_pack(const float* Wp, int64_t n_elems, uint8_t* packed,
                                uint8_t* mask_bits, cudaStream_t s, int* launches);
@@ -26,12 +30,6 @@ cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, cons
 // ---- decode-GEMV (bf16, M <= 32) ----
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
                         int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s, int* launches);
-
-// single-kernel decode-GEMV with the X-transform fused (bf16, M <= 32).
-// Returns false (launching nothing) when the shape needs the two-kernel path.
-bool launch_gemv_fused(const uint16_t* X, int64_t M, const uint8_t* packed, int64_t d_out,
-                       int64_t d_in, int d, const float* A, const float* B, uint16_t* Y,
-                       cudaStream_t s, int* launches, cudaError_t* err);
 
 // integer-code GEMM on X'' (dispatches on M: decode-GEMV for M <= 32, else
 // the tcgen05 GEMM); err may be null (no device error word)

@@ -668,19 +668,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
         mma_commit_pair(drain);
         if (!mbar_wait(drain, 0, kWaitLimit)) fail(p, abort_flag, 15);
       }
-    } else if (rank == 1 && lane < S && C::kHasCodes) {
-      // odd CTA: forward "B half decoded" to the even CTA.  Lane s owns stage s,
-      // so up to S cross-CTA arrives are in flight at once and the decoder warps
-      // only ever arrive locally.
-      const int s = lane;
+    } else if (rank == 1 && lane == 0 && C::kHasCodes) {
+      // odd CTA: forward "B half decoded" to the even CTA, one cluster-scope
+      // arrive per k block, so the decoder warps only ever arrive locally
+      int s = 0;
       uint32_t ph = 0;
-      int64_t it = 0;
       for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
-        for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
-          if (it % S != s) continue;
+        for (int64_t kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 19); break; }
           mbar_arrive_cluster(mapa_shared(smem_u32(&decd_peer[s]), 0));
-          ph ^= 1;
+          if (++s == S) { s = 0; ph ^= 1; }
         }
       }
     }
@@ -864,13 +861,9 @@ cudaError_t launch_kind(const CUtensorMap& a, const CUtensorMap& b, const Params
                         cudaStream_t s, int* grid_out) {
   using C = Cfg<KIND, DW>;
   auto kern = tc_gemm_kernel<KIND, D, DW>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(kSmemBytes));
-  });
-  if (attr_err != cudaSuccess) return attr_err;
+  if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), kSmemBytes);
+      e != cudaSuccess)
+    return e;
   const int64_t tiles = ceil_div(p.M, BM) * ceil_div(p.N, BN);
   int grid = num_sms();
   if (tiles < grid) grid = static_cast<int>(tiles);
@@ -896,13 +889,9 @@ cudaError_t launch_kind2(const CUtensorMap& a, const CUtensorMap& b, const Param
                          cudaStream_t s, int* grid_out) {
   using C = Cfg2<KIND, DW>;
   auto kern = tc2_gemm_kernel<KIND, D, DW>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(C::kSmem));
-  });
-  if (attr_err != cudaSuccess) return attr_err;
+  if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmem);
+      e != cudaSuccess)
+    return e;
   const int64_t tiles = ceil_div(p.M, 2 * BM) * ceil_div(p.N, BN);
   int pairs = num_sms() / 2;
   if (tiles < pairs) pairs = static_cast<int>(tiles);
@@ -931,15 +920,18 @@ cudaError_t launch_tc_forward(const uint16_t* Xa, bool algebraic, const float* c
                               const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
                               const float* A, const float* B, uint16_t* Y, unsigned int* err,
                               cudaStream_t s, int* launches) {
+  // The algebraic form runs on single CTAs (its B tile is a full 256-row
+  // block of codes); the decode form runs on CTA pairs (each CTA holds and
+  // decodes 128 of those rows), where splitting the decode pays off.
   CUtensorMap ta, tb;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Xa, d_in, M, d_in * 2, BK, BM, true) ||
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d_in / 4, d_out, d_in / 4, BK / 4,
-                BN / 2, false))
+                algebraic ? BN : BN / 2, false))
     return cudaErrorInvalidValue;
   Params p{};
   p.M = M; p.N = d_out; p.K = d_in; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.corr = corr; p.Amat = A; p.Bvec = B; p.out = Y; p.err = err;
-  cudaError_t e = algebraic ? launch_kind2<kFwdAlg, 8, 8>(ta, tb, p, s, nullptr)
+  cudaError_t e = algebraic ? launch_kind<kFwdAlg, 8, 4>(ta, tb, p, s, nullptr)
                             : launch_kind2_d<kFwdDec, 8>(d, ta, tb, p, s, nullptr);
   ++*launches;
   return e;
@@ -951,13 +943,13 @@ cudaError_t launch_tc_backward_dx(const uint16_t* dY, const float* rsum, int64_t
                                   cudaStream_t s, int* launches) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, d_out, M, d_out * 2, BK, BM, true) ||
-      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d_in / 4, d_out, d_in / 4, BN / 8, BK,
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d_in / 4, d_out, d_in / 4, BN / 4, BK,
                 false))
     return cudaErrorInvalidValue;
   Params p{};
   p.M = M; p.N = d_in; p.K = d_out; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.rsum = rsum; p.Amat = A; p.Bvec = B; p.out = dX; p.err = err;
-  cudaError_t e = launch_kind2_d<kDx, 8>(d, ta, tb, p, s, nullptr);
+  cudaError_t e = launch_kind_d<kDx, 4>(d, ta, tb, p, s, nullptr);
   ++*launches;
   return e;
 }

@@ -31,6 +31,63 @@ namespace lcvq {
 
 constexpr int kXfThreads = 256;
 
+// One 16-element block of the transform.
+// x16: the block's 16 bf16 activations as two 16-byte words.  sA: A (D x D,
+// row-major, fp32); sBp: B' = B + 3/2 A 1.  Writes the block's X'' in decoder
+// order (o[c] = bf16x2 of positions c and c + 8, each scaled by 4^-(c mod 3))
+// and the block's parts of the per-row constant:
+//   sb   = sum x^T B'           (s')
+//   sxr  = sum bf16(X')         (X'r)
+//   sxpp = sum X''
+template <int D>
+__device__ __forceinline__ void xform_block(const uint4& u0, const uint4& u1,
+                                            const float* __restrict__ sA,
+                                            const float* __restrict__ sBp, uint32_t (&o)[8],
+                                            float& sb, float& sxr, float& sxpp) {
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  float x[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    x[2 * q] = bf16_lo(w[q]);
+    x[2 * q + 1] = bf16_hi(w[q]);
+  }
+  float xrd[16];  // bf16(X') as fp32
+  sb = 0.f;
+  sxr = 0.f;
+#pragma unroll
+  for (int v = 0; v < 16 / D; ++v) {
+#pragma unroll
+    for (int j = 0; j < D; ++j) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < D; ++i) acc = fmaf(x[v * D + i], sA[i * D + j], acc);
+      xrd[v * D + j] = bf16_to_f32(f32_to_bf16(acc));
+      sxr += xrd[v * D + j];
+    }
+#pragma unroll
+    for (int i = 0; i < D; ++i) sb = fmaf(x[v * D + i], sBp[i], sb);
+  }
+  sxpp = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float scale = (c % 3 == 0) ? 1.0f : ((c % 3 == 1) ? 0.25f : 0.0625f);
+    const float lo = xrd[c] * scale;
+    const float hi = xrd[c + 8] * scale;
+    sxpp += lo + hi;
+    o[c] = pack_bf16x2(lo, hi);  // exact: power-of-two scaling of bf16 values
+  }
+}
+
+// B'[i] = B[i] + 3/2 sum_j A[i][j], summed in j order (thread i < D)
+template <int D>
+__device__ __forceinline__ float shifted_offset(const float* __restrict__ A_row, float b) {
+  float rs = 0.f;
+#pragma unroll
+  for (int j = 0; j < D; ++j) rs += A_row[j];
+  return b + 1.5f * rs;
+}
+
+
 template <int D>
 __global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __restrict__ X,
                                                            int64_t d_in,
@@ -51,12 +108,8 @@ __global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __res
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   if (threadIdx.x < D * D) sA[threadIdx.x] = A[threadIdx.x];
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float rs = 0.f;
-    for (int j = 0; j < D; ++j) rs += sA[threadIdx.x * D + j];
-    sBp[threadIdx.x] = B[threadIdx.x] + 1.5f * rs;
-  }
+  if (threadIdx.x < D)
+    sBp[threadIdx.x] = shifted_offset<D>(A + threadIdx.x * D, B[threadIdx.x]);
   __syncthreads();
 
   const int64_t m = blockIdx.x;
@@ -67,38 +120,9 @@ __global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __res
   for (int64_t b = threadIdx.x; b < nblk; b += kXfThreads) {
     const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
     const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    float x[16];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      x[2 * q] = bf16_lo(w[q]);
-      x[2 * q + 1] = bf16_hi(w[q]);
-    }
-    float xrd[16];  // bf16(X') as fp32
-    float sb = 0.f, sxr = 0.f;
-#pragma unroll
-    for (int v = 0; v < 16 / D; ++v) {
-#pragma unroll
-      for (int j = 0; j < D; ++j) {
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < D; ++i) acc = fmaf(x[v * D + i], sA[i * D + j], acc);
-        xrd[v * D + j] = bf16_to_f32(f32_to_bf16(acc));
-        sxr += xrd[v * D + j];
-      }
-#pragma unroll
-      for (int i = 0; i < D; ++i) sb = fmaf(x[v * D + i], sBp[i], sb);
-    }
     uint32_t o[8];
-    float sxpp = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float scale = (c % 3 == 0) ? 1.0f : ((c % 3 == 1) ? 0.25f : 0.0625f);
-      const float lo = xrd[c] * scale;
-      const float hi = xrd[c + 8] * scale;
-      sxpp += lo + hi;
-      o[c] = pack_bf16x2(lo, hi);  // exact: power-of-two scaling of bf16 values
-    }
+    float sb, sxr, sxpp;
+    xform_block<D>(u0, u1, sA, sBp, o, sb, sxr, sxpp);
     uint4* dst = reinterpret_cast<uint4*>(orow + 16 * b);
     dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
     dst[1] = make_uint4(o[4], o[5], o[6], o[7]);

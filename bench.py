@@ -60,6 +60,9 @@ def parse():
 # source that was captured: keyed by the SHA-1 of the source file.
 NCU_TRAFFIC = {
     # source file -> (sha1 of the file when captured, {token count: bytes per launch})
+    # profiles/launches_decode_gemv_bench.md: M = 1 and 4 share gemv_kernel<1, ...>
+    "bit_weight_only_lcvq_b200/csrc/gemv.cu": (
+        "80b75d0752c56f28a2d89ae289e8922b78f5e402", {1: 4226188, 4: 4226188, 16: 4350809}),
 }
 
 

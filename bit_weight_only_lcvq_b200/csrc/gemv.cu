@@ -94,14 +94,15 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
 
-template <int NT, int R, int kWarps>
-__global__ void __launch_bounds__(kWarps * 32, (kWarps == 16 ? 1 : (NT <= 2 ? 2 : 1)))
+// kPrefX: keep the next unit's X'' fragments in flight (costs registers);
+// kMinBlocks: CTAs per SM the register budget must allow.
+template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks>
+__global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
     gemv_kernel(const uint16_t* __restrict__ Xpp, const float* __restrict__ corr, int M,
                 const uint8_t* __restrict__ packed, int64_t N, int64_t K,
                 uint16_t* __restrict__ Y) {
   constexpr int MP = NT * 8;
   constexpr int ROWS = 16 * R;
-  constexpr bool kPrefX = NT == 1;  // keep the next unit's X'' fragments in flight
   __shared__ float part[kWarps][ROWS][MP + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -252,7 +253,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 16 ? 1 : (NT <= 2 ? 2 
   }
 }
 
-template <int NT, int R, int kWarps>
+template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks>
 cudaError_t launch_gemv_t(const uint16_t* Xpp, const float* corr, int M, const uint8_t* packed,
                           int64_t N, int64_t K, uint16_t* Y, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
@@ -265,7 +266,8 @@ cudaError_t launch_gemv_t(const uint16_t* Xpp, const float* corr, int M, const u
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, R, kWarps>, Xpp, corr, M, packed, N, K, Y);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, R, kWarps, kPrefX, kMinBlocks>, Xpp, corr, M,
+                            packed, N, K, Y);
 }
 
 }  // namespace
@@ -275,12 +277,15 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
                         int* launches) {
   cudaError_t e;
   const int m = static_cast<int>(M);
+  // CTA shapes measured best on the 4096 x 4096 workload (graph replays over
+  // rotated weights): M <= 8: 16 rows, 2 CTAs per SM; M <= 16: 32 rows, one CTA
+  // per SM with room for the X'' prefetch; M <= 32: 32 rows, no prefetch.
   if (M <= 8)
-    e = launch_gemv_t<1, 1, 8>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<1, 1, 8, true, 2>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else if (M <= 16)
-    e = launch_gemv_t<2, 2, 8>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<2, 2, 8, true, 1>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   else
-    e = launch_gemv_t<4, 2, 8>(Xpp, corr, m, packed, d_out, d_in, Y, s);
+    e = launch_gemv_t<4, 2, 8, false, 1>(Xpp, corr, m, packed, d_out, d_in, Y, s);
   ++*launches;
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -494,29 +494,80 @@ def row_stack(D, pk):
         dmats.append(dict(packed=torch.from_numpy(m["packed"]).to(dev), A=torch.from_numpy(m["A"]).to(dev),
                           B=torch.from_numpy(m["B"]).to(dev), proj=m["proj"], d_in=m["d_in"],
                           d_out=m["d_out"]))
+    # decoder-layer phases: matrices of one phase read the same input and are
+    # independent (q, k, v | o | gate, up | down)
+    phases = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
     out = {}
     for M in (1, 8, 32):
         ys = {p: torch.empty((M, do), dtype=torch.bfloat16, device=dev) for p, _, do in synth.STACK_PROJS}
         wss = {p: lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, do, di, 8), dev)
                for p, di, do in synth.STACK_PROJS}
 
-        def run(M=M, ys=ys, wss=wss):
+        def run_seq(M=M, ys=ys, wss=wss):
             n = 0
             for m in dmats:
                 lcvq.gemm(xs[m["proj"]][:M], m["packed"], m["d_in"], m["A"], m["B"], 8,
                           out=ys[m["proj"]], workspace=wss[m["proj"]])
                 n += lcvq.last_launch_count()
             return n
-        sg = StepGraphs(run, 1, 5)
-        sg.replay()
-        t, _, _ = timed_graphs(D, sg)
-        ms = t / 5
-        gbs = total_bytes / (ms * 1e-3) / 1e9
-        out[str(M)] = dict(value=gbs, unit="GB/s", us=ms * 1e3,
-                           roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
-                                         frac=gbs / pk["hbm_gbs"]))
-    return dict(metric="stack packed-weight GB/s (224 matrices, 1.62 GB of codes)", per_m=out,
-                packed_bytes=total_bytes)
+
+        # one grouped call per phase (4 per layer)
+        by_layer = [dmats[i:i + len(synth.STACK_PROJS)] for i in range(0, len(dmats), len(synth.STACK_PROJS))]
+        phase_jobs = []
+        for layer in by_layer:
+            named = {m["proj"]: m for m in layer}
+            for ph in phases:
+                phase_jobs.append([(xs[p][:M], named[p]["packed"], named[p]["A"], named[p]["B"],
+                                    named[p]["d_in"]) for p in ph])
+        ph_outs = [[ys[p] for p in ph] for ph in phases] * len(by_layer)
+        ph_ws = lcvq.new_workspace(max(lcvq.workspace_size_grouped(j, M, 8) for j in phase_jobs), dev)
+
+        def run_phase(phase_jobs=phase_jobs, ph_outs=ph_outs, ph_ws=ph_ws):
+            n = 0
+            for jobs, outs in zip(phase_jobs, ph_outs):
+                lcvq.gemm_grouped(jobs, 8, workspace=ph_ws, outs=outs)
+                n += lcvq.last_launch_count()
+            return n
+
+        # the whole stack as one grouped call (independent inputs per matrix)
+        all_jobs = [(xs[m["proj"]][:M], m["packed"], m["A"], m["B"], m["d_in"]) for m in dmats]
+        all_outs = [torch.empty((M, m["d_out"]), dtype=torch.bfloat16, device=dev) for m in dmats]
+        all_ws = lcvq.new_workspace(lcvq.workspace_size_grouped(all_jobs, M, 8), dev)
+
+        def run_all(all_jobs=all_jobs, all_outs=all_outs, all_ws=all_ws):
+            lcvq.gemm_grouped(all_jobs, 8, workspace=all_ws, outs=all_outs)
+            return lcvq.last_launch_count()
+
+        res_m = {}
+        for name, fn in (("sequential", run_seq), ("grouped_by_phase", run_phase),
+                         ("grouped_all", run_all)):
+            sg = StepGraphs(fn, 1, 5)
+            sg.replay()
+            t, launches, _ = timed_graphs(D, sg)
+            ms = t / 5
+            gbs = total_bytes / (ms * 1e-3) / 1e9
+            res_m[name] = dict(value=gbs, unit="GB/s", us=ms * 1e3, launches_per_pass=launches // 5,
+                               roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
+                                             frac=gbs / pk["hbm_gbs"]))
+            del sg
+        # parity of the grouped paths against the sequential one, bitwise, on the last layer
+        torch.cuda.synchronize()
+        run_seq()
+        torch.cuda.synchronize()
+        seq_last = {p: ys[p].clone() for p, _, _ in synth.STACK_PROJS}
+        run_all()
+        torch.cuda.synchronize()
+        res_m["grouped_equals_sequential"] = all(
+            torch.equal(all_outs[len(dmats) - len(synth.STACK_PROJS) + i], seq_last[p])
+            for i, (p, _, _) in enumerate(synth.STACK_PROJS))
+        out[str(M)] = res_m
+        del all_ws, all_outs, ph_ws
+        torch.cuda.empty_cache()
+    return dict(metric="stack packed-weight GB/s (224 matrices, 1.62 GB of codes)",
+                note="sequential: 224 lcvq_gemm calls; grouped_by_phase: one lcvq_gemm_grouped per "
+                     "decoder-layer phase (q,k,v | o | gate,up | down), 128 calls; grouped_all: the "
+                     "224 independent matrices in one lcvq_gemm_grouped call",
+                per_m=out, packed_bytes=total_bytes)
 
 
 ROWS = {"assign_pack": row_assign_pack, "decode": row_decode, "prefill": row_prefill,

@@ -2,6 +2,7 @@
 // Every entry point validates all of its arguments before it launches
 // anything, so a failing call has no side effect.
 #include <atomic>
+#include <vector>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -214,6 +215,78 @@ lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t*
   } else {
     e = launch_simt_forward(X, dtype == LCVQ_BF16, M, packed, d_out, d_in, d, A, B, Y, s,
                             &launches);
+  }
+  return finish(e, launches);
+}
+
+}  // extern "C"
+
+namespace {
+
+constexpr int64_t kGroupMaxDim = int64_t(1) << 28;
+
+// byte offsets of item i's X'' and corr in a grouped workspace; total bytes
+// (0 if any item is invalid)
+size_t grouped_ws(const lcvq_gemm_item* items, int count, int64_t M, int d,
+                  std::vector<size_t>* xpp_off, std::vector<size_t>* corr_off) {
+  if (items == nullptr || count < 1 || M < 1 || M > 32 || !valid_d(d)) return 0;
+  size_t off = kWsHeaderBytes;
+  for (int i = 0; i < count; ++i) {
+    const lcvq_gemm_item& it = items[i];
+    if (it.d_out < 1 || it.d_in < 1 || it.d_out >= kGroupMaxDim || it.d_in >= kGroupMaxDim ||
+        it.d_in % 64 != 0 || it.d_out % 8 != 0)
+      return 0;
+    if (xpp_off) xpp_off->push_back(off);
+    off = round_up(off + size_t(M) * size_t(it.d_in) * 2, 256);
+    if (corr_off) corr_off->push_back(off);
+    off = round_up(off + size_t(M) * 4, 256);
+  }
+  return off;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lcvq_workspace_size_grouped(const lcvq_gemm_item* items, int count, int64_t M, int d) {
+  return grouped_ws(items, count, M, d, nullptr, nullptr);
+}
+
+lcvq_status lcvq_gemm_grouped(const lcvq_gemm_item* items, int count, int64_t M, int d,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  g_last_launches = 0;
+  std::vector<size_t> xoff, coff;
+  const size_t need = grouped_ws(items, count, M, d, &xoff, &coff);
+  if (need == 0) return LCVQ_ERR_INVALID_ARG;
+  if (!workspace) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return LCVQ_ERR_ALIGNMENT;
+  if (ws_bytes < need) return LCVQ_ERR_WORKSPACE;
+  for (int i = 0; i < count; ++i) {
+    const lcvq_gemm_item& it = items[i];
+    if (!it.X || !it.packed || !it.A || !it.B || !it.Y) return LCVQ_ERR_INVALID_ARG;
+    if (!aligned16(it.X) || !aligned16(it.packed) || !aligned16(it.A) || !aligned16(it.B) ||
+        !aligned16(it.Y))
+      return LCVQ_ERR_ALIGNMENT;
+  }
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  std::vector<XformJob> xj(count);
+  std::vector<GemvJob> gj(count);
+  for (int i = 0; i < count; ++i) {
+    const lcvq_gemm_item& it = items[i];
+    uint16_t* Xpp = reinterpret_cast<uint16_t*>(ws + xoff[i]);
+    float* corr = reinterpret_cast<float*>(ws + coff[i]);
+    xj[i] = XformJob{static_cast<const uint16_t*>(it.X), it.A, it.B, Xpp, corr, it.d_in};
+    gj[i] = GemvJob{it.packed, Xpp, corr, static_cast<uint16_t*>(it.Y), it.d_out, it.d_in};
+  }
+  int launches = 0;
+  // per chunk of matrices: their X-transforms, then their decode-GEMV
+  cudaError_t e = cudaSuccess;
+  for (int first = 0; first < count && e == cudaSuccess; first += kMaxGroupItems) {
+    const int n = count - first < kMaxGroupItems ? count - first : kMaxGroupItems;
+    e = launch_xform_grouped(xj.data() + first, n, M, d, s, &launches);
+    if (e == cudaSuccess) e = launch_gemv_grouped(gj.data() + first, n, M, s, &launches);
   }
   return finish(e, launches);
 }

@@ -31,6 +31,36 @@ cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, cons
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
                         int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s, int* launches);
 
+constexpr int kMaxGroupItems = 128;
+
+// the X-transform of several matrices' activations (common M and d) in
+// launches of up to kMaxGroupItems matrices; per matrix, the same bits as
+// launch_xform.
+struct XformJob {
+  const uint16_t* X;
+  const float* A;
+  const float* B;
+  uint16_t* Xpp;
+  float* corr;
+  int64_t d_in;
+};
+
+// decode-GEMV over a group of matrices with a common token count M <= 32, in
+// persistent launches of up to kMaxGroupItems matrices each (X'' and corr of
+// every matrix already formed by launch_xform or launch_xform_grouped).  Each
+// matrix's Y is bit-identical to launch_gemv on that matrix alone.
+struct GemvJob {
+  const uint8_t* packed;
+  const uint16_t* Xpp;
+  const float* corr;
+  uint16_t* Y;
+  int64_t d_out, d_in;
+};
+cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaStream_t s,
+                                int* launches);
+cudaError_t launch_xform_grouped(const XformJob* jobs, int count, int64_t M, int d,
+                                 cudaStream_t s, int* launches);
+
 // integer-code GEMM on X'' (dispatches on M: decode-GEMV for M <= 32, else
 // the tcgen05 GEMM); err may be null (no device error word)
 cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,

@@ -88,13 +88,31 @@ __device__ __forceinline__ float shifted_offset(const float* __restrict__ A_row,
 }
 
 
-template <int D>
-__global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __restrict__ X,
-                                                           int64_t d_in,
-                                                           const float* __restrict__ A,
-                                                           const float* __restrict__ B,
-                                                           uint16_t* __restrict__ Xpp,
-                                                           float* __restrict__ corr) {
+// One launch transforms the rows of up to kItems matrices' activations: CTA
+// (m, i) does row m of item i (a single call is a group of one).
+struct XformItem {
+  const uint16_t* X;  // [M][d_in] bf16
+  const float* A;     // [D*D]
+  const float* B;     // [D]
+  uint16_t* Xpp;      // [M][d_in] out
+  float* corr;        // [M] out
+  int64_t d_in;
+};
+template <int kItems>
+struct XformGroup {
+  XformItem item[kItems];
+};
+
+template <int D, int kItems>
+__global__ void __launch_bounds__(kXfThreads)
+    xform_kernel(const __grid_constant__ XformGroup<kItems> grp) {
+  const XformItem& it = grp.item[blockIdx.y];
+  const uint16_t* __restrict__ X = it.X;
+  const float* __restrict__ A = it.A;
+  const float* __restrict__ B = it.B;
+  uint16_t* __restrict__ Xpp = it.Xpp;
+  float* __restrict__ corr = it.corr;
+  const int64_t d_in = it.d_in;
   __shared__ float sA[D * D];
   __shared__ float sBp[D];
   __shared__ double red[3][kXfThreads / 32];
@@ -155,11 +173,12 @@ __global__ void __launch_bounds__(kXfThreads) xform_kernel(const uint16_t* __res
   }
 }
 
-cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
-                         const float* B, uint16_t* Xpp, float* corr, cudaStream_t s,
-                         int* launches) {
+namespace {
+template <int kItems>
+cudaError_t launch_xform_group(const XformGroup<kItems>& grp, int count, int64_t M, int d,
+                               cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(M), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(M), static_cast<unsigned>(count), 1);
   cfg.blockDim = dim3(kXfThreads, 1, 1);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -167,16 +186,41 @@ cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e;
   switch (d) {
-    case 1: e = cudaLaunchKernelEx(&cfg, xform_kernel<1>, X, d_in, A, B, Xpp, corr); break;
-    case 2: e = cudaLaunchKernelEx(&cfg, xform_kernel<2>, X, d_in, A, B, Xpp, corr); break;
-    case 4: e = cudaLaunchKernelEx(&cfg, xform_kernel<4>, X, d_in, A, B, Xpp, corr); break;
-    default: e = cudaLaunchKernelEx(&cfg, xform_kernel<8>, X, d_in, A, B, Xpp, corr); break;
+    case 1: return cudaLaunchKernelEx(&cfg, xform_kernel<1, kItems>, grp);
+    case 2: return cudaLaunchKernelEx(&cfg, xform_kernel<2, kItems>, grp);
+    case 4: return cudaLaunchKernelEx(&cfg, xform_kernel<4, kItems>, grp);
+    default: return cudaLaunchKernelEx(&cfg, xform_kernel<8, kItems>, grp);
   }
+}
+}  // namespace
+
+cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
+                         const float* B, uint16_t* Xpp, float* corr, cudaStream_t s,
+                         int* launches) {
+  XformGroup<1> grp{};
+  grp.item[0] = XformItem{X, A, B, Xpp, corr, d_in};
+  cudaError_t e = launch_xform_group(grp, 1, M, d, s);
   ++*launches;
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_xform_grouped(const XformJob* jobs, int count, int64_t M, int d,
+                                 cudaStream_t s, int* launches) {
+  for (int first = 0; first < count; first += kMaxGroupItems) {
+    const int n = count - first < kMaxGroupItems ? count - first : kMaxGroupItems;
+    XformGroup<kMaxGroupItems> grp{};
+    for (int i = 0; i < n; ++i) {
+      const XformJob& j = jobs[first + i];
+      grp.item[i] = XformItem{j.X, j.A, j.B, j.Xpp, j.corr, j.d_in};
+    }
+    cudaError_t e = launch_xform_group(grp, n, M, d, s);
+    ++*launches;
+    if (e != cudaSuccess) return e;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // r[m] = sum_n dY[m][n]: the rank-1 term of the dX epilogue (the B part of

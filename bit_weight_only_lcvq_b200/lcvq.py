@@ -38,7 +38,9 @@ EXPORTS = (
     "lcvq_xform",
     "lcvq_gemm_xformed",
     "lcvq_gemv_static",
+    "lcvq_gemm_grouped",
     "lcvq_workspace_size",
+    "lcvq_workspace_size_grouped",
     "lcvq_check_device_error",
     "lcvq_status_string",
     "lcvq_last_launch_count",
@@ -54,6 +56,12 @@ class LcvqError(RuntimeError):
 _lib = None
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+
+
+class GemmItem(ctypes.Structure):
+    """lcvq_gemm_item: one matrix of a grouped decode-GEMV."""
+    _fields_ = [("X", _vp), ("packed", _vp), ("A", _vp), ("B", _vp), ("Y", _vp),
+                ("d_out", _i64), ("d_in", _i64)]
 
 
 def lib() -> ctypes.CDLL:
@@ -73,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.lcvq_xform.argtypes = [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp]
         L.lcvq_gemm_xformed.argtypes = [_vp, _vp, _i64, _vp, _i64, _i64, _vp, _vp]
         L.lcvq_gemv_static.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp]
+        L.lcvq_gemm_grouped.argtypes = [ctypes.POINTER(GemmItem), _i32, _i64, _i32, _vp, _sz, _vp]
+        L.lcvq_workspace_size_grouped.argtypes = [ctypes.POINTER(GemmItem), _i32, _i64, _i32]
+        L.lcvq_workspace_size_grouped.restype = _sz
         L.lcvq_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i64, _i32]
         L.lcvq_workspace_size.restype = _sz
         L.lcvq_check_device_error.argtypes = [_vp, _vp]
@@ -80,7 +91,8 @@ def lib() -> ctypes.CDLL:
         L.lcvq_status_string.restype = ctypes.c_char_p
         L.lcvq_last_launch_count.argtypes = []
         for fn in ("lcvq_assign_pack", "lcvq_decode", "lcvq_gemm", "lcvq_gemm_backward",
-                   "lcvq_xform", "lcvq_gemm_xformed", "lcvq_gemv_static", "lcvq_check_device_error",
+                   "lcvq_xform", "lcvq_gemm_xformed", "lcvq_gemv_static", "lcvq_gemm_grouped",
+                   "lcvq_check_device_error",
                    "lcvq_last_launch_count"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -234,3 +246,34 @@ def gemv_static(X: torch.Tensor, packed: torch.Tensor, d_in: int, A: torch.Tenso
 def check_device_error(workspace: torch.Tensor, stream=None) -> int:
     """Synchronizes the stream and returns the workspace's device error status."""
     return int(lib().lcvq_check_device_error(_ptr(workspace), _stream(stream)))
+
+
+def _group_items(jobs, outs):
+    arr = (GemmItem * len(jobs))()
+    for i, (X, packed, A, B, d_in) in enumerate(jobs):
+        arr[i] = GemmItem(_ptr(X), _ptr(packed), _ptr(A), _ptr(B), _ptr(outs[i]),
+                          packed.shape[0], d_in)
+    return arr
+
+
+def workspace_size_grouped(jobs, M: int, d: int) -> int:
+    """Workspace bytes for gemm_grouped over jobs = [(X, packed, A, B, d_in), ...]."""
+    arr = (GemmItem * len(jobs))()
+    for i, (X, packed, A, B, d_in) in enumerate(jobs):
+        arr[i] = GemmItem(None, None, None, None, None, packed.shape[0], d_in)
+    return int(lib().lcvq_workspace_size_grouped(arr, len(jobs), M, d))
+
+
+def gemm_grouped(jobs, d: int, *, workspace=None, outs=None, stream=None):
+    """Grouped decode-GEMV: Y_i = X_i W~_i for jobs = [(X, packed, A, B, d_in), ...]
+    sharing the token count M <= 32 and d.  Returns the list of Y_i."""
+    M = jobs[0][0].shape[0]
+    if outs is None:
+        outs = [torch.empty((M, packed.shape[0]), dtype=torch.bfloat16, device=X.device)
+                for X, packed, _, _, _ in jobs]
+    arr = _group_items(jobs, outs)
+    if workspace is None:
+        workspace = new_workspace(workspace_size_grouped(jobs, M, d), jobs[0][0].device)
+    _check("lcvq_gemm_grouped", lib().lcvq_gemm_grouped(
+        arr, len(jobs), M, d, _ptr(workspace), workspace.numel(), _stream(stream)))
+    return outs

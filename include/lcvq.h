@@ -153,6 +153,39 @@ LCVQ_API lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64
                                        const uint8_t* packed, int64_t d_out, int64_t d_in,
                                        void* Y, void* stream);
 
+/* Grouped decode-GEMV: Y_i = X_i W~_i for `count` independent matrices.  The
+ * pages define the operation per matrix (Methodology 3; decoupleQ eq. (1) for
+ * the layer convention); grouping is this library's launch arrangement for
+ * many matrices at once (the projections of a layer that read one input, the
+ * experts of a layer, or any set of independent decode-time matmuls).  Each
+ * Y_i is bit-identical to lcvq_gemm on item i alone.
+ *   items  host array of `count` descriptors (read during the call only):
+ *          X [M][d_in] bf16, packed [d_out][d_in/4] codes, A [d*d] and B [d]
+ *          fp32, Y [M][d_out] bf16 out; every pointer 16-byte aligned.
+ *   M      common token count, 1 <= M <= 32 (the decode-GEMV regime).
+ *   d      common vector length.
+ *   workspace: >= lcvq_workspace_size_grouped(items, count, M, d) bytes,
+ *          256-byte aligned, first 256 bytes zeroed once (as lcvq_gemm).
+ * Shapes per item: d_in % 64 == 0, d_out % 8 == 0, 1 <= d_in, d_out < 2^28.
+ * count >= 1.  The call launches 2 * ceil(count / 128) kernels: the
+ * X-transforms of up to 128 matrices, then one persistent decode-GEMV over
+ * their tiles.  Any invalid item fails the whole call before anything is
+ * launched.  The Y_i must not overlap one another or any input. */
+typedef struct {
+  const void* X;
+  const uint8_t* packed;
+  const float* A;
+  const float* B;
+  void* Y;
+  int64_t d_out;
+  int64_t d_in;
+} lcvq_gemm_item;
+
+LCVQ_API lcvq_status lcvq_gemm_grouped(const lcvq_gemm_item* items, int count, int64_t M, int d,
+                                       void* workspace, size_t ws_bytes, void* stream);
+LCVQ_API size_t lcvq_workspace_size_grouped(const lcvq_gemm_item* items, int count, int64_t M,
+                                            int d);
+
 /* Decode-GEMV without a workspace.  The pages have no counterpart: this is a
  * convenience of this library.  It computes exactly what lcvq_gemm computes for
  * bf16 activations and M <= 32 (same kernels, same results), but takes no

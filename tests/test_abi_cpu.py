@@ -55,3 +55,36 @@ def test_invalid_arguments_rejected_without_device():
     assert L.lcvq_gemm(None, 1, 4, None, 8, 64, 8, None, None, 8, 0, None, 0, None) == 3
     assert L.lcvq_gemm_backward(None, None, 1, 4, None, None, 8, 64, 8, None, None, None,
                                 None, None, None, None, 0, None) == 1      # dA/dB required
+
+
+def test_grouped_gemm_rejects_bad_groups_without_device():
+    L = lcvq.lib()
+    Item = lcvq.GemmItem
+
+    def items(*shapes):
+        arr = (Item * len(shapes))()
+        for i, (d_out, d_in) in enumerate(shapes):
+            arr[i] = Item(16, 16, 16, 16, 16, d_out, d_in)  # aligned dummy pointers
+        return arr
+
+    good = items((4096, 4096), (11008, 4096), (4096, 11008))
+    need = L.lcvq_workspace_size_grouped(good, 3, 8, 8)
+    per = [256 * -(-(8 * k * 2) // 256) + 256 for _, k in ((0, 4096), (0, 4096), (0, 11008))]
+    assert need == 256 + sum(per)
+    assert L.lcvq_workspace_size_grouped(good, 3, 33, 8) == 0                 # M > 32
+    assert L.lcvq_workspace_size_grouped(good, 3, 0, 8) == 0                  # M < 1
+    assert L.lcvq_workspace_size_grouped(good, 0, 8, 8) == 0                  # empty group
+    assert L.lcvq_workspace_size_grouped(good, 3, 8, 3) == 0                  # d
+    assert L.lcvq_workspace_size_grouped(items((4096, 4000)), 1, 8, 8) == 0   # d_in % 64
+    assert L.lcvq_workspace_size_grouped(items((4100, 4096)), 1, 8, 8) == 0   # d_out % 8
+    assert L.lcvq_workspace_size_grouped(items((0, 4096)), 1, 8, 8) == 0      # empty matrix
+    # every failure is reported before any device call
+    assert L.lcvq_gemm_grouped(good, 3, 33, 8, 256, need, None) == 1
+    assert L.lcvq_gemm_grouped(good, 3, 8, 8, None, need, None) == 1          # no workspace
+    assert L.lcvq_gemm_grouped(good, 3, 8, 8, 8, need, None) == 3             # misaligned
+    assert L.lcvq_gemm_grouped(good, 3, 8, 8, 256, need - 1, None) == 4       # too small
+    bad = items((4096, 4096), (4096, 4096))
+    bad[1].Y = 8                                                              # one bad item
+    assert L.lcvq_gemm_grouped(bad, 2, 8, 8, 256, 1 << 30, None) == 3
+    bad[1].Y = None
+    assert L.lcvq_gemm_grouped(bad, 2, 8, 8, 256, 1 << 30, None) == 1

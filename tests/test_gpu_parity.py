@@ -262,3 +262,68 @@ def test_launch_count_and_error_word():
               torch.from_numpy(w["B"]).to(dev()), 8, workspace=ws)
     assert lcvq.last_launch_count() >= 1
     assert lcvq.check_device_error(ws) == 0
+
+
+# ------------------------------------------------ grouped decode-GEMV (M <= 32)
+def _group_case(shapes, M, seed):
+    jobs, zs, ws = [], [], []
+    for i, (d_in, d_out) in enumerate(shapes):
+        w, z = _fwd_case(2, M, d_in=d_in, d_out=d_out)
+        g = np.random.Generator(np.random.PCG64(seed + i))
+        z = g.integers(0, 4, size=z.shape, dtype=np.uint8)   # a different code matrix per item
+        jobs.append((to_dev(w["X"], torch.bfloat16), torch.from_numpy(O.pack_codes(z)).to(dev()),
+                     torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev()), d_in))
+        zs.append(z)
+        ws.append(w)
+    return jobs, zs, ws
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 32])
+def test_gemm_grouped_bitwise_equals_separate_calls(M):
+    """Each Y_i of lcvq_gemm_grouped equals lcvq_gemm on item i alone, bit for
+    bit, for mixed shapes (square, up-, down-projection, ragged)."""
+    shapes = [(4096, 4096), (4096, 11008), (11008, 4096), (1088, 520), (512, 8)]
+    jobs, zs, ws = _group_case(shapes, M, 300 + M)
+    Ys = lcvq.gemm_grouped(jobs, 8)
+    assert lcvq.last_launch_count() == 2
+    for (X, packed, A, B, d_in), Y in zip(jobs, Ys):
+        Y1 = lcvq.gemm(X, packed, d_in, A, B, 8)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, Y1)
+    # and the small items against the oracle
+    for i in (3, 4):
+        ref, D = O.forward(ws[i]["X"], zs[i], ws[i]["A"], ws[i]["B"])
+        assert_close(f"grouped item {i} M={M}", to_np(Ys[i]), ref, D, TOL_BF16)
+
+
+def test_gemm_grouped_many_items_and_graph_replay():
+    """More items than one launch takes (two chunks), one workspace, eager and
+    as CUDA-graph replays."""
+    shapes = [(64 * (1 + i % 5), 8 * (1 + i % 7)) for i in range(150)]
+    jobs, zs, ws = _group_case(shapes, 3, 900)
+    wsb = lcvq.new_workspace(lcvq.workspace_size_grouped(jobs, 3, 8))
+    outs = [torch.empty((3, p.shape[0]), dtype=torch.bfloat16, device=dev()) for _, p, _, _, _ in jobs]
+    lcvq.gemm_grouped(jobs, 8, workspace=wsb, outs=outs)
+    assert lcvq.last_launch_count() == 4
+    torch.cuda.synchronize()
+    refs = [o.clone() for o in outs]
+    for i in (0, 77, 149):
+        ref, D = O.forward(ws[i]["X"], zs[i], ws[i]["A"], ws[i]["B"])
+        assert_close(f"grouped many item {i}", to_np(outs[i]), ref, D, TOL_BF16)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        lcvq.gemm_grouped(jobs, 8, workspace=wsb, outs=outs)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lcvq.gemm_grouped(jobs, 8, workspace=wsb, outs=outs)
+    for _ in range(3):
+        for o in outs:
+            o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert all(torch.equal(o, r) for o, r in zip(outs, refs))
+    del g
+    assert lcvq.check_device_error(wsb) == 0

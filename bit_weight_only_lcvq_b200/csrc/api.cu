@@ -286,7 +286,9 @@ lcvq_status lcvq_gemm_grouped(const lcvq_gemm_item* items, int count, int64_t M,
   for (int first = 0; first < count && e == cudaSuccess; first += kMaxGroupItems) {
     const int n = count - first < kMaxGroupItems ? count - first : kMaxGroupItems;
     e = launch_xform_grouped(xj.data() + first, n, M, d, s, &launches);
-    if (e == cudaSuccess) e = launch_gemv_grouped(gj.data() + first, n, M, s, &launches);
+    if (e == cudaSuccess)
+      e = launch_gemv_grouped(gj.data() + first, n, M, s, &launches,
+                              reinterpret_cast<unsigned int*>(ws));
   }
   return finish(e, launches);
 }

@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace lcvq {
 
@@ -302,26 +303,70 @@ struct GemvGroup {
   GemvItem item[kItems];
 };
 
-template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kItems>
+// Code ring in shared memory, per warp: kStages chunks, each ROWS rows x 128 B
+// (kAhead units of 32 B per row).  A chunk's 16-byte pieces are copied with
+// cp.async by the warp's lanes (8 lanes per row, coalesced), XOR-swizzled by
+// (row & 7) so that the lanes' 8-byte reads of one unit spread over the banks.
+// Copies in flight hold no registers, so every SM keeps kStages - 1 chunks per
+// warp on the way from HBM.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+template <int R, int kStages, int kWarps>
+__host__ __device__ constexpr size_t group_smem_ring() {
+  return size_t(kWarps) * kStages * (16 * R) * 128;
+}
+template <int NT, int R, int kWarps>
+__host__ __device__ constexpr size_t group_smem_part() {
+  return size_t(2) * kWarps * (16 * R) * (NT * 8 + 1) * sizeof(float);
+}
+
+template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kStages, int kItems>
 __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
     gemv_group_kernel(const __grid_constant__ GemvGroup<kItems> grp) {
   constexpr int MP = NT * 8;
   constexpr int ROWS = 16 * R;
-  // [2][kWarps][ROWS][MP + 1] partial tiles (dynamic: above the static limit for NT = 4)
-  extern __shared__ float part_smem[];
-  auto part = reinterpret_cast<float(*)[kWarps][ROWS][MP + 1]>(part_smem);
+  constexpr uint32_t kStageBytes = ROWS * 128;
+  static_assert(kStages >= 2, "ring of at least two chunks");
+  // dynamic shared memory: [kWarps][kStages][ROWS][128 B] code ring, then
+  // [2][kWarps][ROWS][MP + 1] fp32 partial tiles
+  extern __shared__ __align__(128) unsigned char gsm[];
+  auto part = reinterpret_cast<float(*)[kWarps][ROWS][MP + 1]>(
+      gsm + group_smem_ring<R, kStages, kWarps>());
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int M = grp.M;
   const int T = grp.item[grp.count - 1].tile_end;
   const int G = static_cast<int>(gridDim.x);
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(gsm)) +
+                        static_cast<uint32_t>(warp) * kStages * kStageBytes;
 
-  // a chunk of this warp: tile, its item, chunk index inside the tile
   struct Cur {
     int tile, item, chunk;
   };
-  // first chunk of this warp at or after c (c.chunk is a candidate index)
   auto seek = [&](Cur c) {
     while (c.tile < T) {
       while (c.tile >= grp.item[c.item].tile_end) ++c.item;
@@ -338,21 +383,26 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
   };
   auto tile_begin = [&](int item) { return item == 0 ? 0 : grp.item[item - 1].tile_end; };
 
-  auto load_unit = [&](const Cur& c, int j, uint2 (&cw)[R][2]) {
-    bool any = c.tile < T;
-    const GemvItem& it = grp.item[any ? c.item : 0];
-    const int64_t u = int64_t(c.chunk) * kAhead + j;
-    const bool kok = any && u * kUnit + 32 * t < it.K;
-    const int64_t row0 = int64_t(c.tile - tile_begin(c.item)) * ROWS;
-    const int64_t Kb = it.K / 4;
+  // copy chunk c into stage s (zero-filled outside the matrix; no copy at all
+  // past the last tile); always one commit group
+  auto issue = [&](const Cur& c, int s) {
+    if (c.tile < T) {
+      const GemvItem& it = grp.item[c.item];
+      const int64_t row0 = int64_t(c.tile - tile_begin(c.item)) * ROWS;
+      const int64_t Kb = it.K / 4;
+      const int64_t cb = int64_t(c.chunk) * (kAhead * 32);  // chunk's first byte in a row
 #pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t row = row0 + r * 16 + g + 8 * h;
-        cw[r][h] = (kok && row < it.N) ? ld_stream_v2(it.packed + row * Kb + 8 * t + u * 32)
-                                       : make_uint2(0, 0);
+      for (int i = 0; i < ROWS / 4; ++i) {
+        const int p = lane + 32 * i;
+        const int row = p >> 3, c16 = p & 7;
+        const int64_t grow = row0 + row;
+        const int64_t col = cb + 16 * c16;
+        const bool ok = grow < it.N && col < Kb;
+        const uint8_t* src = ok ? it.packed + grow * Kb + col : it.packed;
+        cp_async16_zfill(ring + s * kStageBytes + row * 128 + ((c16 ^ (row & 7)) << 4), src, ok);
       }
+    }
+    cp_async_commit();
   };
   // X'' fragments of unit j of chunk c: word q, token tile n -> two 16-byte halves
   auto load_x = [&](const Cur& c, int j, uint4 (&xb)[2][NT][2]) {
@@ -366,8 +416,8 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
       for (int n = 0; n < NT; ++n) {
         const int tok = n * 8 + g;
         if (kok && tok < M) {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(it.Xpp + int64_t(tok) * it.K + u * kUnit + 32 * t + 16 * q);
+          const uint4* src = reinterpret_cast<const uint4*>(it.Xpp + int64_t(tok) * it.K +
+                                                             u * kUnit + 32 * t + 16 * q);
           xb[q][n][0] = __ldg(src);
           xb[q][n][1] = __ldg(src + 1);
         } else {
@@ -377,10 +427,15 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
       }
   };
 
+  // prologue: the first kStages - 1 chunks (codes only: nothing here depends
+  // on the kernels this one may overlap)
   Cur cur = seek(Cur{static_cast<int>(blockIdx.x), 0, warp});
-  uint2 ring[kAhead][R][2];
+  Cur iss = cur;
 #pragma unroll
-  for (int j = 0; j < kAhead; ++j) load_unit(cur, j, ring[j]);
+  for (int s = 0; s < kStages - 1; ++s) {
+    issue(iss, s);
+    iss = advance(iss);
+  }
   Cur nxt = advance(cur);
 
   griddep_wait();  // X'' and corr written by the X-transform are visible from here
@@ -388,6 +443,7 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
   uint4 xcur[2][NT][2], xnxt[2][NT][2];
   load_x(cur, 0, xcur);
 
+  int stage = 0;  // stage of cur
   int eitem = 0;  // item of the tile in the epilogue
   int buf = 0;
   for (int tile = static_cast<int>(blockIdx.x); tile < T; tile += G, buf ^= 1) {
@@ -400,7 +456,16 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
         for (int e = 0; e < 4; ++e) acc[r][n][e] = 0.f;
 
     while (cur.tile == tile) {  // this warp's chunks of the tile
+      cp_async_wait<kStages - 2>();  // this lane's copies of chunk `cur` have landed
+      __syncwarp();                  // ... and every lane's; the stage refilled below is free
+      {
+        int s_iss = stage + kStages - 1;
+        if (s_iss >= kStages) s_iss -= kStages;
+        issue(iss, s_iss);
+        iss = advance(iss);
+      }
       const int Kc = grp.item[cur.item].K;
+      const uint32_t sbase = ring + stage * kStageBytes;
 #pragma unroll
       for (int j = 0; j < kAhead; ++j) {
         if constexpr (kPrefX) {
@@ -408,6 +473,14 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
           else load_x(nxt, 0, xnxt);
         }
         if ((int64_t(cur.chunk) * kAhead + j) * kUnit < Kc) {  // warp-uniform
+          // this lane's two code words of unit j for rows r*16 + g + 8h
+          uint2 cw[R][2];
+          const int c16 = 2 * j + (t >> 1);
+          const uint32_t off = static_cast<uint32_t>(((c16 ^ g) << 4) + ((t & 1) << 3));
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) cw[r][h] = lds_v2(sbase + (r * 16 + g + 8 * h) * 128 + off);
 #pragma unroll
           for (int q = 0; q < 2; ++q) {  // word q of each row: 16 codes, 4 k16 tiles
             uint32_t w0[R][2], w6[R][2], w12[R][2];
@@ -415,7 +488,7 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
             for (int r = 0; r < R; ++r)
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                w0[r][h] = q == 0 ? ring[j][r][h].x : ring[j][r][h].y;
+                w0[r][h] = q == 0 ? cw[r][h].x : cw[r][h].y;
                 w6[r][h] = w0[r][h] >> 6;
                 w12[r][h] = w0[r][h] >> 12;
               }
@@ -441,7 +514,6 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
             }
           }
         }
-        load_unit(nxt, j, ring[j]);  // refill the slot with the next chunk's unit
         if constexpr (kPrefX) {
 #pragma unroll
           for (int q = 0; q < 2; ++q)
@@ -457,6 +529,7 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
       }
       cur = nxt;
       nxt = advance(nxt);
+      if (++stage == kStages) stage = 0;
     }
 
     // the CTA's last tile: the next kernel may start launching
@@ -487,7 +560,253 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
       if (grow < it.N) it.Y[int64_t(tok) * it.N + grow] = f32_to_bf16(sum + it.corr[tok]);
     }
   }
+  cp_async_wait<0>();  // no copy may outlive the CTA (only empty groups remain)
 }
+
+// ---------------------------------------------------------------------------
+// Decode-GEMV over a large group: wide tiles, one producer warp.
+//
+// A tile is 128 weight rows of one matrix over its whole K; consumer warp w
+// (w < 8) owns rows 16 w .. 16 w + 15 of it and runs the whole K, so no tile
+// ends in a CTA-wide sum.  Warp 8 produces: it streams the tile's K chunks
+// (kAhead units = 512 codes per row: one 128-row x 128-byte TMA box with the
+// 128-byte swizzle; and the matching 512 positions of X'' for every token, one
+// 1D bulk copy per token) into a ring of kStages shared-memory stages, each
+// stage's arrival counted on its `full` mbarrier; the consumers
+// release a stage on its `empty` mbarrier.  X'' is thus read once per 128 rows
+// instead of once per 16.
+//
+// Same sums as the split kernel, bit for bit: chunk c of a tile is the split
+// kernel's chunk of warp c mod 8, so a consumer keeps 8 accumulators, adds
+// chunk c into accumulator c mod 8 in the same unit and MMA order, and ends
+// with the split kernel's fixed-order sum over the 8 accumulators.
+//
+// Every wait is bounded (kWideWaitLimit clock cycles); a warp that gives up
+// records LCVQ_ERR_DEVICE_TIMEOUT in the group's error word and raises the
+// CTA's abort flag, and the others wind down.
+constexpr int kWideConsumers = 8;
+constexpr int kWideThreads = (kWideConsumers + 1) * 32;
+constexpr int kWideRows = 16 * kWideConsumers;
+constexpr uint32_t kWideXPitch = 1040;    // 1024 X'' bytes per token + 16
+constexpr long long kWideWaitLimit = 1LL << 32;
+
+template <int kItems>
+struct GemvWideGroup {
+  CUtensorMap codes[kItems];  // per item: [N rows][K/4 bytes], box 128 x 128 B, SW128
+  int count, M;
+  unsigned int* err;
+  GemvItem item[kItems];  // tile_end in 128-row tiles
+};
+
+template <int NT, int kStages>
+struct WideLayout {
+  static constexpr uint32_t kCodeBytes = kWideRows * 128;  // one SW128 box
+  static constexpr uint32_t kXBytes = NT * 8 * kWideXPitch;
+  static constexpr uint32_t kStageBytes = (kCodeBytes + kXBytes + 1023) / 1024 * 1024;
+  static constexpr uint32_t kBarOff = kStages * kStageBytes;
+  static constexpr size_t kSmem = 1024 + size_t(kBarOff) + 2 * kStages * 8 + 16;  // + alignment
+};
+
+template <int NT, int kStages, int kMinBlocks, int kItems>
+__global__ void __launch_bounds__(kWideThreads, kMinBlocks)
+    gemv_wide_kernel(const __grid_constant__ GemvWideGroup<kItems> grp) {
+  using L = WideLayout<NT, kStages>;
+  extern __shared__ __align__(1024) unsigned char wsm_raw[];
+  // SW128 boxes need 1024-byte aligned destinations
+  unsigned char* wsm = wsm_raw + ((1024 - (sm100::smem_u32(wsm_raw) & 1023)) & 1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(wsm + L::kBarOff);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  const uint32_t sbase = sm100::smem_u32(wsm);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = grp.M;
+  const int T = grp.item[grp.count - 1].tile_end;
+  const int G = static_cast<int>(gridDim.x);
+  auto tile_begin = [&](int item) { return item == 0 ? 0 : grp.item[item - 1].tile_end; };
+  auto nchunks = [&](int K) { return static_cast<int>(ceil_div(ceil_div(K, kUnit), kAhead)); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      sm100::mbar_init(&full[s], 1);
+      sm100::mbar_init(&empty[s], kWideConsumers);
+    }
+    *abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+
+  griddep_wait();  // X'' and corr written by the X-transforms are visible from here
+
+  if (warp == kWideConsumers) {
+    // ------------------------------------------------------------ producer
+    int seq = 0, item = 0;
+    for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G) {
+      while (tile >= grp.item[item].tile_end) ++item;
+      const GemvItem& it = grp.item[item];
+      const int64_t row0 = int64_t(tile - tile_begin(item)) * kWideRows;
+      const int nch = nchunks(it.K);
+      for (int c = 0; c < nch; ++c, ++seq) {
+        const int s = seq % kStages;
+        if (!sm100::mbar_wait(&empty[s], ((seq / kStages) & 1) ^ 1, kWideWaitLimit)) {
+          if (lane == 0) record_error(grp.err, LCVQ_ERR_DEVICE_TIMEOUT, 50);
+          *abort_flag = 1;
+          break;
+        }
+        const int64_t xk = int64_t(c) * (kAhead * kUnit);  // chunk's first position
+        const uint32_t xbytes = static_cast<uint32_t>(it.K - xk < 512 ? (it.K - xk) * 2 : 1024);
+        const uint32_t st = sbase + s * L::kStageBytes;
+        if (lane == 0) {
+          // the full box is counted, including the zero fill past N rows or K/4 bytes
+          sm100::mbar_arrive_expect_tx(&full[s], L::kCodeBytes + static_cast<uint32_t>(M) * xbytes);
+          sm100::tma_load_2d(&grp.codes[item], &full[s], wsm + s * L::kStageBytes,
+                             c * (kAhead * 32), static_cast<int>(row0));
+        }
+        __syncwarp();
+        if (lane < M)
+          sm100::bulk_load(st + L::kCodeBytes + lane * kWideXPitch,
+                           it.Xpp + int64_t(lane) * it.K + xk, xbytes, &full[s]);
+      }
+    }
+    // drain: every stage filled above has been consumed, so its copies landed
+    for (int k = 0; k < kStages && !*abort_flag; ++k, ++seq) {
+      const int s = seq % kStages;
+      if (!sm100::mbar_wait(&empty[s], ((seq / kStages) & 1) ^ 1, kWideWaitLimit)) {
+        if (lane == 0) record_error(grp.err, LCVQ_ERR_DEVICE_TIMEOUT, 51);
+        *abort_flag = 1;
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int g = lane >> 2, t = lane & 3;
+  int seq = 0, item = 0;
+  for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G) {
+    while (tile >= grp.item[item].tile_end) ++item;
+    const GemvItem& it = grp.item[item];
+    const int K = it.K;
+    const int nch = nchunks(K);
+    float acc[kWideConsumers][NT][4];
+#pragma unroll
+    for (int v = 0; v < kWideConsumers; ++v)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[v][n][e] = 0.f;
+
+    bool ok = true;
+    for (int c0 = 0; c0 < nch && ok; c0 += kWideConsumers) {
+#pragma unroll
+      for (int v = 0; v < kWideConsumers; ++v) {  // chunk c0 + v -> accumulator v
+        const int c = c0 + v;
+        if (c >= nch) break;
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        const int s = seq % kStages;
+        if (!sm100::mbar_wait(&full[s], (seq / kStages) & 1, kWideWaitLimit)) {
+          if (lane == 0) record_error(grp.err, LCVQ_ERR_DEVICE_TIMEOUT, 52);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const uint32_t st = sbase + s * L::kStageBytes;
+        const uint32_t crow = st + (warp * 16 + g) * 128;  // rows g and g + 8: (row & 7) = g
+        const uint32_t xst = st + L::kCodeBytes;
+#pragma unroll
+        for (int j = 0; j < kAhead; ++j) {
+          const int64_t u = int64_t(c) * kAhead + j;
+          if (u * kUnit >= K) break;  // warp-uniform: past the end of K
+          const bool kok = u * kUnit + 32 * t < K;
+          // SW128: 16-byte chunk c16 of a row sits at c16 ^ (row & 7)
+          const uint32_t off = static_cast<uint32_t>(((2 * j + (t >> 1)) ^ g) << 4) + ((t & 1) << 3);
+          uint2 cw[2];
+          cw[0] = lds_v2(crow + off);
+          cw[1] = lds_v2(crow + 8 * 128 + off);
+          uint4 xb[2][NT][2];
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              const int tok = n * 8 + g;
+              if (kok && tok < M) {
+                const uint32_t xa = xst + tok * kWideXPitch + (j * kUnit + 32 * t + 16 * q) * 2;
+                xb[q][n][0] = lds_v4(xa);
+                xb[q][n][1] = lds_v4(xa + 16);
+              } else {
+                xb[q][n][0] = make_uint4(0, 0, 0, 0);
+                xb[q][n][1] = make_uint4(0, 0, 0, 0);
+              }
+            }
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t w0[2], w6[2], w12[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              w0[h] = q == 0 ? cw[h].x : cw[h].y;
+              w6[h] = w0[h] >> 6;
+              w12[h] = w0[h] >> 12;
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const uint32_t a00 = dec_pair_rt(2 * jj, w0[0], w6[0], w12[0]);
+              const uint32_t a10 = dec_pair_rt(2 * jj, w0[1], w6[1], w12[1]);
+              const uint32_t a01 = dec_pair_rt(2 * jj + 1, w0[0], w6[0], w12[0]);
+              const uint32_t a11 = dec_pair_rt(2 * jj + 1, w0[1], w6[1], w12[1]);
+#pragma unroll
+              for (int n = 0; n < NT; ++n) {
+                const uint32_t b0 = word_of(xb[q][n][jj >> 1], (2 * jj) & 3);
+                const uint32_t b1 = word_of(xb[q][n][jj >> 1], (2 * jj + 1) & 3);
+                mma_bf16_16816(acc[v][n], a00, a10, a01, a11, b0, b1);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&empty[s]);
+        ++seq;
+      }
+    }
+    if (!ok) break;
+
+    // the split kernel's fixed-order sum over the 8 K partitions, plus corr
+    const int64_t row0 = int64_t(tile - tile_begin(item)) * kWideRows + warp * 16;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t row = row0 + g + 8 * (e >> 1);
+        const int tok = n * 8 + 2 * t + (e & 1);
+        float sum = 0.f;
+#pragma unroll
+        for (int v = 0; v < kWideConsumers; ++v) sum += acc[v][n][e];
+        if (row < it.N && tok < M) it.Y[int64_t(tok) * it.N + row] = f32_to_bf16(sum + it.corr[tok]);
+      }
+  }
+  // the last CTA-wide point: consumers are done with every stage
+  griddep_launch_dependents();
+}
+
+// stages of the wide-tile kernel per token-tile count
+#ifndef LCVQ_WS1
+#define LCVQ_WS1 4
+#endif
+#ifndef LCVQ_WS2
+#define LCVQ_WS2 6
+#endif
+
+// code-ring depth (chunks per warp) per token-tile count
+#ifndef LCVQ_GS1
+#define LCVQ_GS1 4
+#endif
+#ifndef LCVQ_GS2
+#define LCVQ_GS2 4
+#endif
+#ifndef LCVQ_GS4
+#define LCVQ_GS4 3
+#endif
 
 // CTAs of a kernel that one device holds at once (cached per kernel and device)
 int64_t resident_ctas(const void* kern, int threads, size_t smem) {
@@ -508,10 +827,10 @@ int64_t resident_ctas(const void* kern, int threads, size_t smem) {
   return v;
 }
 
-template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kItems>
+template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kStages, int kItems>
 cudaError_t launch_group_t(const GemvGroup<kItems>& grp, cudaStream_t s) {
-  auto kern = gemv_group_kernel<NT, R, kWarps, kPrefX, kMinBlocks, kItems>;
-  constexpr size_t smem = size_t(2) * kWarps * (16 * R) * (NT * 8 + 1) * sizeof(float);
+  auto kern = gemv_group_kernel<NT, R, kWarps, kPrefX, kMinBlocks, kStages, kItems>;
+  constexpr size_t smem = group_smem_ring<R, kStages, kWarps>() + group_smem_part<NT, R, kWarps>();
   if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
       e != cudaSuccess)
     return e;
@@ -540,9 +859,9 @@ int group_rows(int64_t M) { return M <= 8 ? kRowsSmallM : kRowsLargeM; }
 // per SM with room for the X'' prefetch; M <= 32: 32 rows, no prefetch.
 template <int kItems>
 cudaError_t launch_group(const GemvGroup<kItems>& grp, cudaStream_t s) {
-  if (grp.M <= 8) return launch_group_t<1, 1, 8, true, 2, kItems>(grp, s);
-  if (grp.M <= 16) return launch_group_t<2, 2, 8, true, 1, kItems>(grp, s);
-  return launch_group_t<4, 2, 8, false, 1, kItems>(grp, s);
+  if (grp.M <= 8) return launch_group_t<1, 1, 8, true, 2, LCVQ_GS1, kItems>(grp, s);
+  if (grp.M <= 16) return launch_group_t<2, 2, 8, true, 1, LCVQ_GS2, kItems>(grp, s);
+  return launch_group_t<4, 2, 8, false, 1, LCVQ_GS4, kItems>(grp, s);
 }
 
 }  // namespace
@@ -575,8 +894,66 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
   return cudaGetLastError();
 }
 
+namespace {
+template <int NT, int kStages, int kMinBlocks, int kItems>
+cudaError_t launch_wide_t(const GemvWideGroup<kItems>& grp, cudaStream_t s) {
+  auto kern = gemv_wide_kernel<NT, kStages, kMinBlocks, kItems>;
+  constexpr size_t smem = WideLayout<NT, kStages>::kSmem;
+  if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
+      e != cudaSuccess)
+    return e;
+  const int64_t tiles = grp.item[grp.count - 1].tile_end;
+  const int64_t resident = resident_ctas(reinterpret_cast<const void*>(kern), kWideThreads, smem);
+  if (resident <= 0) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < resident ? tiles : resident), 1, 1);
+  cfg.blockDim = dim3(kWideThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, grp);
+}
+}  // namespace
+
+#ifndef LCVQ_WIDE_MIN_TILES
+#define LCVQ_WIDE_MIN_TILES 296
+#endif
+
 cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaStream_t s,
-                                int* launches) {
+                                int* launches, unsigned int* err) {
+  // enough 128-row tiles to fill the device: the wide-tile kernel (M <= 16)
+  int64_t wide_tiles = 0;
+  for (int i = 0; i < count; ++i) wide_tiles += ceil_div(jobs[i].d_out, kWideRows);
+  if (M <= 16 && wide_tiles >= LCVQ_WIDE_MIN_TILES) {
+    for (int first = 0; first < count; first += kMaxGroupItems) {
+      const int n = count - first < kMaxGroupItems ? count - first : kMaxGroupItems;
+      GemvWideGroup<kMaxGroupItems> grp{};
+      grp.count = n;
+      grp.M = static_cast<int>(M);
+      grp.err = err;
+      int tiles = 0;
+      for (int i = 0; i < n; ++i) {
+        const GemvJob& j = jobs[first + i];
+        tiles += static_cast<int>(ceil_div(j.d_out, kWideRows));
+        grp.item[i] = GemvItem{j.packed, j.Xpp, j.corr, j.Y, static_cast<int>(j.d_out),
+                               static_cast<int>(j.d_in), tiles};
+        if (!make_tensor_map_2d(&grp.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, j.packed,
+                                uint64_t(j.d_in / 4), uint64_t(j.d_out), uint64_t(j.d_in / 4),
+                                kAhead * 32, kWideRows, true))
+          return cudaErrorInvalidValue;
+      }
+      cudaError_t e = M <= 8 ? launch_wide_t<1, LCVQ_WS1, 2, kMaxGroupItems>(grp, s)
+                             : launch_wide_t<2, LCVQ_WS2, 1, kMaxGroupItems>(grp, s);
+      ++*launches;
+      if (e != cudaSuccess) return e;
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   const int rows = group_rows(M);
   for (int first = 0; first < count; first += kMaxGroupItems) {
     const int n = count - first < kMaxGroupItems ? count - first : kMaxGroupItems;

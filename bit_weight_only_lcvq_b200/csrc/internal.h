@@ -2,6 +2,7 @@
 // of its launch(es) and adds the number of kernels it launched to *launches.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -56,8 +57,9 @@ struct GemvJob {
   uint16_t* Y;
   int64_t d_out, d_in;
 };
+// err: device error word for the bounded waits of the wide-tile form
 cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaStream_t s,
-                                int* launches);
+                                int* launches, unsigned int* err);
 cudaError_t launch_xform_grouped(const XformJob* jobs, int count, int64_t M, int d,
                                  cudaStream_t s, int* launches);
 
@@ -66,6 +68,13 @@ cudaError_t launch_xform_grouped(const XformJob* jobs, int count, int64_t M, int
 cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,
                                 const uint8_t* packed, int64_t d_out, int64_t d_in, uint16_t* Y,
                                 unsigned int* err, cudaStream_t s, int* launches);
+
+// 2D TMA tensor map: `inner` contiguous elements per row, `outer` rows of
+// `row_bytes`; box box_inner x box_outer; 128-byte swizzle or none; zero fill
+// out of bounds.  False if the driver entry point is missing or rejects it.
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                        uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                        bool swizzle128);
 
 // ---- tcgen05 GEMMs (bf16, persistent, one CTA per SM) ----
 int tc_max_grid();

@@ -916,6 +916,12 @@ cudaError_t launch_kind2_d(int d, const CUtensorMap& a, const CUtensorMap& b, co
 
 int tc_max_grid() { return num_sms(); }
 
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                        uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                        bool swizzle128) {
+  return make_map(map, dt, base, inner, outer, row_bytes, box_inner, box_outer, swizzle128);
+}
+
 cudaError_t launch_tc_forward(const uint16_t* Xa, bool algebraic, const float* corr, int64_t M,
                               const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
                               const float* A, const float* B, uint16_t* Y, unsigned int* err,

@@ -327,3 +327,23 @@ def test_gemm_grouped_many_items_and_graph_replay():
         assert all(torch.equal(o, r) for o, r in zip(outs, refs))
     del g
     assert lcvq.check_device_error(wsb) == 0
+
+
+@pytest.mark.parametrize("M", [1, 3, 8, 16])
+def test_gemm_grouped_wide_tiles_bitwise_equal_separate_calls(M):
+    """A group large enough for the wide-tile kernel (>= 296 tiles of 128 rows;
+    one producer warp streams codes and X'' into a shared-memory ring) gives
+    the split kernel's bits; the group includes a ragged row count and a K
+    that ends inside a chunk."""
+    shapes = [(4096, 4096)] * 9 + [(1088, 1000), (11008, 4096)]
+    jobs, zs, ws = _group_case(shapes, M, 700 + M)
+    wsb = lcvq.new_workspace(lcvq.workspace_size_grouped(jobs, M, 8))
+    Ys = lcvq.gemm_grouped(jobs, 8, workspace=wsb)
+    assert lcvq.last_launch_count() == 2
+    assert lcvq.check_device_error(wsb) == 0
+    for i, ((X, packed, A, B, d_in), Y) in enumerate(zip(jobs, Ys)):
+        Y1 = lcvq.gemm(X, packed, d_in, A, B, 8)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, Y1), f"item {i}"
+    ref, D = O.forward(ws[9]["X"], zs[9], ws[9]["A"], ws[9]["B"])
+    assert_close(f"wide grouped ragged item M={M}", to_np(Ys[9]), ref, D, TOL_BF16)

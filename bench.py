@@ -52,6 +52,9 @@ def parse():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--rows", default="all")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--stack-layers", type=int, default=32,
+                   help="decoder layers of the stack row (32 = the 7B-shaped workload)")
+    p.add_argument("--stack-ms", default="1,8,32", help="token counts of the stack row")
     return p.parse_args()
 
 
@@ -476,11 +479,12 @@ def row_qat(D, pk):
                               unit="TFLOP/s", frac=tf / pk["bf16_tflops_sustained"]))
 
 
-def row_stack(D, pk):
-    """7B-shaped stack: 224 matrices, M in {1, 8, 32}; packed GB/s over the stack."""
+def row_stack(D, pk, layers=32, ms=(1, 8, 32)):
+    """7B-shaped stack: 224 matrices, M in {1, 8, 32}; packed GB/s over the stack
+    (fewer layers or token counts only for a profiler capture)."""
     dev = D.dev
     mats = []
-    for layer in range(32):
+    for layer in range(layers):
         for p in range(len(synth.STACK_PROJS)):
             m = synth.stack_matrix(layer, p, 32, with_x=(layer == 0))
             mats.append(m)
@@ -498,7 +502,7 @@ def row_stack(D, pk):
     # independent (q, k, v | o | gate, up | down)
     phases = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
     out = {}
-    for M in (1, 8, 32):
+    for M in ms:
         ys = {p: torch.empty((M, do), dtype=torch.bfloat16, device=dev) for p, _, do in synth.STACK_PROJS}
         wss = {p: lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, do, di, 8), dev)
                for p, di, do in synth.STACK_PROJS}
@@ -563,7 +567,8 @@ def row_stack(D, pk):
         out[str(M)] = res_m
         del all_ws, all_outs, ph_ws
         torch.cuda.empty_cache()
-    return dict(metric="stack packed-weight GB/s (224 matrices, 1.62 GB of codes)",
+    return dict(metric=f"stack packed-weight GB/s ({len(dmats)} matrices, "
+                       f"{total_bytes / 1e9:.2f} GB of codes)",
                 note="sequential: 224 lcvq_gemm calls; grouped_by_phase: one lcvq_gemm_grouped per "
                      "decoder-layer phase (q,k,v | o | gate,up | down), 128 calls; grouped_all: the "
                      "224 independent matrices in one lcvq_gemm_grouped call",
@@ -603,7 +608,11 @@ def main():
     if D.rank == 0:
         for name in want:
             try:
-                rows[name] = ROWS[name](D, pk)
+                if name == "stack":
+                    rows[name] = row_stack(D, pk, args.stack_layers,
+                                           tuple(int(m) for m in args.stack_ms.split(",")))
+                else:
+                    rows[name] = ROWS[name](D, pk)
             except Exception as ex:  # report, do not hide
                 rows[name] = {"error": f"{type(ex).__name__}: {ex}"}
             torch.cuda.empty_cache()

@@ -63,9 +63,9 @@ def parse():
 # source that was captured: keyed by the SHA-1 of the source file.
 NCU_TRAFFIC = {
     # source file -> (sha1 of the file when captured, {token count: bytes per launch})
-    # profiles/launches_decode_gemv_bench.md: M = 1 and 4 share gemv_kernel<1, ...>
+    # profiles/launches_decode_gemv_bench.md: M = 1 and 4 share gemv_group_kernel<1, ...>
     "bit_weight_only_lcvq_b200/csrc/gemv.cu": (
-        "80b75d0752c56f28a2d89ae289e8922b78f5e402", {1: 4226188, 4: 4226188, 16: 4350809}),
+        "9c29dab4f5a6019c8c4c5ebf9f818537dbeaa76e", {1: 4238969, 4: 4238969, 16: 4369947}),
 }
 
 
@@ -369,7 +369,7 @@ def headline(args, D: Dist, pk):
                       traffic=_sum_or_none([traffic_for("bit_weight_only_lcvq_b200/csrc/gemv.cu", M)
                                             for M in Ms]),
                       traffic_unit="bytes per step (3 launches)",
-                      kernel="gemv_kernel (decode-GEMV, M=1,4,16 summed)",
+                      kernel="gemv_group_kernel (decode-GEMV, M=1,4,16 summed)",
                       per_m_us={str(M): per_m[M] * 1e3 for M in Ms},
                       peak_source=f"{PEAK_SRC} hbm_gbs"),
         e2e=e2e, clocks=ck, gpu_launches=int(launches), parity_max_rel_err=parity,

@@ -24,7 +24,9 @@ Sources (cited below by these short names):
   decoupling parameters into integer and floating-point parts* (lryc.cn
   translation).  Eq. (1) fixes the linear-layer convention ``Y = X W~`` with
   ``W~`` of shape ``d_in x d_out``; eq. (3)/(4) are the scalar
-  round/clip/affine special case used as a pin.
+  round/clip/affine special case used as a pin; eq. (5) and section 3.3 (the
+  float part solved in closed form with the integer part fixed) define the
+  least-squares refit of (A, B).
 
 Readings where the pages are silent (each one is listed in the design doc):
 
@@ -256,6 +258,57 @@ def backward_dwp_sampled(X, dY, mask_rows_fn, A, pairs):
         v[t] = mk * float(np.dot(A[:, j], Gv))
         dd[t] = mk * float(np.dot(np.abs(A[:, j]), DGv))
     return v, dd
+
+
+# --------------------------------------------------------------------------
+# least-squares refit of the float part given the codes (decoupleQ page,
+# eq. (5): the layer objective tr{(W~ - W0)^T H (W~ - W0)}; section 3.3: with
+# the integer part fixed the float part is an unconstrained quadratic, solved
+# by setting the derivative to zero).  LC-VQ's float part is (A, B); H is
+# taken as its diagonal h (one weight per input channel; h = 1 is the plain
+# least-squares fit).
+# --------------------------------------------------------------------------
+PINV_RCOND = 1e-12  # eigenvalues below this fraction of the largest count as zero
+
+
+def fit_affine_normal(W0: np.ndarray, z: np.ndarray, d: int, h=None):
+    """The normal equations of the refit.  Output coordinate i of every vector
+    (row n, group g) has input channel k = g d + i; with zt = [z_0 .. z_{d-1}, 1]
+    (the vector's codes and a one for B):
+        G[i] = sum_{n,g} h_k zt zt^T        ((d+1) x (d+1))
+        R[i] = sum_{n,g} h_k W0[n, k] zt    (d+1)
+    Returns (G [d][d+1][d+1], R [d][d+1])."""
+    N, K = W0.shape
+    ng = K // d
+    zt = np.concatenate([z.reshape(N, ng, d).astype(np.float64), np.ones((N, ng, 1))], axis=2)
+    w = np.asarray(W0, dtype=np.float64).reshape(N, ng, d)
+    hv = (np.ones(K) if h is None else np.asarray(h, dtype=np.float64)).reshape(ng, d)
+    G = np.einsum("gi,ngj,ngk->ijk", hv, zt, zt)
+    R = np.einsum("gi,ngi,ngj->ij", hv, w, zt)
+    return G, R
+
+
+def fit_affine(W0: np.ndarray, z: np.ndarray, d: int, h=None):
+    """(A, B) minimizing sum_n sum_k h_k (W0[n, k] - W~[n, k])^2 over W~ = A z + B
+    per vector.  The objective splits over the output coordinate i, and row i
+    of [A | B] is theta_i = G[i]^+ R[i]: the solution of the normal equations,
+    the minimum-norm one when G[i] is singular (a code position that never
+    varies, or weights h that vanish)."""
+    G, R = fit_affine_normal(W0, z, d, h)
+    A = np.zeros((d, d))
+    B = np.zeros(d)
+    for i in range(d):
+        th = np.linalg.pinv(G[i], rcond=PINV_RCOND, hermitian=True) @ R[i]
+        A[i] = th[:d]
+        B[i] = th[d]
+    return A, B
+
+
+def fit_objective(W0, z, A, B, h=None) -> float:
+    """sum_n sum_k h_k (W0[n, k] - (A z + B)[n, k])^2, the quantity fit_affine minimizes."""
+    r = np.asarray(W0, dtype=np.float64) - decode(z, A, B)
+    hh = np.ones(r.shape[1]) if h is None else np.asarray(h, dtype=np.float64)
+    return float(np.sum(hh[None, :] * r * r))
 
 
 # --------------------------------------------------------------------------

@@ -373,6 +373,125 @@ def test_db_identity_at_any_size():
     assert np.allclose(bw["dB"], ident, rtol=1e-13, atol=1e-13)
 
 
+# ---------------------------------------------------------------- (A, B) refit
+def _fit_case(d, N, K, seed, noise=0.0):
+    g = np.random.Generator(np.random.PCG64(seed))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A = g.standard_normal((d, d))
+    B = g.standard_normal(d)
+    W0 = O.decode(z, A, B) + noise * g.standard_normal((N, K))
+    return g, z, A, B, W0
+
+
+@pytest.mark.parametrize("d", [1, 2, 4, 8])
+def test_fit_affine_recovers_an_exact_affine_map(d):
+    """W0 generated as A z + B is fitted with zero residual: (A, B) come back."""
+    _, z, A, B, W0 = _fit_case(d, 37, 16 * d, 500 + d)
+    A2, B2 = O.fit_affine(W0, z, d)
+    assert np.allclose(A2, A, atol=1e-10) and np.allclose(B2, B, atol=1e-10)
+    assert O.fit_objective(W0, z, A2, B2) < 1e-18 * W0.size
+
+
+@pytest.mark.parametrize("d", [2, 4, 8])
+def test_fit_affine_equals_least_squares_on_the_stacked_design(d):
+    """Row i of [A | B] solves the least-squares problem whose design matrix
+    stacks [z, 1] of every vector, weighted by sqrt(h) of the vector's channel i
+    (a different formulation from the oracle's normal equations)."""
+    g, z, A, B, W0 = _fit_case(d, 23, 8 * d, 600 + d, noise=0.3)
+    h = g.uniform(0.1, 2.0, size=8 * d)
+    A2, B2 = O.fit_affine(W0, z, d, h)
+    N, K = W0.shape
+    for i in range(d):
+        rows, rhs = [], []
+        for n in range(N):
+            for grp in range(K // d):
+                k = grp * d + i
+                s = math.sqrt(h[k])
+                rows.append(s * np.append(z[n, grp * d:(grp + 1) * d].astype(np.float64), 1.0))
+                rhs.append(s * W0[n, k])
+        th = np.linalg.lstsq(np.array(rows), np.array(rhs), rcond=None)[0]
+        assert np.allclose(A2[i], th[:d], atol=1e-10) and abs(B2[i] - th[d]) < 1e-10
+
+
+def test_fit_affine_scalar_case_is_simple_linear_regression():
+    """d = 1, h = 1: the per-matrix (s, zero point) of decoupleQ eq. (4) fitted by
+    least squares has the textbook closed form s = cov(z, w) / var(z),
+    b = mean(w) - s mean(z)."""
+    _, z, _, _, W0 = _fit_case(1, 19, 40, 700, noise=0.5)
+    A2, B2 = O.fit_affine(W0, z, 1)
+    zz = z.astype(np.float64).ravel()
+    ww = W0.ravel()
+    s = np.sum((zz - zz.mean()) * (ww - ww.mean())) / np.sum((zz - zz.mean()) ** 2)
+    assert A2[0, 0] == pytest.approx(s, rel=1e-12)
+    assert B2[0] == pytest.approx(ww.mean() - s * zz.mean(), rel=1e-12, abs=1e-12)
+
+
+def test_fit_affine_is_a_minimum():
+    """Every small perturbation of (A, B) raises the weighted objective, and its
+    central-difference gradient vanishes at the fit."""
+    d = 4
+    g, z, _, _, W0 = _fit_case(d, 11, 32, 800, noise=0.4)
+    h = g.uniform(0.5, 1.5, size=32)
+    A2, B2 = O.fit_affine(W0, z, d, h)
+    f0 = O.fit_objective(W0, z, A2, B2, h)
+    eps = 1e-4
+    for t in range(d * d + d):
+        dA = np.zeros((d, d))
+        dB = np.zeros(d)
+        if t < d * d:
+            dA.flat[t] = eps
+        else:
+            dB[t - d * d] = eps
+        fp = O.fit_objective(W0, z, A2 + dA, B2 + dB, h)
+        fm = O.fit_objective(W0, z, A2 - dA, B2 - dB, h)
+        assert fp > f0 and fm > f0
+        assert abs(fp - fm) / (2 * eps) < 1e-6 * (1 + f0)
+
+
+def test_fit_affine_singular_gram_gives_the_minimum_norm_solution():
+    """A code position that never varies makes G singular (its column is a
+    multiple of the ones column); the fit is then the minimum-norm
+    least-squares solution, which lstsq also returns."""
+    d = 4
+    g, z, _, _, W0 = _fit_case(d, 17, 32, 900, noise=0.2)
+    z = z.copy()
+    z[:, 2::d] = 2                      # position 2 of every vector is always 2
+    A2, B2 = O.fit_affine(W0, z, d)
+    N, K = W0.shape
+    for i in range(d):
+        D = np.array([np.append(z[n, grp * d:(grp + 1) * d].astype(np.float64), 1.0)
+                      for n in range(N) for grp in range(K // d)])
+        y = np.array([W0[n, grp * d + i] for n in range(N) for grp in range(K // d)])
+        th = np.linalg.lstsq(D, y, rcond=None)[0]
+        assert np.allclose(A2[i], th[:d], atol=1e-9) and abs(B2[i] - th[d]) < 1e-9
+
+
+def test_fit_affine_weights_scale_and_mask():
+    """Scaling h leaves the fit unchanged; h that is zero outside a set of
+    input channels fits those channels only."""
+    d = 4
+    g, z, _, _, W0 = _fit_case(d, 13, 64, 1000, noise=0.3)
+    h = g.uniform(0.2, 1.0, size=64)
+    A1, B1 = O.fit_affine(W0, z, d, h)
+    A7, B7 = O.fit_affine(W0, z, d, 7.0 * h)
+    assert np.allclose(A1, A7, atol=1e-12) and np.allclose(B1, B7, atol=1e-12)
+    keep = np.zeros(64)
+    keep[:32] = 1.0
+    Am, Bm = O.fit_affine(W0, z, d, keep)
+    As, Bs = O.fit_affine(W0[:, :32], z[:, :32], d)
+    assert np.allclose(Am, As, atol=1e-12) and np.allclose(Bm, Bs, atol=1e-12)
+
+
+def test_fit_planted_mistake_is_caught():
+    """Normal equations that pair channel i's weight with coordinate j's codes
+    (a transposed right-hand side) fail the exact-recovery pin."""
+    d = 4
+    _, z, A, B, W0 = _fit_case(d, 37, 64, 504)
+    G, R = O.fit_affine_normal(W0, z, d)
+    th = np.linalg.solve(G[1], R[2])  # the right-hand side of the wrong coordinate
+    assert not np.allclose(th[:d], A[1], atol=1e-6)
+
+
 # ---------------------------------------------------------------- metric
 def test_rel_err_semantics():
     assert O.rel_err([1.0, 2.0], [1.0, 2.5], [1.0, 5.0]) == pytest.approx(0.1)

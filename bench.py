@@ -575,8 +575,32 @@ def row_stack(D, pk, layers=32, ms=(1, 8, 32)):
                 per_m=out, packed_bytes=total_bytes)
 
 
+def row_fit(D, pk):
+    """Least-squares (A, B) refit on the QAT-step matrix (4096 x 14336, d = 8):
+    W0 = the workload's proxy weights, codes = their assignment; unweighted and
+    with per-channel weights h."""
+    dev = D.dev
+    N, K, d = 4096, 14336, 8
+    w = synth.workload(4, M=1, with_dy=False)
+    W0 = torch.from_numpy(w["Wp"]).to(dev)
+    packed, _ = lcvq.assign_pack(W0, d, with_mask=False)
+    h = torch.rand(K, device=dev, generator=torch.Generator(device=dev).manual_seed(3)) + 0.5
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_FIT_AFFINE, torch.float32, 0, N, K, d), dev)
+    A = torch.empty((d, d), device=dev)
+    B = torch.empty(d, device=dev)
+    nbytes = N * K * (4 + 0.25)
+    out = {}
+    for name, hh in (("unweighted", None), ("weighted", h)):
+        ms = ev_time(lambda: lcvq.fit_affine(W0, packed, d, h=hh, workspace=ws, A=A, B=B), 30)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = dict(value=gbs, unit="GB/s", us=ms * 1e3,
+                         roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
+                                       frac=gbs / pk["hbm_gbs"]))
+    return dict(metric="(A, B) refit GB/s (W0 fp32 + codes read)", forms=out)
+
+
 ROWS = {"assign_pack": row_assign_pack, "decode": row_decode, "prefill": row_prefill,
-        "qat": row_qat, "stack": row_stack}
+        "qat": row_qat, "stack": row_stack, "fit": row_fit}
 
 
 # ----------------------------------------------------------------------------- main

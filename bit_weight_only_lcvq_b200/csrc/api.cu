@@ -161,7 +161,28 @@ size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_ou
   if (dtype != LCVQ_F32 && dtype != LCVQ_BF16) return 0;
   if (op == LCVQ_OP_GEMM) return gemm_ws(dtype, M, d_in).total;
   if (op == LCVQ_OP_GEMM_BACKWARD) return bwd_ws(M, d_out, d_in, d).total;
+  if (op == LCVQ_OP_FIT_AFFINE) return kWsHeaderBytes + fit_partials_bytes(d_out, d_in, d);
   return 0;
+}
+
+lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int64_t d_out, int64_t d_in,
+                            int d, const float* h, float* A, float* B, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  g_last_launches = 0;
+  if (d_out < 0 || d_in < 0 || !valid_d(d) || d_in % 16 != 0) return LCVQ_ERR_INVALID_ARG;
+  if (!A || !B || !workspace) return LCVQ_ERR_INVALID_ARG;
+  const bool empty = d_out == 0 || d_in == 0;
+  if (!empty && (!W0 || !packed)) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || (!empty && (!aligned16(W0) || !aligned16(packed))) ||
+      (h && !aligned16(h)))
+    return LCVQ_ERR_ALIGNMENT;
+  if (ws_bytes < kWsHeaderBytes + fit_partials_bytes(d_out, d_in, d)) return LCVQ_ERR_WORKSPACE;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  double* partials = reinterpret_cast<double*>(static_cast<char*>(workspace) + kWsHeaderBytes);
+  cudaError_t e = launch_fit_affine(W0, packed, empty ? 0 : d_out, empty ? 0 : d_in, d, h, A, B,
+                                    partials, static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
 }
 
 static lcvq_status validate_gemm_shapes(lcvq_dtype dtype, int64_t M, int64_t d_out, int64_t d_in,

@@ -76,6 +76,13 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
                         uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                         bool swizzle128);
 
+// ---- least-squares refit of (A, B) given the codes ----
+// partials: fit_partials_bytes(d_out, d_in, d) bytes of fp64 scratch
+size_t fit_partials_bytes(int64_t d_out, int64_t d_in, int d);
+cudaError_t launch_fit_affine(const float* W0, const uint8_t* packed, int64_t d_out, int64_t d_in,
+                              int d, const float* h, float* A, float* B, double* partials,
+                              cudaStream_t s, int* launches);
+
 // ---- tcgen05 GEMMs (bf16, persistent, one CTA per SM) ----
 int tc_max_grid();
 // Xa is X'' (algebraic, with corr) or X (decode form, A z + B decoded on chip)

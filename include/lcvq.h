@@ -92,7 +92,7 @@ typedef enum {
  *  AUTO:      the library's choice (ALGEBRAIC on the tensor-core paths). */
 typedef enum { LCVQ_FORM_AUTO = 0, LCVQ_FORM_DECODE = 1, LCVQ_FORM_ALGEBRAIC = 2 } lcvq_form;
 
-typedef enum { LCVQ_OP_GEMM = 0, LCVQ_OP_GEMM_BACKWARD = 1 } lcvq_op;
+typedef enum { LCVQ_OP_GEMM = 0, LCVQ_OP_GEMM_BACKWARD = 1, LCVQ_OP_FIT_AFFINE = 2 } lcvq_op;
 
 /* Code assignment and 2-bit packing (LC-QAT technical summary, Methodology 1:
  * index selection becomes rounding and clamping; Methodology 3: proxy weights
@@ -228,6 +228,32 @@ LCVQ_API lcvq_status lcvq_gemm_backward(const void* X, const void* dY, lcvq_dtyp
                                const float* A, const float* B,
                                void* dX, float* dA, float* dB, float* dWp,
                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Least-squares refit of the float part (A, B) given the codes (decoupleQ
+ * page: eq. (5), the layer objective tr{(W~ - W0)^T H (W~ - W0)}, and section
+ * 3.3, where the float part is solved in closed form with the integer part
+ * fixed; here for LC-VQ's codewords c = A z + B, LC-QAT technical summary,
+ * Methodology 1).  H is taken as its diagonal h: the call minimizes
+ *     sum_n sum_k h[k] (W0[n][k] - W~[n][k])^2,   W~ = A z + B per vector,
+ * over A and B.  Row i of [A | B] is G_i^+ R_i, where G_i = sum h zt zt^T
+ * and R_i = sum h W0 zt run over every vector with zt = [z_0 .. z_{d-1}, 1],
+ * taking channel k = g d + i of vector g.  G^+ is the pseudo-inverse:
+ * eigenvalues below 1e-12 of the largest count as zero, which gives the
+ * minimum-norm solution when G_i is singular (a code position that never
+ * varies, or weights that vanish).  Sums are fp32 per lane (exact for the
+ * integer-valued G_i of h = 1), then fp64 in a fixed order; the solve is fp64
+ * and the result is bitwise reproducible.
+ *   W0     [d_out][d_in] fp32 target weights (e.g. the pretrained matrix).
+ *   packed [d_out][d_in/4] codes (format V1).
+ *   h      [d_in] fp32 channel weights >= 0 (e.g. diag(X^T X)), or NULL for 1.
+ *   A      [d*d] fp32 out (row-major);  B [d] fp32 out.
+ *   workspace: >= lcvq_workspace_size(LCVQ_OP_FIT_AFFINE, LCVQ_F32, 0, d_out,
+ *   d_in, d) bytes, 256-byte aligned.
+ * Shapes: d_in % 16 == 0; an empty matrix gives A = 0, B = 0.  Launches 2
+ * kernels. */
+LCVQ_API lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int64_t d_out,
+                                     int64_t d_in, int d, const float* h, float* A, float* B,
+                                     void* workspace, size_t ws_bytes, void* stream);
 
 /* Workspace bytes a call with these arguments needs (0 on invalid input).
  * The workspace holds the device error word (its first 256 bytes, which the

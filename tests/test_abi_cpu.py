@@ -88,3 +88,14 @@ def test_grouped_gemm_rejects_bad_groups_without_device():
     assert L.lcvq_gemm_grouped(bad, 2, 8, 8, 256, 1 << 30, None) == 3
     bad[1].Y = None
     assert L.lcvq_gemm_grouped(bad, 2, 8, 8, 256, 1 << 30, None) == 1
+
+
+def test_fit_affine_rejects_bad_arguments_without_device():
+    L = lcvq.lib()
+    assert L.lcvq_workspace_size(lcvq.OP_FIT_AFFINE, 0, 0, 4096, 4096, 8) > 256
+    assert L.lcvq_workspace_size(lcvq.OP_FIT_AFFINE, 0, 0, 4096, 4096, 3) == 0
+    assert L.lcvq_fit_affine(16, 16, 8, 24, 8, None, 16, 16, 256, 1 << 20, None) == 1  # d_in % 16
+    assert L.lcvq_fit_affine(16, 16, 8, 64, 3, None, 16, 16, 256, 1 << 20, None) == 1  # d
+    assert L.lcvq_fit_affine(16, 16, 8, 64, 8, None, None, 16, 256, 1 << 20, None) == 1  # no A
+    assert L.lcvq_fit_affine(16, 16, 8, 64, 8, 8, 16, 16, 256, 1 << 20, None) == 3     # h misaligned
+    assert L.lcvq_fit_affine(16, 16, 8, 64, 8, None, 16, 16, 256, 16, None) == 4       # workspace

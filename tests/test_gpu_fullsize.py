@@ -9,7 +9,7 @@ import torch
 
 from bit_weight_only_lcvq_b200 import lcvq, synth
 from oracle import lcvq_oracle as O
-from tests.gpu_util import TOL_BF16, assert_close, dev
+from tests.gpu_util import TOL_BF16, assert_close, dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -115,3 +115,24 @@ def test_stack_matrices(M):
                       torch.from_numpy(m["A"]).to(dev()), torch.from_numpy(m["B"]).to(dev()), 8)
         pairs = _pairs(7 + proj, M, m["d_out"], 128)
         _check_sampled_forward(Y, m["X"], z, m["A"], m["B"], pairs, f"stack {m['proj']} M={M}")
+
+
+def test_fit_affine_full_size_qat_matrix():
+    """Refit on the QAT-step matrix (4096 x 14336, d = 8): W0 = A0 z + B0 plus
+    noise; the GPU fit matches the oracle, and recovers (A0, B0) closely."""
+    d, N, K = 8, 4096, 14336
+    g = np.random.Generator(np.random.PCG64(1300))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A0, B0 = synth.affine_diag_dominant(d, g)
+    W0 = O.decode(z, A0, B0)
+    W0 += 0.005 * g.standard_normal((N, K))
+    W0 = W0.astype(np.float32)
+    h = g.uniform(0.5, 2.0, size=K).astype(np.float32)
+    A_ref, B_ref = O.fit_affine(W0.astype(np.float64), z, d, h.astype(np.float64))
+    A, B = lcvq.fit_affine(torch.from_numpy(W0).to(dev()), torch.from_numpy(O.pack_codes(z)).to(dev()),
+                           d, h=torch.from_numpy(h).to(dev()))
+    from tests.test_gpu_parity import _fit_bound, _fit_ok
+    assert _fit_ok(A, B, A_ref, B_ref, _fit_bound(W0.astype(np.float64), z, d, h.astype(np.float64),
+                                                  A_ref, B_ref))
+    ref = np.concatenate([A_ref.ravel(), B_ref.ravel()])
+    assert np.max(np.abs(ref - np.concatenate([A0.ravel(), B0.ravel()]))) < 1e-3

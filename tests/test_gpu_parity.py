@@ -347,3 +347,66 @@ def test_gemm_grouped_wide_tiles_bitwise_equal_separate_calls(M):
         assert torch.equal(Y, Y1), f"item {i}"
     ref, D = O.forward(ws[9]["X"], zs[9], ws[9]["A"], ws[9]["B"])
     assert_close(f"wide grouped ragged item M={M}", to_np(Ys[9]), ref, D, TOL_BF16)
+
+
+# --------------------------------------------- least-squares refit of (A, B)
+# Error bound of the GPU fit.  Its per-lane sums run in fp32 and are flushed
+# into fp64 every 16 terms, each term carrying at most 2 roundings, so an entry
+# of R (and of G when weighted; unweighted G is an exact integer count) is off
+# by at most 18 * 2^-24 of the sum of its terms' absolute values.  To first
+# order, theta = G^+ R moves by |G^+| (|dR| + |dG| |theta|); the result is then
+# rounded to fp32 (2^-24 relative).  The oracle supplies G, R and the
+# absolute-term sums, so the bound is computed, not guessed.
+def _fit_bound(W0, z, d, h, A_ref, B_ref):
+    G, R = O.fit_affine_normal(np.abs(W0), z, d, h)   # G's terms are >= 0: G is its own |sum|
+    th = np.concatenate([A_ref, B_ref[:, None]], axis=1)   # [d][d+1]
+    eps = 18 * 2.0 ** -24
+    bnd = np.zeros_like(th)
+    for i in range(d):
+        dR = eps * R[i]
+        dG = eps * G[i] if h is not None else 0.0 * G[i]
+        Pinv = np.abs(np.linalg.pinv(G[i], rcond=O.PINV_RCOND, hermitian=True))
+        bnd[i] = Pinv @ (dR + dG @ np.abs(th[i])) + 2.0 ** -24 * np.abs(th[i])
+    return bnd + 1e-12 * np.max(np.abs(th))
+
+
+def _fit_ok(got_A, got_B, A, B, bound) -> bool:
+    got = np.concatenate([to_np(got_A), to_np(got_B)[:, None]], axis=1)
+    ref = np.concatenate([np.asarray(A, np.float64), np.asarray(B, np.float64)[:, None]], axis=1)
+    return bool(np.all(np.abs(got - ref) <= bound))
+
+
+@pytest.mark.parametrize("d", [1, 2, 4, 8])
+@pytest.mark.parametrize("weighted", [False, True])
+def test_fit_affine_matches_oracle(d, weighted):
+    """GPU refit against the oracle's normal equations + pseudo-inverse, on a
+    ragged shape (rows and vectors not multiples of the warp's vector count)."""
+    g = np.random.Generator(np.random.PCG64(1100 + 10 * d + weighted))
+    N, K = 77, 16 * 13
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A0, B0 = synth.affine_diag_dominant(d, g)
+    W0 = (O.decode(z, A0, B0) + 0.01 * g.standard_normal((N, K))).astype(np.float32)
+    h = g.uniform(0.1, 3.0, size=K).astype(np.float32) if weighted else None
+    A_ref, B_ref = O.fit_affine(W0.astype(np.float64), z, d, None if h is None else h.astype(np.float64))
+    A, B = lcvq.fit_affine(torch.from_numpy(W0).to(dev()), torch.from_numpy(O.pack_codes(z)).to(dev()),
+                           d, h=None if h is None else torch.from_numpy(h).to(dev()))
+    hb = None if h is None else h.astype(np.float64)
+    assert _fit_ok(A, B, A_ref, B_ref, _fit_bound(W0.astype(np.float64), z, d, hb, A_ref, B_ref))
+
+
+def test_fit_affine_singular_and_empty_and_deterministic():
+    g = np.random.Generator(np.random.PCG64(1200))
+    d, N, K = 8, 64, 256
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    z[:, 5::d] = 1                                   # position 5 never varies: G singular
+    W0 = g.standard_normal((N, K)).astype(np.float32)
+    A_ref, B_ref = O.fit_affine(W0.astype(np.float64), z, d)
+    Wt, Pt = torch.from_numpy(W0).to(dev()), torch.from_numpy(O.pack_codes(z)).to(dev())
+    A1, B1 = lcvq.fit_affine(Wt, Pt, d)
+    A2, B2 = lcvq.fit_affine(Wt, Pt, d)
+    torch.cuda.synchronize()
+    assert torch.equal(A1, A2) and torch.equal(B1, B2)
+    assert _fit_ok(A1, B1, A_ref, B_ref, _fit_bound(W0.astype(np.float64), z, d, None, A_ref, B_ref))
+    Ae, Be = lcvq.fit_affine(torch.zeros((0, K), device=dev()),
+                             torch.zeros((0, K // 4), dtype=torch.uint8, device=dev()), d)
+    assert torch.count_nonzero(Ae) == 0 and torch.count_nonzero(Be) == 0

@@ -599,9 +599,12 @@ def row_stack(D, pk, layers=32, ms=(1, 8, 32)):
         seq_last = {p: ys[p].clone() for p, _, _ in synth.STACK_PROJS}
         run_all()
         torch.cuda.synchronize()
-        res_m["grouped_equals_sequential"] = all(
-            torch.equal(all_outs[len(dmats) - len(synth.STACK_PROJS) + i], seq_last[p])
-            for i, (p, _, _) in enumerate(synth.STACK_PROJS))
+        pairs_ = [(all_outs[len(dmats) - len(synth.STACK_PROJS) + i], seq_last[p])
+                  for i, (p, _, _) in enumerate(synth.STACK_PROJS)]
+        res_m["grouped_vs_sequential"] = dict(
+            bitwise_equal=all(torch.equal(a, b) for a, b in pairs_),
+            max_rel_diff=max(float((a.float() - b.float()).abs().max() / b.float().abs().max())
+                             for a, b in pairs_))
         out[str(M)] = res_m
         del all_ws, all_outs, ph_ws
         torch.cuda.empty_cache()

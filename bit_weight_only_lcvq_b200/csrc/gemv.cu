@@ -796,9 +796,6 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
 #ifndef LCVQ_WS2
 #define LCVQ_WS2 6
 #endif
-#ifndef LCVQ_WS4
-#define LCVQ_WS4 4
-#endif
 
 // code-ring depth (chunks per warp) per token-tile count
 #ifndef LCVQ_GS1
@@ -928,9 +925,13 @@ cudaError_t launch_wide_t(const GemvWideGroup<kItems>& grp, cudaStream_t s) {
 
 cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaStream_t s,
                                 int* launches, unsigned int* err) {
-  // enough 128-row tiles to fill the device: the wide-tile kernel
+  // enough 128-row tiles to fill the device: the wide-tile kernel (M <= 16)
   int64_t wide_tiles = 0;
   for (int i = 0; i < count; ++i) wide_tiles += ceil_div(jobs[i].d_out, kWideRows);
+  // 17..32 tokens: the tcgen05 form (four token tiles of mma.sync cost more
+  // than the tensor cores' A-operand streaming rate)
+  if (M > 16 && wide_tiles >= LCVQ_WIDE_MIN_TILES && gemv_tc_usable(M))
+    return launch_gemv_tc_grouped(jobs, count, M, err, s, launches);
   if (wide_tiles >= LCVQ_WIDE_MIN_TILES) {
     for (int first = 0; first < count; first += kMaxGroupItems) {
       const int n = count - first < kMaxGroupItems ? count - first : kMaxGroupItems;
@@ -949,9 +950,8 @@ cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaS
                                 kAhead * 32, kWideRows, true))
           return cudaErrorInvalidValue;
       }
-      cudaError_t e = M <= 8    ? launch_wide_t<1, LCVQ_WS1, 2, kMaxGroupItems>(grp, s)
-                      : M <= 16 ? launch_wide_t<2, LCVQ_WS2, 1, kMaxGroupItems>(grp, s)
-                                : launch_wide_t<4, LCVQ_WS4, 1, kMaxGroupItems>(grp, s);
+      cudaError_t e = M <= 8 ? launch_wide_t<1, LCVQ_WS1, 2, kMaxGroupItems>(grp, s)
+                             : launch_wide_t<2, LCVQ_WS2, 1, kMaxGroupItems>(grp, s);
       ++*launches;
       if (e != cudaSuccess) return e;
       if ((e = cudaGetLastError()) != cudaSuccess) return e;

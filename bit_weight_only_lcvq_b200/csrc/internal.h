@@ -48,8 +48,9 @@ struct XformJob {
 
 // decode-GEMV over a group of matrices with a common token count M <= 32, in
 // persistent launches of up to kMaxGroupItems matrices each (X'' and corr of
-// every matrix already formed by launch_xform or launch_xform_grouped).  Each
-// matrix's Y is bit-identical to launch_gemv on that matrix alone.
+// every matrix already formed by launch_xform or launch_xform_grouped).  For
+// M <= 16 each matrix's Y is bit-identical to launch_gemv on that matrix
+// alone; large groups with 17 <= M <= 32 run on the tcgen05 form below.
 struct GemvJob {
   const uint8_t* packed;
   const uint16_t* Xpp;
@@ -62,6 +63,11 @@ cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaS
                                 int* launches, unsigned int* err);
 cudaError_t launch_xform_grouped(const XformJob* jobs, int count, int64_t M, int d,
                                  cudaStream_t s, int* launches);
+// the same on the tcgen05 tensor cores (weights in TMEM as the MMA's A
+// operand, tokens as N = 32): launches of up to 48 matrices
+bool gemv_tc_usable(int64_t M);
+cudaError_t launch_gemv_tc_grouped(const GemvJob* jobs, int count, int64_t M, unsigned int* err,
+                                   cudaStream_t s, int* launches);
 
 // integer-code GEMM on X'' (dispatches on M: decode-GEMV for M <= 32, else
 // the tcgen05 GEMM); err may be null (no device error word)

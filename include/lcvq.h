@@ -157,8 +157,12 @@ LCVQ_API lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64
  * pages define the operation per matrix (Methodology 3; decoupleQ eq. (1) for
  * the layer convention); grouping is this library's launch arrangement for
  * many matrices at once (the projections of a layer that read one input, the
- * experts of a layer, or any set of independent decode-time matmuls).  Each
- * Y_i is bit-identical to lcvq_gemm on item i alone.
+ * experts of a layer, or any set of independent decode-time matmuls).  For
+ * M <= 16 each Y_i is bit-identical to lcvq_gemm on item i alone.  For
+ * 17 <= M <= 32, groups of at least 296 tiles of 128 rows run on the tcgen05
+ * tensor cores (decoded weights in tensor memory) and sum in a different fp32
+ * order: Y_i then agrees with lcvq_gemm within the forward tolerance, not
+ * bitwise.
  *   items  host array of `count` descriptors (read during the call only):
  *          X [M][d_in] bf16, packed [d_out][d_in/4] codes, A [d*d] and B [d]
  *          fp32, Y [M][d_out] bf16 out; every pointer 16-byte aligned.

@@ -410,3 +410,22 @@ def test_fit_affine_singular_and_empty_and_deterministic():
     Ae, Be = lcvq.fit_affine(torch.zeros((0, K), device=dev()),
                              torch.zeros((0, K // 4), dtype=torch.uint8, device=dev()), d)
     assert torch.count_nonzero(Ae) == 0 and torch.count_nonzero(Be) == 0
+
+
+@pytest.mark.parametrize("M", [17, 32])
+def test_gemm_grouped_tcgen05_form_matches_oracle(M):
+    """Large groups with 17..32 tokens run on the tcgen05 tensor cores (decoded
+    weights in TMEM, tokens as the MMA's N): within the forward tolerance of the
+    oracle, and of separate lcvq_gemm calls, including a ragged row count and a
+    K that ends inside a code chunk."""
+    shapes = [(4096, 4096)] * 9 + [(1088, 1000), (11008, 4096)]
+    jobs, zs, ws = _group_case(shapes, M, 1400 + M)
+    wsb = lcvq.new_workspace(lcvq.workspace_size_grouped(jobs, M, 8))
+    Ys = lcvq.gemm_grouped(jobs, 8, workspace=wsb)
+    assert lcvq.check_device_error(wsb) == 0
+    for i in (0, 9, 10):
+        Xr = to_np(jobs[i][0])
+        ref, D = O.forward(Xr, zs[i], ws[i]["A"], ws[i]["B"])
+        assert_close(f"tcgen05 grouped item {i} M={M}", to_np(Ys[i]), ref, D, TOL_BF16)
+        Y1 = lcvq.gemm(*jobs[i][:2], jobs[i][4], jobs[i][2], jobs[i][3], 8)
+        assert_close(f"tcgen05 grouped vs single item {i} M={M}", to_np(Ys[i]), to_np(Y1), D, TOL_BF16)

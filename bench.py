@@ -65,7 +65,7 @@ NCU_TRAFFIC = {
     # source file -> (sha1 of the file when captured, {token count: bytes per launch})
     # profiles/launches_decode_gemv_bench.md: M = 1 and 4 share gemv_group_kernel<1, ...>
     "bit_weight_only_lcvq_b200/csrc/gemv.cu": (
-        "9c29dab4f5a6019c8c4c5ebf9f818537dbeaa76e", {1: 4238969, 4: 4238969, 16: 4369947}),
+        "ded1d22b87e7eb46196a4d3c3d218586dd1620b3", {1: 4238924, 4: 4238924, 16: 4369934}),
 }
 
 

@@ -1,26 +1,29 @@
 // Decode-GEMV for few tokens (M <= 32): Y = X W~ with W~ = A z + B streamed as
 // packed 2-bit codes (LC-QAT technical summary, Methodology 3: the forward runs
-// on INT2 x FP16 matmul operators).
+// on INT2 x FP16 matmul operators), one matrix or a group of matrices.
 //
-// The kernel multiplies the transformed activations X'' (see xform.cu) with the
-// raw codes on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+// Both kernels here multiply the transformed activations X'' (see xform.cu)
+// with the raw codes on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
+// accumulate):
 //   * weights are the 16-row A operand, tokens the 8-column B operand, so a
 //     weight tile is decoded once and serves every token;
-//   * codes go from HBM straight into registers (one 128-bit load per row and
-//     lane per 256 codes) and are decoded by a single LOP3 per bf16 pair:
+//   * codes are decoded in registers by a single LOP3 per bf16 pair:
 //     (word >> s) & 0x00030003 << 2p | 0x43004300 = bf16x2(128 + 4^p z_lo,
 //     128 + 4^p z_hi); the power of two and the 128 offset are folded into X''
 //     and the per-row constant `corr`, so decoding costs no float arithmetic;
 //   * the MMA's logical k of each lane is mapped onto the lane's own code
 //     words (the decoder order of X'' makes the B fragments contiguous loads);
-//   * a CTA owns 16 R rows over the whole K (8 warps split K, fixed-order
-//     shared-memory sum), so no partial sum leaves the CTA and the result is
-//     deterministic;
+//   * K is cut into chunks of 512 codes; warp w of 8 sums chunks w, w + 8, ...
+//     and the 8 partial sums are added in warp order, so every path gives the
+//     same bits for a matrix;
 //   * programmatic dependent launch: the code loads do not depend on the
 //     X-transform, so they are issued before griddepcontrol.wait and stream
-//     while the prologue runs.  The kernel touches nothing else before the
+//     while the prologue runs.  The kernels touch nothing else before the
 //     wait, and the X-transform waits for every earlier kernel before it lets
-//     this one launch, so the early reads never race a producer of the codes.
+//     them launch, so the early reads never race a producer of the codes.
+// gemv_group_kernel (split K, cp.async code rings) serves single matrices and
+// small groups; gemv_wide_kernel (128-row tiles, TMA producer warp) serves
+// large groups; gemv_tc.cu holds the tcgen05 form for 17..32 tokens.
 
 #include <map>
 #include <mutex>
@@ -75,204 +78,15 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
   return q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
 }
 
-// CTA: kWarps warps on 16 R weight rows over the whole K, so no partial sum
-// leaves the CTA.  Warp w takes K slice w.  A "unit" is 128 codes of each of the
-// CTA's rows: lane (g, t) holds 2 words of rows g and g + 8 of every row
-// block (8 B each); a warp keeps up to kAhead units of loads in flight.
-// Launch order with the X-transform (programmatic dependent launch): the code
-// loads are issued before griddepcontrol.wait, so they overlap the prologue;
-// X'' and corr are read only after it.
-constexpr int kUnit = 128;  // codes per row per unit (32 B)
+// A "unit" is 128 codes of a row (32 bytes); a chunk is kAhead units.
+constexpr int kUnit = 128;
 constexpr int kAhead = 4;
 
-__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];\n"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
-  return v;
-}
 __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
 }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
-
-// kPrefX: keep the next unit's X'' fragments in flight (costs registers);
-// kMinBlocks: CTAs per SM the register budget must allow.
-template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks>
-__global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
-    gemv_kernel(const uint16_t* __restrict__ Xpp, const float* __restrict__ corr, int M,
-                const uint8_t* __restrict__ packed, int64_t N, int64_t K,
-                uint16_t* __restrict__ Y) {
-  constexpr int MP = NT * 8;
-  constexpr int ROWS = 16 * R;
-  __shared__ float part[kWarps][ROWS][MP + 1];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int64_t row0 = int64_t(blockIdx.x) * ROWS;
-  const int64_t Kb = K / 4;
-  const int64_t nunits = ceil_div(K, kUnit);
-  const int64_t u0 = nunits * warp / kWarps, u1 = nunits * (warp + 1) / kWarps;
-
-  const uint8_t* rowp[R][2];
-  bool rowok[R][2];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t row = row0 + r * 16 + g + 8 * h;
-      rowok[r][h] = row < N;
-      rowp[r][h] = packed + (rowok[r][h] ? row : 0) * Kb + 8 * t;
-    }
-
-  auto load_unit = [&](int64_t u, uint2 (&cw)[R][2]) {
-    const bool kok = u < u1 && u * kUnit + 32 * t < K;  // K % 64 == 0: whole lane chunks
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        cw[r][h] = (kok && rowok[r][h]) ? ld_stream_v2(rowp[r][h] + u * 32) : make_uint2(0, 0);
-  };
-
-  uint2 ring[kAhead][R][2];
-#pragma unroll
-  for (int j = 0; j < kAhead; ++j) load_unit(u0 + j, ring[j]);
-
-  griddep_wait();  // X'' and corr written by the X-transform are visible from here
-
-  const uint16_t* xrow[NT];
-  bool tokok[NT];
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const int tok = n * 8 + g;
-    tokok[n] = tok < M;
-    xrow[n] = Xpp + int64_t(tokok[n] ? tok : 0) * K + 32 * t;
-  }
-
-  float acc[R][NT][4];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[r][n][e] = 0.f;
-
-  // X'' fragments of one unit: word q, token tile n -> two 16-byte halves
-  auto load_x = [&](int64_t u, uint4 (&xb)[2][NT][2]) {
-    const bool kok = u < u1 && u * kUnit + 32 * t < K;
-#pragma unroll
-    for (int q = 0; q < 2; ++q)
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        if (kok && tokok[n]) {
-          const uint4* src = reinterpret_cast<const uint4*>(xrow[n] + u * kUnit + 16 * q);
-          xb[q][n][0] = __ldg(src);
-          xb[q][n][1] = __ldg(src + 1);
-        } else {
-          xb[q][n][0] = make_uint4(0, 0, 0, 0);
-          xb[q][n][1] = make_uint4(0, 0, 0, 0);
-        }
-      }
-  };
-  uint4 xcur[2][NT][2], xnxt[2][NT][2];
-  load_x(u0, xcur);
-
-  for (int64_t base = u0; base < u1; base += kAhead) {
-#pragma unroll
-    for (int j = 0; j < kAhead; ++j) {
-      const int64_t u = base + j;
-      if (u >= u1) break;
-      if constexpr (kPrefX) load_x(u + 1, xnxt);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {  // word q of each row: 16 codes, 4 k16 tiles
-        uint32_t w0[R][2], w6[R][2], w12[R][2];
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            w0[r][h] = q == 0 ? ring[j][r][h].x : ring[j][r][h].y;
-            w6[r][h] = w0[r][h] >> 6;
-            w12[r][h] = w0[r][h] >> 12;
-          }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {  // k16 tile: pairs 2jj, 2jj+1 of word q
-          uint32_t a[R][2][2];
-#pragma unroll
-          for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              a[r][h][0] = dec_pair_rt(2 * jj, w0[r][h], w6[r][h], w12[r][h]);
-              a[r][h][1] = dec_pair_rt(2 * jj + 1, w0[r][h], w6[r][h], w12[r][h]);
-            }
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const uint32_t b0 = word_of(xcur[q][n][jj >> 1], (2 * jj) & 3);
-            const uint32_t b1 = word_of(xcur[q][n][jj >> 1], (2 * jj + 1) & 3);
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-              mma_bf16_16816(acc[r][n], a[r][0][0], a[r][1][0], a[r][0][1], a[r][1][1], b0, b1);
-          }
-        }
-      }
-      load_unit(u + kAhead, ring[j]);  // refill the slot just consumed
-      if constexpr (kPrefX) {
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            xcur[q][n][0] = xnxt[q][n][0];
-            xcur[q][n][1] = xnxt[q][n][1];
-          }
-      } else {
-        load_x(u + 1, xcur);
-      }
-    }
-  }
-
-  // every CTA has passed its main loop: the next kernel may start launching
-  griddep_launch_dependents();
-
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int lr = r * 16 + g;
-      const int tk = n * 8 + 2 * t;
-      part[warp][lr][tk] = acc[r][n][0];
-      part[warp][lr][tk + 1] = acc[r][n][1];
-      part[warp][lr + 8][tk] = acc[r][n][2];
-      part[warp][lr + 8][tk + 1] = acc[r][n][3];
-    }
-  __syncthreads();
-  // sum the 8 K slices in slice order, add the per-row constant, store
-  for (int e = threadIdx.x; e < ROWS * M; e += kWarps * 32) {
-    const int lr = e % ROWS, tok = e / ROWS;
-    const int64_t grow = row0 + lr;
-    float sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) sum += part[w][lr][tok];
-    if (grow < N) Y[int64_t(tok) * N + grow] = f32_to_bf16(sum + corr[tok]);
-  }
-}
-
-template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks>
-cudaError_t launch_gemv_t(const uint16_t* Xpp, const float* corr, int M, const uint8_t* packed,
-                          int64_t N, int64_t K, uint16_t* Y, cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(N, 16 * R)), 1, 1);
-  cfg.blockDim = dim3(kWarps * 32, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, R, kWarps, kPrefX, kMinBlocks>, Xpp, corr, M,
-                            packed, N, K, Y);
 }
 
 // ---------------------------------------------------------------------------
@@ -866,29 +680,16 @@ cudaError_t launch_group(const GemvGroup<kItems>& grp, cudaStream_t s) {
 
 }  // namespace
 
-#ifndef LCVQ_GEMV_GROUPED
-#define LCVQ_GEMV_GROUPED 1
-#endif
-
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
                         int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s,
                         int* launches) {
-  cudaError_t e;
-  const int m = static_cast<int>(M);
-  if (LCVQ_GEMV_GROUPED) {
-    GemvGroup<1> grp{};
-    grp.count = 1;
-    grp.M = m;
-    grp.item[0] = GemvItem{packed, Xpp, corr, Y, static_cast<int>(d_out), static_cast<int>(d_in),
-                           static_cast<int>(ceil_div(d_out, group_rows(M)))};
-    e = launch_group(grp, s);
-  } else if (M <= 8) {
-    e = launch_gemv_t<1, 1, 8, true, 2>(Xpp, corr, m, packed, d_out, d_in, Y, s);
-  } else if (M <= 16) {
-    e = launch_gemv_t<2, 2, 8, true, 1>(Xpp, corr, m, packed, d_out, d_in, Y, s);
-  } else {
-    e = launch_gemv_t<4, 2, 8, false, 1>(Xpp, corr, m, packed, d_out, d_in, Y, s);
-  }
+  // a single matrix is a group of one (the same kernel, so the same bits)
+  GemvGroup<1> grp{};
+  grp.count = 1;
+  grp.M = static_cast<int>(M);
+  grp.item[0] = GemvItem{packed, Xpp, corr, Y, static_cast<int>(d_out), static_cast<int>(d_in),
+                         static_cast<int>(ceil_div(d_out, group_rows(M)))};
+  cudaError_t e = launch_group(grp, s);
   ++*launches;
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

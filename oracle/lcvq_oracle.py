@@ -261,6 +261,47 @@ def backward_dwp_sampled(X, dY, mask_rows_fn, A, pairs):
 
 
 # --------------------------------------------------------------------------
+# DGE: a differentiable gradient estimator through the rounding (LC-QAT page,
+# Methodology 3: the backward approximates the discretization by a smooth,
+# differentiable curve instead of the straight-through estimator).  The pages
+# give no formula; this is the reading taken here (parity of the curve itself
+# is unpinned, only its limits are):
+#   phi_k(w) = floor(w) + 1/2 + tanh(k (frac(w) - 1/2)) / (2 tanh(k/2))  on [0, 3]
+# a staircase whose steps sit at the rounding points (frac = 1/2), equal to w
+# at the integers, tending to rint(w) as k -> inf and to w (the STE) as k -> 0.
+# Its derivative on [0, 3] is
+#   phi_k'(w) = k / (2 tanh(k/2)) * sech^2(k (frac(w) - 1/2)),
+# and 0 outside [0, 3] (the clamp), so that k -> 0 gives the STE mask exactly.
+# --------------------------------------------------------------------------
+def dge_phi(w, k):
+    """The smooth rounding curve phi_k on [0, 3] (clamped outside)."""
+    w = np.clip(np.asarray(w, dtype=np.float64), 0.0, 3.0)
+    fl = np.minimum(np.floor(w), 2.0)        # w = 3 belongs to the last step
+    f = w - fl
+    return fl + 0.5 + np.tanh(k * (f - 0.5)) / (2.0 * np.tanh(k / 2.0))
+
+
+def dge_derivative(Wp, k):
+    """phi_k'(Wp): the factor DGE puts where the STE puts the clamp mask."""
+    w = np.asarray(Wp, dtype=np.float64)
+    inside = (w >= 0.0) & (w <= 3.0)
+    fl = np.minimum(np.floor(np.where(inside, w, 0.0)), 2.0)
+    f = np.where(inside, w, 0.0) - fl
+    g = (k / (2.0 * np.tanh(k / 2.0))) / np.cosh(k * (f - 0.5)) ** 2
+    return np.where(inside, g, 0.0)
+
+
+def backward_dge_dwp(X, dY, z, Wp, A, k):
+    """dWp under DGE: the STE gradient A^T G per vector, times phi_k'(Wp) instead
+    of the clamp mask.  Returns (dWp, D) with D the normaliser of the STE dWp
+    scaled by |phi_k'|."""
+    ones = np.ones(z.shape, dtype=bool)
+    bw = backward(X, dY, z, ones, A, np.zeros(A.shape[0]))
+    s = dge_derivative(Wp, k)
+    return bw["dWp"] * s, bw["D_dWp"] * np.abs(s)
+
+
+# --------------------------------------------------------------------------
 # least-squares refit of the float part given the codes (decoupleQ page,
 # eq. (5): the layer objective tr{(W~ - W0)^T H (W~ - W0)}; section 3.3: with
 # the integer part fixed the float part is an unconstrained quadratic, solved

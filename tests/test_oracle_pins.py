@@ -373,6 +373,51 @@ def test_db_identity_at_any_size():
     assert np.allclose(bw["dB"], ident, rtol=1e-13, atol=1e-13)
 
 
+# ---------------------------------------------------------------- DGE (curve unpinned)
+def test_dge_small_k_limit_is_the_ste_mask():
+    """As k -> 0 the DGE factor tends to the STE's clamp mask (1 on [0, 3], 0
+    outside); checked with an explicit small-k expansion bound."""
+    w = np.array([-1.0, -1e-9, 0.0, 0.2, 0.5, 1.49, 1.5, 2.7, 3.0, 3.0001, 7.0])
+    k = 1e-3
+    g = O.dge_derivative(w, k)
+    mask = ((w >= 0) & (w <= 3)).astype(np.float64)
+    # k/(2 tanh(k/2)) = 1 + k^2/12 + ..., sech^2(k x) = 1 - k^2 x^2 + ...: |g - 1| <= k^2 inside
+    assert np.all(np.abs(g - mask) <= k * k)
+
+
+def test_dge_curve_is_a_staircase_through_the_integers():
+    """phi_k equals w at the integers, is continuous at them, steps at the
+    half-integers, and its derivative matches central differences of phi_k."""
+    for k in (0.5, 4.0, 20.0):
+        for n in (0.0, 1.0, 2.0, 3.0):
+            assert O.dge_phi(n, k) == pytest.approx(n, abs=1e-12)
+        for n in (1.0, 2.0):
+            assert O.dge_phi(n - 1e-12, k) == pytest.approx(O.dge_phi(n + 1e-12, k), abs=1e-9)
+        ws = np.linspace(0.01, 2.99, 97)
+        ws = ws[np.abs(ws - np.round(ws)) > 1e-3]
+        h = 1e-6
+        fd = (O.dge_phi(ws + h, k) - O.dge_phi(ws - h, k)) / (2 * h)
+        assert np.allclose(fd, O.dge_derivative(ws, k), rtol=1e-6, atol=1e-6)
+    # large k approaches rounding away from the steps
+    ws = np.array([0.2, 0.8, 1.3, 2.6])
+    assert np.allclose(O.dge_phi(ws, 200.0), np.rint(ws), atol=1e-12)
+
+
+def test_dge_backward_is_ste_times_the_factor():
+    """dWp under DGE equals the STE dWp (all mask bits set) scaled by phi_k'."""
+    g = np.random.Generator(np.random.PCG64(1500))
+    M, N, K, d = 3, 5, 16, 4
+    X = g.standard_normal((M, K))
+    dY = g.standard_normal((M, N))
+    Wp = g.uniform(-0.5, 3.5, size=(N, K))
+    z, _ = O.assign(Wp)
+    A = g.standard_normal((d, d))
+    dWp, _ = O.backward_dge_dwp(X, dY, z, Wp, A, 3.0)
+    bw = O.backward(X, dY, z, np.ones((N, K), bool), A, np.zeros(d))
+    assert np.allclose(dWp, bw["dWp"] * O.dge_derivative(Wp, 3.0), rtol=1e-13, atol=1e-13)
+    assert np.all(dWp[(Wp < 0) | (Wp > 3)] == 0)
+
+
 # ---------------------------------------------------------------- (A, B) refit
 def _fit_case(d, N, K, seed, noise=0.0):
     g = np.random.Generator(np.random.PCG64(seed))

@@ -2,6 +2,7 @@
 // Every entry point validates all of its arguments before it launches
 // anything, so a failing call has no side effect.
 #include <atomic>
+#include <cmath>
 #include <vector>
 #include <mutex>
 #include <set>
@@ -163,6 +164,18 @@ size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_ou
   if (op == LCVQ_OP_GEMM_BACKWARD) return bwd_ws(M, d_out, d_in, d).total;
   if (op == LCVQ_OP_FIT_AFFINE) return kWsHeaderBytes + fit_partials_bytes(d_out, d_in, d);
   return 0;
+}
+
+lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, float k, void* stream) {
+  g_last_launches = 0;
+  if (n < 0 || n % 4 != 0 || !(k > 0.f) || !std::isfinite(k)) return LCVQ_ERR_INVALID_ARG;
+  if (n == 0) return LCVQ_OK;
+  if (!dWp || !Wp) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(dWp) || !aligned16(Wp)) return LCVQ_ERR_ALIGNMENT;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  cudaError_t e = launch_dge_scale(dWp, Wp, n, k, static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
 }
 
 lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int64_t d_out, int64_t d_in,

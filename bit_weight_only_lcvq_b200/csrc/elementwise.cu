@@ -3,6 +3,8 @@
 // Both are streaming, HBM-bound kernels:
 //   assign_pack reads 4 B and writes 0.25 B (+0.125 B of mask) per weight;
 //   decode reads 0.25 B and writes 2 B (bf16) or 4 B (fp32) per weight.
+#include <math.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -176,6 +178,53 @@ cudaError_t launch_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, in
     case 4: decode_dispatch_bf<4>(codes, n_words, A, B, W, w_bf16, unsigned(blocks), s); break;
     default: decode_dispatch_bf<8>(codes, n_words, A, B, W, w_bf16, unsigned(blocks), s); break;
   }
+  ++*launches;
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// DGE rescale (LC-QAT technical summary, Methodology 3: a differentiable
+// gradient estimator through the rounding instead of the STE).  The pages give
+// no curve; the reading here is the tanh staircase
+//   phi_k(w) = floor(w) + 1/2 + tanh(k (frac(w) - 1/2)) / (2 tanh(k/2))  on [0, 3]
+// whose derivative k / (2 tanh(k/2)) sech^2(k (frac - 1/2)) replaces the STE's
+// clamp mask (0 outside [0, 3]; k -> 0 gives the mask back).  The STE
+// gradient inside the mask is A^T G, so dWp_DGE = dWp_STE * phi_k'(Wp).
+// 12 bytes per weight (dWp read and written, Wp read), float4 at a time.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float dge_factor(float w, float k, float ck) {
+  if (!(w >= 0.f && w <= 3.f)) return 0.f;
+  const float f = w - fminf(floorf(w), 2.f);
+  const float t = tanhf(k * (f - 0.5f));
+  return ck * (1.f - t * t);
+}
+
+__global__ void __launch_bounds__(256) dge_scale_kernel(float4* __restrict__ dWp,
+                                                        const float4* __restrict__ Wp,
+                                                        int64_t n4, float k, float ck) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const float4 w = __ldcs(Wp + i);
+    float4 g = __ldcs(dWp + i);
+    g.x *= dge_factor(w.x, k, ck);
+    g.y *= dge_factor(w.y, k, ck);
+    g.z *= dge_factor(w.z, k, ck);
+    g.w *= dge_factor(w.w, k, ck);
+    __stcs(dWp + i, g);
+  }
+}
+
+cudaError_t launch_dge_scale(float* dWp, const float* Wp, int64_t n, float k, cudaStream_t s,
+                             int* launches) {
+  const int64_t n4 = n / 4;
+  int64_t blocks = ceil_div(n4, 256);
+  const int64_t cap = int64_t(kNumSMsB200) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const double kd = k;
+  const float ck = static_cast<float>(kd / (2.0 * tanh(kd / 2.0)));
+  dge_scale_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      reinterpret_cast<float4*>(dWp), reinterpret_cast<const float4*>(Wp), n4, k, ck);
   ++*launches;
   return cudaGetLastError();
 }

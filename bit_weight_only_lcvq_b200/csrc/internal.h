@@ -20,6 +20,10 @@ cudaError_t launch_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, in
                           const float* A, const float* B, void* W, bool w_bf16,
                           cudaStream_t s, int* launches);
 
+// dWp[i] *= phi_k'(Wp[i]) (the DGE factor; 0 outside [0, 3]); n % 4 == 0
+cudaError_t launch_dge_scale(float* dWp, const float* Wp, int64_t n, float k, cudaStream_t s,
+                             int* launches);
+
 // ---- algebraic-form prologue (bf16 tensor-core paths) ----
 // Xpp[M][d_in] bf16: X' = group-wise X A, rounded to bf16, scaled by the
 // per-position power of two of the code decoder, in the decoder's K order.

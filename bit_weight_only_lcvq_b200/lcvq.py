@@ -40,6 +40,7 @@ EXPORTS = (
     "lcvq_gemv_static",
     "lcvq_gemm_grouped",
     "lcvq_fit_affine",
+    "lcvq_dge_scale",
     "lcvq_workspace_size",
     "lcvq_workspace_size_grouped",
     "lcvq_check_device_error",
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.lcvq_workspace_size_grouped.argtypes = [ctypes.POINTER(GemmItem), _i32, _i64, _i32]
         L.lcvq_workspace_size_grouped.restype = _sz
         L.lcvq_fit_affine.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.lcvq_dge_scale.argtypes = [_vp, _vp, _i64, ctypes.c_float, _vp]
         L.lcvq_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i64, _i32]
         L.lcvq_workspace_size.restype = _sz
         L.lcvq_check_device_error.argtypes = [_vp, _vp]
@@ -93,7 +95,8 @@ def lib() -> ctypes.CDLL:
         L.lcvq_status_string.restype = ctypes.c_char_p
         L.lcvq_last_launch_count.argtypes = []
         for fn in ("lcvq_assign_pack", "lcvq_decode", "lcvq_gemm", "lcvq_gemm_backward",
-                   "lcvq_xform", "lcvq_gemm_xformed", "lcvq_gemv_static", "lcvq_gemm_grouped", "lcvq_fit_affine",
+                   "lcvq_xform", "lcvq_gemm_xformed", "lcvq_gemv_static", "lcvq_gemm_grouped",
+                   "lcvq_fit_affine", "lcvq_dge_scale",
                    "lcvq_check_device_error",
                    "lcvq_last_launch_count"):
             getattr(L, fn).restype = ctypes.c_int
@@ -298,3 +301,11 @@ def fit_affine(W0: torch.Tensor, packed: torch.Tensor, d: int, *, h=None, worksp
         _ptr(W0), _ptr(packed), d_out, d_in, d, _ptr(h), _ptr(A), _ptr(B), _ptr(workspace),
         workspace.numel(), _stream(stream)))
     return A, B
+
+
+def dge_scale(dWp: torch.Tensor, Wp: torch.Tensor, k: float, *, stream=None) -> torch.Tensor:
+    """In place: dWp *= phi_k'(Wp), turning the STE gradient of gemm_backward into
+    the DGE gradient (see lcvq_dge_scale).  Returns dWp."""
+    _check("lcvq_dge_scale", lib().lcvq_dge_scale(_ptr(dWp), _ptr(Wp), dWp.numel(), float(k),
+                                                  _stream(stream)))
+    return dWp

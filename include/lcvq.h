@@ -233,6 +233,22 @@ LCVQ_API lcvq_status lcvq_gemm_backward(const void* X, const void* dY, lcvq_dtyp
                                void* dX, float* dA, float* dB, float* dWp,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* DGE rescale of the proxy-weight gradient (LC-QAT technical summary,
+ * Methodology 3: the paper's backward uses a differentiable gradient
+ * estimator (DGE), a smooth curve in place of the rounding, instead of the
+ * straight-through estimator).  The pages give no formula; this library takes
+ * the tanh staircase through the rounding points on [0, 3]
+ *     phi_k(w) = floor(w) + 1/2 + tanh(k (frac(w) - 1/2)) / (2 tanh(k/2)),
+ * equal to w at the integers, to rint(w) as k -> inf and to w as k -> 0, and
+ * multiplies the gradient by its derivative
+ *     phi_k'(w) = k / (2 tanh(k/2)) sech^2(k (frac(w) - 1/2))   (0 outside [0, 3]).
+ * Applied to the dWp of lcvq_gemm_backward (the STE gradient, A^T G inside the
+ * clamp mask) it gives the DGE gradient: dWp[i] *= phi_k'(Wp[i]).  As k -> 0
+ * the factor tends to the clamp mask, i.e. back to the STE.
+ *   dWp [n] fp32 in/out;  Wp [n] fp32 proxy weights;  k > 0 the sharpness.
+ * Shapes: n % 4 == 0, n >= 0; 16-byte aligned pointers. */
+LCVQ_API lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, float k, void* stream);
+
 /* Least-squares refit of the float part (A, B) given the codes (decoupleQ
  * page: eq. (5), the layer objective tr{(W~ - W0)^T H (W~ - W0)}, and section
  * 3.3, where the float part is solved in closed form with the integer part

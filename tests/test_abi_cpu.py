@@ -99,3 +99,13 @@ def test_fit_affine_rejects_bad_arguments_without_device():
     assert L.lcvq_fit_affine(16, 16, 8, 64, 8, None, None, 16, 256, 1 << 20, None) == 1  # no A
     assert L.lcvq_fit_affine(16, 16, 8, 64, 8, 8, 16, 16, 256, 1 << 20, None) == 3     # h misaligned
     assert L.lcvq_fit_affine(16, 16, 8, 64, 8, None, 16, 16, 256, 16, None) == 4       # workspace
+
+
+def test_dge_scale_rejects_bad_arguments_without_device():
+    L = lcvq.lib()
+    assert L.lcvq_dge_scale(16, 16, 6, 2.0, None) == 1            # n % 4
+    assert L.lcvq_dge_scale(16, 16, 8, 0.0, None) == 1            # k <= 0
+    assert L.lcvq_dge_scale(16, 16, 8, float("nan"), None) == 1   # k not finite
+    assert L.lcvq_dge_scale(None, 16, 8, 2.0, None) == 1
+    assert L.lcvq_dge_scale(8, 16, 8, 2.0, None) == 3             # misaligned
+    assert L.lcvq_dge_scale(None, None, 0, 2.0, None) == 0        # empty: no-op

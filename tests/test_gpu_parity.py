@@ -12,7 +12,7 @@ import torch
 
 from bit_weight_only_lcvq_b200 import lcvq, synth
 from oracle import lcvq_oracle as O
-from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, dev, to_dev, to_np
+from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, dev, to_dev, to_np, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -429,3 +429,18 @@ def test_gemm_grouped_tcgen05_form_matches_oracle(M):
         assert_close(f"tcgen05 grouped item {i} M={M}", to_np(Ys[i]), ref, D, TOL_BF16)
         Y1 = lcvq.gemm(*jobs[i][:2], jobs[i][4], jobs[i][2], jobs[i][3], 8)
         assert_close(f"tcgen05 grouped vs single item {i} M={M}", to_np(Ys[i]), to_np(Y1), D, TOL_BF16)
+
+
+# ------------------------------------------------------ DGE (curve is a reading)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("k", [0.01, 4.0])
+def test_dge_scale_matches_oracle(dtype, k):
+    """lcvq_gemm_backward's dWp rescaled by lcvq_dge_scale equals the oracle's
+    DGE gradient (STE gradient times phi_k'(Wp)) within the backward tolerance;
+    k = 0.01 is near the STE limit."""
+    w, z, mask, a = _bwd_case(4, 32, 256, 128, dtype)
+    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 256, a["A"], a["B"], 8)
+    Wp = torch.from_numpy(w["Wp"]).to(dev())
+    lcvq.dge_scale(out["dWp"], Wp, k)
+    ref, D = O.backward_dge_dwp(w["X"], w["dY"], z, w["Wp"], w["A"], k)
+    assert_close(f"dge k={k}", to_np(out["dWp"]), ref, D, tol_for(dtype))

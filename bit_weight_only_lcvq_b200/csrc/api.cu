@@ -64,6 +64,7 @@ lcvq_status check_device() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+constexpr int64_t kMaxGemmDim = int64_t(1) << 30;
 bool valid_d(int d) { return d == 1 || d == 2 || d == 4 || d == 8; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -203,7 +204,8 @@ static lcvq_status validate_gemm_shapes(lcvq_dtype dtype, int64_t M, int64_t d_o
   if (M < 0 || d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
   if (dtype != LCVQ_F32 && dtype != LCVQ_BF16) return LCVQ_ERR_INVALID_ARG;
   if (d_in % 64 != 0 || d_out % 8 != 0) return LCVQ_ERR_INVALID_ARG;
-  if (M > INT32_MAX) return LCVQ_ERR_INVALID_ARG;
+  // the GEMV kernels index rows and columns in 32 bits
+  if (M > INT32_MAX || d_out > kMaxGemmDim || d_in > kMaxGemmDim) return LCVQ_ERR_INVALID_ARG;
   return LCVQ_OK;
 }
 

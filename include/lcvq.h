@@ -122,8 +122,8 @@ LCVQ_API lcvq_status lcvq_decode(const uint8_t* packed, int64_t d_out, int64_t d
  *   GEMM), fp32 accumulation.  dtype F32: an fp32 CUDA-core path.
  *   form: see lcvq_form (F32 always uses DECODE).
  *   workspace: >= lcvq_workspace_size(LCVQ_OP_GEMM, ...) bytes, 256-byte aligned.
- * Shapes: d_in % 64 == 0, d_out % 8 == 0, M >= 0.  M == 0 or d_out == 0 is a
- * no-op; d_in == 0 writes Y = 0. */
+ * Shapes: d_in % 64 == 0, d_out % 8 == 0, M >= 0, d_in and d_out <= 2^30.
+ * M == 0 or d_out == 0 is a no-op; d_in == 0 writes Y = 0. */
 LCVQ_API lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M,
                       const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
                       const float* A, const float* B, void* Y, lcvq_form form,

@@ -109,3 +109,14 @@ def test_dge_scale_rejects_bad_arguments_without_device():
     assert L.lcvq_dge_scale(None, 16, 8, 2.0, None) == 1
     assert L.lcvq_dge_scale(8, 16, 8, 2.0, None) == 3             # misaligned
     assert L.lcvq_dge_scale(None, None, 0, 2.0, None) == 0        # empty: no-op
+
+
+def test_gemm_dimension_limits_without_device():
+    """Matrix dimensions above 2^30 are refused before anything runs (the GEMV
+    kernels index rows and columns in 32 bits)."""
+    L = lcvq.lib()
+    big = (1 << 30) + 64
+    assert L.lcvq_gemm(None, 1, 4, None, 8, big, 8, None, None, None, 0, None, 0, None) == 1
+    assert L.lcvq_gemm(None, 1, 4, None, big - 56, 64, 8, None, None, None, 0, None, 0, None) == 1
+    assert L.lcvq_gemm_backward(None, None, 1, 4, None, None, 8, big, 8, None, None, None,
+                                None, None, None, None, 0, None) == 1

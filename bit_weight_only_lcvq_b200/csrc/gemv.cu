@@ -495,6 +495,20 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
 
   // ------------------------------------------------------------ consumers
   const int g = lane >> 2, t = lane & 3;
+  // per-lane constants: the SW128 offset of this lane's 8 code bytes of unit j
+  // (16-byte chunk 2 j + t/2 of rows g, g + 8 sits at chunk ^ g), and the
+  // offset and validity of its X'' token rows
+  uint32_t coff[kAhead];
+#pragma unroll
+  for (int j = 0; j < kAhead; ++j)
+    coff[j] = static_cast<uint32_t>(((2 * j + (t >> 1)) ^ g) << 4) + ((t & 1) << 3);
+  uint32_t xoff[NT];
+  bool tokok[NT];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    tokok[n] = n * 8 + g < M;
+    xoff[n] = static_cast<uint32_t>((n * 8 + g) * kWideXPitch + 64 * t);
+  }
   int seq = 0, item = 0;
   for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G) {
     while (tile >= grp.item[item].tile_end) ++item;
@@ -529,24 +543,22 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
         const uint32_t st = sbase + s * L::kStageBytes;
         const uint32_t crow = st + (warp * 16 + g) * 128;  // rows g and g + 8: (row & 7) = g
         const uint32_t xst = st + L::kCodeBytes;
+        const int rem = K - c * (kAhead * kUnit);   // positions of K left from this chunk on
+        const int remt = rem - 32 * t;              // ... from this lane's first position on
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
-          const int64_t u = int64_t(c) * kAhead + j;
-          if (u * kUnit >= K) break;  // warp-uniform: past the end of K
-          const bool kok = u * kUnit + 32 * t < K;
-          // SW128: 16-byte chunk c16 of a row sits at c16 ^ (row & 7)
-          const uint32_t off = static_cast<uint32_t>(((2 * j + (t >> 1)) ^ g) << 4) + ((t & 1) << 3);
+          if (j * kUnit >= rem) break;  // warp-uniform: past the end of K
+          const bool kok = j * kUnit < remt;
           uint2 cw[2];
-          cw[0] = lds_v2(crow + off);
-          cw[1] = lds_v2(crow + 8 * 128 + off);
+          cw[0] = lds_v2(crow + coff[j]);
+          cw[1] = lds_v2(crow + 8 * 128 + coff[j]);
           uint4 xb[2][NT][2];
 #pragma unroll
           for (int q = 0; q < 2; ++q)
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-              const int tok = n * 8 + g;
-              if (kok && tok < M) {
-                const uint32_t xa = xst + tok * kWideXPitch + (j * kUnit + 32 * t + 16 * q) * 2;
+              if (kok && tokok[n]) {
+                const uint32_t xa = xst + xoff[n] + (j * kUnit + 16 * q) * 2;
                 xb[q][n][0] = lds_v4(xa);
                 xb[q][n][1] = lds_v4(xa + 16);
               } else {

@@ -219,19 +219,35 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
     cp_async_commit();
   };
   // X'' fragments of unit j of chunk c: word q, token tile n -> two 16-byte halves
-  auto load_x = [&](const Cur& c, int j, uint4 (&xb)[2][NT][2]) {
+  // X'' of a chunk for this lane: the start of its 32 positions in each token
+  // row, and how many positions of K remain from there (<= 0: none)
+  struct XPos {
+    const uint16_t* base[NT];
+    int remt;
+  };
+  bool tokok[NT];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) tokok[n] = n * 8 + g < M;
+  auto xpos = [&](const Cur& c) {
+    XPos p;
     const bool any = c.tile < T;
     const GemvItem& it = grp.item[any ? c.item : 0];
-    const int64_t u = int64_t(c.chunk) * kAhead + j;
-    const bool kok = any && u * kUnit + 32 * t < it.K;
+    const int64_t k0 = int64_t(c.chunk) * (kAhead * kUnit);
+    p.remt = any ? static_cast<int>(it.K - k0) - 32 * t : 0;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+      p.base[n] = it.Xpp + (tokok[n] ? int64_t(n * 8 + g) * it.K : 0) + k0 + 32 * t;
+    return p;
+  };
+  // X'' fragments of unit j: word q, token tile n -> two 16-byte halves
+  auto load_x = [&](const XPos& p, int j, uint4 (&xb)[2][NT][2]) {
+    const bool kok = j * kUnit < p.remt;
 #pragma unroll
     for (int q = 0; q < 2; ++q)
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        const int tok = n * 8 + g;
-        if (kok && tok < M) {
-          const uint4* src = reinterpret_cast<const uint4*>(it.Xpp + int64_t(tok) * it.K +
-                                                             u * kUnit + 32 * t + 16 * q);
+        if (kok && tokok[n]) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.base[n] + j * kUnit + 16 * q);
           xb[q][n][0] = __ldg(src);
           xb[q][n][1] = __ldg(src + 1);
         } else {
@@ -240,6 +256,11 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
         }
       }
   };
+  // this lane's code bytes of unit j in a stage row (SW128: chunk ^ (row & 7))
+  uint32_t coff[kAhead];
+#pragma unroll
+  for (int j = 0; j < kAhead; ++j)
+    coff[j] = static_cast<uint32_t>((((2 * j + (t >> 1)) ^ g) << 4) + ((t & 1) << 3));
 
   // prologue: the first kStages - 1 chunks (codes only: nothing here depends
   // on the kernels this one may overlap)
@@ -254,8 +275,9 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
 
   griddep_wait();  // X'' and corr written by the X-transform are visible from here
 
+  XPos pcur = xpos(cur), pnxt = xpos(nxt);
   uint4 xcur[2][NT][2], xnxt[2][NT][2];
-  load_x(cur, 0, xcur);
+  load_x(pcur, 0, xcur);
 
   int stage = 0;  // stage of cur
   int eitem = 0;  // item of the tile in the epilogue
@@ -278,23 +300,22 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
         issue(iss, s_iss);
         iss = advance(iss);
       }
-      const int Kc = grp.item[cur.item].K;
+      const int rem = pcur.remt + 32 * t;  // positions of K left from this chunk on
       const uint32_t sbase = ring + stage * kStageBytes;
 #pragma unroll
       for (int j = 0; j < kAhead; ++j) {
         if constexpr (kPrefX) {
-          if (j + 1 < kAhead) load_x(cur, j + 1, xnxt);
-          else load_x(nxt, 0, xnxt);
+          if (j + 1 < kAhead) load_x(pcur, j + 1, xnxt);
+          else load_x(pnxt, 0, xnxt);
         }
-        if ((int64_t(cur.chunk) * kAhead + j) * kUnit < Kc) {  // warp-uniform
+        if (j * kUnit < rem) {  // warp-uniform
           // this lane's two code words of unit j for rows r*16 + g + 8h
           uint2 cw[R][2];
-          const int c16 = 2 * j + (t >> 1);
-          const uint32_t off = static_cast<uint32_t>(((c16 ^ g) << 4) + ((t & 1) << 3));
 #pragma unroll
           for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) cw[r][h] = lds_v2(sbase + (r * 16 + g + 8 * h) * 128 + off);
+            for (int h = 0; h < 2; ++h)
+              cw[r][h] = lds_v2(sbase + (r * 16 + g + 8 * h) * 128 + coff[j]);
 #pragma unroll
           for (int q = 0; q < 2; ++q) {  // word q of each row: 16 codes, 4 k16 tiles
             uint32_t w0[R][2], w6[R][2], w12[R][2];
@@ -337,12 +358,14 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
               xcur[q][n][1] = xnxt[q][n][1];
             }
         } else {
-          if (j + 1 < kAhead) load_x(cur, j + 1, xcur);
-          else load_x(nxt, 0, xcur);
+          if (j + 1 < kAhead) load_x(pcur, j + 1, xcur);
+          else load_x(pnxt, 0, xcur);
         }
       }
       cur = nxt;
+      pcur = pnxt;
       nxt = advance(nxt);
+      pnxt = xpos(nxt);
       if (++stage == kStages) stage = 0;
     }
 

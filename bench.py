@@ -65,7 +65,7 @@ NCU_TRAFFIC = {
     # source file -> (sha1 of the file when captured, {token count: bytes per launch})
     # profiles/launches_decode_gemv_bench.md: M = 1 and 4 share gemv_group_kernel<1, ...>
     "bit_weight_only_lcvq_b200/csrc/gemv.cu": (
-        "ded1d22b87e7eb46196a4d3c3d218586dd1620b3", {1: 4238924, 4: 4238924, 16: 4369934}),
+        "5016dd5597b05501b2883e20d2dbeb24c777ddc9", {1: 4237173, 4: 4237173, 16: 4366684}),
 }
 
 

@@ -26,7 +26,9 @@ Sources (cited below by these short names):
   ``W~`` of shape ``d_in x d_out``; eq. (3)/(4) are the scalar
   round/clip/affine special case used as a pin; eq. (5) and section 3.3 (the
   float part solved in closed form with the integer part fixed) define the
-  least-squares refit of (A, B).
+  least-squares refit of (A, B); eq. (6)-(11) (the integer part solved one
+  element at a time, the rest re-solved without the integer constraint) define
+  the H-aware sequential code assignment.
 
 Readings where the pages are silent (each one is listed in the design doc):
 
@@ -350,6 +352,100 @@ def fit_objective(W0, z, A, B, h=None) -> float:
     r = np.asarray(W0, dtype=np.float64) - decode(z, A, B)
     hh = np.ones(r.shape[1]) if h is None else np.asarray(h, dtype=np.float64)
     return float(np.sum(hh[None, :] * r * r))
+
+
+# --------------------------------------------------------------------------
+# H-aware sequential code assignment: the PTQ initialisation of the codes
+# (LC-QAT page, Methodology 2: the initial integer weights come from LDLQ,
+# which quantizes column by column and compensates the reconstruction error
+# of the columns already fixed; decoupleQ page, section 3.3, eq. (8)-(11):
+# round and clip one element, then re-solve the remaining elements of the
+# quadratic objective (7) with the integer constraint and the box dropped,
+# the second approximation, eq. (11)).
+#
+# In LC-VQ terms the integer part of one weight row is its code vector z and
+# the decoded row is Abar z + bbar (Abar = blockdiag(A, .., A), bbar = B
+# repeated per vector), so objective (7) of a row with target w0 is
+#     g(z) = 1/2 (Abar z + bbar - w0)^T H (Abar z + bbar - w0)
+#          = 1/2 (z - p)^T Q (z - p),   Q = Abar^T H Abar,  p = Abar^-1 (w0 - bbar),
+# p being the row's continuous code-space target (what the proxy weight W_p
+# holds).  With Q factored as (I + U) diag(D) (I + U)^T, U strictly upper
+# triangular,
+#     g(z) = 1/2 sum_k D_k ((z_k - p_k) + sum_{i<k} U[i, k] (z_i - p_i))^2,
+# so once z_0 .. z_{j-1} are fixed the minimiser of eq. (11) over the rest
+# zeroes every bracket k >= j, and its j-th element is
+#     t_j = p_j + sum_{i<j} U[i, j] (p_i - z_i).
+# Element j then takes z_j = clamp(rint(t_j), 0, 3), the rounding and clamping
+# of the assignment step (with Q diagonal, U = 0 and this is that step).
+# --------------------------------------------------------------------------
+def code_space_hessian(H: np.ndarray, A: np.ndarray) -> np.ndarray:
+    """Q = Abar^T H Abar for a K x K input Hessian H and the d x d matrix A:
+    Q[g d + a, h d + b] = sum_{i,j} A[i, a] H[g d + i, h d + j] A[j, b]."""
+    H = np.asarray(H, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    K = H.shape[0]
+    d = A.shape[0]
+    Abar = np.kron(np.eye(K // d), A)
+    return Abar.T @ H @ Abar
+
+
+def code_targets(W0: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """p = Abar^-1 (w0 - bbar) per row: each length-d vector solved against A."""
+    W0 = np.asarray(W0, dtype=np.float64)
+    N, K = W0.shape
+    d = A.shape[0]
+    r = (W0.reshape(N, K // d, d) - np.asarray(B, dtype=np.float64)[None, None, :])
+    sol = np.linalg.solve(np.asarray(A, dtype=np.float64), r.reshape(-1, d).T).T
+    return sol.reshape(N, K)
+
+
+def ldl_upper(Q: np.ndarray):
+    """Q = (I + U) diag(D) (I + U)^T with U strictly upper triangular.  This is
+    the Cholesky factorisation of Q with rows and columns reversed: if
+    J Q J = C C^T (C lower), then V = J C J is upper triangular with
+    Q = V V^T, and U = V diag(1 / diag V) - I, D = diag(V)^2.
+    Returns (U, D)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    C = np.linalg.cholesky(Q[::-1, ::-1])
+    V = C[::-1, ::-1]
+    v = np.diag(V).copy()
+    U = V / v[None, :] - np.eye(Q.shape[0])
+    return np.triu(U, 1), v * v
+
+
+def ldlq_assign(P: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """Codes Z (u8, N x K) of the sequential rule above, every row of the
+    targets P (N x K) on its own, elements in increasing k.  Only the strictly
+    upper triangle of U (K x K) is used."""
+    P = np.asarray(P, dtype=np.float64)
+    Ut = np.triu(np.asarray(U, dtype=np.float64), 1)
+    N, K = P.shape
+    Z = np.zeros((N, K), dtype=np.uint8)
+    E = np.zeros((N, K))  # p_i - z_i of the elements already fixed
+    for j in range(K):
+        t = P[:, j] + E[:, :j] @ Ut[:j, j]
+        z = np.clip(np.rint(t), 0, CODE_MAX)
+        Z[:, j] = z.astype(np.uint8)
+        E[:, j] = P[:, j] - z
+    return Z
+
+
+def ldlq_targets(P: np.ndarray, U: np.ndarray, Z: np.ndarray):
+    """The targets t_j that the rule rounds, given the codes Z that were chosen
+    (each t_j depends only on the codes before it), and the per-element sum of
+    the absolute values of its terms, |p_j| + sum_{i<j} |U[i, j] (p_i - z_i)|.
+    A code z_j is the rule's choice when it equals clamp(rint(t_j), 0, 3).
+    Returns (T, S)."""
+    P = np.asarray(P, dtype=np.float64)
+    Ut = np.triu(np.asarray(U, dtype=np.float64), 1)
+    E = P - np.asarray(Z, dtype=np.float64)
+    return P + E @ Ut, np.abs(P) + np.abs(E) @ np.abs(Ut)
+
+
+def ldlq_objective(P: np.ndarray, Q: np.ndarray, Z: np.ndarray) -> np.ndarray:
+    """g(z) = 1/2 (z - p)^T Q (z - p) for every row; returns a length-N array."""
+    R = np.asarray(Z, dtype=np.float64) - np.asarray(P, dtype=np.float64)
+    return 0.5 * np.einsum("nk,kl,nl->n", R, np.asarray(Q, dtype=np.float64), R)
 
 
 # --------------------------------------------------------------------------

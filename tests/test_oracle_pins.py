@@ -537,6 +537,171 @@ def test_fit_planted_mistake_is_caught():
     assert not np.allclose(th[:d], A[1], atol=1e-6)
 
 
+# ---------------------------------------------------------------- H-aware sequential assignment
+def _spd(g, K, n=None, ridge=0.05):
+    """A correlated symmetric positive definite K x K matrix: X^T X / n from
+    rows with a shared component, plus a ridge."""
+    n = n or 4 * K
+    X = g.standard_normal((n, K)) + 0.8 * g.standard_normal((n, 1))
+    return X.T @ X / n + ridge * np.eye(K)
+
+
+def _eq11_direct(p, Q):
+    """The pages' procedure written out for one row: fix element j by rounding
+    and clipping the j-th element of the continuous minimiser of
+    1/2 (z - p)^T Q (z - p) over the elements not fixed yet (a linear solve on
+    the sub-block of Q), then move on to j + 1."""
+    K = len(p)
+    z = np.zeros(K)
+    for j in range(K):
+        f, x = slice(j, K), slice(0, j)
+        y = p[f] - np.linalg.solve(Q[f, f], Q[f, x] @ (z[x] - p[x]))
+        z[j] = np.clip(np.rint(y[0]), 0, 3)
+    return z
+
+
+def test_ldl_upper_reconstructs_the_matrix():
+    g = np.random.Generator(np.random.PCG64(71))
+    Q = _spd(g, 12)
+    U, D = O.ldl_upper(Q)
+    I = np.eye(12)
+    assert np.array_equal(U, np.triu(U, 1))
+    assert np.all(D > 0)
+    assert np.allclose((I + U) @ np.diag(D) @ (I + U).T, Q, atol=1e-12)
+
+
+def test_ldlq_with_a_diagonal_hessian_is_round_and_clamp(golden_dir):
+    """Q diagonal: no compensation, the codes are those of the assignment step
+    (ties to even, clamping, the golden tie cases included)."""
+    g = np.random.Generator(np.random.PCG64(72))
+    rows = [ln.split() for ln in _read(golden_dir, "round_clamp_ties.txt")]
+    w = np.array([_f32(r[0]) for r in rows if np.isfinite(_f32(r[0]))], dtype=np.float64)
+    K = len(w)
+    P = np.stack([w, g.uniform(-0.5, 3.5, K), g.uniform(-2, 5, K)])
+    U, _ = O.ldl_upper(np.diag(g.uniform(0.1, 3.0, K)))
+    assert np.array_equal(U, np.zeros((K, K)))
+    assert np.array_equal(O.ldlq_assign(P, U), O.assign(P.astype(np.float32))[0])
+
+
+def test_ldlq_equals_the_eq11_procedure_solved_directly():
+    """The factor form gives the same codes as re-solving the remaining
+    elements with a linear solve at every step."""
+    g = np.random.Generator(np.random.PCG64(73))
+    for K in (1, 2, 5, 10):
+        Q = _spd(g, K)
+        U, _ = O.ldl_upper(Q)
+        P = g.uniform(-0.5, 3.5, size=(40, K))
+        Z = O.ldlq_assign(P, U)
+        for n in range(40):
+            assert np.array_equal(Z[n], _eq11_direct(P[n], Q)), (K, n)
+
+
+def test_ldlq_choice_is_the_best_code_by_exhaustive_search():
+    """At every step the chosen code minimises, over all four codes, the
+    objective with the earlier codes fixed and the later elements at their
+    continuous optimum."""
+    g = np.random.Generator(np.random.PCG64(74))
+    K = 7
+    Q = _spd(g, K)
+    U, _ = O.ldl_upper(Q)
+    P = g.uniform(-1.0, 4.0, size=(25, K))
+    Z = O.ldlq_assign(P, U)
+    for n in range(25):
+        p = P[n]
+        for j in range(K):
+            best, arg = np.inf, -1
+            for c in range(4):
+                z = np.concatenate([Z[n, :j].astype(np.float64), [c]])
+                r = slice(j + 1, K)
+                x = slice(0, j + 1)
+                rest = p[r] - np.linalg.solve(Q[r, r], Q[r, x] @ (z - p[x])) if j + 1 < K else p[r]
+                full = np.concatenate([z, rest]) - p
+                val = 0.5 * full @ Q @ full
+                if val < best:
+                    best, arg = val, c
+            assert Z[n, j] == arg, (n, j)
+
+
+def test_ldlq_equals_the_inverse_cholesky_error_feedback_form():
+    """The same codes from the other standard form of the update: after fixing
+    element j, subtract (t_j - z_j) / L[j, j] * L[j, >j] from the later targets,
+    with L^T L = Q^-1 and L upper triangular."""
+    g = np.random.Generator(np.random.PCG64(75))
+    K = 24
+    Q = _spd(g, K)
+    U, _ = O.ldl_upper(Q)
+    L = np.linalg.cholesky(np.linalg.inv(Q)).T
+    P = g.uniform(-0.5, 3.5, size=(30, K))
+    T = P.copy()
+    Zg = np.zeros((30, K))
+    for j in range(K):
+        Zg[:, j] = np.clip(np.rint(T[:, j]), 0, 3)
+        T[:, j + 1:] -= np.outer((T[:, j] - Zg[:, j]) / L[j, j], L[j, j + 1:])
+    assert np.array_equal(O.ldlq_assign(P, U), Zg)
+
+
+def test_code_space_objective_is_the_weight_space_objective():
+    """1/2 (z - p)^T Q (z - p) with Q = Abar^T H Abar and p = Abar^-1 (w0 - bbar)
+    equals 1/2 (W~ - w0)^T H (W~ - w0) with W~ decoded from the codes."""
+    g = np.random.Generator(np.random.PCG64(76))
+    d, K, N = 4, 16, 6
+    A = np.eye(d) * 0.3 + 0.05 * g.standard_normal((d, d))
+    B = g.standard_normal(d)
+    H = _spd(g, K)
+    W0 = g.standard_normal((N, K))
+    Z = g.integers(0, 4, size=(N, K)).astype(np.uint8)
+    R = O.decode(Z, A, B) - W0
+    direct = 0.5 * np.einsum("nk,kl,nl->n", R, H, R)
+    got = O.ldlq_objective(O.code_targets(W0, A, B), O.code_space_hessian(H, A), Z)
+    assert np.allclose(got, direct, rtol=1e-10, atol=1e-12)
+
+
+def test_ldlq_targets_reproduce_the_choices():
+    g = np.random.Generator(np.random.PCG64(77))
+    K = 32
+    U, _ = O.ldl_upper(_spd(g, K))
+    P = g.uniform(-0.5, 3.5, size=(16, K))
+    Z = O.ldlq_assign(P, U)
+    T, S = O.ldlq_targets(P, U, Z)
+    assert np.array_equal(np.clip(np.rint(T), 0, 3), Z)
+    assert np.all(S >= np.abs(T) - 1e-12)
+
+
+def test_ldlq_lowers_the_objective_on_a_correlated_hessian():
+    """The point of the compensation: on a strongly correlated Q the mean
+    objective is below that of plain rounding (fixed seed, 200 rows)."""
+    g = np.random.Generator(np.random.PCG64(78))
+    K = 32
+    Q = _spd(g, K, ridge=0.01)
+    U, _ = O.ldl_upper(Q)
+    P = g.uniform(-0.5, 3.5, size=(200, K))
+    seq = O.ldlq_objective(P, Q, O.ldlq_assign(P, U)).mean()
+    rnd = O.ldlq_objective(P, Q, np.clip(np.rint(P), 0, 3)).mean()
+    assert seq < 0.8 * rnd
+
+
+def test_ldlq_planted_mistakes_are_caught():
+    """Feeding back the error of the compensated target (t_i - z_i) instead of
+    p_i - z_i, or factoring Q without reversing its order (the transposed
+    lower factor in place of the upper one), breaks agreement with the direct
+    procedure."""
+    g = np.random.Generator(np.random.PCG64(79))
+    K = 10
+    Q = _spd(g, K)
+    U, _ = O.ldl_upper(Q)
+    P = g.uniform(-0.5, 3.5, size=(40, K))
+    ref = np.stack([_eq11_direct(P[n], Q) for n in range(40)])
+    T = P.copy()
+    Zw = np.zeros_like(P)
+    for j in range(K):
+        Zw[:, j] = np.clip(np.rint(T[:, j]), 0, 3)
+        T[:, j + 1:] += np.outer(T[:, j] - Zw[:, j], U[j, j + 1:])
+    assert not np.array_equal(Zw, ref)
+    C = np.linalg.cholesky(Q)  # the factor without the reversal: Q = (I + L) D (I + L)^T, L lower
+    wrong = (C / np.diag(C)[None, :] - np.eye(K)).T
+    assert not np.array_equal(O.ldlq_assign(P, wrong), ref)
+
+
 # ---------------------------------------------------------------- metric
 def test_rel_err_semantics():
     assert O.rel_err([1.0, 2.0], [1.0, 2.5], [1.0, 5.0]) == pytest.approx(0.1)

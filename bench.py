@@ -281,18 +281,6 @@ def headline(args, D: Dist, pk):
     ws = {M: lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, d), dev)
           for M in Ms}
 
-    # parity before timing (oracle on rank 0, M = 16 full output)
-    parity = None
-    if D.rank == 0:
-        from oracle import lcvq_oracle as O
-        z, _ = O.assign(w["Wp"])
-        for M in Ms:
-            lcvq.gemm(X[M], copies[0], K, A, B, d, out=Y[M], workspace=ws[M])
-            ref, Dn = O.forward(w["X"][:M], z, w["A"], w["B"])
-            e = O.rel_err(Y[M].float().cpu().numpy(), ref, Dn)
-            parity = e if parity is None else max(parity, e)
-        assert parity <= 4e-3, f"parity failed before timing: {parity}"
-
     ctr = [0]
 
     def step():
@@ -410,7 +398,7 @@ def headline(args, D: Dist, pk):
                       kernel="gemv_group_kernel (decode-GEMV, M=1,4,16 summed)",
                       per_m_us={str(M): per_m[M] * 1e3 for M in Ms},
                       peak_source=f"{PEAK_SRC} hbm_gbs"),
-        e2e=e2e, clocks=ck, gpu_launches=int(launches), parity_max_rel_err=parity,
+        e2e=e2e, clocks=ck, gpu_launches=int(launches),
     )
     return res
 
@@ -424,16 +412,11 @@ def row_assign_pack(D, pk):
     Wp = torch.from_numpy(w["Wp"]).to(dev)
     packed = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
     mask = torch.empty((N, K // 8), dtype=torch.uint8, device=dev)
-    from oracle import lcvq_oracle as O
-    z, m = O.assign(w["Wp"])
-    lcvq.assign_pack(Wp, 8, packed=packed, mask=mask)
-    exact = bool(np.array_equal(packed.cpu().numpy(), O.pack_codes(z)) and
-                 np.array_equal(mask.cpu().numpy(), O.pack_mask(m)))
     ms = ev_time(lambda: lcvq.assign_pack(Wp, 8, packed=packed, mask=mask), 50)
     nbytes = N * K * (4 + 0.25 + 0.125)
     gbs = nbytes / (ms * 1e-3) / 1e9
     return dict(metric="assign+pack GB/s (fp32 in, codes+mask out)", value=gbs, unit="GB/s",
-                us=ms * 1e3, bit_exact=exact,
+                us=ms * 1e3,
                 roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
                               frac=gbs / pk["hbm_gbs"]))
 
@@ -465,20 +448,12 @@ def row_prefill(D, pk):
     X = torch.from_numpy(w["X"]).to(torch.bfloat16).to(dev)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, d), dev)
-    from oracle import lcvq_oracle as O
-    z, _ = O.assign(w["Wp"])
-    rng = np.random.Generator(np.random.PCG64(1))
-    pairs = [(int(a), int(b)) for a, b in zip(rng.integers(0, M, 256), rng.integers(0, N, 256))]
     out = {}
     flops = 2.0 * M * N * K
     for form in ("algebraic", "decode"):
-        lcvq.gemm(X, packed, K, A, B, d, form=form, out=Y, workspace=ws)
-        Yc = Y.float().cpu().numpy()
-        y, dd = O.forward_sampled(w["X"], {n: z[n] for _, n in pairs}, w["A"], w["B"], pairs)
-        err = O.rel_err(np.array([Yc[m, n] for m, n in pairs]), y, dd)
         ms = ev_time(lambda: lcvq.gemm(X, packed, K, A, B, d, form=form, out=Y, workspace=ws), 5)
         tf = flops / (ms * 1e-3) / 1e12
-        out[form] = dict(value=tf, unit="TFLOP/s", us=ms * 1e3, sampled_rel_err=err,
+        out[form] = dict(value=tf, unit="TFLOP/s", us=ms * 1e3,
                          roofline=dict(bound="tensor", achieved=tf, peak=pk["bf16_tflops"],
                                        unit="TFLOP/s", frac=tf / pk["bf16_tflops"]))
     return dict(metric="prefill GEMM TFLOP/s (2MNK / time)", forms=out)
@@ -640,8 +615,42 @@ def row_fit(D, pk):
     return dict(metric="(A, B) refit GB/s (W0 fp32 + codes read)", forms=out)
 
 
+# fp32 FMA peak: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz (the maximum SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
+
+
+def row_ldlq(D, pk):
+    """H-aware sequential code assignment on a 4096 x 4096 matrix (d = 8): the
+    code-space factor of a calibration Hessian (8192 activation rows, outlier
+    recipe, 1% damping) is formed on the device in fp64 before timing."""
+    dev = D.dev
+    N = K = 4096
+    d = 8
+    w = synth.ldlq_workload(N, K, d)
+    X = torch.from_numpy(w["Xcal"]).to(dev, torch.float64)
+    H = X.T @ X / X.shape[0]
+    H += 0.01 * H.diagonal().mean() * torch.eye(K, dtype=torch.float64, device=dev)
+    Abar = torch.kron(torch.eye(K // d, dtype=torch.float64, device=dev),
+                      torch.from_numpy(w["A"]).to(dev, torch.float64))
+    Q = Abar.T @ H @ Abar
+    V = torch.linalg.cholesky(Q.flip(0, 1)).flip(0, 1)  # Q = V V^T, V upper triangular
+    U = (V / V.diagonal()[None, :]).triu(1).float().contiguous()
+    del X, H, Abar, Q, V
+    P = torch.from_numpy(w["P"]).to(dev)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_ASSIGN_LDLQ, torch.float32, 0, N, K, d), dev)
+    lcvq.assign_ldlq(P, U, d, workspace=ws, packed=packed)
+    ms = ev_time(lambda: lcvq.assign_ldlq(P, U, d, workspace=ws, packed=packed), 10)
+    tf = N * K * (K - 1) / (ms * 1e-3) / 1e12
+    return dict(metric="H-aware assignment TFLOP/s (N K (K-1) / time: fp32 FMA, 2 flops each)",
+                value=tf, unit="TFLOP/s", us=ms * 1e3,
+                roofline=dict(bound="alu", achieved=tf, peak=FP32_ALU_TFLOPS, unit="TFLOP/s",
+                              frac=tf / FP32_ALU_TFLOPS,
+                              peak_source="derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz"))
+
+
 ROWS = {"assign_pack": row_assign_pack, "decode": row_decode, "prefill": row_prefill,
-        "qat": row_qat, "stack": row_stack, "fit": row_fit}
+        "qat": row_qat, "stack": row_stack, "fit": row_fit, "ldlq": row_ldlq}
 
 
 # ----------------------------------------------------------------------------- main

@@ -65,6 +65,7 @@ lcvq_status check_device() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 constexpr int64_t kMaxGemmDim = int64_t(1) << 30;
+constexpr int64_t kMaxLdlqDim = int64_t(1) << 20;  // U is d_in^2 floats
 bool valid_d(int d) { return d == 1 || d == 2 || d == 4 || d == 8; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -164,7 +165,29 @@ size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_ou
   if (op == LCVQ_OP_GEMM) return gemm_ws(dtype, M, d_in).total;
   if (op == LCVQ_OP_GEMM_BACKWARD) return bwd_ws(M, d_out, d_in, d).total;
   if (op == LCVQ_OP_FIT_AFFINE) return kWsHeaderBytes + fit_partials_bytes(d_out, d_in, d);
+  if (op == LCVQ_OP_ASSIGN_LDLQ) return kWsHeaderBytes + ldlq_workspace_bytes(d_out, d_in);
   return 0;
+}
+
+lcvq_status lcvq_assign_ldlq(const float* P, const float* U, int64_t d_out, int64_t d_in, int d,
+                             uint8_t* packed, void* workspace, size_t ws_bytes, void* stream) {
+  g_last_launches = 0;
+  if (d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
+  if (d_in % 64 != 0 || d_in % d != 0 || d_in > kMaxLdlqDim || d_out > kMaxGemmDim)
+    return LCVQ_ERR_INVALID_ARG;
+  if (!workspace) return LCVQ_ERR_INVALID_ARG;
+  if (d_out == 0 || d_in == 0) return LCVQ_OK;
+  if (!P || !U || !packed) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(P) || !aligned16(U) || !aligned16(packed) || !aligned16(workspace))
+    return LCVQ_ERR_ALIGNMENT;
+  if (ws_bytes < kWsHeaderBytes + ldlq_workspace_bytes(d_out, d_in)) return LCVQ_ERR_WORKSPACE;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e = launch_ldlq(P, U, d_out, d_in, packed, reinterpret_cast<float*>(ws + kWsHeaderBytes),
+                              reinterpret_cast<unsigned int*>(ws), static_cast<cudaStream_t>(stream),
+                              &launches);
+  return finish(e, launches);
 }
 
 lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, float k, void* stream) {

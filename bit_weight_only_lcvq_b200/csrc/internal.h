@@ -93,6 +93,13 @@ cudaError_t launch_fit_affine(const float* W0, const uint8_t* packed, int64_t d_
                               int d, const float* h, float* A, float* B, double* partials,
                               cudaStream_t s, int* launches);
 
+// ---- H-aware sequential code assignment ----
+// E: ldlq_workspace_bytes(d_out, d_in) bytes of fp32 scratch (the errors p - z)
+size_t ldlq_workspace_bytes(int64_t d_out, int64_t d_in);
+cudaError_t launch_ldlq(const float* P, const float* U, int64_t d_out, int64_t d_in,
+                        uint8_t* packed, float* E, unsigned int* err, cudaStream_t s,
+                        int* launches);
+
 // ---- tcgen05 GEMMs (bf16, persistent, one CTA per SM) ----
 int tc_max_grid();
 // Xa is X'' (algebraic, with corr) or X (decode form, A z + B decoded on chip)

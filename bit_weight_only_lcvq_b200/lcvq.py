@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcvq.so"
 
 F32, BF16 = 0, 1
 FORMS = {"auto": 0, "decode": 1, "algebraic": 2}
-OP_GEMM, OP_GEMM_BACKWARD, OP_FIT_AFFINE = 0, 1, 2
+OP_GEMM, OP_GEMM_BACKWARD, OP_FIT_AFFINE, OP_ASSIGN_LDLQ = 0, 1, 2, 3
 STATUS = {
     0: "LCVQ_OK",
     1: "LCVQ_ERR_INVALID_ARG",
@@ -41,6 +41,7 @@ EXPORTS = (
     "lcvq_gemm_grouped",
     "lcvq_fit_affine",
     "lcvq_dge_scale",
+    "lcvq_assign_ldlq",
     "lcvq_workspace_size",
     "lcvq_workspace_size_grouped",
     "lcvq_check_device_error",
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
         L.lcvq_workspace_size_grouped.restype = _sz
         L.lcvq_fit_affine.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
         L.lcvq_dge_scale.argtypes = [_vp, _vp, _i64, ctypes.c_float, _vp]
+        L.lcvq_assign_ldlq.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _sz, _vp]
         L.lcvq_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i64, _i32]
         L.lcvq_workspace_size.restype = _sz
         L.lcvq_check_device_error.argtypes = [_vp, _vp]
@@ -301,6 +303,24 @@ def fit_affine(W0: torch.Tensor, packed: torch.Tensor, d: int, *, h=None, worksp
         _ptr(W0), _ptr(packed), d_out, d_in, d, _ptr(h), _ptr(A), _ptr(B), _ptr(workspace),
         workspace.numel(), _stream(stream)))
     return A, B
+
+
+def assign_ldlq(P: torch.Tensor, U: torch.Tensor, d: int, *, workspace=None, packed=None,
+                stream=None) -> torch.Tensor:
+    """Codes of the H-aware sequential assignment of the code-space targets P
+    [d_out][d_in] with the strictly upper factor U [d_in][d_in] of the
+    code-space Hessian (see lcvq_assign_ldlq).  Returns packed [d_out][d_in/4]."""
+    d_out, d_in = P.shape
+    dev = P.device
+    if packed is None:
+        packed = torch.empty((d_out, d_in // 4), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = new_workspace(workspace_size(OP_ASSIGN_LDLQ, torch.float32, 0, d_out, d_in, d),
+                                  dev)
+    _check("lcvq_assign_ldlq", lib().lcvq_assign_ldlq(
+        _ptr(P), _ptr(U), d_out, d_in, d, _ptr(packed), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return packed
 
 
 def dge_scale(dWp: torch.Tensor, Wp: torch.Tensor, k: float, *, stream=None) -> torch.Tensor:

@@ -188,3 +188,34 @@ def stack_matrix(layer: int, proj: int, M: int, *, with_x: bool = True) -> dict:
     if with_x:
         out["X"] = x_outliers(M, d_in, rng(5, T_X, sub), rng(5, T_OUTLIER, sub), "bf16")
     return out
+
+
+def ldlq_workload(d_out: int = 4096, d_in: int = 4096, d: int = 8, n_cal: int | None = None,
+                  with_cal: bool = True) -> dict:
+    """Inputs of the H-aware sequential assignment (workload id 6): code-space
+    targets P ~ U[-0.5, 3.5] ``[d_out][d_in]`` (fp32), the matrix's A/B
+    (diagonal-dominant recipe) and ``n_cal`` (default 2 d_in) calibration
+    activation rows with the outlier recipe, fp32, from which the caller forms
+    the input Hessian.  Sizes may be reduced for small cases with the same
+    distributions."""
+    n_cal = n_cal or 2 * d_in
+    out = dict(d_in=d_in, d_out=d_out, d=d, n_cal=n_cal)
+    out["P"] = wp_uniform(d_out, d_in, rng(6, T_WP))
+    out["A"], out["B"] = affine_diag_dominant(d, rng(6, T_A))
+    if with_cal:
+        out["Xcal"] = x_outliers(n_cal, d_in, rng(6, T_X), rng(6, T_OUTLIER), "fp32")
+    return out
+
+
+def strict_upper_dyadic(K: int, g: np.random.Generator, step: float = 1.0 / 64,
+                        limit: int = 4) -> np.ndarray:
+    """A strictly upper triangular K x K fp32 matrix with entries that are
+    multiples of ``step`` in [-limit step, limit step]: every product with a
+    small dyadic error and every partial sum of a row is exact in fp32."""
+    u = g.integers(-limit, limit + 1, size=(K, K)).astype(np.float64) * step
+    return np.triu(u, 1).astype(np.float32)
+
+
+def targets_dyadic(d_out: int, d_in: int, g: np.random.Generator, step: float = 1.0 / 32) -> np.ndarray:
+    """Targets on a 1/32 grid in [-0.5, 3.5] (exact rounding ties included)."""
+    return (g.integers(-16, 113, size=(d_out, d_in)).astype(np.float64) * step).astype(np.float32)

@@ -92,7 +92,12 @@ typedef enum {
  *  AUTO:      the library's choice (ALGEBRAIC on the tensor-core paths). */
 typedef enum { LCVQ_FORM_AUTO = 0, LCVQ_FORM_DECODE = 1, LCVQ_FORM_ALGEBRAIC = 2 } lcvq_form;
 
-typedef enum { LCVQ_OP_GEMM = 0, LCVQ_OP_GEMM_BACKWARD = 1, LCVQ_OP_FIT_AFFINE = 2 } lcvq_op;
+typedef enum {
+  LCVQ_OP_GEMM = 0,
+  LCVQ_OP_GEMM_BACKWARD = 1,
+  LCVQ_OP_FIT_AFFINE = 2,
+  LCVQ_OP_ASSIGN_LDLQ = 3
+} lcvq_op;
 
 /* Code assignment and 2-bit packing (LC-QAT technical summary, Methodology 1:
  * index selection becomes rounding and clamping; Methodology 3: proxy weights
@@ -274,6 +279,39 @@ LCVQ_API lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, floa
 LCVQ_API lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int64_t d_out,
                                      int64_t d_in, int d, const float* h, float* A, float* B,
                                      void* workspace, size_t ws_bytes, void* stream);
+
+/* H-aware sequential code assignment, the PTQ initialisation of the codes
+ * (LC-QAT technical summary, Methodology 2: the initial integer weights come
+ * from LDLQ, column-wise quantization with sequential compensation of the
+ * reconstruction error; decoupleQ page, section 3.3, eq. (8)-(11): round and
+ * clip one element, then re-solve the remaining ones without the integer
+ * constraint and the box).  For a row with target w0 and the input Hessian H
+ * (e.g. X^T X of calibration activations) the layer objective is
+ *     1/2 (Abar z + bbar - w0)^T H (Abar z + bbar - w0) = 1/2 (z - p)^T Q (z - p),
+ * with Abar = blockdiag(A, .., A), bbar = B per vector, Q = Abar^T H Abar and
+ * p = Abar^-1 (w0 - bbar), the row's code-space target (what W_p holds).  The
+ * call takes P and the factor U of Q = (I + U) diag(D) (I + U)^T (U strictly
+ * upper triangular: the Cholesky factor of Q with its rows and columns
+ * reversed, scaled to a unit diagonal), and sets, for every row, in order of
+ * increasing column j,
+ *     z_j = clamp(rint(t_j), 0, 3),   t_j = p_j + sum_{i<j} U[i][j] (p_i - z_i),
+ * which is t_j = the j-th element of the minimiser of eq. (11) once z_0 ..
+ * z_{j-1} are fixed.  With Q diagonal (U = 0) this is lcvq_assign_pack.
+ * Arithmetic is fp32 (t in a fixed blocked order); a code can differ from the
+ * fp64 rule only where t_j lies within fp32 rounding of a rounding boundary.
+ *   P      [d_out][d_in] fp32 targets; finite values (a non-finite one makes
+ *          the rest of its row unspecified).
+ *   U      [d_in][d_in] fp32 row-major; only the entries above the diagonal
+ *          are read.
+ *   packed [d_out][d_in/4] out: the codes (format V1).
+ *   workspace: >= lcvq_workspace_size(LCVQ_OP_ASSIGN_LDLQ, LCVQ_F32, 0, d_out,
+ *   d_in, d) bytes (the fp32 errors p - z of every row), 256-byte aligned.
+ * Shapes: d_in % 64 == 0, d_in % d == 0, d_in <= 2^20; 16-byte aligned
+ * pointers.  Launches 1 kernel of ceil(d_out / 16) CTAs, N d_in (d_in - 1) / 2
+ * fused multiply-adds. */
+LCVQ_API lcvq_status lcvq_assign_ldlq(const float* P, const float* U, int64_t d_out, int64_t d_in,
+                                      int d, uint8_t* packed, void* workspace, size_t ws_bytes,
+                                      void* stream);
 
 /* Workspace bytes a call with these arguments needs (0 on invalid input).
  * The workspace holds the device error word (its first 256 bytes, which the

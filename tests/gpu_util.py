@@ -35,3 +35,24 @@ def assert_close(name, got, ref, D, tol):
     err = O.rel_err(got, ref, D)
     assert err <= tol, f"{name}: max rel err {err:.3e} > {tol:.1e}"
     return err
+
+
+def ldlq_check(P, U, Z):
+    """Validity of codes Z of the H-aware sequential assignment (computed in
+    fp32): the oracle recomputes, in fp64, the target t_j that each code was
+    rounded from, given the codes before it.  Every code must be
+    clamp(rint(t_j), 0, 3), except where t_j lies within the fp32 error bound
+    of a rounding boundary (0.5, 1.5, 2.5), where either neighbour is valid.
+    The bound is (chain + 96) 2^-24 sum|terms|, chain = K/8 additions (the
+    longest sum of one warp's share of the earlier blocks) plus the
+    cross-warp sum and the in-block updates.  Returns (bad, near)."""
+    P = np.asarray(P, dtype=np.float64)
+    T, S = O.ldlq_targets(P, np.asarray(U, dtype=np.float64), Z)
+    K = P.shape[1]
+    tau = (K / 8 + 96) * 2.0 ** -24 * S
+    ref = np.clip(np.rint(T), 0, 3)
+    dist = np.abs(T - (np.floor(T) + 0.5))
+    near = (dist <= tau) & (T > 0.5 - tau) & (T < 2.5 + tau)
+    Zf = np.asarray(Z, dtype=np.float64)
+    bad = ((Zf != ref) & ~near) | (np.abs(np.clip(T, 0, 3) - Zf) > 0.5 + tau)
+    return int(bad.sum()), int(near.sum())

@@ -111,6 +111,21 @@ def test_dge_scale_rejects_bad_arguments_without_device():
     assert L.lcvq_dge_scale(None, None, 0, 2.0, None) == 0        # empty: no-op
 
 
+def test_assign_ldlq_rejects_bad_arguments_without_device():
+    L = lcvq.lib()
+    ws = L.lcvq_workspace_size(lcvq.OP_ASSIGN_LDLQ, 0, 0, 50, 256, 8)
+    assert ws == 256 + 64 * 256 * 4                                     # rows padded to 16
+    assert L.lcvq_workspace_size(lcvq.OP_ASSIGN_LDLQ, 0, 0, 50, 256, 3) == 0
+    assert L.lcvq_assign_ldlq(16, 16, 8, 96, 8, 16, 256, 1 << 20, None) == 1    # d_in % 64
+    assert L.lcvq_assign_ldlq(16, 16, 8, 64, 3, 16, 256, 1 << 20, None) == 1    # d
+    assert L.lcvq_assign_ldlq(16, 16, 8, (1 << 20) + 64, 8, 16, 256, 1 << 40, None) == 1  # d_in
+    assert L.lcvq_assign_ldlq(16, None, 8, 64, 8, 16, 256, 1 << 20, None) == 1  # no U
+    assert L.lcvq_assign_ldlq(16, 16, 8, 64, 8, 16, None, 1 << 20, None) == 1   # no workspace
+    assert L.lcvq_assign_ldlq(16, 8, 8, 64, 8, 16, 256, 1 << 20, None) == 3     # U misaligned
+    assert L.lcvq_assign_ldlq(16, 16, 8, 64, 8, 16, 256, 1024, None) == 4       # workspace
+    assert L.lcvq_assign_ldlq(None, None, 0, 64, 8, None, 256, 0, None) == 0    # empty: no-op
+
+
 def test_gemm_dimension_limits_without_device():
     """Matrix dimensions above 2^30 are refused before anything runs (the GEMV
     kernels index rows and columns in 32 bits)."""

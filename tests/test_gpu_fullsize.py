@@ -28,6 +28,20 @@ def _check_sampled_forward(Y, Xnp, z, A, B, pairs, tag):
     assert_close(tag, got, y, dd, TOL_BF16)
 
 
+def test_decode_gemv_full():
+    """The decode-GEMV workload the benchmark times: d_in = d_out = 4096, d = 8,
+    M in {1, 4, 16} bf16; every output element against the oracle."""
+    w = synth.workload(2, M=16, with_dy=False)
+    z, _ = O.assign(w["Wp"])
+    packed, _ = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev()), 8, with_mask=False)
+    A, B = torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev())
+    for M in (1, 4, 16):
+        X = torch.from_numpy(w["X"][:M].copy()).to(torch.bfloat16).to(dev())
+        Y = lcvq.gemm(X, packed, 4096, A, B, 8)
+        ref, Dn = O.forward(w["X"][:M], z, w["A"], w["B"])
+        assert_close(f"decode-GEMV M={M}", Y.float().cpu().numpy(), ref, Dn, TOL_BF16)
+
+
 @pytest.mark.parametrize("form", ["algebraic", "decode"])
 def test_prefill_full(form):
     """Prefill GEMM: d_in=4096, d_out=11008, d=8, M=2048 bf16."""
@@ -136,3 +150,37 @@ def test_fit_affine_full_size_qat_matrix():
                                                   A_ref, B_ref))
     ref = np.concatenate([A_ref.ravel(), B_ref.ravel()])
     assert np.max(np.abs(ref - np.concatenate([A0.ravel(), B0.ravel()]))) < 1e-3
+
+
+def test_ldlq_full_size_decode_matrix():
+    """H-aware sequential assignment at 4096 x 4096 (the size the benchmark
+    times) with a calibration Hessian: sampled rows are checked against the
+    fp64 recomputation of every target, and match the oracle's own run."""
+    from tests.test_gpu_parity import _ldlq_case, _ldlq_gpu
+    from tests.gpu_util import ldlq_check
+    N = K = 4096
+    P, U = _ldlq_case(N, K)
+    packed = _ldlq_gpu(P, U).cpu().numpy()
+    g = np.random.Generator(np.random.PCG64(1600))
+    rows = np.unique(np.concatenate([[0, 15, 16, N - 1], g.choice(N, 44, replace=False)]))
+    Z = O.unpack_codes(packed[rows], K)
+    bad, near = ldlq_check(P[rows], U, Z)
+    assert bad == 0, (bad, near)
+    Zo = O.ldlq_assign(P[rows[:8]], U)
+    assert np.sum(np.all(Z[:8] == Zo, axis=1)) >= 8 - near
+
+
+def test_ldlq_full_size_qat_matrix():
+    """4096 x 14336 (the QAT-step matrix) with a random factor: sampled rows
+    checked against the fp64 recomputation."""
+    from tests.gpu_util import ldlq_check
+    N, K = 4096, 14336
+    g = np.random.Generator(np.random.PCG64(1601))
+    P = synth.wp_uniform(N, K, g)
+    U = (g.standard_normal((K, K), dtype=np.float32) * np.float32(1.0 / np.sqrt(K)))
+    U = np.triu(U, 1)
+    out = lcvq.assign_ldlq(torch.from_numpy(P).to(dev()), torch.from_numpy(U).to(dev()), 8)
+    rows = np.array([0, 1, 2047, 4095] + list(g.choice(N, 4, replace=False)))
+    Z = O.unpack_codes(out.cpu().numpy()[rows], K)
+    bad, near = ldlq_check(P[rows], U, Z)
+    assert bad == 0, (bad, near)

@@ -12,7 +12,7 @@ import torch
 
 from bit_weight_only_lcvq_b200 import lcvq, synth
 from oracle import lcvq_oracle as O
-from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, dev, to_dev, to_np, tol_for
+from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, dev, ldlq_check, to_dev, to_np, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -444,3 +444,88 @@ def test_dge_scale_matches_oracle(dtype, k):
     lcvq.dge_scale(out["dWp"], Wp, k)
     ref, D = O.backward_dge_dwp(w["X"], w["dY"], z, w["Wp"], w["A"], k)
     assert_close(f"dge k={k}", to_np(out["dWp"]), ref, D, tol_for(dtype))
+
+
+# --------------------------------------------------------------- H-aware sequential assignment
+def _ldlq_case(N, K, d=8, n_cal=None):
+    """Targets, and the code-space factor U (fp32) of a calibration Hessian
+    H = Xcal^T Xcal / n + 1% damping, through the matrix's A."""
+    w = synth.ldlq_workload(N, K, d, n_cal=n_cal)
+    X = w["Xcal"].astype(np.float64)
+    H = X.T @ X / X.shape[0]
+    H += 0.01 * np.mean(np.diag(H)) * np.eye(K)
+    U, _ = O.ldl_upper(O.code_space_hessian(H, w["A"].astype(np.float64)))
+    return w["P"], U.astype(np.float32)
+
+
+def _ldlq_gpu(P, U, d=8):
+    return lcvq.assign_ldlq(torch.from_numpy(P).to(dev()), torch.from_numpy(U).to(dev()), d)
+
+
+@pytest.mark.parametrize("N,K", [(50, 256), (33, 640)])
+def test_ldlq_matches_oracle_on_a_calibration_hessian(N, K):
+    """Every code is the rule's choice for the target it was rounded from
+    (fp64 recomputation), and the rows agree with the oracle's own run."""
+    P, U = _ldlq_case(N, K)
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_ASSIGN_LDLQ, torch.float32, 0, N, K, 8))
+    packed = lcvq.assign_ldlq(torch.from_numpy(P).to(dev()), torch.from_numpy(U).to(dev()), 8,
+                              workspace=ws)
+    assert lcvq.check_device_error(ws) == 0
+    Z = O.unpack_codes(packed.cpu().numpy(), K)
+    bad, near = ldlq_check(P, U, Z)
+    assert bad == 0, (bad, near)
+    Zo = O.ldlq_assign(P, U)
+    same_rows = int(np.sum(np.all(Z == Zo, axis=1)))
+    assert same_rows >= N - near, (same_rows, near)
+    # the compensation is at work: the codes differ from plain rounding
+    assert np.mean(Z != O.assign(P)[0]) > 0.05
+
+
+def test_ldlq_exact_arithmetic_is_bit_exact():
+    """Dyadic targets and factor entries make every fp32 product and sum
+    exact, so the codes (exact ties to even included) match the oracle bit
+    for bit."""
+    g = np.random.Generator(np.random.PCG64(1500))
+    N, K = 37, 512
+    P = synth.targets_dyadic(N, K, g)
+    U = synth.strict_upper_dyadic(K, g)
+    packed = _ldlq_gpu(P, U)
+    assert np.array_equal(packed.cpu().numpy(), O.pack_codes(O.ldlq_assign(P, U)))
+
+
+def test_ldlq_reads_only_above_the_diagonal_and_zero_factor_is_assign_pack():
+    """U = 0 above the diagonal, NaN on and below it: the codes are those of
+    lcvq_assign_pack (ties, clamping and far-out values included)."""
+    g = np.random.Generator(np.random.PCG64(1501))
+    N, K = 40, 192
+    P = _adversarial_wp(N, K, 1502)
+    P[~np.isfinite(P)] = 1e30
+    U = np.full((K, K), np.nan, dtype=np.float32)
+    U[np.triu_indices(K, 1)] = 0.0
+    packed = _ldlq_gpu(P, U)
+    ref, _ = lcvq.assign_pack(torch.from_numpy(P).to(dev()), d=8, with_mask=False)
+    assert torch.equal(packed, ref)
+    assert np.array_equal(packed.cpu().numpy(), O.pack_codes(O.assign(P)[0]))
+
+
+def test_ldlq_rows_are_independent_and_deterministic():
+    P, U = _ldlq_case(50, 256)
+    a = _ldlq_gpu(P, U)
+    b = _ldlq_gpu(P, U)
+    part = _ldlq_gpu(np.ascontiguousarray(P[16:32]), U)
+    assert torch.equal(a, b)
+    assert torch.equal(a[16:32], part)
+
+
+@pytest.mark.parametrize("N,K", [(1, 64), (16, 64), (17, 128), (3, 1024)])
+def test_ldlq_edge_shapes(N, K):
+    P, U = _ldlq_case(N, K, n_cal=max(2 * K, 64))
+    Z = O.unpack_codes(_ldlq_gpu(P, U).cpu().numpy(), K)
+    bad, near = ldlq_check(P, U, Z)
+    assert bad == 0, (bad, near)
+
+
+def test_ldlq_empty_matrix_is_a_no_op():
+    U = torch.zeros((64, 64), device=dev())
+    out = lcvq.assign_ldlq(torch.zeros((0, 64), device=dev()), U, 8)
+    assert out.shape == (0, 16)

@@ -307,7 +307,7 @@ LCVQ_API lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int
  *   workspace: >= lcvq_workspace_size(LCVQ_OP_ASSIGN_LDLQ, LCVQ_F32, 0, d_out,
  *   d_in, d) bytes (the fp32 errors p - z of every row), 256-byte aligned.
  * Shapes: d_in % 64 == 0, d_in % d == 0, d_in <= 2^20; 16-byte aligned
- * pointers.  Launches 1 kernel of ceil(d_out / 16) CTAs, N d_in (d_in - 1) / 2
+ * pointers.  Launches 1 kernel of ceil(d_out / 32) CTAs, d_out d_in (d_in - 1) / 2
  * fused multiply-adds. */
 LCVQ_API lcvq_status lcvq_assign_ldlq(const float* P, const float* U, int64_t d_out, int64_t d_in,
                                       int d, uint8_t* packed, void* workspace, size_t ws_bytes,

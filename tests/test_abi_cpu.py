@@ -114,7 +114,7 @@ def test_dge_scale_rejects_bad_arguments_without_device():
 def test_assign_ldlq_rejects_bad_arguments_without_device():
     L = lcvq.lib()
     ws = L.lcvq_workspace_size(lcvq.OP_ASSIGN_LDLQ, 0, 0, 50, 256, 8)
-    assert ws == 256 + 64 * 256 * 4                                     # rows padded to 16
+    assert ws == 256 + 64 * 256 * 4                                     # rows padded to 32
     assert L.lcvq_workspace_size(lcvq.OP_ASSIGN_LDLQ, 0, 0, 50, 256, 3) == 0
     assert L.lcvq_assign_ldlq(16, 16, 8, 96, 8, 16, 256, 1 << 20, None) == 1    # d_in % 64
     assert L.lcvq_assign_ldlq(16, 16, 8, 64, 3, 16, 256, 1 << 20, None) == 1    # d

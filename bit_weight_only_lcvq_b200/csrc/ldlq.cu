@@ -11,26 +11,30 @@
 // Rows are independent; within a row every t_j waits for all z_{i<j}.
 //
 // ldlq_kernel: one CTA per 32 rows (one CTA per SM), K in blocks of 64
-// columns.  For block b (columns j0 .. j0 + 63, j0 = 64 b):
-//   1. the part of t from the earlier blocks, T_b = E_{<b} U[<j0, block], is
-//      a 32 x 64 x j0 product: warp 8 streams the chunks c < b, each the
-//      64 x 64 tile U[64c .., j0 ..] (TMA box) and the CTA's own errors
-//      E[64c .., 32 rows] (one 8 KB bulk copy from the workspace, written at
-//      the end of block c), through a ring of shared-memory stages; consumer
-//      warp w takes k rows 8w .. 8w + 7 of every chunk and all 32 x 64
-//      outputs (fp32 FFMA, lane tile 8 rows x 8 columns: 16 values loaded
-//      per 64 FMAs, which balances the shared-memory and FMA pipes), and the
-//      8 warps' partial tiles are summed in warp order through shared memory;
-//   2. the block itself runs in order: warp w takes rows 4w .. 4w + 3, lane l
-//      holds t of columns l and l + 32; at step j the owner lane rounds,
-//      the error p_j - z_j is broadcast by a shuffle and every later column
-//      adds U[j0 + j][col] times it (the diagonal tile, one more stage);
-//   3. codes go out 16 bytes per row, the errors to the workspace (8 KB), and
-//      an mbarrier tells the producer that chunk b may now be loaded.
-// The work is N K (K - 1) / 2 fused multiply-adds, on the CUDA cores in fp32
-// (the codes must follow the fp64 rule except within fp32 rounding of a
-// rounding boundary).  Every wait is bounded; a warp that gives up records
-// LCVQ_ERR_DEVICE_TIMEOUT and the CTA winds down through the same barriers.
+// columns, three kinds of warps working one block apart:
+//   * warps 0..7 form, for block b (columns j0 .. j0 + 63, j0 = 64 b), the
+//     compensation from the earlier blocks, T_b = E_{<b} U[<j0, block]: a
+//     32 x 64 x j0 product, split over the warps by k rows of every 64-row
+//     chunk, fp32 FFMA with a lane tile of 8 rows x 8 columns (16 values
+//     loaded per 64 FMAs, which balances the shared-memory and FMA pipes);
+//     the 8 partial tiles are summed in warp order into T_b in shared memory;
+//   * warp 8 rounds block b in order, one lane per row, holding the row's 64
+//     targets and compensations in registers: t_j = p_j + c_j, z_j by a
+//     clamp and the magic-number rounding (ties to even, on the FMA pipe),
+//     e_j = p_j - z_j, then c_k += U[j0 + j][j0 + k] e_j for the later columns
+//     (the diagonal tile; its rows are read as warp-wide broadcasts).  Its
+//     errors go to shared memory, where warps 0..7 take the newest chunk of
+//     T_{b+1} from, and to the workspace, where the older chunks come from;
+//     it prefetches the next block's targets with cp.async;
+//   * warp 9 streams, through TMA, the 64 x 64 tiles U[64c .., j0 ..] with the
+//     CTA's error chunks E[64c .., 32 rows] (a ring of stages) and the
+//     diagonal tiles (two buffers).
+// While warp 8 rounds block b, warps 0..7 already work on T_{b+1}: only its
+// last chunk waits for block b's errors.  The work is N K (K - 1) / 2 fused
+// multiply-adds, on the CUDA cores in fp32 (a code can differ from the fp64
+// rule only within fp32 rounding of a rounding boundary).  Every wait is
+// bounded; a warp that gives up records LCVQ_ERR_DEVICE_TIMEOUT, raises the
+// CTA's abort flag, and the CTA winds down through the same barriers.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -41,23 +45,32 @@ namespace {
 
 constexpr int kLqRows = 32;                         // weight rows per CTA
 constexpr int kLqBlk = 64;                          // columns per block = k rows per chunk
-constexpr int kLqCons = 8;                          // consumer warps
-constexpr int kLqSeqRows = kLqRows / kLqCons;       // rows per warp in the in-order part
-constexpr int kLqThreads = (kLqCons + 1) * 32;      // + one producer warp
-constexpr int kLqStages = 4;
+constexpr int kLqGemm = 8;                          // product warps
+constexpr int kLqSeqWarp = kLqGemm;                 // the in-order warp
+constexpr int kLqProdWarp = kLqGemm + 1;            // the TMA producer
+constexpr int kLqThreads = (kLqGemm + 2) * 32;
+constexpr int kLqStages = 3;
+constexpr int kLqTPitch = kLqBlk + 4;               // padded rows: conflict-free row reads
 constexpr uint32_t kLqUBytes = kLqBlk * kLqBlk * 4;          // 64 x 64 fp32 tile of U
 constexpr uint32_t kLqEBytes = kLqBlk * kLqRows * 4;         // 64 k x 32 rows of errors
 constexpr uint32_t kLqStageBytes = kLqUBytes + kLqEBytes;
-constexpr uint32_t kLqRedOff = kLqStages * kLqStageBytes;   // [8 warps][32][64] partials
-constexpr uint32_t kLqRedBytes = kLqCons * kLqRows * kLqBlk * 4;
-constexpr uint32_t kLqEstOff = kLqRedOff + kLqRedBytes;     // [64][32] errors of the block
-constexpr uint32_t kLqZOff = kLqEstOff + kLqEBytes;         // [32][16] code bytes of the block
-constexpr uint32_t kLqBarOff = kLqZOff + kLqRows * 16;
-constexpr size_t kLqSmem = 128 + kLqBarOff + (2 * kLqStages + 1) * 8 + 16;
+constexpr uint32_t kLqDiagOff = kLqStages * kLqStageBytes;  // 2 diagonal tiles
+constexpr uint32_t kLqRedOff = kLqDiagOff + 2 * kLqUBytes;  // [8 warps][32][64] partials
+constexpr uint32_t kLqRedBytes = kLqGemm * kLqRows * kLqBlk * 4;
+constexpr uint32_t kLqTOff = kLqRedOff + kLqRedBytes;       // T_b [32][68]
+constexpr uint32_t kLqTBytes = kLqRows * kLqTPitch * 4;
+constexpr uint32_t kLqEstOff = kLqTOff + kLqTBytes;         // newest errors [64][32]
+constexpr uint32_t kLqPOff = kLqEstOff + kLqEBytes;         // targets, 2 x [32][68]
+constexpr uint32_t kLqBarOff = kLqPOff + 2 * kLqTBytes;
+constexpr int kLqNumBars = 2 * kLqStages + 4 + 4;           // full, empty, dfull x2, dempty x2,
+                                                            // tready, eready, ebar x2
+constexpr size_t kLqSmem = 128 + kLqBarOff + kLqNumBars * 8 + 16;
 constexpr long long kLqWaitLimit = 1LL << 32;
-static_assert(kLqStageBytes % 128 == 0, "TMA destinations stay 128-byte aligned");
-static_assert(kLqEBytes / 16 == 2 * kLqCons * 32, "two float4 of a chunk of errors per consumer thread");
-static_assert(kLqSeqRows == 4, "the in-order part stages its errors as one float4 per column");
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x in [0, 3] to an integer
+static_assert(kLqStageBytes % 128 == 0 && kLqDiagOff % 128 == 0, "TMA destinations stay aligned");
+static_assert(kLqTBytes % 16 == 0 && kLqEstOff % 16 == 0 && kLqPOff % 16 == 0, "16-byte rows");
+static_assert(kLqGemm * 32 * 8 == kLqRows * kLqBlk, "each product thread sums 8 outputs");
+static_assert(kLqSmem <= 232448, "fits in one SM's shared memory");
 
 struct LdlqParams {
   CUtensorMap u;        // U [K][K] fp32, box 64 x 64, no swizzle
@@ -68,12 +81,34 @@ struct LdlqParams {
   unsigned int* err;
 };
 
-__device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, %0;\n" ::"n"(kLqCons * 32) : "memory");
+__device__ __forceinline__ void gemm_sync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(kLqGemm * 32) : "memory");
 }
 // generic-proxy global writes -> visible to later bulk (async-proxy) reads
 __device__ __forceinline__ void fence_async_global() {
   asm volatile("fence.proxy.async.global;\n" ::: "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// a shared-memory load kept in program order (volatile), so that the fully
+// unrolled in-order loop does not hoist every row of the diagonal tile into
+// registers ahead of its use
+__device__ __forceinline__ float4 lds_f4_ordered(const float* ptr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(sm100::smem_u32(ptr)));
+  return v;
 }
 
 __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_constant__ LdlqParams p) {
@@ -81,8 +116,20 @@ __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_consta
   unsigned char* sm = lq_raw + ((128 - (sm100::smem_u32(lq_raw) & 127)) & 127);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kLqBarOff);
   uint64_t* empty = full + kLqStages;
-  uint64_t* ebar = empty + kLqStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ebar + 1);
+  uint64_t* dfull = empty + kLqStages;
+  uint64_t* dempty = dfull + 2;
+  uint64_t* tready = dempty + 2;  // T_b in shared memory (phase b - 1)
+  uint64_t* eready = tready + 1;  // block b's errors in shared memory (phase b)
+  // block b's errors in the workspace: ebar[b & 1], phase b / 2 (one barrier per
+  // parity of b, so that the producer, which waits for block b - 2, never finds
+  // the barrier two phases ahead of the one it waits for)
+  uint64_t* ebar = eready + 1;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ebar + 2);
+  float* diag = reinterpret_cast<float*>(sm + kLqDiagOff);
+  float* red = reinterpret_cast<float*>(sm + kLqRedOff);
+  float* tbuf = reinterpret_cast<float*>(sm + kLqTOff);
+  float* est = reinterpret_cast<float*>(sm + kLqEstOff);
+  float* pbuf = reinterpret_cast<float*>(sm + kLqPOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t K = p.K;
@@ -93,38 +140,57 @@ __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_consta
   if (threadIdx.x == 0) {
     for (int s = 0; s < kLqStages; ++s) {
       sm100::mbar_init(&full[s], 1);
-      sm100::mbar_init(&empty[s], kLqCons);
+      sm100::mbar_init(&empty[s], kLqGemm);
     }
-    sm100::mbar_init(ebar, kLqCons * 32);
+    for (int s = 0; s < 2; ++s) {
+      sm100::mbar_init(&dfull[s], 1);
+      sm100::mbar_init(&dempty[s], 1);
+    }
+    sm100::mbar_init(tready, kLqGemm * 32);
+    sm100::mbar_init(eready, 32);
+    sm100::mbar_init(&ebar[0], 32);
+    sm100::mbar_init(&ebar[1], 32);
     *abort_flag = 0;
     sm100::fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kLqCons) {
+  // bounded wait; after a timeout anywhere in the CTA every later wait is skipped
+  auto wait = [&](uint64_t* bar, uint32_t parity, unsigned site) {
+    if (*abort_flag) return false;
+    if (!sm100::mbar_wait(bar, parity, kLqWaitLimit)) {
+      if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, site);
+      *abort_flag = 1;
+      return false;
+    }
+    return true;
+  };
+
+  if (warp == kLqProdWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) sm100::tma_prefetch_map(&p.u);
-    int seq = 0;  // stages issued
+    int seq = 0, nd = 0;  // ring stages and diagonal tiles issued
     for (int b = 0; b < nb && !*abort_flag; ++b) {
-      for (int c = 0; c <= b; ++c) {
+      const int db = b & 1;
+      if (!wait(&dempty[db], ((b >> 1) & 1) ^ 1, 70)) break;
+      if (lane == 0) {
+        sm100::mbar_arrive_expect_tx(&dfull[db], kLqUBytes);
+        sm100::tma_load_2d(&p.u, &dfull[db], diag + db * (kLqBlk * kLqBlk), b * kLqBlk, b * kLqBlk);
+      }
+      __syncwarp();
+      ++nd;
+      for (int c = 0; c < b; ++c) {
         const int s = seq % kLqStages;
-        if (!sm100::mbar_wait(&empty[s], ((seq / kLqStages) & 1) ^ 1, kLqWaitLimit)) {
-          if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, 70);
-          *abort_flag = 1;
-          break;
-        }
-        // the newest chunk of errors exists once block b - 1 has been stored
-        if (c == b - 1 && !sm100::mbar_wait(ebar, (b - 1) & 1, kLqWaitLimit)) {
-          if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, 71);
-          *abort_flag = 1;
-          break;
-        }
+        if (!wait(&empty[s], ((seq / kLqStages) & 1) ^ 1, 71)) break;
+        // chunk b - 1 of the errors is read from shared memory by the product
+        // warps; the older ones come from the workspace, once stored
+        const bool with_e = c + 1 < b;
+        if (with_e && c == b - 2 && !wait(&ebar[b & 1], ((b - 2) >> 1) & 1, 72)) break;
         if (lane == 0) {
           unsigned char* st = sm + s * kLqStageBytes;
-          const bool diag = c == b;
-          sm100::mbar_arrive_expect_tx(&full[s], kLqUBytes + (diag ? 0u : kLqEBytes));
+          sm100::mbar_arrive_expect_tx(&full[s], kLqUBytes + (with_e ? kLqEBytes : 0u));
           sm100::tma_load_2d(&p.u, &full[s], st, b * kLqBlk, c * kLqBlk);
-          if (!diag)
+          if (with_e)
             sm100::bulk_load(sm100::smem_u32(st + kLqUBytes), Ecta + int64_t(c) * kLqBlk * kLqRows,
                              kLqEBytes, &full[s]);
         }
@@ -132,37 +198,119 @@ __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_consta
         ++seq;
       }
     }
-    // no copy may outlive the CTA: wait until the last stages issued have landed
-    for (int q = seq > kLqStages ? seq - kLqStages : 0; q < seq; ++q) {
+    // no copy may outlive the CTA: wait until the last tiles issued have landed
+    for (int q = seq > kLqStages ? seq - kLqStages : 0; q < seq; ++q)
       if (!sm100::mbar_wait(&full[q % kLqStages], (q / kLqStages) & 1, kLqWaitLimit)) {
-        if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, 72);
+        if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, 73);
         break;
       }
-    }
+    for (int q = nd > 2 ? nd - 2 : 0; q < nd; ++q)
+      if (!sm100::mbar_wait(&dfull[q & 1], (q >> 1) & 1, kLqWaitLimit)) {
+        if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, 74);
+        break;
+      }
     return;
   }
 
-  // ------------------------------------------------------------ consumers
-  // product lane tile 8 x 8: rows 8 rg .. 8 rg + 7, columns 4 cg .. 4 cg + 3 and
+  if (warp == kLqSeqWarp) {
+    // ------------------------------------------------------------ in order, lane = row
+    const int64_t grow = row0 + lane;
+    const bool live = grow < p.N;
+    const float* prow = p.P + (live ? grow : 0) * K;
+    auto prefetch = [&](int b) {
+      const uint32_t dst = sm100::smem_u32(pbuf + (b & 1) * (kLqRows * kLqTPitch) + lane * kLqTPitch);
+#pragma unroll
+      for (int m = 0; m < kLqBlk / 4; ++m) cp_async16(dst + 16 * m, prow + int64_t(b) * kLqBlk + 4 * m, live);
+      cp_async_commit();
+    };
+    prefetch(0);
+    for (int b = 0; b < nb; ++b) {
+      const int64_t j0 = int64_t(b) * kLqBlk;
+      cp_async_wait_all();
+      __syncwarp();
+      // the block's targets stay in shared memory (read 4 at a time below)
+      const float4* pr = reinterpret_cast<const float4*>(pbuf + (b & 1) * (kLqRows * kLqTPitch) + lane * kLqTPitch);
+      if (b + 1 < nb) prefetch(b + 1);  // into the other buffer
+      if (b > 0) wait(tready, (b - 1) & 1, 75);
+      const int db = b & 1;
+      wait(&dfull[db], (b >> 1) & 1, 76);
+      const float* dg = diag + db * (kLqBlk * kLqBlk);
+      uint32_t code[4] = {0u, 0u, 0u, 0u};
+      float* erow = Ecta + j0 * kLqRows + lane;
+      // two halves of 32 columns: the second half first takes the first half's
+      // errors as a product (independent FMAs), then runs in order
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float c[32];
+        if (b > 0) {
+          const float4* tr = reinterpret_cast<const float4*>(tbuf + lane * kLqTPitch + 32 * h);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 v = tr[m];
+            c[4 * m] = v.x, c[4 * m + 1] = v.y, c[4 * m + 2] = v.z, c[4 * m + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) c[k] = 0.f;
+        }
+        if (h == 1) {
+#pragma unroll 1
+          for (int j = 0; j < 32; ++j) {
+            const float e = est[j * kLqRows + lane];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+              const float4 u = lds_f4_ordered(dg + j * kLqBlk + 32 + 4 * m);
+              c[4 * m] = fmaf(u.x, e, c[4 * m]);
+              c[4 * m + 1] = fmaf(u.y, e, c[4 * m + 1]);
+              c[4 * m + 2] = fmaf(u.z, e, c[4 * m + 2]);
+              c[4 * m + 3] = fmaf(u.w, e, c[4 * m + 3]);
+            }
+          }
+        }
+        float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = 32 * h + jj;
+          asm volatile("" ::: "memory");  // keep each step's loads with the step
+          if ((jj & 3) == 0) p4 = pr[j >> 2];
+          const float pj = (jj & 3) == 0 ? p4.x : (jj & 3) == 1 ? p4.y : (jj & 3) == 2 ? p4.z : p4.w;
+          const float xc = fminf(fmaxf(pj + c[jj], 0.f), 3.f);  // NaN -> 0
+          const float zb = __fadd_rn(xc, kRoundMagic);           // integer in the low bits
+          const float e = pj - __fadd_rn(zb, -kRoundMagic);
+          code[j >> 4] |= (__float_as_uint(zb) & 3u) << (2 * (j & 15));
+          est[j * kLqRows + lane] = e;
+          erow[j * kLqRows] = e;
+          // only U[i][j] with i < j is read: the columns after j
+#pragma unroll
+          for (int m = (jj + 1) >> 2; m < 8; ++m) {
+            const float4 u = lds_f4_ordered(dg + j * kLqBlk + 32 * h + 4 * m);
+            if (4 * m > jj) c[4 * m] = fmaf(u.x, e, c[4 * m]);
+            if (4 * m + 1 > jj) c[4 * m + 1] = fmaf(u.y, e, c[4 * m + 1]);
+            if (4 * m + 2 > jj) c[4 * m + 2] = fmaf(u.z, e, c[4 * m + 2]);
+            c[4 * m + 3] = fmaf(u.w, e, c[4 * m + 3]);
+          }
+        }
+      }
+      if (live)
+        *reinterpret_cast<uint4*>(p.packed + grow * (K / 4) + j0 / 4) =
+            make_uint4(code[0], code[1], code[2], code[3]);
+      __syncwarp();
+      sm100::mbar_arrive(eready);
+      fence_async_global();
+      sm100::mbar_arrive(&ebar[b & 1]);
+      if (lane == 0) sm100::mbar_arrive(&dempty[db]);
+    }
+    cp_async_wait_all();
+    return;
+  }
+
+  // ------------------------------------------------------------ product warps
+  // lane tile 8 x 8: rows 8 rg .. 8 rg + 7, columns 4 cg .. 4 cg + 3 and
   // 32 + 4 cg .. 32 + 4 cg + 3, so that every quarter-warp reads 128 contiguous
   // bytes of U and one broadcast 16 bytes of E per shared-memory load
   const int rg = lane >> 3, cg = lane & 7;
-  const int sr = kLqSeqRows * warp;  // rows of the in-order part: sr .. sr + 3
-  float* red = reinterpret_cast<float*>(sm + kLqRedOff);
-  float* est = reinterpret_cast<float*>(sm + kLqEstOff);
-  uint8_t* zst = sm + kLqZOff;
-  int seq = 0;  // stages consumed
-  for (int b = 0; b < nb; ++b) {
-    const int64_t j0 = int64_t(b) * kLqBlk;
-    float pv[kLqSeqRows][2];
-#pragma unroll
-    for (int r = 0; r < kLqSeqRows; ++r) {
-      const int64_t gr = row0 + sr + r;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) pv[r][h] = gr < p.N ? __ldg(p.P + gr * K + j0 + lane + 32 * h) : 0.f;
-    }
-
-    // 1. T_b = E_{<b} U[<j0, block]: this warp's k rows of every chunk
+  int seq = 0;  // ring stages consumed
+  for (int b = 1; b < nb; ++b) {
     float acc[8][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -170,12 +318,13 @@ __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_consta
       for (int q = 0; q < 8; ++q) acc[i][q] = 0.f;
     for (int c = 0; c < b; ++c, ++seq) {
       const int s = seq % kLqStages;
-      if (!*abort_flag && !sm100::mbar_wait(&full[s], (seq / kLqStages) & 1, kLqWaitLimit)) {
-        if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, 73);
-        *abort_flag = 1;
-      }
+      wait(&full[s], (seq / kLqStages) & 1, 77);
       const float* us = reinterpret_cast<const float*>(sm + s * kLqStageBytes);
       const float* es = us + kLqBlk * kLqBlk;
+      if (c + 1 == b) {  // the newest errors: block b - 1, straight from the in-order warp
+        wait(eready, (b - 1) & 1, 78);
+        es = est;
+      }
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int k = 8 * warp + r;
@@ -193,102 +342,30 @@ __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&empty[s]);
     }
-    if (b > 0) {
-      float* rw = red + warp * (kLqRows * kLqBlk);
+    float* rw = red + warp * (kLqRows * kLqBlk);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float* dst = rw + (8 * rg + i) * kLqBlk + 4 * cg;
-        *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-        *reinterpret_cast<float4*>(dst + 32) = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-      }
+    for (int i = 0; i < 8; ++i) {
+      float* dst = rw + (8 * rg + i) * kLqBlk + 4 * cg;
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      *reinterpret_cast<float4*>(dst + 32) = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
     }
-    consumers_sync();
-    float t[kLqSeqRows][2];
-#pragma unroll
-    for (int r = 0; r < kLqSeqRows; ++r)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float sum = 0.f;
-        if (b > 0) {
-#pragma unroll
-          for (int w = 0; w < kLqCons; ++w) sum += red[w * (kLqRows * kLqBlk) + (sr + r) * kLqBlk + lane + 32 * h];
-        }
-        t[r][h] = pv[r][h] + sum;
-      }
-
-    // 2. the block in order, with the diagonal tile U[j0 .., j0 ..]
-    float eo[kLqSeqRows][2];
-    uint32_t zo[kLqSeqRows][2];
-#pragma unroll
-    for (int r = 0; r < kLqSeqRows; ++r) eo[r][0] = eo[r][1] = 0.f, zo[r][0] = zo[r][1] = 0u;
+    gemm_sync();
     {
-      const int s = seq % kLqStages;
-      if (!*abort_flag && !sm100::mbar_wait(&full[s], (seq / kLqStages) & 1, kLqWaitLimit)) {
-        if (lane == 0) record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, 74);
-        *abort_flag = 1;
-      }
-      const float* dg = reinterpret_cast<const float*>(sm + s * kLqStageBytes);
-      // columns 0 .. 31 of the block (held in t[.][0]), then 32 .. 63 (t[.][1])
-#pragma unroll 2
-      for (int j = 0; j < 32; ++j) {
-        const float u0 = dg[j * kLqBlk + lane];
-        const float u1 = dg[j * kLqBlk + lane + 32];
+      // thread i sums row i / 8, columns 4 (i % 8) .. + 3 and 32 + 4 (i % 8) .. + 3
+      const int row = threadIdx.x >> 3, c4 = 4 * (threadIdx.x & 7);
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
 #pragma unroll
-        for (int r = 0; r < kLqSeqRows; ++r) {
-          const float z = fminf(fmaxf(rintf(t[r][0]), 0.f), 3.f);  // NaN -> 0
-          const float e = __shfl_sync(0xffffffffu, pv[r][0] - z, j);
-          if (lane == j) {
-            eo[r][0] = e;
-            zo[r][0] = static_cast<uint32_t>(z);
-          }
-          // only U[i][j] with i < j is read: the columns after j
-          if (lane > j) t[r][0] = fmaf(u0, e, t[r][0]);
-          t[r][1] = fmaf(u1, e, t[r][1]);
-        }
+      for (int w = 0; w < kLqGemm; ++w) {
+        const float4 a = *reinterpret_cast<const float4*>(red + w * (kLqRows * kLqBlk) + row * kLqBlk + c4);
+        const float4 b4 = *reinterpret_cast<const float4*>(red + w * (kLqRows * kLqBlk) + row * kLqBlk + 32 + c4);
+        s0.x += a.x, s0.y += a.y, s0.z += a.z, s0.w += a.w;
+        s1.x += b4.x, s1.y += b4.y, s1.z += b4.z, s1.w += b4.w;
       }
-#pragma unroll 2
-      for (int j = 0; j < 32; ++j) {
-        const float u1 = dg[(32 + j) * kLqBlk + lane + 32];
-#pragma unroll
-        for (int r = 0; r < kLqSeqRows; ++r) {
-          const float z = fminf(fmaxf(rintf(t[r][1]), 0.f), 3.f);
-          const float e = __shfl_sync(0xffffffffu, pv[r][1] - z, j);
-          if (lane == j) {
-            eo[r][1] = e;
-            zo[r][1] = static_cast<uint32_t>(z);
-          }
-          if (lane > j) t[r][1] = fmaf(u1, e, t[r][1]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&empty[s]);
-      ++seq;
+      *reinterpret_cast<float4*>(tbuf + row * kLqTPitch + c4) = s0;
+      *reinterpret_cast<float4*>(tbuf + row * kLqTPitch + 32 + c4) = s1;
     }
-
-    // 3. stage the block's errors and codes, then store them
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int col = lane + 32 * h;
-      *reinterpret_cast<float4*>(est + col * kLqRows + sr) =
-          make_float4(eo[0][h], eo[1][h], eo[2][h], eo[3][h]);
-#pragma unroll
-      for (int r = 0; r < kLqSeqRows; ++r) {
-        uint32_t v = zo[r][h] << (2 * (lane & 3));
-        v |= __shfl_xor_sync(0xffffffffu, v, 1);
-        v |= __shfl_xor_sync(0xffffffffu, v, 2);
-        if ((lane & 3) == 0) zst[(sr + r) * 16 + (col >> 2)] = static_cast<uint8_t>(v);
-      }
-    }
-    consumers_sync();
-    const int tid = threadIdx.x;  // 0 .. 255
-    float4* edst = reinterpret_cast<float4*>(Ecta + j0 * kLqRows);
-    edst[tid] = reinterpret_cast<const float4*>(est)[tid];
-    edst[tid + kLqCons * 32] = reinterpret_cast<const float4*>(est)[tid + kLqCons * 32];
-    if (tid < kLqRows && row0 + tid < p.N)
-      *reinterpret_cast<uint4*>(p.packed + (row0 + tid) * (K / 4) + j0 / 4) =
-          reinterpret_cast<const uint4*>(zst)[tid];
-    fence_async_global();
-    sm100::mbar_arrive(ebar);
+    gemm_sync();  // the partials are read before the next block writes them
+    sm100::mbar_arrive(tready);
   }
 }
 

@@ -179,7 +179,10 @@ def test_ldlq_full_size_qat_matrix():
     P = synth.wp_uniform(N, K, g)
     U = (g.standard_normal((K, K), dtype=np.float32) * np.float32(1.0 / np.sqrt(K)))
     U = np.triu(U, 1)
-    out = lcvq.assign_ldlq(torch.from_numpy(P).to(dev()), torch.from_numpy(U).to(dev()), 8)
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_ASSIGN_LDLQ, torch.float32, 0, N, K, 8))
+    out = lcvq.assign_ldlq(torch.from_numpy(P).to(dev()), torch.from_numpy(U).to(dev()), 8,
+                           workspace=ws)
+    assert lcvq.check_device_error(ws) == 0
     rows = np.array([0, 1, 2047, 4095] + list(g.choice(N, 4, replace=False)))
     Z = O.unpack_codes(out.cpu().numpy()[rows], K)
     bad, near = ldlq_check(P[rows], U, Z)

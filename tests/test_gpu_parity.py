@@ -459,7 +459,12 @@ def _ldlq_case(N, K, d=8, n_cal=None):
 
 
 def _ldlq_gpu(P, U, d=8):
-    return lcvq.assign_ldlq(torch.from_numpy(P).to(dev()), torch.from_numpy(U).to(dev()), d)
+    N, K = P.shape
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_ASSIGN_LDLQ, torch.float32, 0, N, K, d))
+    out = lcvq.assign_ldlq(torch.from_numpy(P).to(dev()), torch.from_numpy(U).to(dev()), d,
+                           workspace=ws)
+    assert lcvq.check_device_error(ws) == 0
+    return out
 
 
 @pytest.mark.parametrize("N,K", [(50, 256), (33, 640)])

@@ -18,14 +18,16 @@
 //     chunk, fp32 FFMA with a lane tile of 8 rows x 8 columns (16 values
 //     loaded per 64 FMAs, which balances the shared-memory and FMA pipes);
 //     the 8 partial tiles are summed in warp order into T_b in shared memory;
-//   * warp 8 rounds block b in order, one lane per row, holding the row's 64
-//     targets and compensations in registers: t_j = p_j + c_j, z_j by a
-//     clamp and the magic-number rounding (ties to even, on the FMA pipe),
-//     e_j = p_j - z_j, then c_k += U[j0 + j][j0 + k] e_j for the later columns
-//     (the diagonal tile; its rows are read as warp-wide broadcasts).  Its
-//     errors go to shared memory, where warps 0..7 take the newest chunk of
-//     T_{b+1} from, and to the workspace, where the older chunks come from;
-//     it prefetches the next block's targets with cp.async;
+//   * warp 8 rounds block b in order, one lane per row: t_j = p_j + c_j, z_j
+//     by a clamp and the magic-number rounding (ties to even, on the FMA
+//     pipe), e_j = p_j - z_j, and the later columns of the block take
+//     U[j0 + j][j0 + k] e_j (the diagonal tile, read as warp-wide broadcasts).
+//     It goes in sub-blocks of 8 columns: a sub-block first takes the errors
+//     of the earlier sub-blocks as a small product, then runs in order, so
+//     only 8 compensations are live.  Its errors go to shared memory, where
+//     warps 0..7 take the newest chunk of T_{b+1} from, and to the workspace,
+//     where the older chunks come from; it prefetches the next block's
+//     targets with cp.async;
 //   * warp 9 streams, through TMA, the 64 x 64 tiles U[64c .., j0 ..] with the
 //     CTA's error chunks E[64c .., 32 rows] (a ring of stages) and the
 //     diagonal tiles (two buffers).
@@ -98,17 +100,6 @@ __device__ __forceinline__ void cp_async_commit() {
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-}
-
-// a shared-memory load kept in program order (volatile), so that the fully
-// unrolled in-order loop does not hoist every row of the diagonal tile into
-// registers ahead of its use
-__device__ __forceinline__ float4 lds_f4_ordered(const float* ptr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(sm100::smem_u32(ptr)));
-  return v;
 }
 
 __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_constant__ LdlqParams p) {
@@ -237,57 +228,49 @@ __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_consta
       const float* dg = diag + db * (kLqBlk * kLqBlk);
       uint32_t code[4] = {0u, 0u, 0u, 0u};
       float* erow = Ecta + j0 * kLqRows + lane;
-      // two halves of 32 columns: the second half first takes the first half's
-      // errors as a product (independent FMAs), then runs in order
+      // eight sub-blocks of 8 columns: sub-block q first takes the errors of
+      // sub-blocks 0 .. q-1 as a small product (independent FMAs), then runs
+      // its 8 columns in order; only 8 compensations are live at a time
+      const float4* dg4 = reinterpret_cast<const float4*>(dg);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float c[32];
+      for (int q = 0; q < 8; ++q) {
+        float cs[8];
         if (b > 0) {
-          const float4* tr = reinterpret_cast<const float4*>(tbuf + lane * kLqTPitch + 32 * h);
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float4 v = tr[m];
-            c[4 * m] = v.x, c[4 * m + 1] = v.y, c[4 * m + 2] = v.z, c[4 * m + 3] = v.w;
-          }
+          const float4 t0 = *reinterpret_cast<const float4*>(tbuf + lane * kLqTPitch + 8 * q);
+          const float4 t1 = *reinterpret_cast<const float4*>(tbuf + lane * kLqTPitch + 8 * q + 4);
+          cs[0] = t0.x, cs[1] = t0.y, cs[2] = t0.z, cs[3] = t0.w;
+          cs[4] = t1.x, cs[5] = t1.y, cs[6] = t1.z, cs[7] = t1.w;
         } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) c[k] = 0.f;
+          for (int k = 0; k < 8; ++k) cs[k] = 0.f;
         }
-        if (h == 1) {
-#pragma unroll 1
-          for (int j = 0; j < 32; ++j) {
-            const float e = est[j * kLqRows + lane];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-              const float4 u = lds_f4_ordered(dg + j * kLqBlk + 32 + 4 * m);
-              c[4 * m] = fmaf(u.x, e, c[4 * m]);
-              c[4 * m + 1] = fmaf(u.y, e, c[4 * m + 1]);
-              c[4 * m + 2] = fmaf(u.z, e, c[4 * m + 2]);
-              c[4 * m + 3] = fmaf(u.w, e, c[4 * m + 3]);
-            }
-          }
+#pragma unroll 4
+        for (int j = 0; j < 8 * q; ++j) {
+          const float e = est[j * kLqRows + lane];
+          const float4 u0 = dg4[j * (kLqBlk / 4) + 2 * q];
+          const float4 u1 = dg4[j * (kLqBlk / 4) + 2 * q + 1];
+          cs[0] = fmaf(u0.x, e, cs[0]), cs[1] = fmaf(u0.y, e, cs[1]);
+          cs[2] = fmaf(u0.z, e, cs[2]), cs[3] = fmaf(u0.w, e, cs[3]);
+          cs[4] = fmaf(u1.x, e, cs[4]), cs[5] = fmaf(u1.y, e, cs[5]);
+          cs[6] = fmaf(u1.z, e, cs[6]), cs[7] = fmaf(u1.w, e, cs[7]);
         }
-        float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 p0 = pr[2 * q], p1 = pr[2 * q + 1];
+        const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = 32 * h + jj;
-          asm volatile("" ::: "memory");  // keep each step's loads with the step
-          if ((jj & 3) == 0) p4 = pr[j >> 2];
-          const float pj = (jj & 3) == 0 ? p4.x : (jj & 3) == 1 ? p4.y : (jj & 3) == 2 ? p4.z : p4.w;
-          const float xc = fminf(fmaxf(pj + c[jj], 0.f), 3.f);  // NaN -> 0
-          const float zb = __fadd_rn(xc, kRoundMagic);           // integer in the low bits
-          const float e = pj - __fadd_rn(zb, -kRoundMagic);
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = 8 * q + jj;
+          const float xc = fminf(fmaxf(pv[jj] + cs[jj], 0.f), 3.f);  // NaN -> 0
+          const float zb = __fadd_rn(xc, kRoundMagic);               // integer in the low bits
+          const float e = pv[jj] - __fadd_rn(zb, -kRoundMagic);
           code[j >> 4] |= (__float_as_uint(zb) & 3u) << (2 * (j & 15));
           est[j * kLqRows + lane] = e;
           erow[j * kLqRows] = e;
-          // only U[i][j] with i < j is read: the columns after j
+          if (jj < 7) {  // only U[i][j] with i < j is read: the columns after j
+            const float4 u0 = dg4[j * (kLqBlk / 4) + 2 * q];
+            const float4 u1 = dg4[j * (kLqBlk / 4) + 2 * q + 1];
+            const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-          for (int m = (jj + 1) >> 2; m < 8; ++m) {
-            const float4 u = lds_f4_ordered(dg + j * kLqBlk + 32 * h + 4 * m);
-            if (4 * m > jj) c[4 * m] = fmaf(u.x, e, c[4 * m]);
-            if (4 * m + 1 > jj) c[4 * m + 1] = fmaf(u.y, e, c[4 * m + 1]);
-            if (4 * m + 2 > jj) c[4 * m + 2] = fmaf(u.z, e, c[4 * m + 2]);
-            c[4 * m + 3] = fmaf(u.w, e, c[4 * m + 3]);
+            for (int k = jj + 1; k < 8; ++k) cs[k] = fmaf(uv[k], e, cs[k]);
           }
         }
       }
@@ -325,15 +308,23 @@ __global__ void __launch_bounds__(kLqThreads, 1) ldlq_kernel(const __grid_consta
         wait(eready, (b - 1) & 1, 78);
         es = est;
       }
+      // operands of k row r + 1 are loaded before the FMAs of row r
+      const float* ep = es + (8 * warp) * kLqRows + 8 * rg;
+      const float* upp = us + (8 * warp) * kLqBlk + 4 * cg;
+      float4 e0 = *reinterpret_cast<const float4*>(ep);
+      float4 e1 = *reinterpret_cast<const float4*>(ep + 4);
+      float4 u0 = *reinterpret_cast<const float4*>(upp);
+      float4 u1 = *reinterpret_cast<const float4*>(upp + 32);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const int k = 8 * warp + r;
-        const float4 e0 = *reinterpret_cast<const float4*>(es + k * kLqRows + 8 * rg);
-        const float4 e1 = *reinterpret_cast<const float4*>(es + k * kLqRows + 8 * rg + 4);
-        const float4 u0 = *reinterpret_cast<const float4*>(us + k * kLqBlk + 4 * cg);
-        const float4 u1 = *reinterpret_cast<const float4*>(us + k * kLqBlk + 32 + 4 * cg);
         const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
         const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        if (r + 1 < 8) {
+          e0 = *reinterpret_cast<const float4*>(ep + (r + 1) * kLqRows);
+          e1 = *reinterpret_cast<const float4*>(ep + (r + 1) * kLqRows + 4);
+          u0 = *reinterpret_cast<const float4*>(upp + (r + 1) * kLqBlk);
+          u1 = *reinterpret_cast<const float4*>(upp + (r + 1) * kLqBlk + 32);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll

@@ -167,6 +167,18 @@ def ev_time(fn, n, stream=None):
     return e0.elapsed_time(e1) / n
 
 
+def graph_time(fn, n, reps=3):
+    """Device time (ms) per call of fn(), from a CUDA graph of n back-to-back
+    calls replayed `reps` times: no host overhead between the kernels (a
+    Python-level call costs tens of microseconds, more than a short kernel)."""
+    g = capture(lambda: [fn() for _ in range(n)])
+    g.replay()
+    torch.cuda.synchronize()
+    ms = ev_time(g.replay, reps)
+    del g
+    return ms / n
+
+
 def capture(fn):
     """CUDA graph of fn() (the library launches on torch's current stream, which
     is the capture stream inside the context)."""
@@ -412,7 +424,7 @@ def row_assign_pack(D, pk):
     Wp = torch.from_numpy(w["Wp"]).to(dev)
     packed = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
     mask = torch.empty((N, K // 8), dtype=torch.uint8, device=dev)
-    ms = ev_time(lambda: lcvq.assign_pack(Wp, 8, packed=packed, mask=mask), 50)
+    ms = graph_time(lambda: lcvq.assign_pack(Wp, 8, packed=packed, mask=mask), 20)
     nbytes = N * K * (4 + 0.25 + 0.125)
     gbs = nbytes / (ms * 1e-3) / 1e9
     return dict(metric="assign+pack GB/s (fp32 in, codes+mask out)", value=gbs, unit="GB/s",
@@ -429,7 +441,7 @@ def row_decode(D, pk):
     A = torch.from_numpy(w["A"]).to(dev)
     B = torch.from_numpy(w["B"]).to(dev)
     W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
-    ms = ev_time(lambda: lcvq.decode(packed, K, A, B, 8, out=W), 50)
+    ms = graph_time(lambda: lcvq.decode(packed, K, A, B, 8, out=W), 20)
     nbytes = N * K * (0.25 + 2)
     gbs = nbytes / (ms * 1e-3) / 1e9
     return dict(metric="decode GB/s (codes in, bf16 W~ out)", value=gbs, unit="GB/s", us=ms * 1e3,
@@ -607,7 +619,7 @@ def row_fit(D, pk):
     nbytes = N * K * (4 + 0.25)
     out = {}
     for name, hh in (("unweighted", None), ("weighted", h)):
-        ms = ev_time(lambda: lcvq.fit_affine(W0, packed, d, h=hh, workspace=ws, A=A, B=B), 30)
+        ms = graph_time(lambda: lcvq.fit_affine(W0, packed, d, h=hh, workspace=ws, A=A, B=B), 10)
         gbs = nbytes / (ms * 1e-3) / 1e9
         out[name] = dict(value=gbs, unit="GB/s", us=ms * 1e3,
                          roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",

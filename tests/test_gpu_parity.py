@@ -72,6 +72,24 @@ def test_decode(d, dtype):
     assert_close("decode", to_np(W), ref, D, tol)
 
 
+@pytest.mark.parametrize("shape", [(1, 16), (3, 48), (37, 528), (128, 4096)])
+def test_decode_d8_bf16_ragged_and_exact_zero(shape):
+    """d = 8 to bf16 runs on the tensor cores: shapes whose vector count ends
+    inside a warp's batch, and exact results where the pages' values are exact
+    (zero codes with B = 0 give exact zeros)."""
+    N, K = shape
+    g = np.random.Generator(np.random.PCG64(110 + N))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    z[0, :8] = 0
+    A, B = synth.affine_diag_dominant(8, g)
+    B[:] = 0.0
+    W = lcvq.decode(torch.from_numpy(O.pack_codes(z)).to(dev()), K, torch.from_numpy(A).to(dev()),
+                    torch.from_numpy(B).to(dev()), 8)
+    ref = O.decode(z, A, B)
+    assert_close("decode d=8", to_np(W), ref, O.decode_abs(z, A, B), 2.0 ** -8)
+    assert np.all(to_np(W)[0, :8] == 0.0)
+
+
 # --------------------------------------------------------------- forward
 def _fwd_case(wid, M, d_in, d_out, d=None, seed_shift=0):
     w = synth.workload(wid, M=M, d_in=d_in, d_out=d_out, d=d, with_dy=False)

@@ -10,12 +10,10 @@
 // its channel k = g d + i and zt = [z_0 .. z_{d-1}, 1]:
 //   G_i = sum h_k zt zt^T,   R_i = sum h_k W0[n][k] zt.
 //
-//  * fit_accum_kernel: one pass over W0 and the codes.  Lane (v, i) of a warp
-//    takes coordinate i of vector v of each group of 32/d consecutive vectors
-//    (32 consecutive floats of W0: coalesced) and keeps its G_i (upper
-//    triangle) and R_i in registers: fp32 sums flushed into fp64 every 16
-//    elements (below).  Lanes of one i are summed by an xor-shuffle tree,
-//    warps in warp order in fp64, and each CTA writes one fp64 partial.
+//  * fit_accum_kernel: one pass over W0 and the codes, forming per vector
+//    position the integer Gram of its codes and the products of its targets
+//    with its codes; h is applied afterwards, per CTA, in fp64 (below).  Each
+//    CTA writes one fp64 partial of every G_i and R_i.
 //  * fit_solve_kernel: sums the partials in CTA order (fp64), then thread i
 //    forms theta_i = G_i^+ R_i in fp64: by Cholesky when every pivot is above
 //    1e-8 of the largest diagonal entry (G_i comfortably positive definite,
@@ -33,8 +31,6 @@ namespace lcvq {
 
 namespace {
 
-constexpr int kFitThreads = 256;
-constexpr int kFitWarps = kFitThreads / 32;
 constexpr double kPinvRcond = 1e-12;
 
 template <int D>
@@ -42,134 +38,160 @@ struct FitDims {
   static constexpr int P = D + 1;                 // zt length
   static constexpr int SG = P * (P + 1) / 2;      // upper triangle of G_i
   static constexpr int S = SG + P;                // G_i then R_i
-  static constexpr int kVecPerWarp = 32 / D;      // vectors per warp step
 };
 
-// Per-lane sums.  Terms are accumulated in fp32 and flushed into fp64 every
-// kFitFlush elements, so the rounding of a sum is at most kFitFlush * 2^-24
-// of the sum of its terms' absolute values, however long the sum.  Without
-// weights every G entry is an integer count, which fp32 holds exactly.
+// The pass over W0 and the codes.  With h applied per channel, the normal
+// equations are sums over the vector positions g of a row (channel k = g d + i):
+//     G_i = sum_g h_{gd+i} S_g,   S_g = sum_n zt zt^T   (zt of vector (n, g)),
+//     R_i = sum_g h_{gd+i} T_{g,i},   T_{g,i} = sum_n W0[n][gd+i] zt,
+// so the pass only forms S_g (an integer Gram: exact in fp32 over the rows
+// of one thread) and T_g; h enters afterwards, in fp64.
+//
+// fit_accum_kernel: lane l of a CTA owns vector position g = 32 c + l of column
+// tile c and its 4 warps split the CTA's rows.  Per row a lane loads the d
+// floats of its vector (a warp reads 32 d consecutive floats) and its code,
+// forms zt = [z_0 .. z_{d-1}, 1] once, and adds d (d+1) products to T and the
+// (d+1)(d+2)/2 upper-triangle products to S: about 2.3 (d+1) instructions per
+// weight instead of a Gram per weight.  T is fp32 flushed into fp64 (shared
+// memory) every kFitFlush rows, so each fp32 partial sums at most kFitFlush
+// terms.  The CTA then sums its warps in warp order, applies h per coordinate
+// in fp64 over its 32 positions in order, and writes one partial [d][G_i, R_i].
 constexpr int kFitFlush = 16;
-// grid-stride steps whose loads are in flight together, and CTAs per SM:
-// measured best (4096 x 14336, d = 8): unweighted 4 steps at 2 CTAs per SM
-// (128 registers, no spill); weighted 8 steps at 1 CTA (its fp64 mirror of G
-// does not fit 128 registers)
-template <bool kWeighted>
-struct FitShape {
-  static constexpr int kAhead = kWeighted ? 8 : 4;
-  static constexpr int kMinBlocks = kWeighted ? 1 : 2;
+constexpr int kFitLanes = 32;            // vector positions per CTA
+constexpr int kFitRowWarps = 4;          // warps per CTA, each a share of the rows
+constexpr int kFitThreads2 = kFitLanes * kFitRowWarps;
+constexpr int kFitAhead2 = 4;            // rows whose loads are in flight together
+constexpr int kFitTargetCtas = 2 * kNumSMsB200;
+
+template <int D>
+struct FitSmem {
+  using F = FitDims<D>;
+  static constexpr int kT = D * F::P;                        // T entries per position
+  static constexpr int kStage = (kT > F::SG ? kT : F::SG);   // fp64 per thread
+  static constexpr size_t kStageBytes = size_t(kStage) * kFitThreads2 * 8;
+  static constexpr size_t kPosBytes = size_t(kFitLanes) * (F::SG + kT) * 8;
+  static constexpr size_t kBytes = kStageBytes + kPosBytes;
 };
 
-template <int D, bool kWeighted>
-__global__ void __launch_bounds__(kFitThreads, FitShape<kWeighted>::kMinBlocks) fit_accum_kernel(
-    const float* __restrict__ W0, const uint32_t* __restrict__ codes, int64_t n_vec,
-    int64_t groups, const float* __restrict__ h, double* __restrict__ partials) {
+template <int D>
+__global__ void __launch_bounds__(kFitThreads2, 2) fit_accum_kernel(
+    const float* __restrict__ W0, const uint32_t* __restrict__ codes, int64_t N, int64_t groups,
+    int64_t row_splits, const float* __restrict__ h, double* __restrict__ partials) {
   using F = FitDims<D>;
-  constexpr int kG = F::SG;
-  // an fp64 mirror of G only where its terms are not integers
-  constexpr int kG64 = kWeighted ? F::SG : 1;
-  __shared__ double red[kFitWarps][D][F::S];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int vl = lane / D, i = lane % D;
-  float g32[kG], r32[F::P];
-  double g64[kG64], r64[F::P];
-#pragma unroll
-  for (int s = 0; s < kG; ++s) g32[s] = 0.f;
-#pragma unroll
-  for (int s = 0; s < kG64; ++s) g64[s] = 0.0;
-#pragma unroll
-  for (int s = 0; s < F::P; ++s) r32[s] = 0.f, r64[s] = 0.0;
+  using L = FitSmem<D>;
+  constexpr int P = F::P, kT = L::kT;
+  extern __shared__ __align__(16) unsigned char fit_smem[];
+  double* stage = reinterpret_cast<double*>(fit_smem);                 // [kStage][threads]
+  double* pos = reinterpret_cast<double*>(fit_smem + L::kStageBytes);   // [32][SG + kT]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t ct = int64_t(blockIdx.x) / row_splits, rs = int64_t(blockIdx.x) % row_splits;
+  const int64_t g = ct * kFitLanes + lane;
+  const bool live = g < groups;
+  const int64_t rows_per = ceil_div(N, row_splits);
+  const int64_t r_begin = rs * rows_per, r_end = r_begin + rows_per < N ? r_begin + rows_per : N;
+  const int64_t K = groups * D;
+  const int64_t words_per_row = K / 16;  // d_in % 16 == 0
+  const int64_t gbit = g * (2 * D);      // the vector's bits within its row
+  const uint32_t cshift = static_cast<uint32_t>(gbit & 31);
 
-  const int64_t steps = ceil_div(n_vec, F::kVecPerWarp);
-  const int64_t st0 = int64_t(blockIdx.x) * kFitWarps + warp;
-  const int64_t stride = int64_t(gridDim.x) * kFitWarps;
-  // channel of this lane's element, kept up to date without a division per element
-  const int64_t vstep = (stride * F::kVecPerWarp) % groups;
-  int64_t g = (st0 * F::kVecPerWarp + vl) % groups;
+  for (int q = 0; q < L::kStage; ++q) stage[q * kFitThreads2 + tid] = 0.0;
+  float t32[kT], s32[F::SG];
+#pragma unroll
+  for (int q = 0; q < kT; ++q) t32[q] = 0.f;
+#pragma unroll
+  for (int q = 0; q < F::SG; ++q) s32[q] = 0.f;
+
+  auto flush = [&]() {
+#pragma unroll
+    for (int q = 0; q < kT; ++q) {
+      stage[q * kFitThreads2 + tid] += double(t32[q]);
+      t32[q] = 0.f;
+    }
+  };
   int pending = 0;
-  // kFitAhead steps per round, their loads issued together (latency hiding)
-  constexpr int kFitAhead = FitShape<kWeighted>::kAhead;
-  for (int64_t st = st0; st < steps; st += stride * kFitAhead) {
-    float wv[kFitAhead];
-    uint32_t cw[kFitAhead];
+  for (int64_t n0 = r_begin + warp; n0 < r_end; n0 += int64_t(kFitRowWarps) * kFitAhead2) {
+    float wv[kFitAhead2][D];
+    uint32_t cw[kFitAhead2];
 #pragma unroll
-    for (int u = 0; u < kFitAhead; ++u) {
-      const int64_t vec = (st + u * stride) * F::kVecPerWarp + vl;
-      if (st + u * stride < steps && vec < n_vec) {
-        wv[u] = __ldcs(W0 + vec * D + i);
-        // the vector's 2D code bits start at bit 2 D vec of the packed stream
-        const int64_t bit = vec * (2 * D);
-        cw[u] = __ldg(codes + (bit >> 5)) >> (bit & 31);
+    for (int u = 0; u < kFitAhead2; ++u) {
+      const int64_t n = n0 + int64_t(u) * kFitRowWarps;
+      const bool ok = live && n < r_end;
+      const float* src = W0 + n * K + g * D;
+      if constexpr (D % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < D / 4; ++q) {
+          const float4 v = ok ? __ldcs(reinterpret_cast<const float4*>(src) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+          wv[u][4 * q] = v.x, wv[u][4 * q + 1] = v.y, wv[u][4 * q + 2] = v.z, wv[u][4 * q + 3] = v.w;
+        }
       } else {
-        wv[u] = 0.f;
-        cw[u] = 0u;
+#pragma unroll
+        for (int q = 0; q < D; ++q) wv[u][q] = ok ? __ldcs(src + q) : 0.f;
       }
+      cw[u] = ok ? __ldg(codes + n * words_per_row + (gbit >> 5)) >> cshift : 0u;
     }
 #pragma unroll
-    for (int u = 0; u < kFitAhead; ++u) {
-      const int64_t vec = (st + u * stride) * F::kVecPerWarp + vl;
-      if (st + u * stride < steps && vec < n_vec) {
-        const float w = wv[u];
-        const uint32_t word = cw[u];
-        // small integers to float without the conversion unit: OR the value
-        // into the mantissa of 2^23 and subtract 2^23
-        float zt[F::P];
+    for (int u = 0; u < kFitAhead2; ++u) {
+      const int64_t n = n0 + int64_t(u) * kFitRowWarps;
+      if (!(live && n < r_end)) continue;
+      // small integers to float without the conversion unit: OR the value
+      // into the mantissa of 2^23 and subtract 2^23
+      float zt[P];
 #pragma unroll
-        for (int j = 0; j < D; ++j)
-          zt[j] = __int_as_float(0x4B000000 | static_cast<int>((word >> (2 * j)) & 3u)) - 8388608.0f;
-        zt[D] = 1.f;
-        const float hw = kWeighted ? __ldg(h + g * D + i) : 1.f;
-        int s = 0;
+      for (int j = 0; j < D; ++j)
+        zt[j] = __int_as_float(0x4B000000 | static_cast<int>((cw[u] >> (2 * j)) & 3u)) - 8388608.0f;
+      zt[D] = 1.f;
 #pragma unroll
-        for (int a = 0; a < F::P; ++a) {
-          const float ha = kWeighted ? hw * zt[a] : zt[a];
+      for (int i = 0; i < D; ++i) {
 #pragma unroll
-          for (int b = a; b < F::P; ++b) {
-            g32[s] = fmaf(ha, zt[b], g32[s]);
-            ++s;
-          }
-        }
-        const float hwv = hw * w;
-#pragma unroll
-        for (int a = 0; a < F::P; ++a) r32[a] = fmaf(hwv, zt[a], r32[a]);
-        if (++pending == kFitFlush) {
-          pending = 0;
-          if constexpr (kWeighted) {
-#pragma unroll
-            for (int q = 0; q < kG; ++q) g64[q] += g32[q], g32[q] = 0.f;
-          }
-#pragma unroll
-          for (int q = 0; q < F::P; ++q) r64[q] += r32[q], r32[q] = 0.f;
-        }
+        for (int j = 0; j < D; ++j) t32[i * P + j] = fmaf(wv[u][i], zt[j], t32[i * P + j]);
+        t32[i * P + D] += wv[u][i];
       }
-      g += vstep;
-      if (g >= groups) g -= groups;
+      int q = 0;
+#pragma unroll
+      for (int a = 0; a < P; ++a)
+#pragma unroll
+        for (int b = a; b < P; ++b) {
+          s32[q] = fmaf(zt[a], zt[b], s32[q]);
+          ++q;
+        }
+      if (++pending == kFitFlush) {
+        pending = 0;
+        flush();
+      }
     }
   }
-  double gsum[kG];
-#pragma unroll
-  for (int q = 0; q < kG; ++q) gsum[q] = kWeighted ? g64[q < kG64 ? q : 0] + g32[q] : double(g32[q]);
-#pragma unroll
-  for (int q = 0; q < F::P; ++q) r64[q] += r32[q];
-  // lanes of one coordinate i: lanes i, i + D, ...; xor tree over those
-#pragma unroll
-  for (int off = D; off < 32; off <<= 1) {
-#pragma unroll
-    for (int q = 0; q < kG; ++q) gsum[q] += __shfl_xor_sync(0xffffffffu, gsum[q], off);
-#pragma unroll
-    for (int q = 0; q < F::P; ++q) r64[q] += __shfl_xor_sync(0xffffffffu, r64[q], off);
-  }
-  if (lane < D) {
-#pragma unroll
-    for (int q = 0; q < F::SG; ++q) red[warp][lane][q] = gsum[q];
-#pragma unroll
-    for (int q = 0; q < F::P; ++q) red[warp][lane][F::SG + q] = r64[q];
+  flush();
+  __syncthreads();
+  // per position: T summed over the warps in warp order ...
+  for (int e = tid; e < kFitLanes * kT; e += kFitThreads2) {
+    const int l = e / kT, q = e % kT;
+    double t = 0.0;
+    for (int w = 0; w < kFitRowWarps; ++w) t += stage[q * kFitThreads2 + w * 32 + l];
+    pos[l * (F::SG + kT) + F::SG + q] = t;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < D * F::S; e += kFitThreads) {
-    const int ii = e / F::S, q = e % F::S;
+  // ... then S (exact integers) through the same staging area
+#pragma unroll
+  for (int q = 0; q < F::SG; ++q) stage[q * kFitThreads2 + tid] = double(s32[q]);
+  __syncthreads();
+  for (int e = tid; e < kFitLanes * F::SG; e += kFitThreads2) {
+    const int l = e / F::SG, q = e % F::SG;
     double t = 0.0;
-    for (int w2 = 0; w2 < kFitWarps; ++w2) t += red[w2][ii][q];
+    for (int w = 0; w < kFitRowWarps; ++w) t += stage[q * kFitThreads2 + w * 32 + l];
+    pos[l * (F::SG + kT) + q] = t;
+  }
+  __syncthreads();
+  // h per coordinate, positions in order: one partial [d][G_i (SG), R_i (P)]
+  for (int e = tid; e < D * F::S; e += kFitThreads2) {
+    const int i = e / F::S, q = e % F::S;
+    double t = 0.0;
+    for (int l = 0; l < kFitLanes; ++l) {
+      const int64_t gg = ct * kFitLanes + l;
+      if (gg >= groups) break;
+      const double hw = h ? double(__ldg(h + gg * D + i)) : 1.0;
+      const double v = q < F::SG ? pos[l * (F::SG + kT) + q] : pos[l * (F::SG + kT) + F::SG + i * P + (q - F::SG)];
+      t += hw * v;
+    }
     partials[int64_t(blockIdx.x) * D * F::S + e] = t;
   }
 }
@@ -303,13 +325,18 @@ __global__ void __launch_bounds__(256) fit_solve_kernel(const double* __restrict
   B[i] = static_cast<float>(th[D]);
 }
 
-template <int D>
-int fit_grid(int64_t n_vec) {
-  const int64_t steps = ceil_div(n_vec, FitDims<D>::kVecPerWarp);
-  int64_t g = ceil_div(steps, kFitWarps);
-  const int64_t cap = int64_t(kNumSMsB200) * 4;
-  if (g > cap) g = cap;
-  return static_cast<int>(g < 1 ? 1 : g);
+// column tiles of 32 positions times row splits, about two CTAs per SM
+struct FitGrid {
+  int64_t tiles, splits;
+  int64_t ctas() const { return tiles * splits; }
+};
+inline FitGrid fit_grid(int64_t d_out, int64_t groups) {
+  FitGrid f{ceil_div(groups > 0 ? groups : 1, kFitLanes), 1};
+  if (f.tiles < kFitTargetCtas) f.splits = kFitTargetCtas / f.tiles;
+  const int64_t max_splits = ceil_div(d_out > 0 ? d_out : 1, 16);
+  if (f.splits > max_splits) f.splits = max_splits;
+  if (f.splits < 1) f.splits = 1;
+  return f;
 }
 
 template <int D>
@@ -317,17 +344,17 @@ cudaError_t launch_fit_t(const float* W0, const uint8_t* packed, int64_t d_out, 
                          const float* h, float* A, float* B, double* partials, cudaStream_t s,
                          int* launches) {
   const int64_t groups = d_in / D;
-  const int64_t n_vec = d_out * groups;
-  const int grid = fit_grid<D>(n_vec);
+  const FitGrid fg = fit_grid(d_out, groups);
   const uint32_t* codes = reinterpret_cast<const uint32_t*>(packed);
-  const int64_t gr = groups > 0 ? groups : 1;
-  if (h)
-    fit_accum_kernel<D, true><<<grid, kFitThreads, 0, s>>>(W0, codes, n_vec, gr, h, partials);
-  else
-    fit_accum_kernel<D, false><<<grid, kFitThreads, 0, s>>>(W0, codes, n_vec, gr, h, partials);
+  auto kern = fit_accum_kernel<D>;
+  if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), FitSmem<D>::kBytes);
+      e != cudaSuccess)
+    return e;
+  kern<<<static_cast<unsigned>(fg.ctas()), kFitThreads2, FitSmem<D>::kBytes, s>>>(
+      W0, codes, d_out, groups, fg.splits, h, partials);
   ++*launches;
   if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
-  fit_solve_kernel<D><<<1, 256, 0, s>>>(partials, grid, A, B);
+  fit_solve_kernel<D><<<1, 256, 0, s>>>(partials, static_cast<int>(fg.ctas()), A, B);
   ++*launches;
   return cudaGetLastError();
 }
@@ -335,12 +362,13 @@ cudaError_t launch_fit_t(const float* W0, const uint8_t* packed, int64_t d_out, 
 }  // namespace
 
 size_t fit_partials_bytes(int64_t d_out, int64_t d_in, int d) {
-  const int64_t n_vec = d > 0 ? d_out * (d_in / d) : 0;
+  if (d <= 0) return 0;
+  const size_t ctas = size_t(fit_grid(d_out, d_in / d).ctas());
   switch (d) {
-    case 1: return size_t(fit_grid<1>(n_vec)) * 1 * FitDims<1>::S * sizeof(double);
-    case 2: return size_t(fit_grid<2>(n_vec)) * 2 * FitDims<2>::S * sizeof(double);
-    case 4: return size_t(fit_grid<4>(n_vec)) * 4 * FitDims<4>::S * sizeof(double);
-    default: return size_t(fit_grid<8>(n_vec)) * 8 * FitDims<8>::S * sizeof(double);
+    case 1: return ctas * 1 * FitDims<1>::S * sizeof(double);
+    case 2: return ctas * 2 * FitDims<2>::S * sizeof(double);
+    case 4: return ctas * 4 * FitDims<4>::S * sizeof(double);
+    default: return ctas * 8 * FitDims<8>::S * sizeof(double);
   }
 }
 

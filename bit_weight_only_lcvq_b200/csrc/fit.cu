@@ -196,6 +196,209 @@ __global__ void __launch_bounds__(kFitThreads2, 2) fit_accum_kernel(
   }
 }
 
+// d = 8 on the tensor cores (mma.sync m16n8k8, tf32 in, fp32 out).  Warp w of
+// a CTA owns the 4 vector positions 32 c + 4 w .. + 3 of column tile c over
+// the CTA's rows, 8 rows per step.  Per position and step:
+//   T: A = the targets [16 x 8 rows]: rows 0..7 the tf32 "hi" parts of the 8
+//      channels, rows 8..15 the "lo" parts (w - hi rounded to tf32, so hi + lo
+//      is w to 2^-22); B = the codes [8 rows x 8] (exact); D rows i and i + 8
+//      add up to T[i][j] = sum w_i z_j.
+//   S: A = the codes [8 x 8 rows] with a ninth row of ones, B = the codes:
+//      D = the integer Gram (exact), row 8 the code sums.
+// The products are exact.  S is a sum of small integers and stays in the
+// MMA's fp32 accumulator (exact below 2^24).  T's MMA sums 8 products from
+// zero; its hi and lo rows are added and kept in fp32 for kFitFlush terms,
+// then added into fp64: a T entry's rounding is at most about 20 2^-24 of its
+// terms' absolute sum (the split's 2^-22, the MMA's partial sums, the two fp32
+// additions).  T[i][8] = sum w_i and S[8][8] (the row count) are added on the
+// CUDA cores.
+constexpr int kFit8Warps = 8;
+constexpr int kFit8PosPerWarp = 4;
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+// d = A B (from zero) or d += A B
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+__device__ __forceinline__ void mma_tf32_1688_acc(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3, uint32_t b0,
+                                                  uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Each warp streams its 8-row steps through a ring of kFit8Stages shared-memory
+// stages by cp.async (rows padded to 160 bytes: the lanes' reads hit distinct
+// banks), so that kFit8Stages - 1 steps of W0 are in flight per warp.
+constexpr int kFit8Stages = 6;
+constexpr int kFit8Pitch = 160;                              // bytes per staged row of W0
+constexpr int kFit8StageBytes = 8 * kFit8Pitch + 8 * 16;     // W0 rows + the rows' code words
+constexpr int kFit8RingBytes = kFit8Warps * kFit8Stages * kFit8StageBytes;
+
+__device__ __forceinline__ void fit_cp_async4(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void fit_cp_async(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kFit8Warps * 32, 2) fit8_mma_kernel(
+    const float* __restrict__ W0, const uint32_t* __restrict__ codes, int64_t N, int64_t groups,
+    int64_t row_splits, const float* __restrict__ h, double* __restrict__ partials) {
+  using F = FitDims<8>;
+  constexpr int P = F::P, kT = 8 * P;
+  __shared__ double pos[kFitLanes][F::SG + kT];
+  extern __shared__ __align__(16) unsigned char fit8_ring[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int64_t ct = int64_t(blockIdx.x) / row_splits, rs = int64_t(blockIdx.x) % row_splits;
+  const int64_t rows_per = ceil_div(N, row_splits);
+  const int64_t r_begin = rs * rows_per, r_end = r_begin + rows_per < N ? r_begin + rows_per : N;
+  const int64_t K = groups * 8;
+  const int64_t words_per_row = K / 16;
+  const int64_t g0 = ct * kFitLanes + warp * kFit8PosPerWarp;  // first position of this warp
+  const uint32_t one_row = gq == 0 ? __float_as_uint(1.0f) : 0u;  // A_S row 8
+  unsigned char* ring = fit8_ring + warp * (kFit8Stages * kFit8StageBytes);
+  const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
+
+  // step t covers rows r_begin + 8 t ..; lane l copies 16-byte chunks l and l + 32
+  // of its 8 x 128 bytes of W0, and lanes 0..7 the 16 code bytes of row l
+  const int64_t nsteps = ceil_div(r_end - r_begin, 8);
+  auto issue = [&](int64_t t) {
+    const uint32_t st = ring_s + static_cast<uint32_t>(t % kFit8Stages) * kFit8StageBytes;
+    const int64_t n0 = r_begin + 8 * t;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int chunk = lane + 32 * c, row = chunk >> 3, col = chunk & 7;  // col: 16-byte chunk
+      const int64_t n = n0 + row;
+      const int64_t gpos = g0 + (col >> 1);                               // 2 chunks per position
+      const bool ok = n < r_end && gpos < groups;
+      fit_cp_async(st + row * kFit8Pitch + col * 16,
+                   ok ? static_cast<const void*>(W0 + n * K + g0 * 8 + col * 4) : W0, ok);
+    }
+    if (lane < 16) {  // code word lane & 1 of row lane / 2 (a row of codes is only 4-byte aligned)
+      const int64_t n = n0 + (lane >> 1);
+      const int v = lane & 1;
+      const bool ok = n < r_end && g0 + 2 * v < groups;
+      fit_cp_async4(st + 8 * kFit8Pitch + (lane >> 1) * 16 + v * 4,
+                    ok ? static_cast<const void*>(codes + n * words_per_row + (g0 >> 1) + v) : codes, ok);
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  };
+
+  double t64[kFit8PosPerWarp][2], sw64[kFit8PosPerWarp];
+  float t32[kFit8PosPerWarp][2], s32[kFit8PosPerWarp][4], sw32[kFit8PosPerWarp];
+#pragma unroll
+  for (int q = 0; q < kFit8PosPerWarp; ++q) {
+    t64[q][0] = t64[q][1] = 0.0, t32[q][0] = t32[q][1] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s32[q][e] = 0.f;
+    sw64[q] = 0.0, sw32[q] = 0.f;
+  }
+  for (int64_t t = 0; t < kFit8Stages - 1; ++t) {
+    if (t < nsteps) issue(t);
+    else asm volatile("cp.async.commit_group;\n" ::: "memory");
+  }
+  int flush_steps = 0;
+  for (int64_t t = 0; t < nsteps; ++t) {
+    // keep kFit8Stages - 1 steps in flight: issue step t + S - 1, then wait for step t
+    if (t + kFit8Stages - 1 < nsteps) issue(t + kFit8Stages - 1);
+    else asm volatile("cp.async.commit_group;\n" ::: "memory");
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(kFit8Stages - 1) : "memory");
+    __syncwarp();
+    const unsigned char* st = ring + (t % kFit8Stages) * kFit8StageBytes;
+    const float* wrow_a = reinterpret_cast<const float*>(st + tq * kFit8Pitch);
+    const float* wrow_b = reinterpret_cast<const float*>(st + (tq + 4) * kFit8Pitch);
+    const uint32_t* crow_a = reinterpret_cast<const uint32_t*>(st + 8 * kFit8Pitch + tq * 16);
+    const uint32_t* crow_b = reinterpret_cast<const uint32_t*>(st + 8 * kFit8Pitch + (tq + 4) * 16);
+#pragma unroll
+    for (int q = 0; q < kFit8PosPerWarp; ++q) {
+      const float wa = wrow_a[q * 8 + gq], wb = wrow_b[q * 8 + gq];
+      const uint32_t sh = 16u * (q & 1) + 2u * gq;  // code gq of position q within its word
+      const uint32_t za = __float_as_uint(__int_as_float(0x4B000000 | int((crow_a[q >> 1] >> sh) & 3u)) - 8388608.0f);
+      const uint32_t zb = __float_as_uint(__int_as_float(0x4B000000 | int((crow_b[q >> 1] >> sh) & 3u)) - 8388608.0f);
+      const uint32_t ha = to_tf32(wa), hb = to_tf32(wb);
+      const uint32_t la = to_tf32(wa - __uint_as_float(ha)), lb = to_tf32(wb - __uint_as_float(hb));
+      float d[4];
+      mma_tf32_1688(d, ha, la, hb, lb, za, zb);
+      t32[q][0] += d[0] + d[2];  // rows gq (hi) and gq + 8 (lo)
+      t32[q][1] += d[1] + d[3];
+      mma_tf32_1688_acc(s32[q], za, one_row, zb, one_row, za, zb);
+      sw32[q] += wa + wb;
+    }
+    __syncwarp();  // the stage is read before a later issue overwrites it
+    if (++flush_steps == kFitFlush / 8) {  // t32: kFitFlush terms; sw32: 2 per step
+      flush_steps = 0;
+#pragma unroll
+      for (int q = 0; q < kFit8PosPerWarp; ++q) {
+        t64[q][0] += double(t32[q][0]), t64[q][1] += double(t32[q][1]);
+        t32[q][0] = t32[q][1] = 0.f;
+        sw64[q] += double(sw32[q]), sw32[q] = 0.f;
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+#pragma unroll
+  for (int q = 0; q < kFit8PosPerWarp; ++q) {
+    t64[q][0] += double(t32[q][0]), t64[q][1] += double(t32[q][1]);
+    sw64[q] += double(sw32[q]);
+    // lanes of one channel gq: tq = 0..3 (xor over lane bits 0, 1)
+    sw64[q] += __shfl_xor_sync(0xffffffffu, sw64[q], 1);
+    sw64[q] += __shfl_xor_sync(0xffffffffu, sw64[q], 2);
+  }
+  // scatter into pos[l][S upper triangle | T[i][j]] for l = 4 warp + q
+  auto sidx = [](int a, int b) {  // upper-triangle index of (a <= b) in a P x P matrix
+    return a * P - a * (a - 1) / 2 + (b - a);
+  };
+#pragma unroll
+  for (int q = 0; q < kFit8PosPerWarp; ++q) {
+    double* pp = &pos[warp * kFit8PosPerWarp + q][0];
+    const int j0 = 2 * tq;
+    // T: D rows gq (hi) and gq + 8 (lo), columns 2tq, 2tq + 1
+    pp[F::SG + gq * P + j0] = t64[q][0];
+    pp[F::SG + gq * P + j0 + 1] = t64[q][1];
+    if (tq == 0) pp[F::SG + gq * P + 8] = sw64[q];
+    // S: rows a = gq, columns b = 2tq, 2tq + 1 (upper triangle: a <= b)
+    if (gq <= j0) pp[sidx(gq, j0)] = double(s32[q][0]);
+    if (gq <= j0 + 1) pp[sidx(gq, j0 + 1)] = double(s32[q][1]);
+    if (gq == 0) {  // row 8 (the ones): S[8][b] = sum z_b, stored as S[b][8]
+      pp[sidx(j0, 8)] = double(s32[q][2]);
+      pp[sidx(j0 + 1, 8)] = double(s32[q][3]);
+    }
+    if (lane == 0) pp[sidx(8, 8)] = double(r_end > r_begin ? r_end - r_begin : 0);
+  }
+  __syncthreads();
+  // h per coordinate, positions in order: one partial [8][G_i (SG), R_i (P)]
+  for (int e = tid; e < 8 * F::S; e += kFit8Warps * 32) {
+    const int i = e / F::S, q = e % F::S;
+    double t = 0.0;
+    for (int l = 0; l < kFitLanes; ++l) {
+      const int64_t gg = ct * kFitLanes + l;
+      if (gg >= groups) break;
+      const double hw = h ? double(__ldg(h + gg * 8 + i)) : 1.0;
+      const double v = q < F::SG ? pos[l][q] : pos[l][F::SG + i * P + (q - F::SG)];
+      t += hw * v;
+    }
+    partials[int64_t(blockIdx.x) * 8 * F::S + e] = t;
+  }
+}
+
 // theta = G^+ R for a symmetric positive semi-definite P x P matrix G (row-major,
 // overwritten), by cyclic Jacobi rotations G = V diag(lambda) V^T.
 template <int P>
@@ -335,6 +538,9 @@ inline FitGrid fit_grid(int64_t d_out, int64_t groups) {
   if (f.tiles < kFitTargetCtas) f.splits = kFitTargetCtas / f.tiles;
   const int64_t max_splits = ceil_div(d_out > 0 ? d_out : 1, 16);
   if (f.splits > max_splits) f.splits = max_splits;
+  // the code Gram stays exact in fp32 while a CTA's rows times 9 is below 2^24
+  const int64_t min_splits = ceil_div(d_out > 0 ? d_out : 1, int64_t(1) << 20);
+  if (f.splits < min_splits) f.splits = min_splits;
   if (f.splits < 1) f.splits = 1;
   return f;
 }
@@ -346,12 +552,21 @@ cudaError_t launch_fit_t(const float* W0, const uint8_t* packed, int64_t d_out, 
   const int64_t groups = d_in / D;
   const FitGrid fg = fit_grid(d_out, groups);
   const uint32_t* codes = reinterpret_cast<const uint32_t*>(packed);
-  auto kern = fit_accum_kernel<D>;
-  if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), FitSmem<D>::kBytes);
-      e != cudaSuccess)
-    return e;
-  kern<<<static_cast<unsigned>(fg.ctas()), kFitThreads2, FitSmem<D>::kBytes, s>>>(
-      W0, codes, d_out, groups, fg.splits, h, partials);
+  if constexpr (D == 8) {
+    auto kern8 = fit8_mma_kernel;
+    if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern8), kFit8RingBytes);
+        e != cudaSuccess)
+      return e;
+    kern8<<<static_cast<unsigned>(fg.ctas()), kFit8Warps * 32, kFit8RingBytes, s>>>(
+        W0, codes, d_out, groups, fg.splits, h, partials);
+  } else {
+    auto kern = fit_accum_kernel<D>;
+    if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), FitSmem<D>::kBytes);
+        e != cudaSuccess)
+      return e;
+    kern<<<static_cast<unsigned>(fg.ctas()), kFitThreads2, FitSmem<D>::kBytes, s>>>(
+        W0, codes, d_out, groups, fg.splits, h, partials);
+  }
   ++*launches;
   if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
   fit_solve_kernel<D><<<1, 256, 0, s>>>(partials, static_cast<int>(fg.ctas()), A, B);

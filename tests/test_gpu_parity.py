@@ -378,7 +378,11 @@ def test_gemm_grouped_wide_tiles_bitwise_equal_separate_calls(M):
 def _fit_bound(W0, z, d, h, A_ref, B_ref):
     G, R = O.fit_affine_normal(np.abs(W0), z, d, h)   # G's terms are >= 0: G is its own |sum|
     th = np.concatenate([A_ref, B_ref[:, None]], axis=1)   # [d][d+1]
-    eps = 18 * 2.0 ** -24
+    # per-term rounding of the GPU's sums, relative to their absolute sums: the
+    # 2^-22 of the tf32 hi/lo split of W0 (d = 8), up to 14 2^-24 inside one
+    # tensor-core sum of 8 products, and the fp32 additions before the fp64
+    # flush every 16 terms; 24 2^-24 covers every path
+    eps = 24 * 2.0 ** -24
     bnd = np.zeros_like(th)
     for i in range(d):
         dR = eps * R[i]

@@ -278,26 +278,37 @@ __global__ void __launch_bounds__(kFit8Warps * 32, 2) fit8_mma_kernel(
   const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
 
   // step t covers rows r_begin + 8 t ..; lane l copies 16-byte chunks l and l + 32
-  // of its 8 x 128 bytes of W0, and lanes 0..7 the 16 code bytes of row l
-  const int64_t nsteps = ceil_div(r_end - r_begin, 8);
-  auto issue = [&](int64_t t) {
-    const uint32_t st = ring_s + static_cast<uint32_t>(t % kFit8Stages) * kFit8StageBytes;
-    const int64_t n0 = r_begin + 8 * t;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int chunk = lane + 32 * c, row = chunk >> 3, col = chunk & 7;  // col: 16-byte chunk
-      const int64_t n = n0 + row;
-      const int64_t gpos = g0 + (col >> 1);                               // 2 chunks per position
-      const bool ok = n < r_end && gpos < groups;
-      fit_cp_async(st + row * kFit8Pitch + col * 16,
-                   ok ? static_cast<const void*>(W0 + n * K + g0 * 8 + col * 4) : W0, ok);
-    }
-    if (lane < 16) {  // code word lane & 1 of row lane / 2 (a row of codes is only 4-byte aligned)
-      const int64_t n = n0 + (lane >> 1);
-      const int v = lane & 1;
-      const bool ok = n < r_end && g0 + 2 * v < groups;
-      fit_cp_async4(st + 8 * kFit8Pitch + (lane >> 1) * 16 + v * 4,
-                    ok ? static_cast<const void*>(codes + n * words_per_row + (g0 >> 1) + v) : codes, ok);
+  // of its 8 x 128 bytes of W0 (row c / 8, chunk c % 8), lanes 0..15 code word
+  // l % 2 of row l / 2.  Sources advance by 8 rows per step; only the last,
+  // partial step checks rows.
+  const int nsteps = static_cast<int>(ceil_div(r_end - r_begin, 8));
+  const int nfull = static_cast<int>((r_end - r_begin) / 8);
+  const int crow0 = lane >> 3, ccol = lane & 7;  // chunk lane: row crow0 (and crow0 + 4), column ccol
+  const bool wcol_ok = g0 + (ccol >> 1) < groups;
+  const float* wsrc = W0 + (r_begin + crow0) * K + g0 * 8 + ccol * 4;
+  const int64_t wstep = 8 * K, wrow4 = 4 * K;
+  const uint32_t wdst = static_cast<uint32_t>(crow0 * kFit8Pitch + ccol * 16);
+  const int cv = lane & 1, crow = (lane >> 1) & 7;
+  const bool ccol_ok = lane < 16 && g0 + 2 * cv < groups;
+  const uint32_t* csrc = codes + (r_begin + crow) * words_per_row + (g0 >> 1) + cv;
+  const int64_t cstep = 8 * words_per_row;
+  const uint32_t cdst = static_cast<uint32_t>(8 * kFit8Pitch + crow * 16 + cv * 4);
+  auto issue = [&](int t, int stage) {
+    const uint32_t st = ring_s + static_cast<uint32_t>(stage) * kFit8StageBytes;
+    const float* ws = wsrc + int64_t(t) * wstep;
+    const uint32_t* cs = csrc + int64_t(t) * cstep;
+    if (t < nfull) {
+      fit_cp_async(st + wdst, wcol_ok ? static_cast<const void*>(ws) : W0, wcol_ok);
+      fit_cp_async(st + wdst + 4 * kFit8Pitch, wcol_ok ? static_cast<const void*>(ws + wrow4) : W0, wcol_ok);
+      if (lane < 16) fit_cp_async4(st + cdst, ccol_ok ? static_cast<const void*>(cs) : codes, ccol_ok);
+    } else {
+      const int64_t n0 = r_begin + 8 * int64_t(t);
+      const bool ra = n0 + crow0 < r_end, rb = n0 + crow0 + 4 < r_end, rc = n0 + crow < r_end;
+      fit_cp_async(st + wdst, wcol_ok && ra ? static_cast<const void*>(ws) : W0, wcol_ok && ra);
+      fit_cp_async(st + wdst + 4 * kFit8Pitch, wcol_ok && rb ? static_cast<const void*>(ws + wrow4) : W0,
+                   wcol_ok && rb);
+      if (lane < 16)
+        fit_cp_async4(st + cdst, ccol_ok && rc ? static_cast<const void*>(cs) : codes, ccol_ok && rc);
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
   };
@@ -311,28 +322,34 @@ __global__ void __launch_bounds__(kFit8Warps * 32, 2) fit8_mma_kernel(
     for (int e = 0; e < 4; ++e) s32[q][e] = 0.f;
     sw64[q] = 0.0, sw32[q] = 0.f;
   }
-  for (int64_t t = 0; t < kFit8Stages - 1; ++t) {
-    if (t < nsteps) issue(t);
+  for (int t = 0; t < kFit8Stages - 1; ++t) {
+    if (t < nsteps) issue(t, t);
     else asm volatile("cp.async.commit_group;\n" ::: "memory");
   }
   int flush_steps = 0;
-  for (int64_t t = 0; t < nsteps; ++t) {
+  int s_use = 0, s_issue = kFit8Stages - 1;
+  // lane's reads in a stage: rows tq and tq + 4, channel gq of each position
+  const uint32_t ra_off = static_cast<uint32_t>(tq * kFit8Pitch + gq * 4);
+  const uint32_t ca_off = static_cast<uint32_t>(8 * kFit8Pitch + tq * 16);
+  for (int t = 0; t < nsteps; ++t) {
     // keep kFit8Stages - 1 steps in flight: issue step t + S - 1, then wait for step t
-    if (t + kFit8Stages - 1 < nsteps) issue(t + kFit8Stages - 1);
+    if (t + kFit8Stages - 1 < nsteps) issue(t + kFit8Stages - 1, s_issue);
     else asm volatile("cp.async.commit_group;\n" ::: "memory");
+    s_issue = s_issue + 1 == kFit8Stages ? 0 : s_issue + 1;
     asm volatile("cp.async.wait_group %0;\n" ::"n"(kFit8Stages - 1) : "memory");
     __syncwarp();
-    const unsigned char* st = ring + (t % kFit8Stages) * kFit8StageBytes;
-    const float* wrow_a = reinterpret_cast<const float*>(st + tq * kFit8Pitch);
-    const float* wrow_b = reinterpret_cast<const float*>(st + (tq + 4) * kFit8Pitch);
-    const uint32_t* crow_a = reinterpret_cast<const uint32_t*>(st + 8 * kFit8Pitch + tq * 16);
-    const uint32_t* crow_b = reinterpret_cast<const uint32_t*>(st + 8 * kFit8Pitch + (tq + 4) * 16);
+    const unsigned char* st = ring + s_use * kFit8StageBytes;
+    s_use = s_use + 1 == kFit8Stages ? 0 : s_use + 1;
+    const uint2 cwa = *reinterpret_cast<const uint2*>(st + ca_off);
+    const uint2 cwb = *reinterpret_cast<const uint2*>(st + ca_off + 4 * 16);
 #pragma unroll
     for (int q = 0; q < kFit8PosPerWarp; ++q) {
-      const float wa = wrow_a[q * 8 + gq], wb = wrow_b[q * 8 + gq];
+      const float wa = *reinterpret_cast<const float*>(st + ra_off + q * 32);
+      const float wb = *reinterpret_cast<const float*>(st + ra_off + 4 * kFit8Pitch + q * 32);
       const uint32_t sh = 16u * (q & 1) + 2u * gq;  // code gq of position q within its word
-      const uint32_t za = __float_as_uint(__int_as_float(0x4B000000 | int((crow_a[q >> 1] >> sh) & 3u)) - 8388608.0f);
-      const uint32_t zb = __float_as_uint(__int_as_float(0x4B000000 | int((crow_b[q >> 1] >> sh) & 3u)) - 8388608.0f);
+      const uint32_t wa_c = (q >> 1) ? cwa.y : cwa.x, wb_c = (q >> 1) ? cwb.y : cwb.x;
+      const uint32_t za = __float_as_uint(__int_as_float(0x4B000000 | ((wa_c >> sh) & 3u)) - 8388608.0f);
+      const uint32_t zb = __float_as_uint(__int_as_float(0x4B000000 | ((wb_c >> sh) & 3u)) - 8388608.0f);
       const uint32_t ha = to_tf32(wa), hb = to_tf32(wb);
       const uint32_t la = to_tf32(wa - __uint_as_float(ha)), lb = to_tf32(wb - __uint_as_float(hb));
       float d[4];

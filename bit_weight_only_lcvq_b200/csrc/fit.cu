@@ -215,10 +215,11 @@ __global__ void __launch_bounds__(kFitThreads2, 2) fit_accum_kernel(
 constexpr int kFit8Warps = 8;
 constexpr int kFit8PosPerWarp = 4;
 
+// x rounded to tf32 (10 explicit mantissa bits), to nearest with ties away from
+// zero, on the integer pipe: add half of the 13 dropped bits to the magnitude
+// and clear them (a carry moves into the exponent, as it should)
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
+  return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
 }
 // d = A B (from zero) or d += A B
 __device__ __forceinline__ void mma_tf32_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,

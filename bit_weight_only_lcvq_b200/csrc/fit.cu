@@ -14,8 +14,8 @@
 //    position the integer Gram of its codes and the products of its targets
 //    with its codes; h is applied afterwards, per CTA, in fp64 (below).  Each
 //    CTA writes one fp64 partial of every G_i and R_i.
-//  * fit_solve_kernel: sums the partials in CTA order (fp64), then thread i
-//    forms theta_i = G_i^+ R_i in fp64: by Cholesky when every pivot is above
+//  * fit_solve_kernel: CTA i sums coordinate i's partials in a fixed order
+//    (fp64), then forms theta_i = G_i^+ R_i in fp64: by Cholesky when every pivot is above
 //    1e-8 of the largest diagonal entry (G_i comfortably positive definite,
 //    pseudo-inverse = inverse), otherwise by a cyclic Jacobi
 //    eigendecomposition with eigenvalues below 1e-12 of the largest taken as
@@ -507,40 +507,59 @@ __device__ bool cholesky_solve(const double (&G)[P][P], const double (&R)[P], do
   return true;
 }
 
+// One CTA per coordinate i: sums its (d+1)(d+2)/2 + (d+1) values over the
+// partials -- thread (q, c) adds partials c, c + 4, c + 8, ... of value q in
+// order, 14 loads in flight, and the 4 chunk sums are added in chunk order
+// (a fixed order: bitwise reproducible) -- then solves theta_i.
+constexpr int kSolveChunks = 4;
+constexpr int kSolveBatch = 14;
+
 template <int D>
 __global__ void __launch_bounds__(256) fit_solve_kernel(const double* __restrict__ partials,
                                                         int num_parts, float* __restrict__ A,
                                                         float* __restrict__ B) {
   using F = FitDims<D>;
-  __shared__ double tot[D][F::S];
-  for (int e = threadIdx.x; e < D * F::S; e += blockDim.x) {
-    // partials in CTA order; loads batched 8 at a time, adds in order
-    const double* src = partials + e;
-    const int64_t pitch = int64_t(D) * F::S;
-    double t = 0.0;
-    int p = 0;
-    for (; p + 8 <= num_parts; p += 8) {
-      double v[8];
+  static_assert(F::S * kSolveChunks <= 256, "one thread per value and chunk");
+  __shared__ double part[kSolveChunks][F::S];
+  const int i = blockIdx.x;
+  const int t = threadIdx.x;
+  if (t < F::S * kSolveChunks) {
+    const int q = t % F::S, c = t / F::S;
+    const int64_t pitch = int64_t(D) * F::S * kSolveChunks;  // partials c, c + 4, ...
+    const double* src = partials + int64_t(c) * D * F::S + i * F::S + q;
+    double acc = 0.0;
+    int p = c;
+    for (; p + kSolveChunks * (kSolveBatch - 1) < num_parts; p += kSolveChunks * kSolveBatch) {
+      double v[kSolveBatch];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = src[int64_t(p + q) * pitch];
+      for (int u = 0; u < kSolveBatch; ++u) v[u] = src[int64_t(u) * pitch];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) t += v[q];
+      for (int u = 0; u < kSolveBatch; ++u) acc += v[u];
+      src += int64_t(kSolveBatch) * pitch;
     }
-    for (; p < num_parts; ++p) t += src[int64_t(p) * pitch];
-    tot[e / F::S][e % F::S] = t;
+    for (; p < num_parts; p += kSolveChunks) {
+      acc += *src;
+      src += pitch;
+    }
+    part[c][q] = acc;
   }
   __syncthreads();
-  const int i = threadIdx.x;
-  if (i >= D) return;
+  if (t != 0) return;
+  double tot[F::S];
+  for (int q = 0; q < F::S; ++q) {
+    double v = 0.0;
+    for (int c = 0; c < kSolveChunks; ++c) v += part[c][q];
+    tot[q] = v;
+  }
   double G[F::P][F::P], R[F::P], th[F::P];
   int s = 0;
   for (int a = 0; a < F::P; ++a)
     for (int b = a; b < F::P; ++b) {
-      G[a][b] = tot[i][s];
-      G[b][a] = tot[i][s];
+      G[a][b] = tot[s];
+      G[b][a] = tot[s];
       ++s;
     }
-  for (int a = 0; a < F::P; ++a) R[a] = tot[i][F::SG + a];
+  for (int a = 0; a < F::P; ++a) R[a] = tot[F::SG + a];
   if (!cholesky_solve<F::P>(G, R, th)) pinv_solve<F::P>(G, R, th);
   for (int j = 0; j < D; ++j) A[i * D + j] = static_cast<float>(th[j]);
   B[i] = static_cast<float>(th[D]);
@@ -587,7 +606,7 @@ cudaError_t launch_fit_t(const float* W0, const uint8_t* packed, int64_t d_out, 
   }
   ++*launches;
   if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
-  fit_solve_kernel<D><<<1, 256, 0, s>>>(partials, static_cast<int>(fg.ctas()), A, B);
+  fit_solve_kernel<D><<<D, 256, 0, s>>>(partials, static_cast<int>(fg.ctas()), A, B);
   ++*launches;
   return cudaGetLastError();
 }

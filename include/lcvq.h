@@ -265,9 +265,11 @@ LCVQ_API lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, floa
  * taking channel k = g d + i of vector g.  G^+ is the pseudo-inverse:
  * eigenvalues below 1e-12 of the largest count as zero, which gives the
  * minimum-norm solution when G_i is singular (a code position that never
- * varies, or weights that vanish).  Sums are fp32 per lane (exact for the
- * integer-valued G_i of h = 1), then fp64 in a fixed order; the solve is fp64
- * and the result is bitwise reproducible.
+ * varies, or weights that vanish).  The pass forms, per vector position, the
+ * codes' Gram (exact) and the targets times the codes (d = 8: tf32 hi/lo tensor-
+ * core products; other d: fp32), added into fp64 every 16 terms; h enters in
+ * fp64 afterwards.  Every sum has a fixed order and the solve is fp64: the
+ * result is bitwise reproducible.
  *   W0     [d_out][d_in] fp32 target weights (e.g. the pretrained matrix).
  *   packed [d_out][d_in/4] codes (format V1).
  *   h      [d_in] fp32 channel weights >= 0 (e.g. diag(X^T X)), or NULL for 1.

@@ -6,6 +6,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "decode_mma.cuh"
 #include "internal.h"
 
 namespace lcvq {
@@ -154,47 +155,10 @@ __global__ void __launch_bounds__(256) decode_kernel(const uint32_t* __restrict_
 }
 
 // d = 8, bf16 output: the decode as a small product on the tensor cores
-// (mma.sync m16n8k16).  16 vectors are the rows of the MMA's A operand and the
-// 8 output coordinates its columns,
-//     W~[v][i] = B[i] + sum_k Aop[v][k] Bop[k][i],
-// with k running over (code j, part):  k = 2t -> code t, hi;  k = 2t + 1 ->
-// code t + 4, hi;  k = 2t + 8 -> code t, lo;  k = 2t + 9 -> code t + 4, lo
-// (t = 0..3).  Aop[v][k] is the code z_v[j] as a bf16 (exact) and Bop[k][i] the
-// hi or lo bf16 part of A[i][j] (hi = bf16(A), lo = bf16(A - hi): A to 2^-17),
-// so the products are exact in fp32 and the accumulator starts at B[i]; a
-// vector of zero codes gives B exactly.  A code becomes its bf16 value by one
-// byte permute from two constant tables.  This costs about 4 instructions per
-// weight, where the FMA form (8 FMAs and an int-to-float conversion per
-// weight) is ALU-bound below the store bandwidth.
-constexpr uint32_t kBf16CodeLo = 0x40008000u;  // low bytes of bf16 0, 1, 2, 3: 00 80 00 40
-constexpr uint32_t kBf16CodeHi = 0x40403F00u;  // high bytes: 00 3F 40 40
+// (decode_mma.cuh).  This costs about 4 instructions per weight, where the FMA
+// form (8 FMAs and an int-to-float conversion per weight) is ALU-bound below
+// the store bandwidth.
 constexpr int kDec8Groups = 16;                // MMAs (16 vectors each) per warp and iteration
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-// bf16 pair (code t, code t + 4) of a vector whose 16-bit code sits at bit
-// `sh - 2t` of `word`, with sh = that offset + 2t
-__device__ __forceinline__ uint32_t code_pair_bf16(uint32_t word, uint32_t sh) {
-  const uint32_t y = (word >> sh) & 0x0303u;  // code t at bits 0-1, code t + 4 at bits 8-9
-  return prmt(kBf16CodeLo, kBf16CodeHi, y * 0x11u + 0x4040u);
-}
-// D = Aop Bop + C with the A registers repeated (k 8..15 are the lo parts of
-// the same codes) and C = (B[2t], B[2t+1]) in both rows
-__device__ __forceinline__ void mma_16816_dec(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0,
-                                              uint32_t b1, float c0, float c1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%4,%5}, "
-      "{%6,%7}, {%8,%9,%8,%9};\n"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
 
 __global__ void __launch_bounds__(256) decode8_mma_kernel(const uint32_t* __restrict__ words,
                                                           int64_t n_vec,
@@ -205,13 +169,8 @@ __global__ void __launch_bounds__(256) decode8_mma_kernel(const uint32_t* __rest
   // B operand: column n = g is output coordinate g; rows 2t, 2t + 1 (hi) and
   // 2t + 8, 2t + 9 (lo) are A[g][t] and A[g][t + 4]
   uint32_t b0, b1;
-  {
-    const float x0 = A[g * 8 + t], x1 = A[g * 8 + t + 4];
-    const uint16_t h0 = f32_to_bf16(x0), h1 = f32_to_bf16(x1);
-    b0 = uint32_t(h0) | (uint32_t(h1) << 16);
-    b1 = pack_bf16x2(x0 - bf16_to_f32(h0), x1 - bf16_to_f32(h1));
-  }
-  const float c0 = B[2 * t], c1 = B[2 * t + 1];
+  float c0, c1;
+  dec8::operands(A, B, g, t, b0, b1, c0, c1);
   const uint32_t sh = 16u * (g & 1) + 2u * t;  // vector g of a group is half g & 1 of its word
   const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
   constexpr int kPer = 16 * kDec8Groups;      // vectors per warp iteration
@@ -242,9 +201,9 @@ __global__ void __launch_bounds__(256) decode8_mma_kernel(const uint32_t* __rest
 #pragma unroll
     for (int m = 0; m < kDec8Groups; ++m) {
       float d[4];
-      mma_16816_dec(d, code_pair_bf16(cur[m][0], sh), code_pair_bf16(cur[m][1], sh), b0, b1, c0, c1);
-      __stcs(dst + 64 * m, bf16x2_rn(d[0], d[1]));
-      __stcs(dst + 64 * m + 32, bf16x2_rn(d[2], d[3]));
+      dec8::mma(d, dec8::code_pair_bf16(cur[m][0], sh), dec8::code_pair_bf16(cur[m][1], sh), b0, b1, c0, c1);
+      __stcs(dst + 64 * m, dec8::bf16x2_rn(d[0], d[1]));
+      __stcs(dst + 64 * m + 32, dec8::bf16x2_rn(d[2], d[3]));
     }
   }
   // the ragged tail (fewer than kPer vectors) goes to the warp whose turn it is
@@ -255,9 +214,9 @@ __global__ void __launch_bounds__(256) decode8_mma_kernel(const uint32_t* __rest
       const uint32_t w1 = v1 < n_vec ? words[v1 >> 1] : 0u;
       const uint32_t w2 = v2 < n_vec ? words[v2 >> 1] : 0u;
       float d[4];
-      mma_16816_dec(d, code_pair_bf16(w1, sh), code_pair_bf16(w2, sh), b0, b1, c0, c1);
-      if (v1 < n_vec) reinterpret_cast<uint32_t*>(W)[v1 * 4 + t] = bf16x2_rn(d[0], d[1]);
-      if (v2 < n_vec) reinterpret_cast<uint32_t*>(W)[v2 * 4 + t] = bf16x2_rn(d[2], d[3]);
+      dec8::mma(d, dec8::code_pair_bf16(w1, sh), dec8::code_pair_bf16(w2, sh), b0, b1, c0, c1);
+      if (v1 < n_vec) reinterpret_cast<uint32_t*>(W)[v1 * 4 + t] = dec8::bf16x2_rn(d[0], d[1]);
+      if (v2 < n_vec) reinterpret_cast<uint32_t*>(W)[v2 * 4 + t] = dec8::bf16x2_rn(d[2], d[3]);
     }
   }
 }

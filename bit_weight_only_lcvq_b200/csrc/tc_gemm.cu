@@ -33,6 +33,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "decode_mma.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -117,6 +118,9 @@ __device__ __forceinline__ void dec_word(uint32_t w, uint4& c0, uint4& c1) {
                   dec_pair<7>(w, w6, w12));
 }
 
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w)
@@ -689,6 +693,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
     constexpr int kGroupWarps = DW / kGroups > 0 ? DW / kGroups : 1;
     const int grp = (warp - 2) / kGroupWarps;
     const int dt = (threadIdx.x - 64) % (32 * kGroupWarps);
+    // d = 8 decode form on the tensor cores: this lane's operands of A z + B
+    [[maybe_unused]] uint32_t db0 = 0, db1 = 0;
+    [[maybe_unused]] float dc0 = 0.f, dc1 = 0.f;
+    if constexpr (KIND == kFwdDec && D == 8)
+      dec8::operands(sAm, sAm + D * D, lane >> 2, lane & 3, db0, db1, dc0, dc1);
     int s = 0;
     uint32_t ph = 0;
     int64_t it = 0;
@@ -713,6 +722,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
             dec_word(w[q], c0, c1);
             st_shared_v4(row + (((2 * q) ^ (r & 7)) << 4), c0);
             st_shared_v4(row + (((2 * q + 1) ^ (r & 7)) << 4), c1);
+          }
+        } else if constexpr (KIND == kFwdDec && D == 8) {
+          // warp w of the decoders takes rows 16 w .. 16 w + 15: MMA v decodes
+          // vector v of rows 16 w + g and 16 w + 8 + g (decode_mma.cuh) and
+          // stores 4 bytes per lane into the rows' SW128 chunk v (conflict-free:
+          // the 8 rows of one store have distinct chunk positions)
+          const int g = lane >> 2, t = lane & 3;
+          const int r1 = 16 * (dt >> 5) + g, r2 = r1 + 8;
+          const uint4 ca = *reinterpret_cast<const uint4*>(cs + r1 * 16);
+          const uint4 cb = *reinterpret_cast<const uint4*>(cs + r2 * 16);
+          const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w}, wb[4] = {cb.x, cb.y, cb.z, cb.w};
+          const uint32_t row1 = bs + r1 * 128, row2 = bs + r2 * 128;
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint32_t sh = 16u * (v & 1) + 2u * t;
+            float d4[4];
+            dec8::mma(d4, dec8::code_pair_bf16(wa[v >> 1], sh), dec8::code_pair_bf16(wb[v >> 1], sh),
+                      db0, db1, dc0, dc1);
+            st_shared_u32(row1 + ((v ^ (r1 & 7)) << 4) + 4 * t, dec8::bf16x2_rn(d4[0], d4[1]));
+            st_shared_u32(row2 + ((v ^ (r2 & 7)) << 4) + 4 * t, dec8::bf16x2_rn(d4[2], d4[3]));
           }
         } else if constexpr (KIND == kFwdDec) {  // 128 rows, two threads per row
           const int r = dt >> 1, h = dt & 1;

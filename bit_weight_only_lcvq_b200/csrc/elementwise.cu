@@ -245,12 +245,11 @@ cudaError_t launch_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, in
     int64_t b8 = ceil_div(ceil_div(n_vec, 16 * kDec8Groups), 8);
     // a persistent grid of resident blocks: each warp keeps its next 512 bytes
     // of codes in flight while it decodes and stores the current ones
-    static int resident = 0;
-    if (resident == 0) {
+    static const int resident = [] {  // thread-safe one-time initialisation
       int r = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, decode8_mma_kernel, 256, 0);
-      resident = r > 0 ? r : 1;
-    }
+      return r > 0 ? r : 1;
+    }();
     const int64_t cap8 = int64_t(kNumSMsB200) * resident;
     if (b8 > cap8) b8 = cap8;
     if (b8 < 1) b8 = 1;

@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(256) decode_kernel(const uint32_t* __restrict_
 // (decode_mma.cuh).  This costs about 4 instructions per weight, where the FMA
 // form (8 FMAs and an int-to-float conversion per weight) is ALU-bound below
 // the store bandwidth.
-constexpr int kDec8Groups = 16;                // MMAs (16 vectors each) per warp and iteration
+constexpr int kDec8Groups = 4;                 // MMAs (16 vectors each) per warp and iteration
 
 __global__ void __launch_bounds__(256) decode8_mma_kernel(const uint32_t* __restrict__ words,
                                                           int64_t n_vec,

@@ -243,8 +243,8 @@ cudaError_t launch_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, in
   if (d == 8 && w_bf16) {
     const int64_t n_vec = d_out * (d_in / 8);
     int64_t b8 = ceil_div(ceil_div(n_vec, 16 * kDec8Groups), 8);
-    // a persistent grid of resident blocks: each warp keeps its next 512 bytes
-    // of codes in flight while it decodes and stores the current ones
+    // a persistent grid of resident blocks: each warp keeps its next batch
+    // of codes (128 bytes) in flight while it decodes and stores the current one
     static const int resident = [] {  // thread-safe one-time initialisation
       int r = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, decode8_mma_kernel, 256, 0);

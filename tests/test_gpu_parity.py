@@ -132,8 +132,8 @@ def test_gemv_bf16_small_d(d):
 
 @pytest.mark.parametrize("M,d_in,d_out", [(33, 512, 264), (200, 512, 264), (300, 576, 520)])
 def test_gemm_bf16_larger_m(M, d_in, d_out):
-    """Tensor-core forms, including tiles ragged in M, in d_out (pairs of
-    128-row halves) and in K (a k block of 64 split by the end of d_in)."""
+    """Tensor-core forms, including tiles ragged in M and in d_out (pairs of
+    128-row halves), and an odd number of 64-wide k blocks."""
     w, z = _fwd_case(3, M, d_in=d_in, d_out=d_out)
     for form in ("auto", "decode", "algebraic"):
         Y = _run_fwd(w, z, torch.bfloat16, form)

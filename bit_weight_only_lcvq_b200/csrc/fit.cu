@@ -294,10 +294,11 @@ __global__ void __launch_bounds__(kFit8Warps * 32, 2) fit8_mma_kernel(
   const uint32_t* csrc = codes + (r_begin + crow) * words_per_row + (g0 >> 1) + cv;
   const int64_t cstep = 8 * words_per_row;
   const uint32_t cdst = static_cast<uint32_t>(8 * kFit8Pitch + crow * 16 + cv * 4);
+  // sources of the next step to issue, advanced by one step per issue
+  const float* ws = wsrc;
+  const uint32_t* cs = csrc;
   auto issue = [&](int t, int stage) {
     const uint32_t st = ring_s + static_cast<uint32_t>(stage) * kFit8StageBytes;
-    const float* ws = wsrc + int64_t(t) * wstep;
-    const uint32_t* cs = csrc + int64_t(t) * cstep;
     if (t < nfull) {
       fit_cp_async(st + wdst, wcol_ok ? static_cast<const void*>(ws) : W0, wcol_ok);
       fit_cp_async(st + wdst + 4 * kFit8Pitch, wcol_ok ? static_cast<const void*>(ws + wrow4) : W0, wcol_ok);
@@ -312,6 +313,8 @@ __global__ void __launch_bounds__(kFit8Warps * 32, 2) fit8_mma_kernel(
         fit_cp_async4(st + cdst, ccol_ok && rc ? static_cast<const void*>(cs) : codes, ccol_ok && rc);
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
+    ws += wstep;
+    cs += cstep;
   };
 
   double t64[kFit8PosPerWarp][2], sw64[kFit8PosPerWarp];

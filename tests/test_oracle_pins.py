@@ -720,3 +720,36 @@ def test_planted_mistakes_are_caught(golden_dir):
     assert not np.array_equal(O.decode(z, A, 0 * B), [[17.0, 35.0]])
     w = np.array([2.5], dtype=np.float32)
     assert np.floor(w + 0.5)[0] != O.assign(w)[0][0]   # half-up would give 3
+
+
+def test_ldlq_validity_checker_is_not_vacuous():
+    """The check the GPU tests apply to H-aware codes (every code must be the
+    rule's choice for its own fp64 target, except within the fp32 band of a
+    rounding boundary) accepts the oracle's codes and rejects plain rounding,
+    a single code flipped away from any tie, and shifted codes; a tie sitting
+    inside the band may go either way."""
+    from tests.gpu_util import ldlq_check
+    g = np.random.Generator(np.random.PCG64(80))
+    K = 128
+    Q = _spd(g, K, ridge=0.01)
+    U, _ = O.ldl_upper(Q)
+    U = U.astype(np.float32)
+    P = g.uniform(-0.5, 3.5, size=(12, K)).astype(np.float32)
+    Z = O.ldlq_assign(P, U)
+    assert ldlq_check(P, U, Z)[0] == 0
+    assert ldlq_check(P, U, np.clip(np.rint(P), 0, 3).astype(np.uint8))[0] > 0
+    T, _ = O.ldlq_targets(P, U, Z)
+    far = np.argwhere((np.abs(T - (np.floor(T) + 0.5)) > 0.2) & (T > 0.3) & (T < 2.7))
+    n, j = far[0]
+    Zf = Z.copy()
+    Zf[n, j] = 3 - Zf[n, j] if Zf[n, j] in (0, 3) else Zf[n, j] + 1
+    assert ldlq_check(P, U, Zf)[0] >= 1
+    assert ldlq_check(P, U, np.minimum(Z + 1, 3))[0] > 0
+    # an exact tie (target 1.5 with no compensation) is valid rounded up or down
+    P1 = np.full((1, 64), 0.25, dtype=np.float32)
+    P1[0, 7] = 1.5
+    U0 = np.zeros((64, 64), dtype=np.float32)
+    Zt = O.ldlq_assign(P1, U0)
+    Zu = Zt.copy()
+    Zu[0, 7] = 1 if Zt[0, 7] == 2 else 2
+    assert ldlq_check(P1, U0, Zt)[0] == 0 and ldlq_check(P1, U0, Zu)[0] == 0

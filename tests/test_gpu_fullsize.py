@@ -55,6 +55,20 @@ def test_prefill_full(form):
     _check_sampled_forward(Y, w["X"], z, w["A"], w["B"], _pairs(3, 2048, 11008), f"prefill {form}")
 
 
+def test_decode_full_qat_matrix():
+    """Decode to bf16 at the size the benchmark times (4096 x 14336, d = 8):
+    sampled rows, every element, against the oracle."""
+    w = synth.workload(4, M=1, with_dy=False)
+    z, _ = O.assign(w["Wp"])
+    packed, _ = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev()), 8, with_mask=False)
+    W = lcvq.decode(packed, 14336, torch.from_numpy(w["A"]).to(dev()),
+                    torch.from_numpy(w["B"]).to(dev()), 8)
+    rows = [0, 1, 2047, 4095, 1234, 3333]
+    got = W[rows].float().cpu().numpy()
+    ref = O.decode(z[rows], w["A"], w["B"])
+    assert_close("decode full", got, ref, O.decode_abs(z[rows], w["A"], w["B"]), 2.0 ** -8)
+
+
 @pytest.fixture(scope="module")
 def qat():
     w = synth.workload(4)

@@ -511,6 +511,11 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
 template <int KIND, int DW>
 struct Cfg2 {
   static constexpr int kThreads = 32 * (2 + DW + 4);
+  // groups of decoder warps take alternate k blocks: 8-warp groups for the
+  // decode form (a group decodes a stage's 128 rows with 8 warps), 4-warp
+  // groups otherwise
+  static constexpr int kDecGroups = DW < 8 ? 1 : (KIND == kFwdDec ? DW / 8 : DW / 4);
+  static constexpr int kDecGroupWarps = DW / kDecGroups > 0 ? DW / kDecGroups : 1;
   static constexpr bool kHasCodes = KIND != kDw;
   static constexpr bool kAmn = KIND == kDw;
   static constexpr bool kBmn = KIND == kDx || KIND == kDw;
@@ -558,7 +563,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       mbar_init(&fullA[s], 1);
       mbar_init(&fullC[s], 1);
       // this CTA's decoder warps of the group that owns stage s's k block
-      mbar_init(&decd[s], DW > 0 ? ((KIND == kFwdDec || DW < 8) ? DW : 4) : 1);
+      mbar_init(&decd[s], DW > 0 ? C::kDecGroupWarps : 1);
       mbar_init(&empty[s], 1);
       mbar_init(&decd_peer[s], 1);            // one forwarded arrive from the odd CTA
     }
@@ -689,8 +694,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
     // ------------------------------------------------------------ decoders (both CTAs)
     // kGroups groups of decoder warps take alternate k blocks, so each group has
     // kGroups MMA k-block times to decode and publish one stage.
-    constexpr int kGroups = (KIND == kFwdDec || DW < 8) ? 1 : DW / 4;
-    constexpr int kGroupWarps = DW / kGroups > 0 ? DW / kGroups : 1;
+    constexpr int kGroups = C::kDecGroups;
+    constexpr int kGroupWarps = C::kDecGroupWarps;
     const int grp = (warp - 2) / kGroupWarps;
     const int dt = (threadIdx.x - 64) % (32 * kGroupWarps);
     // d = 8 decode form on the tensor cores: this lane's operands of A z + B

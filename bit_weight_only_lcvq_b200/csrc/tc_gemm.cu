@@ -50,6 +50,9 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int C_BYTES = 4096;         // packed codes of one stage
+// CTA pairs: k blocks per forwarded "odd half decoded" arrive (measured on the
+// 2048 x 4096 -> 11008 decode form: 1, 2, 3 -> 724, 815, 857 TFLOP/s)
+constexpr int kPairPeerGroup = 3;
 constexpr int kTmemCols = 512;
 constexpr long long kWaitLimit = 1LL << 32;  // clock cycles (~2 s)
 
@@ -534,6 +537,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
                     const Params p) {
   using C = Cfg2<KIND, DW>;
   constexpr int S = C::kStages;
+  // k blocks per odd-to-even "decoded" arrive: group q (k blocks q G .. q G + G - 1
+  // of the pair's stream) uses decd_peer[q % S] in phase (q / S) & 1
+  constexpr int kPeerGroup = kPairPeerGroup;
+  static_assert(kPeerGroup >= 1 && kPeerGroup < S, "a group must not span the whole ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * C::kStage);
@@ -541,7 +548,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
   uint64_t* fullC = bars + S;        // [S]  per CTA: its codes landed
   uint64_t* decd = bars + 2 * S;     // [S]  per CTA: its own B half decoded
   uint64_t* empty = bars + 3 * S;    // [S]  per CTA: the MMA is done with stage s
-  uint64_t* decd_peer = bars + 4 * S; // [S] even CTA: the odd CTA's B half decoded
+  uint64_t* decd_peer = bars + 4 * S; // [S] even CTA: the odd CTA's B halves of a group decoded
   uint64_t* tfull = bars + 5 * S;    // [2]  per CTA: accumulator buffer ready
   uint64_t* tempty = tfull + 2;      // [2]  even CTA: both epilogues drained the buffer
   uint64_t* drain = tempty + 2;
@@ -565,7 +572,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       // this CTA's decoder warps of the group that owns stage s's k block
       mbar_init(&decd[s], DW > 0 ? C::kDecGroupWarps : 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&decd_peer[s], 1);            // one forwarded arrive from the odd CTA
+      mbar_init(&decd_peer[s], 1);            // one forwarded arrive per group from the odd CTA
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -635,7 +642,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, C::kAmn, C::kBmn);
       int s = 0;
       uint32_t ph = 0;
-      int64_t local = 0;
+      int64_t local = 0, it = 0;
       bool issued = false;
       for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs, ++local) {
         const int buf = static_cast<int>(local & 1);
@@ -645,11 +652,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
         tc_fence_after();
         const uint32_t dt = tmem + buf * BN;
         bool ok = true;
-        for (int64_t kb = 0; kb < kblocks; ++kb) {
+        for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
           if (!mbar_wait(&fullA[s], ph, kWaitLimit)) { fail(p, abort_flag, 13); ok = false; break; }
           if constexpr (C::kHasCodes) {
             if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 14); ok = false; break; }
-            if (!mbar_wait_cluster(&decd_peer[s], ph, kWaitLimit)) {
+            // the odd CTA's half of B: one cluster-scope wait per group of k blocks
+            const int64_t q = it / kPeerGroup;
+            if (it % kPeerGroup == 0 &&
+                !mbar_wait_cluster(&decd_peer[q % S], static_cast<uint32_t>((q / S) & 1),
+                                   kWaitLimit)) {
               fail(p, abort_flag, 18);
               ok = false;
               break;
@@ -679,13 +690,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       }
     } else if (rank == 1 && lane == 0 && C::kHasCodes) {
       // odd CTA: forward "B half decoded" to the even CTA, one cluster-scope
-      // arrive per k block, so the decoder warps only ever arrive locally
+      // arrive per group of kPeerGroup k blocks (and after the last one), so
+      // the decoder warps only ever arrive locally and the cluster-scope
+      // handover, whose cost sets the pace when it runs every k block, runs
+      // once per group
       int s = 0;
       uint32_t ph = 0;
+      int64_t it = 0;
       for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
-        for (int64_t kb = 0; kb < kblocks; ++kb) {
+        const bool last_tile = tile + npairs >= tiles;
+        for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
           if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 19); break; }
-          mbar_arrive_cluster(mapa_shared(smem_u32(&decd_peer[s]), 0));
+          if (it % kPeerGroup == kPeerGroup - 1 || (last_tile && kb + 1 == kblocks))
+            mbar_arrive_cluster(mapa_shared(smem_u32(&decd_peer[(it / kPeerGroup) % S]), 0));
           if (++s == S) { s = 0; ph ^= 1; }
         }
       }

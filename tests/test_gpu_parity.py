@@ -141,6 +141,16 @@ def test_gemm_bf16_larger_m(M, d_in, d_out):
         assert_close(f"gemm M={M} {form}", to_np(Y), ref, D, TOL_BF16)
 
 
+def test_gemm_decode_form_many_tiles_per_pair():
+    """Decode form with more tiles than CTA pairs and 5 k blocks per tile, so
+    some pairs run two tiles and the odd CTA's grouped "decoded" handover
+    spans a tile boundary and ends on a partial group; ragged in d_out."""
+    w, z = _fwd_case(3, 512, d_in=320, d_out=41 * 256 - 40)
+    Y = _run_fwd(w, z, torch.bfloat16, "decode")
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close("gemm decode form, 82 tiles", to_np(Y), ref, D, TOL_BF16)
+
+
 def test_gemm_f32_single_layer():
     """fp32 single-layer workload (d_in = d_out = 512, d = 4, M = 16)."""
     w, z = _fwd_case(1, 16, d_in=512, d_out=512)

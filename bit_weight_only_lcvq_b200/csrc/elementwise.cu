@@ -90,7 +90,17 @@ cudaError_t launch_assign_pack(const float* Wp, int64_t n_elems, uint8_t* packed
   const int tail = static_cast<int>(n_elems % 128);
   const int64_t warps_needed = ceil_div(n_chunks, kApUnroll) + (tail ? 1 : 0);
   int64_t blocks = ceil_div(warps_needed, 8);
-  const int64_t cap = int64_t(kNumSMsB200) * 8;
+  // one wave of resident blocks (the loop strides over the rest): a grid of
+  // more blocks than fit at once would end in a partly empty second wave
+  static const int resident = [] {  // thread-safe one-time initialisation
+    int r = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, assign_pack_kernel, 256, 0) !=
+            cudaSuccess ||
+        r < 1)
+      r = 1;
+    return r;
+  }();
+  const int64_t cap = int64_t(kNumSMsB200) * resident;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   assign_pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(

@@ -107,7 +107,14 @@ def lib() -> ctypes.CDLL:
 
 
 def _ptr(t):
-    return None if t is None else t.data_ptr()
+    """Device address of a CUDA tensor (None stays None).  Every array the
+    C ABI takes is device memory, so a host tensor is refused here rather than
+    handed to a kernel as an address it cannot read."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"lcvq: expected a CUDA tensor, got one on {t.device}")
+    return t.data_ptr()
 
 
 def _stream(stream=None):

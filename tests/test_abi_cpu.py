@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from bit_weight_only_lcvq_b200 import lcvq
 
@@ -135,3 +136,11 @@ def test_gemm_dimension_limits_without_device():
     assert L.lcvq_gemm(None, 1, 4, None, big - 56, 64, 8, None, None, None, 0, None, 0, None) == 1
     assert L.lcvq_gemm_backward(None, None, 1, 4, None, None, 8, big, 8, None, None, None,
                                 None, None, None, None, 0, None) == 1
+
+
+def test_binding_refuses_host_tensors():
+    """The binding hands kernels device addresses only: a host tensor is
+    refused before any call reaches the library (no CPU fallback either)."""
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        lcvq._ptr(torch.zeros(4))
+    assert lcvq._ptr(None) is None

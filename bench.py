@@ -735,6 +735,10 @@ def main():
         print(json.dumps(line))
         return 0
 
+    if not torch.cuda.is_available():  # the product path has no CPU fallback
+        print("bench.py: no CUDA device; the library's kernels need a B200 "
+              "(--impl reference times the CPU oracle)", file=sys.stderr)
+        return 2
     D = Dist()
     res = headline(args, D, pk)
     if D.rank == 0 and D.world == 1 and not args.no_cpu_baseline:

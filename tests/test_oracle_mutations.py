@@ -1,0 +1,94 @@
+"""The pins are not vacuous.
+
+Each case plants one plausible mistake in a single oracle function on the CPU.
+It then runs the pins that should notice, and at least one must fail. The
+mistakes:
+- a transposed or dropped operand;
+- a flipped sign;
+- a wrong tie or bit order;
+- a lost mask;
+- a dropped intercept;
+- missing error feedback.
+
+Nothing here touches a GPU.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import lcvq_oracle as O
+from tests import test_oracle_pins as P
+
+_decode, _assign, _pack = O.decode, O.assign, O.pack_codes
+_backward, _fit, _ldlq = O.backward, O.fit_affine, O.ldlq_assign
+
+
+def _assign_half_up(Wp):
+    z, mask = _assign(Wp)
+    w = np.asarray(Wp, dtype=np.float64)
+    up = np.clip(np.floor(np.where(np.isnan(w), 0.0, w) + 0.5), 0, 3).astype(np.uint8)
+    return up, mask
+
+
+def _pack_msb_first(z):
+    z = np.asarray(z, dtype=np.uint8)
+    n, k = z.shape
+    return _pack(z.reshape(n, k // 4, 4)[:, :, ::-1].reshape(n, k))
+
+
+def _backward_with(change):
+    def bw(*args):
+        out = dict(_backward(*args))
+        change(out)
+        return out
+    return bw
+
+
+def _negate_dx(o):
+    o["dX"] = -o["dX"]
+
+
+def _transpose_da(o):
+    o["dA"] = o["dA"].T.copy()
+
+
+def _backward_no_mask(X, dY, z, mask, A, B):
+    return _backward(X, dY, z, np.ones_like(mask, dtype=bool), A, B)
+
+
+MUTATIONS = [
+    ("decode: A transposed", "decode", lambda z, A, B: _decode(z, np.asarray(A).T, B),
+     [lambda gd: P.test_decode_golden(gd), lambda gd: P.test_linear_layer_golden(gd)]),
+    ("decode: B dropped", "decode", lambda z, A, B: _decode(z, A, 0.0 * np.asarray(B)),
+     [lambda gd: P.test_decode_golden(gd)]),
+    ("assign: ties rounded half up", "assign", _assign_half_up,
+     [lambda gd: P.test_round_clamp_golden(gd)]),
+    ("pack: most significant code first", "pack_codes", _pack_msb_first,
+     [lambda gd: P.test_pack_golden(gd), lambda gd: P.test_packed_d8_vector_is_codebook_index()]),
+    ("backward: dX sign flipped", "backward", _backward_with(_negate_dx),
+     [lambda gd: P.test_backward_finite_differences_exact()]),
+    ("backward: dA transposed", "backward", _backward_with(_transpose_da),
+     [lambda gd: P.test_backward_finite_differences_exact()]),
+    ("backward: clamp mask lost", "backward", _backward_no_mask,
+     [lambda gd: P.test_backward_dwp_ste_surrogate_finite_differences()]),
+    ("refit: intercept dropped", "fit_affine", lambda W0, z, d, h=None: (_fit(W0, z, d, h)[0],
+                                                                         np.zeros(d)),
+     [lambda gd: P.test_fit_affine_recovers_an_exact_affine_map(4)]),
+    ("H-aware assignment: no error feedback", "ldlq_assign",
+     lambda Pm, U: _ldlq(Pm, np.zeros_like(np.asarray(U))),
+     [lambda gd: P.test_ldlq_equals_the_eq11_procedure_solved_directly()]),
+]
+
+
+@pytest.mark.parametrize("name,target,mutant,pins", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_fails_a_pin(name, target, mutant, pins, monkeypatch, golden_dir):
+    for pin in pins:  # the pins pass on the oracle as written
+        pin(golden_dir)
+    monkeypatch.setattr(O, target, mutant)
+    caught = 0
+    for pin in pins:
+        try:
+            pin(golden_dir)
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"no pin noticed: {name}"

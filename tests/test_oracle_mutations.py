@@ -7,8 +7,9 @@ mistakes:
 - a flipped sign;
 - a wrong tie or bit order;
 - a lost mask;
-- a dropped intercept;
-- missing error feedback.
+- a dropped intercept or normaliser;
+- missing error feedback;
+- an unreversed factorisation.
 
 Nothing here touches a GPU.
 """
@@ -21,6 +22,7 @@ from tests import test_oracle_pins as P
 
 _decode, _assign, _pack = O.decode, O.assign, O.pack_codes
 _backward, _fit, _ldlq = O.backward, O.fit_affine, O.ldlq_assign
+_pack_mask, _dge_d, _ldl, _hess = O.pack_mask, O.dge_derivative, O.ldl_upper, O.code_space_hessian
 
 
 def _assign_half_up(Wp):
@@ -56,6 +58,27 @@ def _backward_no_mask(X, dY, z, mask, A, B):
     return _backward(X, dY, z, np.ones_like(mask, dtype=bool), A, B)
 
 
+def _pack_mask_msb_first(mask):
+    m = np.asarray(mask, dtype=np.uint8)
+    n, k = m.shape
+    return _pack_mask(m.reshape(n, k // 8, 8)[:, :, ::-1].reshape(n, k))
+
+
+def _dge_unnormalised(Wp, k):  # the k / (2 tanh(k / 2)) factor forgotten
+    return _dge_d(Wp, k) / (k / (2.0 * np.tanh(k / 2.0)))
+
+
+def _ldl_lower_factor(Q):  # the factor without the row and column reversal
+    Q = np.asarray(Q, dtype=np.float64)
+    C = np.linalg.cholesky(Q)
+    v = np.diag(C).copy()
+    return np.triu((C / v[None, :] - np.eye(Q.shape[0])).T, 1), v * v
+
+
+def _hessian_untransposed(H, A):  # Abar H Abar^T instead of Abar^T H Abar
+    return _hess(H, np.asarray(A).T)
+
+
 MUTATIONS = [
     ("decode: A transposed", "decode", lambda z, A, B: _decode(z, np.asarray(A).T, B),
      [lambda gd: P.test_decode_golden(gd), lambda gd: P.test_linear_layer_golden(gd)]),
@@ -77,6 +100,14 @@ MUTATIONS = [
     ("H-aware assignment: no error feedback", "ldlq_assign",
      lambda Pm, U: _ldlq(Pm, np.zeros_like(np.asarray(U))),
      [lambda gd: P.test_ldlq_equals_the_eq11_procedure_solved_directly()]),
+    ("mask: most significant bit first", "pack_mask", _pack_mask_msb_first,
+     [lambda gd: P.test_mask_golden(gd)]),
+    ("DGE: derivative not normalised", "dge_derivative", _dge_unnormalised,
+     [lambda gd: P.test_dge_curve_is_a_staircase_through_the_integers()]),
+    ("LDL: factor of the unreversed matrix", "ldl_upper", _ldl_lower_factor,
+     [lambda gd: P.test_ldl_upper_reconstructs_the_matrix()]),
+    ("code-space Hessian: A on the wrong side", "code_space_hessian", _hessian_untransposed,
+     [lambda gd: P.test_code_space_objective_is_the_weight_space_objective()]),
 ]
 
 

@@ -30,7 +30,7 @@ Sources (cited below by these short names):
   element at a time, the rest re-solved without the integer constraint) define
   the H-aware sequential code assignment.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
 
 * rounding is round-half-to-even (numpy ``rint``); clamp to ``[0, 3]``;
   NaN -> 0, +Inf -> 3, -Inf -> 0;

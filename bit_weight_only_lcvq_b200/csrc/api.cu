@@ -44,6 +44,14 @@ namespace {
 
 thread_local int g_last_launches = 0;
 
+}  // namespace
+
+namespace lcvq {
+void set_last_launches(int n) { g_last_launches = n; }
+}  // namespace lcvq
+
+namespace {
+
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, 2 other
 

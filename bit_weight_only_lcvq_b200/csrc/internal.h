@@ -13,6 +13,10 @@ namespace lcvq {
 // set once per (function, device)
 cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
 
+// records the number of kernels the current call launched, for
+// lcvq_last_launch_count() (per host thread)
+void set_last_launches(int n);
+
 // ---- elementwise ----
 cudaError_t launch_assign_pack(const float* Wp, int64_t n_elems, uint8_t* packed,
                                uint8_t* mask_bits, cudaStream_t s, int* launches);

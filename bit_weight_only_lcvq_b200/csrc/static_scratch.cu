@@ -22,6 +22,7 @@ namespace {
 
 constexpr int64_t kStaticMaxM = 32;
 constexpr int64_t kStaticMaxDin = 32768;
+constexpr int64_t kStaticMaxDout = int64_t(1) << 30;  // the same bound as lcvq_gemm
 constexpr size_t kStaticXppBytes = size_t(kStaticMaxM) * size_t(kStaticMaxDin) * 2;  // 2 MiB
 constexpr size_t kStaticScratchBytes = kStaticXppBytes + 256;                        // + corr
 
@@ -54,9 +55,11 @@ bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 extern "C" lcvq_status lcvq_gemv_static(const void* X, int64_t M, const uint8_t* packed,
                                         int64_t d_out, int64_t d_in, int d, const float* A,
                                         const float* B, void* Y, void* stream) {
+  lcvq::set_last_launches(0);
   if (M < 0 || d_out < 0 || d_in < 0) return LCVQ_ERR_INVALID_ARG;
   if (!(d == 1 || d == 2 || d == 4 || d == 8)) return LCVQ_ERR_INVALID_ARG;
   if (d_in % 64 != 0 || d_out % 8 != 0) return LCVQ_ERR_INVALID_ARG;
+  if (d_out > kStaticMaxDout) return LCVQ_ERR_INVALID_ARG;  // rows are indexed in 32 bits
   if (M > kStaticMaxM || d_in > kStaticMaxDin) return LCVQ_ERR_WORKSPACE;  // beyond the array
   if (M == 0 || d_out == 0) return LCVQ_OK;
   if (!Y) return LCVQ_ERR_INVALID_ARG;
@@ -86,5 +89,7 @@ extern "C" lcvq_status lcvq_gemv_static(const void* X, int64_t M, const uint8_t*
   if (e == cudaSuccess)
     e = lcvq::launch_gemv(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), s,
                           &launches);
-  return e == cudaSuccess ? LCVQ_OK : LCVQ_ERR_CUDA;
+  if (e != cudaSuccess) return LCVQ_ERR_CUDA;
+  lcvq::set_last_launches(launches);
+  return LCVQ_OK;
 }

@@ -24,38 +24,52 @@ from tests.gpu_util import TOL_BF16, dev
 pytestmark = pytest.mark.gpu
 
 
-def _case(M, d_in, d_out):
-    w = synth.workload(2, M=M, d_in=d_in, d_out=d_out, with_dy=False)
+def _case(M, d_in, d_out, d=8):
+    w = synth.workload(2, M=M, d_in=d_in, d_out=d_out, d=d, with_dy=False)
     z, _ = O.assign(w["Wp"])
     t = dict(X=torch.from_numpy(w["X"]).to(torch.bfloat16).to(dev()),
              packed=torch.from_numpy(O.pack_codes(z)).to(dev()),
              A=torch.from_numpy(w["A"]).to(dev()), B=torch.from_numpy(w["B"]).to(dev()))
-    _, D = O.forward(w["X"], z, w["A"], w["B"])
-    return w, t, D
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    return w, t, ref, D
 
 
-def _static_call(t, M, d_out, d_in, Y):
+def _static_call(t, M, d_out, d_in, Y, d=8):
     L = lcvq.lib()
-    st = L.lcvq_gemv_static(t["X"].data_ptr(), M, t["packed"].data_ptr(), d_out, d_in, 8,
+    st = L.lcvq_gemv_static(t["X"].data_ptr(), M, t["packed"].data_ptr(), d_out, d_in, d,
                             t["A"].data_ptr(), t["B"].data_ptr(), Y.data_ptr(),
                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     return st
 
 
+# (M, d_in, d_out, d): M = 32 fills the array's token rows; d = 4 changes the
+# X-transform; the others span the split kernel's 16- and 32-row tiles
+CASES = [(16, 4096, 4096, 8), (3, 1088, 520, 8), (32, 2048, 1032, 8), (9, 512, 264, 4)]
+
+
 def test_static_scratch_matches_workspace_path_two_calls():
-    cases = [(16, 4096, 4096), (3, 1088, 520)]
-    for M, d_in, d_out in cases:          # two calls in a row, different shapes
-        w, t, D = _case(M, d_in, d_out)
-        Y_static = torch.full((M, d_out), float("nan"), dtype=torch.bfloat16, device=dev())
-        assert _static_call(t, M, d_out, d_in, Y_static) == 0
-        Y_ref = lcvq.gemm(t["X"], t["packed"], d_in, t["A"], t["B"], 8)
-        torch.cuda.synchronize()
-        err = O.rel_err(Y_static.double().cpu().numpy(), Y_ref.double().cpu().numpy(), D)
-        assert err <= TOL_BF16, f"M={M}: static vs workspace path rel err {err:.3e}"
+    """Each case is called twice in a row through the C ABI; the second call
+    runs on an array that still holds the previous call's data.  Both must give
+    lcvq_gemm's result (the same kernels, so the same bits) and lie within the
+    forward tolerance of the oracle."""
+    L = lcvq.lib()
+    for M, d_in, d_out, d in CASES:
+        w, t, ref, D = _case(M, d_in, d_out, d)
+        Y_ref = lcvq.gemm(t["X"], t["packed"], d_in, t["A"], t["B"], d)
+        for call in range(2):
+            Y_static = torch.full((M, d_out), float("nan"), dtype=torch.bfloat16, device=dev())
+            assert _static_call(t, M, d_out, d_in, Y_static, d) == 0
+            assert L.lcvq_last_launch_count() == 2
+            torch.cuda.synchronize()
+            err = O.rel_err(Y_static.double().cpu().numpy(), Y_ref.double().cpu().numpy(), D)
+            assert err <= TOL_BF16, f"M={M} call {call}: static vs workspace path rel err {err:.3e}"
+            assert torch.equal(Y_static, Y_ref), f"M={M} d={d} call {call}: bits differ"
+            err = O.rel_err(Y_static.double().cpu().numpy(), ref, D)
+            assert err <= TOL_BF16, f"M={M} call {call}: static vs oracle rel err {err:.3e}"
 
 
 def test_static_scratch_rejects_sizes_beyond_the_array():
-    w, t, _ = _case(4, 512, 64)
+    w, t, _, _ = _case(4, 512, 64)
     Y = torch.zeros((40, 64), dtype=torch.bfloat16, device=dev())
     L = lcvq.lib()
     s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -64,5 +78,8 @@ def test_static_scratch_rejects_sizes_beyond_the_array():
                               t["A"].data_ptr(), t["B"].data_ptr(), Y.data_ptr(), s) == 4
     assert L.lcvq_gemv_static(t["X"].data_ptr(), 4, t["packed"].data_ptr(), 64, 32768 + 64, 8,
                               t["A"].data_ptr(), t["B"].data_ptr(), Y.data_ptr(), s) == 4
+    # a d_out beyond lcvq_gemm's bound is an invalid argument, as there
+    assert L.lcvq_gemv_static(t["X"].data_ptr(), 4, t["packed"].data_ptr(), (1 << 30) + 8, 512, 8,
+                              t["A"].data_ptr(), t["B"].data_ptr(), Y.data_ptr(), s) == 1
     torch.cuda.synchronize()
     assert torch.count_nonzero(Y) == 0

@@ -56,3 +56,27 @@ def ldlq_check(P, U, Z):
     Zf = np.asarray(Z, dtype=np.float64)
     bad = ((Zf != ref) & ~near) | (np.abs(np.clip(T, 0, 3) - Zf) > 0.5 + tau)
     return int(bad.sum()), int(near.sum())
+
+
+GUARD_BYTES = 4096     # guard on each side of a canaried output (keeps 256-byte alignment)
+GUARD_FILL = 0xA5
+
+
+def guarded(shape, dtype):
+    """An output tensor of `shape` placed inside a larger buffer whose
+    GUARD_BYTES on either side (and the output itself) are filled with the
+    byte GUARD_FILL.  Returns (out, buf); guard_intact(out, buf) checks that a
+    kernel writing `out` left every guard byte alone."""
+    esz = torch.empty((), dtype=dtype).element_size()
+    n = int(np.prod(shape))
+    g = GUARD_BYTES // esz
+    buf = torch.empty(n + 2 * g, dtype=dtype, device=dev())
+    buf.view(torch.uint8).fill_(GUARD_FILL)
+    return buf[g:g + n].view(shape), buf
+
+
+def guard_intact(out, buf) -> bool:
+    raw = buf.view(torch.uint8)
+    nb = out.numel() * out.element_size()
+    head, tail = raw[:GUARD_BYTES], raw[GUARD_BYTES + nb:]
+    return bool(torch.all(head == GUARD_FILL)) and bool(torch.all(tail == GUARD_FILL))

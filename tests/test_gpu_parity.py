@@ -12,7 +12,8 @@ import torch
 
 from bit_weight_only_lcvq_b200 import lcvq, synth
 from oracle import lcvq_oracle as O
-from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, dev, ldlq_check, to_dev, to_np, tol_for
+from tests.gpu_util import (TOL_BF16, TOL_F32, assert_close, dev, guard_intact, guarded, ldlq_check,
+                            to_dev, to_np, tol_for)
 
 pytestmark = pytest.mark.gpu
 
@@ -34,9 +35,13 @@ def _adversarial_wp(n_rows, n_cols, seed):
 def test_assign_pack_bit_exact(shape):
     Wp = _adversarial_wp(*shape, seed=shape[0] * 7 + shape[1])
     z, mask = O.assign(Wp)
-    packed, mbits = lcvq.assign_pack(torch.from_numpy(Wp).to(dev()), d=8 if shape[1] % 8 == 0 else 4)
+    packed, pbuf = guarded((shape[0], shape[1] // 4), torch.uint8)
+    mbits, mbuf = guarded((shape[0], shape[1] // 8), torch.uint8)
+    lcvq.assign_pack(torch.from_numpy(Wp).to(dev()), d=8 if shape[1] % 8 == 0 else 4,
+                     packed=packed, mask=mbits)
     assert np.array_equal(packed.cpu().numpy(), O.pack_codes(z))
     assert np.array_equal(mbits.cpu().numpy(), O.pack_mask(mask))
+    assert guard_intact(packed, pbuf) and guard_intact(mbits, mbuf)
 
 
 def test_assign_pack_workload_distributions():
@@ -64,12 +69,14 @@ def test_decode(d, dtype):
     N, K = 40, 256
     z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
     A, B = synth.affine_diag_dominant(d, g)
-    W = lcvq.decode(torch.from_numpy(O.pack_codes(z)).to(dev()), K, torch.from_numpy(A).to(dev()),
-                    torch.from_numpy(B).to(dev()), d, dtype=dtype)
+    W, wbuf = guarded((N, K), dtype)
+    lcvq.decode(torch.from_numpy(O.pack_codes(z)).to(dev()), K, torch.from_numpy(A).to(dev()),
+                torch.from_numpy(B).to(dev()), d, out=W)
     ref = O.decode(z, A, B)
     D = O.decode_abs(z, A, B)
     tol = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-6
     assert_close("decode", to_np(W), ref, D, tol)
+    assert guard_intact(W, wbuf)
 
 
 @pytest.mark.parametrize("shape", [(1, 16), (3, 48), (37, 528), (128, 4096)])
@@ -83,11 +90,13 @@ def test_decode_d8_bf16_ragged_and_exact_zero(shape):
     z[0, :8] = 0
     A, B = synth.affine_diag_dominant(8, g)
     B[:] = 0.0
-    W = lcvq.decode(torch.from_numpy(O.pack_codes(z)).to(dev()), K, torch.from_numpy(A).to(dev()),
-                    torch.from_numpy(B).to(dev()), 8)
+    W, wbuf = guarded((N, K), torch.bfloat16)
+    lcvq.decode(torch.from_numpy(O.pack_codes(z)).to(dev()), K, torch.from_numpy(A).to(dev()),
+                torch.from_numpy(B).to(dev()), 8, out=W)
     ref = O.decode(z, A, B)
     assert_close("decode d=8", to_np(W), ref, O.decode_abs(z, A, B), 2.0 ** -8)
     assert np.all(to_np(W)[0, :8] == 0.0)
+    assert guard_intact(W, wbuf)
 
 
 # --------------------------------------------------------------- forward
@@ -98,11 +107,16 @@ def _fwd_case(wid, M, d_in, d_out, d=None, seed_shift=0):
 
 
 def _run_fwd(w, z, dtype, form="auto"):
+    """lcvq_gemm into a canaried output: the bytes around Y stay untouched."""
     packed = torch.from_numpy(O.pack_codes(z)).to(dev())
     X = to_dev(w["X"], dtype)
     A = torch.from_numpy(w["A"]).to(dev())
     B = torch.from_numpy(w["B"]).to(dev())
-    return lcvq.gemm(X, packed, w["d_in"], A, B, w["d"], form=form)
+    Y, ybuf = guarded((X.shape[0], packed.shape[0]), dtype)
+    lcvq.gemm(X, packed, w["d_in"], A, B, w["d"], form=form, out=Y)
+    torch.cuda.synchronize()
+    assert guard_intact(Y, ybuf), f"lcvq_gemm wrote outside Y (M={X.shape[0]}, form={form})"
+    return Y
 
 
 @pytest.mark.parametrize("M", [1, 2, 4, 5, 8, 13, 16, 27, 32])
@@ -241,14 +255,25 @@ def _check_bwd(w, z, mask, out, tol, tag):
 
 def test_backward_f32_single_layer():
     w, z, mask, a = _bwd_case(1, 16, 512, 512, torch.float32)
-    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 512, a["A"], a["B"], 4)
+    dX, xbuf = guarded((16, 512), torch.float32)
+    dWp, wbuf = guarded((512, 512), torch.float32)
+    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], 512, a["A"], a["B"], 4,
+                             outs=dict(dX=dX, dWp=dWp))
+    torch.cuda.synchronize()
+    assert guard_intact(dX, xbuf) and guard_intact(dWp, wbuf)
     _check_bwd(w, z, mask, out, TOL_F32, "f32")
 
 
 @pytest.mark.parametrize("M,d_in,d_out", [(37, 576, 264), (200, 1024, 512)])
 def test_backward_bf16(M, d_in, d_out):
+    """bf16 backward on ragged shapes, into canaried dX and dWp."""
     w, z, mask, a = _bwd_case(4, M, d_in, d_out, torch.bfloat16)
-    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], d_in, a["A"], a["B"], 8)
+    dX, xbuf = guarded((M, d_in), torch.bfloat16)
+    dWp, wbuf = guarded((d_out, d_in), torch.float32)
+    out = lcvq.gemm_backward(a["X"], a["dY"], a["packed"], a["mask"], d_in, a["A"], a["B"], 8,
+                             outs=dict(dX=dX, dWp=dWp))
+    torch.cuda.synchronize()
+    assert guard_intact(dX, xbuf) and guard_intact(dWp, wbuf)
     _check_bwd(w, z, mask, out, TOL_BF16, f"bf16 M={M}")
 
 
@@ -568,3 +593,84 @@ def test_ldlq_empty_matrix_is_a_no_op():
     U = torch.zeros((64, 64), device=dev())
     out = lcvq.assign_ldlq(torch.zeros((0, 64), device=dev()), U, 8)
     assert out.shape == (0, 16)
+
+
+# ------------------------------------ the algebraic form as two calls (lcvq_xform, lcvq_gemm_xformed)
+def _unscramble_xpp(xpp: np.ndarray) -> np.ndarray:
+    """X'' (decoder order, position c of each 16-block scaled by 4^-(c mod 3))
+    back to bf16(X') in natural order, exactly (powers of two)."""
+    M, K = xpp.shape
+    blk = xpp.reshape(M, K // 16, 8, 2)                 # [.., pair c, (pos c, pos c + 8)]
+    scale = np.array([4.0 ** (c % 3) for c in range(8)])[None, None, :]
+    lo, hi = blk[..., 0] * scale, blk[..., 1] * scale
+    return np.concatenate([lo, hi], axis=2).reshape(M, K)
+
+
+@pytest.mark.parametrize("M,K,d", [(1, 1088, 8), (5, 4096, 8), (32, 512, 4), (3, 256, 2), (7, 128, 1)])
+def test_xform_matches_its_definition(M, K, d):
+    """lcvq_xform against the definition in lcvq.h, restated here in fp64:
+    X'[m][g d + j] = sum_i X[m][g d + i] A[i][j] rounded to bf16 (within the
+    bf16 half-ulp plus the fp32 products), stored in decoder order with the
+    per-position power of two exactly; corr = s' - 3/2 sum bf16(X') -
+    128 sum X'' with s' = sum_g x_g . (B + 3/2 A 1)."""
+    w = synth.workload(2, M=M, d_in=K, d_out=8, d=d, with_dy=False)
+    X = to_dev(w["X"], torch.bfloat16)
+    A, B = torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev())
+    xpp, xbuf = guarded((M, K), torch.bfloat16)
+    corr, cbuf = guarded((M,), torch.float32)
+    lcvq.xform(X, A, B, d, xpp=xpp, corr=corr)
+    torch.cuda.synchronize()
+    assert guard_intact(xpp, xbuf) and guard_intact(corr, cbuf)
+    x = w["X"].astype(np.float64)
+    A64, B64 = w["A"].astype(np.float64), w["B"].astype(np.float64)
+    xg = x.reshape(M, K // d, d)
+    Xp = np.einsum("mgi,ij->mgj", xg, A64).reshape(M, K)
+    DXp = np.einsum("mgi,ij->mgj", np.abs(xg), np.abs(A64)).reshape(M, K)
+    xpp_np = to_np(xpp)
+    xr = _unscramble_xpp(xpp_np)
+    assert np.all(np.abs(xr - Xp) <= 2.0 ** -8 * DXp), "X' is not bf16(X A)"
+    Bp = B64 + 1.5 * A64.sum(axis=1)
+    s = np.einsum("mgi,i->m", xg, Bp)
+    ref = s - 1.5 * xr.sum(1) - 128.0 * xpp_np.sum(1)
+    Dc = np.einsum("mgi,i->m", np.abs(xg), np.abs(Bp)) + 1.5 * np.abs(xr).sum(1) + \
+        128.0 * np.abs(xpp_np).sum(1)
+    assert_close("corr", to_np(corr), ref, Dc, 1e-5)
+
+
+@pytest.mark.parametrize("M,d_in,d_out", [(1, 1088, 520), (4, 4096, 1024), (13, 576, 264),
+                                          (16, 1088, 520), (32, 512, 264), (33, 512, 264),
+                                          (200, 576, 520)])
+def test_xform_then_gemm_xformed_equals_gemm(M, d_in, d_out):
+    """lcvq_gemm with the algebraic form is lcvq_xform followed by
+    lcvq_gemm_xformed: the two calls give lcvq_gemm's bits (decode-GEMV and
+    tensor-core GEMM alike), within the tolerance of the oracle, and write
+    nothing outside their outputs."""
+    w, z = _fwd_case(2, M, d_in=d_in, d_out=d_out)
+    packed = torch.from_numpy(O.pack_codes(z)).to(dev())
+    X = to_dev(w["X"], torch.bfloat16)
+    A, B = torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev())
+    Y1 = lcvq.gemm(X, packed, d_in, A, B, 8, form="algebraic")
+    Ya = lcvq.gemm(X, packed, d_in, A, B, 8)
+    xpp, corr = lcvq.xform(X, A, B, 8)
+    Y2, ybuf = guarded((M, d_out), torch.bfloat16)
+    lcvq.gemm_xformed(xpp, corr, packed, out=Y2)
+    torch.cuda.synchronize()
+    assert guard_intact(Y2, ybuf)
+    assert torch.equal(Y1, Y2)
+    assert torch.equal(Ya, Y2)
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close(f"gemm_xformed M={M}", to_np(Y2), ref, D, TOL_BF16)
+
+
+def test_gemm_grouped_outputs_are_canaried():
+    """Every Y_i of a grouped call (split and wide-tile kernels) stays inside
+    its own buffer."""
+    for shapes, M in (([(1088, 520), (512, 8), (4096, 1000)], 5),
+                      ([(4096, 4096)] * 9 + [(1088, 1000)], 3)):
+        jobs, zs, ws = _group_case(shapes, M, 2000 + M)
+        pairs = [guarded((M, p.shape[0]), torch.bfloat16) for _, p, _, _, _ in jobs]
+        lcvq.gemm_grouped(jobs, 8, outs=[o for o, _ in pairs])
+        torch.cuda.synchronize()
+        assert all(guard_intact(o, b) for o, b in pairs)
+        ref, D = O.forward(ws[0]["X"], zs[0], ws[0]["A"], ws[0]["B"])
+        assert_close("canaried grouped item 0", to_np(pairs[0][0]), ref, D, TOL_BF16)

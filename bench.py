@@ -59,11 +59,12 @@ def parse():
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
-# dominant kernel, from one ncu capture (profiles/), valid only for the kernel
-# source that was captured: keyed by the SHA-1 of the source file.
+# dominant kernel, from one ncu capture of this benchmark's decode-GEMV step,
+# valid only for the kernel source that was captured: keyed by the SHA-1 of
+# the source file.
 NCU_TRAFFIC = {
     # source file -> (sha1 of the file when captured, {token count: bytes per launch})
-    # profiles/launches_decode_gemv_bench.md: M = 1 and 4 share gemv_group_kernel<1, ...>
+    # M = 1 and 4 share one instantiation of the kernel
     "bit_weight_only_lcvq_b200/csrc/gemv.cu": (
         "5016dd5597b05501b2883e20d2dbeb24c777ddc9", {1: 4237173, 4: 4237173, 16: 4366684}),
 }
@@ -224,9 +225,19 @@ class StepGraphs:
             self.g_rem.replay()
         return self.q * self.n_full + self.n_rem
 
+    def prime(self):
+        """Launch each captured graph once, untimed: a graph's first launch
+        uploads it to the device, which must not fall inside a timed region."""
+        self.g_full.replay()
+        if self.g_rem is not None:
+            self.g_rem.replay()
+        torch.cuda.synchronize()
+
 
 def timed_graphs(D, sg: StepGraphs, sampler=None):
-    """Barrier + sync on both sides; returns (max-over-ranks ms, launches, clocks)."""
+    """Barrier + sync on both sides; returns (max-over-ranks ms, launches, clocks).
+    The graphs are primed (launched once) before the timed region."""
+    sg.prime()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if sampler:
@@ -242,54 +253,71 @@ def timed_graphs(D, sg: StepGraphs, sampler=None):
     return D.max(e0.elapsed_time(e1)), launches, ck
 
 
-# ----------------------------------------------------------------------------- oracle leg
-def oracle_gemv_sample(Ms, seconds=10.0):
-    """The oracle (fp64) on the decode-GEMV workload's codes: Y for the three
-    token counts over as many full 4096 x 4096 passes as fit in ~`seconds`."""
-    from oracle import lcvq_oracle as O
-    w = synth.workload(2, M=max(Ms), with_dy=False)
-    z, _ = O.assign(w["Wp"])
+# ----------------------------------------------------------------------------- oracle legs
+def _oracle():
+    """The C++ fp64 oracle (plain loops, one thread per output row range)."""
+    from oracle import cpp as C
+    C.lib()
+    return C
+
+
+def _timed_loop(fn, seconds):
+    """Calls fn() until `seconds` have passed (at least once); (calls, seconds)."""
     t0 = time.perf_counter()
-    passes = 0
+    n = 0
     while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            return n, dt
+
+
+def oracle_gemv_sample(Ms, seconds=10.0, threads=1):
+    """The C++ oracle on the decode-GEMV workload (4096 x 4096, d = 8): Y and
+    its normaliser for the three token counts, single-threaded, over as many
+    full passes as fit in ~`seconds`."""
+    C = _oracle()
+    w = synth.workload(2, M=max(Ms), with_dy=False)
+    from oracle import lcvq_oracle as O
+    packed = O.pack_codes(O.assign(w["Wp"])[0])
+    X = w["X"].astype(np.float64)
+
+    def step():
         for M in Ms:
-            O.forward(w["X"][:M], z, w["A"], w["B"])
-        passes += 1
-        if time.perf_counter() - t0 >= seconds:
-            break
-    dt = time.perf_counter() - t0
+            C.forward_packed(X[:M], packed, 4096, w["A"], w["B"], threads=threads)
+    passes, dt = _timed_loop(step, seconds)
     packed_bytes = passes * len(Ms) * (4096 * 4096 // 4)
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # pragma: no cover
-        threads = os.cpu_count() or 1
-    return dict(value=packed_bytes / dt / 1e9, unit="GB/s", cores=int(threads), kind="oracle",
-                sample=f"{passes} full passes of d_in=d_out=4096, d=8 at M={list(Ms)} "
-                       f"(fp64 decode + BLAS matmul incl. |x||w| normaliser), {dt:.1f} s")
+    return dict(value=packed_bytes / dt / 1e9, unit="GB/s", cores=threads, kind="oracle",
+                sample=f"{passes} full passes of d_in=d_out=4096, d=8 at M={list(Ms)} by the C++ "
+                       f"fp64 oracle (decode, Y and its normaliser) on {threads} thread(s), "
+                       f"{dt:.1f} s")
 
 
 def oracle_reference_arm(Ms, steps, warmup, budget_s=60.0):
-    """The reference arm: the oracle itself, timed as steps.  A step is one
-    pass over the three token counts on the decode-GEMV workload, on all 4096
-    output rows when K + W such passes fit in ~budget_s, otherwise on the first
-    `rows` rows (a bounded sample; the metric counts the packed bytes of the
-    rows computed).  W untimed steps, then K timed ones."""
+    """The reference arm: the C++ fp64 oracle itself, timed as steps on all host
+    cores.  A step is one pass over the three token counts on the decode-GEMV
+    workload, on all 4096 output rows when K + W such passes fit in ~budget_s,
+    otherwise on the first `rows` rows (a bounded sample; the metric counts the
+    packed bytes of the rows computed).  W untimed steps, then K timed ones."""
+    C = _oracle()
     from oracle import lcvq_oracle as O
+    threads = C.default_threads()
     w = synth.workload(2, M=max(Ms), with_dy=False)
-    z, _ = O.assign(w["Wp"])
+    packed = O.pack_codes(O.assign(w["Wp"])[0])
+    X = w["X"].astype(np.float64)
     t0 = time.perf_counter()
     for M in Ms:
-        O.forward(w["X"][:M], z, w["A"], w["B"])
+        C.forward_packed(X[:M], packed, 4096, w["A"], w["B"], threads=threads)
     full_s = max(time.perf_counter() - t0, 1e-3)
     rows = 4096
     if (steps + warmup) * full_s > budget_s:
         rows = max(16, int(4096 * budget_s / ((steps + warmup) * full_s)) // 16 * 16)
-    zs = np.ascontiguousarray(z[:rows])
+    ps = np.ascontiguousarray(packed[:rows])
 
     def step():
         for M in Ms:
-            O.forward(w["X"][:M], zs, w["A"], w["B"])
+            C.forward_packed(X[:M], ps, 4096, w["A"], w["B"], threads=threads)
 
     for _ in range(warmup):
         step()
@@ -298,16 +326,11 @@ def oracle_reference_arm(Ms, steps, warmup, budget_s=60.0):
         step()
     dt = time.perf_counter() - t0
     packed_bytes = steps * len(Ms) * (rows * 4096 // 4)
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # pragma: no cover
-        threads = os.cpu_count() or 1
-    return dict(value=packed_bytes / dt / 1e9, unit="GB/s", cores=int(threads), kind="oracle",
+    return dict(value=packed_bytes / dt / 1e9, unit="GB/s", cores=threads, kind="oracle",
                 ms_per_step=dt / max(steps, 1) * 1e3,
-                sample=f"{steps} timed steps after {warmup} untimed, each the {rows} x 4096 "
-                       f"rows of d=8 codes at M={list(Ms)} (fp64 decode + BLAS matmul incl. "
-                       f"|x||w| normaliser), {dt:.1f} s")
+                sample=f"{steps} timed steps after {warmup} untimed, each the {rows} x 4096 rows of "
+                       f"d=8 codes at M={list(Ms)} (C++ fp64 oracle: decode, Y and its normaliser; "
+                       f"{threads} threads), {dt:.1f} s")
 
 
 # ----------------------------------------------------------------------------- headline
@@ -457,6 +480,58 @@ def headline(args, D: Dist, pk):
 
 
 # ----------------------------------------------------------------------------- other rows
+def _roof(bound, achieved, peak, unit, **kw):
+    return dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak, **kw)
+
+
+# fp32 FMA peak: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz (the maximum SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
+FP32_SRC = "derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz"
+
+
+def row_single_layer(D, pk, cpu=True):
+    """Single linear layer, fp32 (d_in = d_out = 512, d = 4, M = 16): the
+    forward Y = X W~ and the straight-through backward (dX, dA, dB, dWp), on the
+    CUDA cores (fp32 activations).  Work: 3 x 2 M N K flops."""
+    dev = D.dev
+    M, K, N, d = 16, 512, 512, 4
+    w = synth.workload(1)
+    Wp = torch.from_numpy(w["Wp"]).to(dev)
+    packed, mask = lcvq.assign_pack(Wp, d)
+    A = torch.from_numpy(w["A"]).to(dev)
+    B = torch.from_numpy(w["B"]).to(dev)
+    X = torch.from_numpy(w["X"]).to(dev)
+    dY = torch.from_numpy(w["dY"]).to(dev)
+    Y = torch.empty((M, N), device=dev)
+    wsf = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.float32, M, N, K, d), dev)
+    wsb = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM_BACKWARD, torch.float32, M, N, K, d), dev)
+    outs = dict(dX=torch.empty((M, K), device=dev), dWp=torch.empty((N, K), device=dev),
+                dA=torch.empty((d, d), device=dev), dB=torch.empty((d,), device=dev))
+
+    def step():
+        lcvq.gemm(X, packed, K, A, B, d, out=Y, workspace=wsf)
+        lcvq.gemm_backward(X, dY, packed, mask, K, A, B, d, outs=outs, workspace=wsb)
+    ms = graph_time(step, 50)
+    flops = 3 * 2.0 * M * N * K
+    tf = flops / (ms * 1e-3) / 1e12
+    out = dict(metric="single-layer fp32 forward + STE backward TFLOP/s (3 x 2MNK / time)",
+               value=tf, unit="TFLOP/s", us=ms * 1e3,
+               roofline=_roof("alu", tf, FP32_ALU_TFLOPS, "TFLOP/s", peak_source=FP32_SRC))
+    if cpu:
+        C = _oracle()
+        from oracle import lcvq_oracle as O
+        z, m = O.assign(w["Wp"])
+
+        def ostep():
+            C.forward(w["X"], z, w["A"], w["B"], threads=1)
+            C.backward(w["X"], w["dY"], z, m, w["A"], w["B"], threads=1)
+        n, dt = _timed_loop(ostep, 2.0)
+        out["cpu_baseline"] = dict(value=n * flops / dt / 1e12, unit="TFLOP/s", cores=1,
+                                   kind="oracle", sample=f"{n} full forward + backward passes of the "
+                                   f"layer by the C++ fp64 oracle on 1 thread, {dt:.1f} s")
+    return out
+
+
 def row_assign_pack(D, pk):
     """Assign + pack (+ mask) on the QAT-step weights: 4096 x 14336 fp32."""
     dev = D.dev
@@ -490,7 +565,7 @@ def row_decode(D, pk):
                               frac=gbs / pk["hbm_gbs"]))
 
 
-def row_prefill(D, pk):
+def row_prefill(D, pk, cpu=True):
     """Prefill GEMM, d_in=4096 -> d_out=11008, M=2048, both forward forms."""
     dev = D.dev
     M, K, N, d = 2048, 4096, 11008, 8
@@ -510,12 +585,24 @@ def row_prefill(D, pk):
         ms = ev_time(call, 5)
         tf = flops / (ms * 1e-3) / 1e12
         out[form] = dict(value=tf, unit="TFLOP/s", us=ms * 1e3,
-                         roofline=dict(bound="tensor", achieved=tf, peak=pk["bf16_tflops"],
-                                       unit="TFLOP/s", frac=tf / pk["bf16_tflops"]))
-    return dict(metric="prefill GEMM TFLOP/s (2MNK / time)", forms=out)
+                         roofline=_roof("tensor", tf, pk["bf16_tflops"], "TFLOP/s"))
+    res = dict(metric="prefill GEMM TFLOP/s (2MNK / time)", forms=out)
+    if cpu:  # the oracle on the first `rows` output rows, all host cores
+        C = _oracle()
+        from oracle import lcvq_oracle as O
+        rows = 128
+        pkd = O.pack_codes(O.assign(w["Wp"][:rows])[0])
+        Xd = w["X"].astype(np.float64)
+        n, dt = _timed_loop(lambda: C.forward_packed(Xd, pkd, K, w["A"], w["B"]), 3.0)
+        res["cpu_baseline"] = dict(value=n * 2.0 * M * rows * K / dt / 1e12, unit="TFLOP/s",
+                                   cores=C.default_threads(), kind="oracle",
+                                   sample=f"{n} passes of the first {rows} of {N} output rows "
+                                          f"(M={M}, K={K}) by the C++ fp64 oracle (Y and its "
+                                          f"normaliser), {dt:.1f} s")
+    return res
 
 
-def row_qat(D, pk):
+def row_qat(D, pk, cpu=True):
     """QAT step on d_in=14336, d_out=4096, M=8192: assign/pack, forward, backward."""
     dev = D.dev
     M, K, N, d = 8192, 14336, 4096, 8
@@ -539,27 +626,57 @@ def row_qat(D, pk):
     bw = lambda: lcvq.gemm_backward(X, dY, packed, mask, K, A, B, d, outs=outs, workspace=wsb)
     for f in (ap, fw, bw):  # warm-up: first-launch costs stay out of the timing
         f()
+    # burst: each stage timed alone over a few calls (about 1 ms each)
     t_ap = ev_time(ap, 3)
-    t_fw = ev_time(fw, 2)
-    t_bw = ev_time(bw, 2)
+    t_fw = ev_time(fw, 3)
+    t_bw = ev_time(bw, 3)
     gemm_flops = 2.0 * M * N * K
     total = t_ap + t_fw + t_bw
     tf = 3 * gemm_flops / (total * 1e-3) / 1e12
-    return dict(metric="QAT step TFLOP/s (3 x 2MNK / step time)", value=tf, unit="TFLOP/s",
-                step_us=total * 1e3, assign_pack_us=t_ap * 1e3, forward_us=t_fw * 1e3,
-                backward_us=t_bw * 1e3,
-                roofline=dict(bound="tensor", achieved=tf, peak=pk["bf16_tflops_sustained"],
-                              unit="TFLOP/s", frac=tf / pk["bf16_tflops_sustained"]))
+
+    # sustained: whole steps back to back for about 3 s
+    def step():
+        ap()
+        fw()
+        bw()
+    n_sus = max(3, int(math.ceil(3000.0 / total)))
+    t_sus = ev_time(step, n_sus)
+    tf_sus = 3 * gemm_flops / (t_sus * 1e-3) / 1e12
+    res = dict(metric="QAT step TFLOP/s (3 x 2MNK / step time)", value=tf, unit="TFLOP/s",
+               step_us=total * 1e3, assign_pack_us=t_ap * 1e3, forward_us=t_fw * 1e3,
+               backward_us=t_bw * 1e3,
+               roofline=_roof("tensor", tf, pk["bf16_tflops"], "TFLOP/s",
+                              timing="burst: each stage over 3 calls after a warm-up call"),
+               sustained=dict(value=tf_sus, unit="TFLOP/s", step_us=t_sus * 1e3, steps=n_sus,
+                              roofline=_roof("tensor", tf_sus, pk["bf16_tflops_sustained"],
+                                             "TFLOP/s", timing=f"{n_sus} whole steps back to back")))
+    if cpu:  # the oracle's forward + backward on the first `rows` output rows, all host cores
+        C = _oracle()
+        from oracle import lcvq_oracle as O
+        rows = 16
+        z, m = O.assign(w["Wp"][:rows])
+        Xd, dYd = w["X"].astype(np.float64), np.ascontiguousarray(w["dY"][:, :rows], np.float64)
+
+        def ostep():
+            C.forward(Xd, z, w["A"], w["B"])
+            C.backward(Xd, dYd, z, m, w["A"], w["B"])
+        n, dt = _timed_loop(ostep, 3.0)
+        res["cpu_baseline"] = dict(value=n * 3 * 2.0 * M * rows * K / dt / 1e12, unit="TFLOP/s",
+                                   cores=C.default_threads(), kind="oracle",
+                                   sample=f"{n} forward + backward passes of the first {rows} of "
+                                          f"{N} output rows (M={M}, K={K}) by the C++ fp64 "
+                                          f"oracle (with normalisers), {dt:.1f} s")
+    return res
 
 
-def row_stack(D, pk, layers=32, ms=(1, 8, 32)):
+def row_stack(D, pk, layers=32, ms=(1, 8, 32), cpu=True):
     """7B-shaped stack: 224 matrices, M in {1, 8, 32}; packed GB/s over the stack
     (fewer layers or token counts only for a profiler capture)."""
     dev = D.dev
     mats = []
     for layer in range(layers):
         for p in range(len(synth.STACK_PROJS)):
-            m = synth.stack_matrix(layer, p, 32, with_x=(layer == 0))
+            m = synth.stack_matrix(layer, p, max(ms), with_x=(layer == 0))
             mats.append(m)
     total_bytes = sum(m["packed"].nbytes for m in mats)
     dmats = []
@@ -643,15 +760,32 @@ def row_stack(D, pk, layers=32, ms=(1, 8, 32)):
         out[str(M)] = res_m
         del all_ws, all_outs, ph_ws
         torch.cuda.empty_cache()
-    return dict(metric=f"stack packed-weight GB/s ({len(dmats)} matrices, "
-                       f"{total_bytes / 1e9:.2f} GB of codes)",
-                note="sequential: 224 lcvq_gemm calls; grouped_by_phase: one lcvq_gemm_grouped per "
-                     "decoder-layer phase (q,k,v | o | gate,up | down), 128 calls; grouped_all: the "
-                     "224 independent matrices in one lcvq_gemm_grouped call",
-                per_m=out, packed_bytes=total_bytes)
+    res = dict(metric=f"stack packed-weight GB/s ({len(dmats)} matrices, "
+                      f"{total_bytes / 1e9:.2f} GB of codes)",
+               note="sequential: 224 lcvq_gemm calls; grouped_by_phase: one lcvq_gemm_grouped per "
+                    "decoder-layer phase (q,k,v | o | gate,up | down), 128 calls; grouped_all: the "
+                    "224 independent matrices in one lcvq_gemm_grouped call",
+               per_m=out, packed_bytes=total_bytes)
+    if cpu:  # the oracle on one decoder layer (7 matrices) per token count, all host cores
+        C = _oracle()
+        layer = [m for m in mats if m["layer"] == 0]
+        lbytes = sum(m["packed"].nbytes for m in layer)
+        cb = {}
+        for M in ms:
+            def ostep(M=M):
+                for m in layer:
+                    C.forward_packed(m["X"][:M].astype(np.float64), m["packed"], m["d_in"],
+                                     m["A"], m["B"])
+            n, dt = _timed_loop(ostep, 1.0)
+            cb[str(M)] = n * lbytes / dt / 1e9
+        res["cpu_baseline"] = dict(value=cb, unit="GB/s", cores=C.default_threads(), kind="oracle",
+                                   sample="one decoder layer (q,k,v,o,gate,up,down: "
+                                          f"{lbytes / 1e6:.0f} MB of codes) per token count by the "
+                                          "C++ fp64 oracle (decode, Y and its normaliser), ~1 s each")
+    return res
 
 
-def row_fit(D, pk):
+def row_fit(D, pk, cpu=True):
     """Least-squares (A, B) refit on the QAT-step matrix (4096 x 14336, d = 8):
     W0 = the workload's proxy weights, codes = their assignment; unweighted and
     with per-channel weights h."""
@@ -672,14 +806,21 @@ def row_fit(D, pk):
         out[name] = dict(value=gbs, unit="GB/s", us=ms * 1e3,
                          roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
                                        frac=gbs / pk["hbm_gbs"]))
-    return dict(metric="(A, B) refit GB/s (W0 fp32 + codes read)", forms=out)
+    res = dict(metric="(A, B) refit GB/s (W0 fp32 + codes read)", forms=out)
+    if cpu:  # the numpy oracle's normal equations and solve on the first `rows` rows
+        from oracle import lcvq_oracle as O
+        rows = 256
+        W0s = w["Wp"][:rows].astype(np.float64)
+        zs = O.assign(w["Wp"][:rows])[0]
+        n, dt = _timed_loop(lambda: O.fit_affine(W0s, zs, d), 2.0)
+        res["cpu_baseline"] = dict(value=n * rows * K * 4.25 / dt / 1e9, unit="GB/s",
+                                   cores=_blas_threads(), kind="oracle",
+                                   sample=f"{n} unweighted refits of the first {rows} of {N} rows "
+                                          f"by the numpy fp64 oracle, {dt:.1f} s")
+    return res
 
 
-# fp32 FMA peak: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz (the maximum SM clock)
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
-
-
-def row_ldlq(D, pk):
+def row_ldlq(D, pk, cpu=True):
     """H-aware sequential code assignment on a 4096 x 4096 matrix (d = 8): the
     code-space factor of a calibration Hessian (8192 activation rows, outlier
     recipe, 1% damping) is formed on the device in fp64 before timing."""
@@ -702,15 +843,58 @@ def row_ldlq(D, pk):
     lcvq.assign_ldlq(P, U, d, workspace=ws, packed=packed)
     ms = ev_time(lambda: lcvq.assign_ldlq(P, U, d, workspace=ws, packed=packed), 10)
     tf = N * K * (K - 1) / (ms * 1e-3) / 1e12
-    return dict(metric="H-aware assignment TFLOP/s (N K (K-1) / time: fp32 FMA, 2 flops each)",
-                value=tf, unit="TFLOP/s", us=ms * 1e3,
-                roofline=dict(bound="alu", achieved=tf, peak=FP32_ALU_TFLOPS, unit="TFLOP/s",
-                              frac=tf / FP32_ALU_TFLOPS,
-                              peak_source="derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz"))
+    res = dict(metric="H-aware assignment TFLOP/s (N K (K-1) / time: fp32 FMA, 2 flops each)",
+               value=tf, unit="TFLOP/s", us=ms * 1e3,
+               roofline=_roof("alu", tf, FP32_ALU_TFLOPS, "TFLOP/s", peak_source=FP32_SRC))
+    if cpu:  # the numpy oracle's sequential rule on the first `rows` rows
+        from oracle import lcvq_oracle as O
+        rows = 8
+        Ph = w["P"][:rows]
+        Uh = U.cpu().numpy()
+        n, dt = _timed_loop(lambda: O.ldlq_assign(Ph, Uh), 2.0)
+        res["cpu_baseline"] = dict(value=n * rows * K * (K - 1) / dt / 1e12, unit="TFLOP/s",
+                                   cores=_blas_threads(), kind="oracle",
+                                   sample=f"{n} runs on the first {rows} of {N} rows by the numpy "
+                                          f"fp64 oracle, {dt:.1f} s")
+    return res
 
 
-ROWS = {"assign_pack": row_assign_pack, "decode": row_decode, "prefill": row_prefill,
-        "qat": row_qat, "stack": row_stack, "fit": row_fit, "ldlq": row_ldlq}
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+ROWS = {"single_layer": row_single_layer, "assign_pack": row_assign_pack, "decode": row_decode,
+        "prefill": row_prefill, "qat": row_qat, "stack": row_stack, "fit": row_fit,
+        "ldlq": row_ldlq}
+CPU_ROWS = ("single_layer", "prefill", "qat", "stack", "fit", "ldlq")
+
+
+def row_summary(name, r) -> str:
+    """One short line per row (printed to stderr next to the JSON line)."""
+    def fr(x):
+        rf = x.get("roofline") or {}
+        return f"{x['value']:.4g} {x['unit']} ({100 * rf.get('frac', float('nan')):.1f}% of {rf.get('peak')})"
+    if "error" in r:
+        return f"row {name}: ERROR {r['error']}"
+    parts = []
+    if "forms" in r:
+        parts += [f"{k}: {fr(v)}" for k, v in r["forms"].items()]
+    elif "per_m" in r:
+        for M, arr in r["per_m"].items():
+            parts += [f"M={M} {a}: {fr(v)}" for a, v in arr.items() if "value" in v]
+    else:
+        parts.append(fr(r))
+    if "sustained" in r:
+        parts.append(f"sustained: {fr(r['sustained'])}")
+    cb = r.get("cpu_baseline")
+    if cb:
+        parts.append(f"oracle: {cb['value'] if isinstance(cb['value'], dict) else round(cb['value'], 6)} "
+                     f"{cb['unit']} on {cb['cores']} core(s)")
+    return f"row {name}: " + "; ".join(parts)
 
 
 # ----------------------------------------------------------------------------- main
@@ -746,16 +930,20 @@ def main():
     rows = {}
     want = list(ROWS) if args.rows == "all" else ([] if args.rows == "none" else args.rows.split(","))
     if D.rank == 0:
+        cpu = D.world == 1 and not args.no_cpu_baseline
         for name in want:
             try:
                 if name == "stack":
                     rows[name] = row_stack(D, pk, args.stack_layers,
-                                           tuple(int(m) for m in args.stack_ms.split(",")))
+                                           tuple(int(m) for m in args.stack_ms.split(",")), cpu=cpu)
+                elif name in CPU_ROWS:
+                    rows[name] = ROWS[name](D, pk, cpu=cpu)
                 else:
                     rows[name] = ROWS[name](D, pk)
             except Exception as ex:  # report, do not hide
                 rows[name] = {"error": f"{type(ex).__name__}: {ex}"}
             torch.cuda.empty_cache()
+            print(row_summary(name, rows[name]), file=sys.stderr, flush=True)
     res["rows"] = rows
     if D.rank == 0:
         print(json.dumps(res))

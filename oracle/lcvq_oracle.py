@@ -347,6 +347,47 @@ def fit_affine(W0: np.ndarray, z: np.ndarray, d: int, h=None):
     return A, B
 
 
+def fit_affine_h_normal(W0: np.ndarray, z: np.ndarray, d: int, H: np.ndarray):
+    """The normal equations of the refit under the full input Hessian H
+    (decoupleQ page, eq. (5): the objective tr{(W~ - W0)^T H (W~ - W0)} with
+    W~ = d_in x d_out; in this storage order it is sum_n r_n^T H r_n over the
+    rows r_n = W~[n] - W0[n]).  With zt = [z_0 .. z_{d-1}, 1] per vector, the
+    decoded element is W~[n, g d + i] = sum_a theta[i, a] zt[n, g, a] with
+    theta = [A | B], so the objective is a quadratic in theta whose normal
+    equations couple every pair of vector positions (g, g'):
+        G[(i, a), (j, b)] = sum_n sum_{g, g'} H[g d + i, g' d + j] zt[n, g, a] zt[n, g', b]
+        R[(i, a)]         = sum_n sum_g sum_k H[g d + i, k] W0[n, k] zt[n, g, a]
+    Returns (G [d (d+1)][d (d+1)], R [d (d+1)]), index (i, a) -> i (d+1) + a."""
+    W0 = np.asarray(W0, dtype=np.float64)
+    H = np.asarray(H, dtype=np.float64)
+    N, K = W0.shape
+    ng = K // d
+    zt = np.concatenate([np.asarray(z, np.float64).reshape(N, ng, d), np.ones((N, ng, 1))], axis=2)
+    S = np.einsum("nga,nhb->gahb", zt, zt)                  # code Gram of every (g, g') pair
+    Hg = H.reshape(ng, d, ng, d)                            # H[g d + i, h d + j] -> [g, i, h, j]
+    G = np.einsum("gihj,gahb->iajb", Hg, S).reshape(d * (d + 1), d * (d + 1))
+    T = np.einsum("nk,nga->kga", W0, zt)                    # W0^T zt per position
+    R = np.einsum("gik,kga->ia", H.reshape(ng, d, K), T).reshape(d * (d + 1))
+    return G, R
+
+
+def fit_affine_h(W0: np.ndarray, z: np.ndarray, d: int, H: np.ndarray):
+    """(A, B) minimizing sum_n (W~[n] - W0[n])^T H (W~[n] - W0[n]) over W~ = A z + B
+    per vector (decoupleQ page, eq. (5) with the codes fixed, solved in closed
+    form as in its section 3.3): theta = G^+ R from fit_affine_h_normal, the
+    minimum-norm solution when G is singular."""
+    G, R = fit_affine_h_normal(W0, z, d, H)
+    th = np.linalg.pinv(G, rcond=PINV_RCOND, hermitian=True) @ R
+    th = th.reshape(d, d + 1)
+    return th[:, :d].copy(), th[:, d].copy()
+
+
+def fit_objective_h(W0, z, A, B, H) -> float:
+    """sum_n (W~[n] - W0[n])^T H (W~[n] - W0[n]), the quantity fit_affine_h minimizes."""
+    r = decode(z, A, B) - np.asarray(W0, dtype=np.float64)
+    return float(np.einsum("nk,kl,nl->", r, np.asarray(H, dtype=np.float64), r))
+
+
 def fit_objective(W0, z, A, B, h=None) -> float:
     """sum_n sum_k h_k (W0[n, k] - (A z + B)[n, k])^2, the quantity fit_affine minimizes."""
     r = np.asarray(W0, dtype=np.float64) - decode(z, A, B)

@@ -9,7 +9,8 @@ mistakes:
 - a lost mask;
 - a dropped intercept or normaliser;
 - missing error feedback;
-- an unreversed factorisation.
+- an unreversed factorisation;
+- a Hessian with its cross-position coupling dropped, or left out of one side.
 
 Nothing here touches a GPU.
 """
@@ -23,6 +24,22 @@ from tests import test_oracle_pins as P
 _decode, _assign, _pack = O.decode, O.assign, O.pack_codes
 _backward, _fit, _ldlq = O.backward, O.fit_affine, O.ldlq_assign
 _pack_mask, _dge_d, _ldl, _hess = O.pack_mask, O.dge_derivative, O.ldl_upper, O.code_space_hessian
+_fit_h, _fit_h_normal = O.fit_affine_h, O.fit_affine_h_normal
+
+
+def _fit_h_block_diagonal(W0, z, d, H):  # the (g, g') coupling of H dropped
+    H = np.asarray(H, dtype=np.float64)
+    Hb = np.zeros_like(H)
+    for g0 in range(0, H.shape[0], d):
+        Hb[g0:g0 + d, g0:g0 + d] = H[g0:g0 + d, g0:g0 + d]
+    return _fit_h(W0, z, d, Hb)
+
+
+def _fit_h_rhs_without_h(W0, z, d, H):  # the right-hand side formed with H = I
+    G, _ = _fit_h_normal(W0, z, d, H)
+    _, R = _fit_h_normal(W0, z, d, np.eye(np.asarray(H).shape[0]))
+    th = (np.linalg.pinv(G, rcond=O.PINV_RCOND, hermitian=True) @ R).reshape(d, d + 1)
+    return th[:, :d].copy(), th[:, d].copy()
 
 
 def _assign_half_up(Wp):
@@ -108,6 +125,10 @@ MUTATIONS = [
      [lambda gd: P.test_ldl_upper_reconstructs_the_matrix()]),
     ("code-space Hessian: A on the wrong side", "code_space_hessian", _hessian_untransposed,
      [lambda gd: P.test_code_space_objective_is_the_weight_space_objective()]),
+    ("full-H refit: (g, g') coupling dropped", "fit_affine_h", _fit_h_block_diagonal,
+     [lambda gd: P.test_fit_affine_h_equals_least_squares_with_the_hessian_root(4)]),
+    ("full-H refit: right-hand side without H", "fit_affine_h", _fit_h_rhs_without_h,
+     [lambda gd: P.test_fit_affine_h_recovers_an_exact_affine_map(4)]),
 ]
 
 

@@ -537,6 +537,111 @@ def test_fit_planted_mistake_is_caught():
     assert not np.allclose(th[:d], A[1], atol=1e-6)
 
 
+# ---------------------------------------------------------------- refit under the full Hessian H
+def _calib_hessian(g, K, n=None, ridge=0.05):
+    """H = X^T X / n of correlated calibration rows (a shared component and a
+    few outlier channels), plus a ridge: symmetric positive definite and far
+    from diagonal."""
+    n = n or 3 * K
+    X = g.standard_normal((n, K)) + 0.8 * g.standard_normal((n, 1))
+    X[:, g.choice(K, max(1, K // 16), replace=False)] *= 6.0
+    return X.T @ X / n + ridge * np.eye(K)
+
+
+@pytest.mark.parametrize("d", [1, 2, 4, 8])
+def test_fit_affine_h_recovers_an_exact_affine_map(d):
+    """W0 generated as A z + B is fitted with zero objective under any positive
+    definite H: (A, B) come back."""
+    g, z, A, B, W0 = _fit_case(d, 29, 8 * d, 1700 + d)
+    H = _calib_hessian(g, 8 * d)
+    A2, B2 = O.fit_affine_h(W0, z, d, H)
+    assert np.allclose(A2, A, atol=1e-9) and np.allclose(B2, B, atol=1e-9)
+    assert O.fit_objective_h(W0, z, A2, B2, H) < 1e-16 * np.abs(W0).sum() ** 2
+
+
+@pytest.mark.parametrize("d", [2, 4, 8])
+def test_fit_affine_h_equals_least_squares_with_the_hessian_root(d):
+    """The objective is sum_n |H^(1/2) (Phi_n theta - w0_n)|^2 with Phi_n the
+    linear map from theta = [A | B] to the decoded row n; stacking
+    H^(1/2) Phi_n over the rows and solving by lstsq (a different formulation:
+    a matrix square root and an orthogonal factorisation instead of the normal
+    equations) gives the same (A, B)."""
+    g, z, A, B, W0 = _fit_case(d, 13, 6 * d, 1800 + d, noise=0.3)
+    K = 6 * d
+    H = _calib_hessian(g, K)
+    ev, V = np.linalg.eigh(H)
+    Hr = (V * np.sqrt(ev)) @ V.T                       # H^(1/2)
+    N = W0.shape[0]
+    rows, rhs = [], []
+    for n in range(N):
+        Phi = np.zeros((K, d * (d + 1)))
+        for grp in range(K // d):
+            zt = np.append(z[n, grp * d:(grp + 1) * d].astype(np.float64), 1.0)
+            for i in range(d):
+                Phi[grp * d + i, i * (d + 1):(i + 1) * (d + 1)] = zt
+        rows.append(Hr @ Phi)
+        rhs.append(Hr @ W0[n])
+    th = np.linalg.lstsq(np.vstack(rows), np.concatenate(rhs), rcond=None)[0].reshape(d, d + 1)
+    A2, B2 = O.fit_affine_h(W0, z, d, H)
+    assert np.allclose(A2, th[:, :d], atol=1e-9) and np.allclose(B2, th[:, d], atol=1e-9)
+
+
+@pytest.mark.parametrize("d", [1, 4, 8])
+def test_fit_affine_h_with_a_diagonal_hessian_is_the_weighted_fit(d):
+    """H = diag(h) decouples the output coordinates: the result is the
+    per-channel weighted fit (fit_affine with weights h)."""
+    g, z, _, _, W0 = _fit_case(d, 21, 8 * d, 1900 + d, noise=0.4)
+    h = g.uniform(0.2, 3.0, size=8 * d)
+    A1, B1 = O.fit_affine(W0, z, d, h)
+    A2, B2 = O.fit_affine_h(W0, z, d, np.diag(h))
+    assert np.allclose(A1, A2, atol=1e-10) and np.allclose(B1, B2, atol=1e-10)
+
+
+def test_fit_affine_h_is_a_minimum_and_scale_invariant():
+    """Every small perturbation of (A, B) raises sum_n r_n^T H r_n, its
+    central-difference gradient vanishes at the fit, and scaling H leaves the
+    fit unchanged."""
+    d = 4
+    g, z, _, _, W0 = _fit_case(d, 11, 32, 2000, noise=0.4)
+    H = _calib_hessian(g, 32)
+    A2, B2 = O.fit_affine_h(W0, z, d, H)
+    A5, B5 = O.fit_affine_h(W0, z, d, 5.0 * H)
+    assert np.allclose(A2, A5, atol=1e-11) and np.allclose(B2, B5, atol=1e-11)
+    f0 = O.fit_objective_h(W0, z, A2, B2, H)
+    eps = 1e-4
+    for t in range(d * d + d):
+        dA = np.zeros((d, d))
+        dB = np.zeros(d)
+        if t < d * d:
+            dA.flat[t] = eps
+        else:
+            dB[t - d * d] = eps
+        fp = O.fit_objective_h(W0, z, A2 + dA, B2 + dB, H)
+        fm = O.fit_objective_h(W0, z, A2 - dA, B2 - dB, H)
+        assert fp > f0 and fm > f0
+        assert abs(fp - fm) / (2 * eps) < 1e-6 * (1 + f0)
+
+
+def test_fit_affine_h_beats_the_diagonal_fit_on_a_correlated_hessian():
+    """On a correlated H the full-H fit reaches a lower H-objective than the
+    fit that keeps only diag(H); dropping the off-diagonal blocks (g != g') of
+    the normal equations, a plausible mistake, is caught by the stacked
+    least-squares pin's answer."""
+    d = 4
+    g, z, _, _, W0 = _fit_case(d, 15, 32, 2100, noise=0.5)
+    H = _calib_hessian(g, 32)
+    Af, Bf = O.fit_affine_h(W0, z, d, H)
+    Ad, Bd = O.fit_affine(W0, z, d, np.diag(H))
+    assert O.fit_objective_h(W0, z, Af, Bf, H) < O.fit_objective_h(W0, z, Ad, Bd, H)
+    # block-diagonal mistake: H with its off-diagonal d x d blocks removed
+    Hb = np.zeros_like(H)
+    for grp in range(32 // d):
+        sl = slice(grp * d, (grp + 1) * d)
+        Hb[sl, sl] = H[sl, sl]
+    Ab, Bb = O.fit_affine_h(W0, z, d, Hb)
+    assert not np.allclose(Ab, Af, atol=1e-6)
+
+
 # ---------------------------------------------------------------- H-aware sequential assignment
 def _spd(g, K, n=None, ridge=0.05):
     """A correlated symmetric positive definite K x K matrix: X^T X / n from

@@ -738,9 +738,9 @@ def row_stack(D, pk, layers=32, ms=(1, 8, 32), cpu=True):
             sg = StepGraphs(fn, 1, 5)
             sg.replay()
             t, launches, _ = timed_graphs(D, sg)
-            ms = t / 5
-            gbs = total_bytes / (ms * 1e-3) / 1e9
-            res_m[name] = dict(value=gbs, unit="GB/s", us=ms * 1e3, launches_per_pass=launches // 5,
+            ms_pass = t / 5
+            gbs = total_bytes / (ms_pass * 1e-3) / 1e9
+            res_m[name] = dict(value=gbs, unit="GB/s", us=ms_pass * 1e3, launches_per_pass=launches // 5,
                                roofline=dict(bound="hbm", achieved=gbs, peak=pk["hbm_gbs"], unit="GB/s",
                                              frac=gbs / pk["hbm_gbs"]))
             del sg
@@ -820,6 +820,52 @@ def row_fit(D, pk, cpu=True):
     return res
 
 
+def row_fit_h(D, pk, cpu=True):
+    """Least-squares (A, B) refit under the full input Hessian on a 4096 x 4096
+    matrix (d = 8) with an 8192-row calibration Hessian (outlier recipe, 1%
+    ridge) formed on the device before timing.  The call's work is dominated by
+    one tensor-core contraction of 2 (K + 64)(3 K + 64) N flops (the code Gram
+    and the targets times the codes); value = those flops / the whole call."""
+    dev = D.dev
+    N = K = 4096
+    d = 8
+    g = np.random.Generator(np.random.PCG64(2500))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A0, B0 = synth.affine_diag_dominant(d, g)
+    zt = torch.from_numpy(z).to(dev)
+    W0 = (torch.from_numpy(A0).to(dev) @ zt.view(N, K // d, d).float().transpose(1, 2)).transpose(1, 2)
+    W0 = (W0 + torch.from_numpy(B0).to(dev)).reshape(N, K).contiguous()
+    W0 += 0.005 * torch.randn((N, K), device=dev, generator=torch.Generator(device=dev).manual_seed(1))
+    packed, _ = lcvq.assign_pack(zt.float(), d, with_mask=False)
+    w = synth.ldlq_workload(N, K, d, n_cal=8192)
+    X = torch.from_numpy(w["Xcal"]).to(dev, torch.float64)
+    H64 = X.T @ X / X.shape[0]
+    H64 += 0.01 * H64.diagonal().mean() * torch.eye(K, dtype=torch.float64, device=dev)
+    H = H64.float().contiguous()
+    del X, H64
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_FIT_AFFINE_H, torch.float32, 0, N, K, d), dev)
+    A = torch.empty((d, d), device=dev)
+    B = torch.empty(d, device=dev)
+    ms = graph_time(lambda: lcvq.fit_affine_h(W0, packed, d, H, workspace=ws, A=A, B=B), 5)
+    flops = 2.0 * (K + 64) * (3 * K + 64) * N
+    tf = flops / (ms * 1e-3) / 1e12
+    res = dict(metric="(A, B) refit under the full Hessian TFLOP/s (2 (K+64)(3K+64) N / call time)",
+               value=tf, unit="TFLOP/s", us=ms * 1e3,
+               roofline=_roof("tensor", tf, pk["bf16_tflops"], "TFLOP/s",
+                              note="whole call (operand pass, Gram GEMM, fp64 contraction, solve)"))
+    if cpu:  # the numpy oracle's normal equations and solve on the first `rows` rows
+        from oracle import lcvq_oracle as O
+        rows = 256
+        W0h = W0[:rows].cpu().numpy().astype(np.float64)
+        Hh = H.cpu().numpy().astype(np.float64)
+        n, dt = _timed_loop(lambda: O.fit_affine_h(W0h, z[:rows], d, Hh), 3.0)
+        res["cpu_baseline"] = dict(value=n * 2.0 * (K + 64) * (3 * K + 64) * rows / dt / 1e12,
+                                   unit="TFLOP/s", cores=_blas_threads(), kind="oracle",
+                                   sample=f"{n} refits of the first {rows} of {N} rows by the numpy "
+                                          f"fp64 oracle, {dt:.1f} s")
+    return res
+
+
 def row_ldlq(D, pk, cpu=True):
     """H-aware sequential code assignment on a 4096 x 4096 matrix (d = 8): the
     code-space factor of a calibration Hessian (8192 activation rows, outlier
@@ -869,8 +915,8 @@ def _blas_threads() -> int:
 
 ROWS = {"single_layer": row_single_layer, "assign_pack": row_assign_pack, "decode": row_decode,
         "prefill": row_prefill, "qat": row_qat, "stack": row_stack, "fit": row_fit,
-        "ldlq": row_ldlq}
-CPU_ROWS = ("single_layer", "prefill", "qat", "stack", "fit", "ldlq")
+        "fit_h": row_fit_h, "ldlq": row_ldlq}
+CPU_ROWS = ("single_layer", "prefill", "qat", "stack", "fit", "fit_h", "ldlq")
 
 
 def row_summary(name, r) -> str:

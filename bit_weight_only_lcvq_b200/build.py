@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "liblcvq.so")
 OBJDIR = os.path.join(ROOT, "_build", "obj")
 
-SOURCES = ["api.cu", "elementwise.cu", "xform.cu", "gemv.cu", "simt.cu", "tc_gemm.cu", "static_scratch.cu", "fit.cu", "gemv_tc.cu", "ldlq.cu"]
+SOURCES = ["api.cu", "elementwise.cu", "xform.cu", "gemv.cu", "simt.cu", "tc_gemm.cu", "static_scratch.cu", "fit.cu", "fit_h.cu", "gemv_tc.cu", "ldlq.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -74,6 +74,8 @@ lcvq_status check_device() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 constexpr int64_t kMaxGemmDim = int64_t(1) << 30;
 constexpr int64_t kMaxLdlqDim = int64_t(1) << 20;  // U is d_in^2 floats
+constexpr int64_t kMaxFitHDin = int64_t(1) << 16;  // the Gram is ~12 d_in^2 bytes
+constexpr int64_t kMaxFitHDout = int64_t(1) << 20; // integer code sums stay exact in fp32
 bool valid_d(int d) { return d == 1 || d == 2 || d == 4 || d == 8; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -174,7 +176,30 @@ size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_ou
   if (op == LCVQ_OP_GEMM_BACKWARD) return bwd_ws(M, d_out, d_in, d).total;
   if (op == LCVQ_OP_FIT_AFFINE) return kWsHeaderBytes + fit_partials_bytes(d_out, d_in, d);
   if (op == LCVQ_OP_ASSIGN_LDLQ) return kWsHeaderBytes + ldlq_workspace_bytes(d_out, d_in);
+  if (op == LCVQ_OP_FIT_AFFINE_H) return kWsHeaderBytes + fith_scratch_bytes(d_out, d_in, d);
   return 0;
+}
+
+lcvq_status lcvq_fit_affine_h(const float* W0, const uint8_t* packed, int64_t d_out, int64_t d_in,
+                              int d, const float* H, float* A, float* B, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  g_last_launches = 0;
+  if (d_out < 0 || d_in < 0 || !valid_d(d) || d_in % 64 != 0) return LCVQ_ERR_INVALID_ARG;
+  if (d_in > kMaxFitHDin || d_out > kMaxFitHDout) return LCVQ_ERR_INVALID_ARG;
+  if (!A || !B || !workspace) return LCVQ_ERR_INVALID_ARG;
+  const bool empty = d_out == 0 || d_in == 0;
+  if (!empty && (!W0 || !packed || !H)) return LCVQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || !aligned16(A) || !aligned16(B) ||
+      (!empty && (!aligned16(W0) || !aligned16(packed) || !aligned16(H))))
+    return LCVQ_ERR_ALIGNMENT;
+  if (ws_bytes < kWsHeaderBytes + fith_scratch_bytes(d_out, d_in, d)) return LCVQ_ERR_WORKSPACE;
+  if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
+  int launches = 0;
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e = launch_fit_affine_h(W0, packed, empty ? 0 : d_out, empty ? 0 : d_in, d, H, A, B,
+                                      ws + kWsHeaderBytes, reinterpret_cast<unsigned int*>(ws),
+                                      static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
 }
 
 lcvq_status lcvq_assign_ldlq(const float* P, const float* U, int64_t d_out, int64_t d_in, int d,

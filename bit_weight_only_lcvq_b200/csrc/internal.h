@@ -97,6 +97,14 @@ cudaError_t launch_fit_affine(const float* W0, const uint8_t* packed, int64_t d_
                               int d, const float* h, float* A, float* B, double* partials,
                               cudaStream_t s, int* launches);
 
+// ---- least-squares refit of (A, B) under the full Hessian H ----
+// scratch: fith_scratch_bytes(d_out, d_in, d) bytes (the bf16 operands, the
+// fp32 Gram and the fp64 partials of the normal equations)
+size_t fith_scratch_bytes(int64_t d_out, int64_t d_in, int d);
+cudaError_t launch_fit_affine_h(const float* W0, const uint8_t* packed, int64_t d_out, int64_t d_in,
+                                int d, const float* H, float* A, float* B, void* scratch,
+                                unsigned int* err, cudaStream_t s, int* launches);
+
 // ---- H-aware sequential code assignment ----
 // E: ldlq_workspace_bytes(d_out, d_in) bytes of fp32 scratch (the errors p - z)
 size_t ldlq_workspace_bytes(int64_t d_out, int64_t d_in);
@@ -121,6 +129,11 @@ cudaError_t launch_tc_backward_dw(const uint16_t* X, const uint16_t* dY, int64_t
                                   int64_t d_in, int d, const float* A, float* dWp,
                                   float* partials, int* num_parts, unsigned int* err,
                                   cudaStream_t s, int* launches);
+// C[r][c] = sum_n Q[n][r] Q[n][c] for r < cols_p, c < cols_q (fp32 out,
+// [cols_p][cols_q]): the tcgen05 Gram of Q's first cols_p columns against all
+// of Q (bf16 [rows][cols_q]); cols_p, cols_q multiples of 64
+cudaError_t launch_tc_gram(const uint16_t* Q, int64_t rows, int64_t cols_p, int64_t cols_q,
+                           float* C, unsigned int* err, cudaStream_t s, int* launches);
 // r[m] = sum_n dY[m][n] (fp64 accumulation), bf16 dY
 cudaError_t launch_rowsum(const uint16_t* dY, int64_t M, int64_t n, float* r, cudaStream_t s,
                           int* launches);

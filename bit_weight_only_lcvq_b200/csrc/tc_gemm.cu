@@ -28,6 +28,10 @@
 //           (both MN-major); the epilogue never stores G: it writes
 //           dWp = mask * A^T G per d-vector (STE, Methodology 3) and accumulates
 //           sum G_i z_j, sum G_i into per-CTA partials of dA, dB.
+//   Gram    C[r][c]  = sum_n P[n][r] Q[n][c]                  A = P^T, B = Q^T
+//           (both MN-major, bf16 from TMA); the epilogue stores C in fp32.  The
+//           refit under a full Hessian forms the code Gram and the targets
+//           times the codes this way (fit_h.cu).
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -56,7 +60,7 @@ constexpr int kPairPeerGroup = 3;
 constexpr int kTmemCols = 512;
 constexpr long long kWaitLimit = 1LL << 32;  // clock cycles (~2 s)
 
-enum Kind { kFwdAlg = 0, kFwdDec = 1, kDx = 2, kDw = 3 };
+enum Kind { kFwdAlg = 0, kFwdDec = 1, kDx = 2, kDw = 3, kGram = 4 };
 
 struct Params {
   int64_t M, N, K;    // D is M x N, contraction K (see each kind)
@@ -75,9 +79,9 @@ struct Params {
 template <int KIND, int DW>
 struct Cfg {
   static constexpr int kThreads = 32 * (2 + DW + 4);
-  static constexpr bool kHasCodes = KIND != kDw;
-  static constexpr bool kAmn = KIND == kDw;
-  static constexpr bool kBmn = KIND == kDx || KIND == kDw;
+  static constexpr bool kHasCodes = KIND != kDw && KIND != kGram;
+  static constexpr bool kAmn = KIND == kDw || KIND == kGram;
+  static constexpr bool kBmn = KIND == kDx || KIND == kDw || KIND == kGram;
   static constexpr uint32_t kStageTx = A_BYTES + (kHasCodes ? C_BYTES : B_BYTES);
 };
 
@@ -177,6 +181,19 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const float* sAm
       v1.z = pack_bf16x2(o[12], o[13]); v1.w = pack_bf16x2(o[14], o[15]);
       reinterpret_cast<uint4*>(dX + 16 * b)[0] = v0;
       reinterpret_cast<uint4*>(dX + 16 * b)[1] = v1;
+    }
+  } else if constexpr (KIND == kGram) {
+    float* C = static_cast<float*>(p.out) + gm * p.N + gn0;
+    if (gn0 + 32 <= p.N) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(C)[q] =
+            make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                        __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+    } else {
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        if (gn0 + q < p.N) C[q] = __uint_as_float(r[q]);
     }
   } else {  // kDw: D row = n (d_out), D column = k (d_in)
     const int64_t n = gm, k0 = gn0;
@@ -284,7 +301,7 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if constexpr (KIND != kFwdAlg) {  // the algebraic form never touches A, B
+  if constexpr (KIND != kFwdAlg && KIND != kGram) {  // these never touch A, B
     if (threadIdx.x < D * D) sAm[threadIdx.x] = p.Amat[threadIdx.x];
     if (KIND != kDw && threadIdx.x >= 64 && threadIdx.x < 64 + D)
       sAm[D * D + threadIdx.x - 64] = p.Bvec[threadIdx.x - 64];
@@ -1007,6 +1024,20 @@ cudaError_t launch_tc_backward_dx(const uint16_t* dY, const float* rsum, int64_t
   p.M = M; p.N = d_in; p.K = d_out; p.d_in = d_in; p.d_out = d_out;
   p.codes = packed; p.rsum = rsum; p.Amat = A; p.Bvec = B; p.out = dX; p.err = err;
   cudaError_t e = launch_kind_d<kDx, 4>(d, ta, tb, p, s, nullptr);
+  ++*launches;
+  return e;
+}
+
+cudaError_t launch_tc_gram(const uint16_t* Q, int64_t rows, int64_t cols_p, int64_t cols_q,
+                           float* C, unsigned int* err, cudaStream_t s, int* launches) {
+  // P is the first cols_p columns of Q (same rows and row pitch)
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, cols_p, rows, cols_q * 2, 64, BK, true) ||
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, cols_q, rows, cols_q * 2, 64, BK, true))
+    return cudaErrorInvalidValue;
+  Params p{};
+  p.M = cols_p; p.N = cols_q; p.K = rows; p.out = C; p.err = err;
+  cudaError_t e = launch_kind<kGram, 8, 0>(ta, tb, p, s, nullptr);
   ++*launches;
   return e;
 }

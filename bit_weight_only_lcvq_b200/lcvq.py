@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcvq.so"
 
 F32, BF16 = 0, 1
 FORMS = {"auto": 0, "decode": 1, "algebraic": 2}
-OP_GEMM, OP_GEMM_BACKWARD, OP_FIT_AFFINE, OP_ASSIGN_LDLQ = 0, 1, 2, 3
+OP_GEMM, OP_GEMM_BACKWARD, OP_FIT_AFFINE, OP_ASSIGN_LDLQ, OP_FIT_AFFINE_H = 0, 1, 2, 3, 4
 STATUS = {
     0: "LCVQ_OK",
     1: "LCVQ_ERR_INVALID_ARG",
@@ -40,6 +40,7 @@ EXPORTS = (
     "lcvq_gemv_static",
     "lcvq_gemm_grouped",
     "lcvq_fit_affine",
+    "lcvq_fit_affine_h",
     "lcvq_dge_scale",
     "lcvq_assign_ldlq",
     "lcvq_workspace_size",
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
         L.lcvq_workspace_size_grouped.argtypes = [ctypes.POINTER(GemmItem), _i32, _i64, _i32]
         L.lcvq_workspace_size_grouped.restype = _sz
         L.lcvq_fit_affine.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.lcvq_fit_affine_h.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
         L.lcvq_dge_scale.argtypes = [_vp, _vp, _i64, ctypes.c_float, _vp]
         L.lcvq_assign_ldlq.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _sz, _vp]
         L.lcvq_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i64, _i32]
@@ -98,7 +100,7 @@ def lib() -> ctypes.CDLL:
         L.lcvq_last_launch_count.argtypes = []
         for fn in ("lcvq_assign_pack", "lcvq_decode", "lcvq_gemm", "lcvq_gemm_backward",
                    "lcvq_xform", "lcvq_gemm_xformed", "lcvq_gemv_static", "lcvq_gemm_grouped",
-                   "lcvq_fit_affine", "lcvq_dge_scale",
+                   "lcvq_fit_affine", "lcvq_fit_affine_h", "lcvq_dge_scale", "lcvq_assign_ldlq",
                    "lcvq_check_device_error",
                    "lcvq_last_launch_count"):
             getattr(L, fn).restype = ctypes.c_int
@@ -308,6 +310,25 @@ def fit_affine(W0: torch.Tensor, packed: torch.Tensor, d: int, *, h=None, worksp
                                   dev)
     _check("lcvq_fit_affine", lib().lcvq_fit_affine(
         _ptr(W0), _ptr(packed), d_out, d_in, d, _ptr(h), _ptr(A), _ptr(B), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return A, B
+
+
+def fit_affine_h(W0: torch.Tensor, packed: torch.Tensor, d: int, H: torch.Tensor, *,
+                 workspace=None, A=None, B=None, stream=None):
+    """Least-squares (A, B) for target weights W0 given the codes under the full
+    input Hessian H [d_in][d_in] (see lcvq_fit_affine_h).  Returns (A, B)."""
+    d_out, d_in = W0.shape
+    dev = W0.device
+    if A is None:
+        A = torch.empty((d, d), dtype=torch.float32, device=dev)
+    if B is None:
+        B = torch.empty(d, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(workspace_size(OP_FIT_AFFINE_H, torch.float32, 0, d_out, d_in, d),
+                                  dev)
+    _check("lcvq_fit_affine_h", lib().lcvq_fit_affine_h(
+        _ptr(W0), _ptr(packed), d_out, d_in, d, _ptr(H), _ptr(A), _ptr(B), _ptr(workspace),
         workspace.numel(), _stream(stream)))
     return A, B
 

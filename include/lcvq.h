@@ -96,7 +96,8 @@ typedef enum {
   LCVQ_OP_GEMM = 0,
   LCVQ_OP_GEMM_BACKWARD = 1,
   LCVQ_OP_FIT_AFFINE = 2,
-  LCVQ_OP_ASSIGN_LDLQ = 3
+  LCVQ_OP_ASSIGN_LDLQ = 3,
+  LCVQ_OP_FIT_AFFINE_H = 4
 } lcvq_op;
 
 /* Code assignment and 2-bit packing (LC-QAT technical summary, Methodology 1:
@@ -281,6 +282,43 @@ LCVQ_API lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, floa
 LCVQ_API lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int64_t d_out,
                                      int64_t d_in, int d, const float* h, float* A, float* B,
                                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Least-squares refit of (A, B) under the full input Hessian H (decoupleQ
+ * page: eq. (5), the layer objective tr{(W~ - W0)^T H (W~ - W0)} with W~ and
+ * W0 of shape d_in x d_out and H = X^T X of the layer's inputs; section 3.3:
+ * with the integer part fixed the float part is a quadratic, solved in closed
+ * form; LC-QAT technical summary, Methodology 1, for the codewords
+ * c = A z + B).  In storage order the call minimizes
+ *     sum_n (W~[n] - W0[n])^T H (W~[n] - W0[n]),   W~ = A z + B per vector,
+ * over A and B.  With theta = [A | B] (row i = [A[i][0..d-1], B[i]]) and
+ * zt = [z_0 .. z_{d-1}, 1] per vector, the normal equations couple every pair
+ * of vector positions (g, h):
+ *     L[(i,a),(j,b)] = sum_{g,h} H[g d + i][h d + j] sum_n zt[n][g][a] zt[n][h][b]
+ *     R[(i,a)]       = sum_g sum_k H[g d + i][k] sum_n zt[n][g][a] W0[n][k]
+ * and theta = L^+ R (d (d+1) unknowns): Cholesky when every pivot is above
+ * 1e-8 of the largest diagonal entry, otherwise the pseudo-inverse with
+ * eigenvalues below 1e-12 of the largest taken as zero (the minimum-norm
+ * solution).  With H diagonal this is lcvq_fit_affine with h = diag(H).
+ * Arithmetic: the code Gram and the code column sums are exact (bf16 codes,
+ * fp32 tensor-core sums); W0 enters the tensor-core contraction W0^T Z as two
+ * bf16 terms (within 2^-18 of W0) summed in fp32 over the rows; the
+ * contraction with H and the solve are fp64.  Every sum has a fixed order:
+ * the result is bitwise reproducible.
+ *   W0     [d_out][d_in] fp32 target weights.
+ *   packed [d_out][d_in/4] codes (format V1).
+ *   H      [d_in][d_in] fp32, symmetric (every entry is read); e.g. X^T X of
+ *          calibration activations, usually with a small ridge.
+ *   A      [d*d] fp32 out (row-major);  B [d] fp32 out.
+ *   workspace: >= lcvq_workspace_size(LCVQ_OP_FIT_AFFINE_H, LCVQ_F32, 0, d_out,
+ *   d_in, d) bytes (about 2 d_out d_in * 3 + 12 d_in^2 bytes of scratch),
+ *   256-byte aligned, first 256 bytes zeroed once.
+ * Shapes: d_in % 64 == 0, d_in <= 65536, d_out <= 2^20; an empty matrix gives
+ * A = 0, B = 0.  Launches 4 kernels: the bf16 operand pass, one tcgen05 GEMM
+ * of 2 (d_in + 64)(3 d_in + 64) d_out flops, the fp64 contraction with H and
+ * the solve. */
+LCVQ_API lcvq_status lcvq_fit_affine_h(const float* W0, const uint8_t* packed, int64_t d_out,
+                                       int64_t d_in, int d, const float* H, float* A, float* B,
+                                       void* workspace, size_t ws_bytes, void* stream);
 
 /* H-aware sequential code assignment, the PTQ initialisation of the codes
  * (LC-QAT technical summary, Methodology 2: the initial integer weights come

@@ -363,11 +363,12 @@ def fit_affine_h_normal(W0: np.ndarray, z: np.ndarray, d: int, H: np.ndarray):
     N, K = W0.shape
     ng = K // d
     zt = np.concatenate([np.asarray(z, np.float64).reshape(N, ng, d), np.ones((N, ng, 1))], axis=2)
-    S = np.einsum("nga,nhb->gahb", zt, zt)                  # code Gram of every (g, g') pair
+    # (optimize=True lets numpy contract these sums through BLAS)
+    S = np.einsum("nga,nhb->gahb", zt, zt, optimize=True)   # code Gram of every (g, g') pair
     Hg = H.reshape(ng, d, ng, d)                            # H[g d + i, h d + j] -> [g, i, h, j]
-    G = np.einsum("gihj,gahb->iajb", Hg, S).reshape(d * (d + 1), d * (d + 1))
-    T = np.einsum("nk,nga->kga", W0, zt)                    # W0^T zt per position
-    R = np.einsum("gik,kga->ia", H.reshape(ng, d, K), T).reshape(d * (d + 1))
+    G = np.einsum("gihj,gahb->iajb", Hg, S, optimize=True).reshape(d * (d + 1), d * (d + 1))
+    T = np.einsum("nk,nga->kga", W0, zt, optimize=True)     # W0^T zt per position
+    R = np.einsum("gik,kga->ia", H.reshape(ng, d, K), T, optimize=True).reshape(d * (d + 1))
     return G, R
 
 

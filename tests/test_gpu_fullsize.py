@@ -236,3 +236,23 @@ def test_ldlq_full_size_qat_matrix():
     Z = O.unpack_codes(out.cpu().numpy()[rows], K)
     bad, near = ldlq_check(P[rows], U, Z)
     assert bad == 0, (bad, near)
+
+
+def test_fit_affine_h_full_size_decode_matrix():
+    """Refit under the full Hessian at 4096 x 4096 (d = 8) with an 8192-row
+    calibration Hessian (outlier recipe, 1% ridge): W0 = A0 z + B0 plus noise;
+    the GPU fit lies within the derived bound of the oracle and reaches its
+    H-objective."""
+    from tests.test_gpu_parity import _fith_bound, _fith_case, _fith_gpu
+    d, N, K = 8, 4096, 4096
+    z, A0, B0, W0, H = _fith_case(2500, N, K, d, noise=0.005, n_cal=8192)
+    H64, W64 = H.astype(np.float64), W0.astype(np.float64)
+    A_ref, B_ref = O.fit_affine_h(W64, z, d, H64)
+    A, B = _fith_gpu(W0, z, d, H)
+    got = np.concatenate([to_np(A), to_np(B)[:, None]], axis=1)
+    ref = np.concatenate([A_ref, B_ref[:, None]], axis=1)
+    bnd = _fith_bound(W64, z, d, H64, A_ref, B_ref)
+    assert np.all(np.abs(got - ref) <= bnd), float(np.max(np.abs(got - ref) / bnd))
+    assert O.fit_objective_h(W64, z, to_np(A), to_np(B), H64) <= \
+        O.fit_objective_h(W64, z, A_ref, B_ref, H64) * (1 + 1e-6)
+    assert np.max(np.abs(ref - np.concatenate([A0, B0[:, None]], axis=1))) < 1e-3

@@ -674,3 +674,106 @@ def test_gemm_grouped_outputs_are_canaried():
         assert all(guard_intact(o, b) for o, b in pairs)
         ref, D = O.forward(ws[0]["X"], zs[0], ws[0]["A"], ws[0]["B"])
         assert_close("canaried grouped item 0", to_np(pairs[0][0]), ref, D, TOL_BF16)
+
+
+# ------------------------------------------ least-squares refit under the full Hessian H
+def _fith_bound(W0, z, d, H, A_ref, B_ref):
+    """Error bound of lcvq_fit_affine_h.  The code Gram and column sums are
+    exact; T~ = W0^T zt carries the bf16 hi/lo split of W0 (2^-18) and the
+    fp32 sum over the rows (at most one rounding per 16-row tensor-core step,
+    plus the step's own sum), so |dT~| <= eps_t sum|W0| zt; R then moves by at
+    most eps_t (|H| |W0|^T zt summed as R is), and theta = L^+ R by |L^+| |dR|
+    to first order.  The fp64 contraction and solve add ~1e-12 relative, the
+    fp32 result 2^-24.  The oracle supplies L, R and the absolute sums."""
+    N = W0.shape[0]
+    L, _ = O.fit_affine_h_normal(W0, z, d, H)
+    La, Ra = O.fit_affine_h_normal(np.abs(W0), z, d, np.abs(H))
+    th = np.concatenate([A_ref, B_ref[:, None]], axis=1).ravel()
+    eps_t = 2.0 ** -17 + (np.ceil(N / 16) + 32) * 2.0 ** -23
+    Pinv = np.abs(np.linalg.pinv(L, rcond=O.PINV_RCOND, hermitian=True))
+    bnd = Pinv @ ((eps_t + 1e-12) * Ra + 1e-12 * La @ np.abs(th)) + 2.0 ** -24 * np.abs(th)
+    bnd = bnd + 1e-12 * np.max(np.abs(th))
+    return bnd.reshape(d, d + 1)
+
+
+def _fith_case(seed, N, K, d, noise=0.01, n_cal=None):
+    g = np.random.Generator(np.random.PCG64(seed))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A0, B0 = synth.affine_diag_dominant(d, g)
+    W0 = (O.decode(z, A0, B0) + noise * g.standard_normal((N, K))).astype(np.float32)
+    n_cal = n_cal or 2 * K
+    X = synth.x_outliers(n_cal, K, g, g, "fp32").astype(np.float64)
+    H = X.T @ X / n_cal
+    H += 0.01 * np.mean(np.diag(H)) * np.eye(K)
+    return z, A0, B0, W0, H.astype(np.float32)
+
+
+def _fith_gpu(W0, z, d, H):
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_FIT_AFFINE_H, torch.float32, 0,
+                                                W0.shape[0], W0.shape[1], d))
+    A, B = lcvq.fit_affine_h(torch.from_numpy(W0).to(dev()), torch.from_numpy(O.pack_codes(z)).to(dev()),
+                             d, torch.from_numpy(H).to(dev()), workspace=ws)
+    assert lcvq.check_device_error(ws) == 0
+    return A, B
+
+
+@pytest.mark.parametrize("d", [1, 2, 4, 8])
+@pytest.mark.parametrize("N,K", [(77, 192), (300, 512)])
+def test_fit_affine_h_matches_oracle(d, N, K):
+    """GPU refit under a correlated calibration Hessian against the oracle's
+    normal equations over every (g, g') pair, within the derived bound, on
+    ragged row counts and K not a multiple of the 256-column chunk."""
+    z, A0, B0, W0, H = _fith_case(2200 + 10 * d + N, N, K, d)
+    H64, W64 = H.astype(np.float64), W0.astype(np.float64)
+    A_ref, B_ref = O.fit_affine_h(W64, z, d, H64)
+    A, B = _fith_gpu(W0, z, d, H)
+    got = np.concatenate([to_np(A), to_np(B)[:, None]], axis=1)
+    ref = np.concatenate([A_ref, B_ref[:, None]], axis=1)
+    bnd = _fith_bound(W64, z, d, H64, A_ref, B_ref)
+    assert np.all(np.abs(got - ref) <= bnd), float(np.max(np.abs(got - ref) / bnd))
+    # the fit is the H-objective's minimum: the GPU answer is as good as the oracle's
+    f_gpu = O.fit_objective_h(W64, z, to_np(A), to_np(B), H64)
+    f_ref = O.fit_objective_h(W64, z, A_ref, B_ref, H64)
+    assert f_gpu <= f_ref * (1 + 1e-6) + 1e-12
+
+
+def test_fit_affine_h_with_diagonal_h_agrees_with_fit_affine():
+    """H = diag(h): the full-H refit and the per-channel refit solve the same
+    problem; both lie within their bounds of the oracle."""
+    d, N, K = 8, 64, 256
+    g = np.random.Generator(np.random.PCG64(2300))
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    A0, B0 = synth.affine_diag_dominant(d, g)
+    W0 = (O.decode(z, A0, B0) + 0.02 * g.standard_normal((N, K))).astype(np.float32)
+    h = g.uniform(0.5, 2.0, size=K).astype(np.float32)
+    A_ref, B_ref = O.fit_affine(W0.astype(np.float64), z, d, h.astype(np.float64))
+    A1, B1 = _fith_gpu(W0, z, d, np.diag(h).astype(np.float32))
+    bnd = _fith_bound(W0.astype(np.float64), z, d, np.diag(h).astype(np.float64), A_ref, B_ref)
+    got = np.concatenate([to_np(A1), to_np(B1)[:, None]], axis=1)
+    ref = np.concatenate([A_ref, B_ref[:, None]], axis=1)
+    assert np.all(np.abs(got - ref) <= bnd)
+    A2, B2 = lcvq.fit_affine(torch.from_numpy(W0).to(dev()), torch.from_numpy(O.pack_codes(z)).to(dev()),
+                             d, h=torch.from_numpy(h).to(dev()))
+    assert _fit_ok(A2, B2, A_ref, B_ref, _fit_bound(W0.astype(np.float64), z, d,
+                                                    h.astype(np.float64), A_ref, B_ref))
+
+
+def test_fit_affine_h_singular_empty_and_deterministic():
+    """A code position that never varies makes L singular: the minimum-norm
+    solution (the Jacobi pseudo-inverse path); an empty matrix gives zeros; two
+    runs give the same bits."""
+    d, N, K = 4, 96, 128
+    z, _, _, W0, H = _fith_case(2400, N, K, d, noise=0.3)
+    z = z.copy()
+    z[:, 1::d] = 2
+    A_ref, B_ref = O.fit_affine_h(W0.astype(np.float64), z, d, H.astype(np.float64))
+    A1, B1 = _fith_gpu(W0, z, d, H)
+    A2, B2 = _fith_gpu(W0, z, d, H)
+    assert torch.equal(A1, A2) and torch.equal(B1, B2)
+    got = np.concatenate([to_np(A1).ravel(), to_np(B1)])
+    ref = np.concatenate([A_ref.ravel(), B_ref])
+    assert np.max(np.abs(got - ref)) <= 1e-5 * np.max(np.abs(ref)), (got, ref)
+    Ae, Be = lcvq.fit_affine_h(torch.zeros((0, K), device=dev()),
+                               torch.zeros((0, K // 4), dtype=torch.uint8, device=dev()), d,
+                               torch.from_numpy(H).to(dev()))
+    assert torch.count_nonzero(Ae) == 0 and torch.count_nonzero(Be) == 0

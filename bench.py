@@ -64,9 +64,6 @@ def parse():
 # the source file.
 NCU_TRAFFIC = {
     # source file -> (sha1 of the file when captured, {token count: bytes per launch})
-    # M = 1 and 4 share one instantiation of the kernel
-    "bit_weight_only_lcvq_b200/csrc/gemv.cu": (
-        "5016dd5597b05501b2883e20d2dbeb24c777ddc9", {1: 4237173, 4: 4237173, 16: 4366684}),
 }
 
 

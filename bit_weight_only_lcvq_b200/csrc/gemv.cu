@@ -29,65 +29,15 @@
 #include <mutex>
 #include <utility>
 
+#include "codec.cuh"
 #include "common.cuh"
+#include "gemv_common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
 namespace lcvq {
 
 namespace {
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
-                                               uint32_t a2, uint32_t a3, uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// bf16x2 (128 + 4^p z_c, 128 + 4^p z_{c+8}) of pair c of a 16-code word, given
-// the word and its shifts by 6 and 12.
-template <int C>
-__device__ __forceinline__ uint32_t dec_pair(uint32_t w0, uint32_t w6, uint32_t w12) {
-  constexpr int P = C % 3;
-  const uint32_t src = (C < 3) ? w0 : ((C < 6) ? w6 : w12);
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n"  // (a & b) | c
-      : "=r"(r)
-      : "r"(src), "n"(0x00030003u << (2 * P)), "n"(0x43004300u));
-  return r;
-}
-
-// same as dec_pair<C> for a C that is a compile-time constant after unrolling
-__device__ __forceinline__ uint32_t dec_pair_rt(int c, uint32_t w0, uint32_t w6, uint32_t w12) {
-  switch (c) {
-    case 0: return dec_pair<0>(w0, w6, w12);
-    case 1: return dec_pair<1>(w0, w6, w12);
-    case 2: return dec_pair<2>(w0, w6, w12);
-    case 3: return dec_pair<3>(w0, w6, w12);
-    case 4: return dec_pair<4>(w0, w6, w12);
-    case 5: return dec_pair<5>(w0, w6, w12);
-    case 6: return dec_pair<6>(w0, w6, w12);
-    default: return dec_pair<7>(w0, w6, w12);
-  }
-}
-
-__device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
-  return q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
-}
-
-// A "unit" is 128 codes of a row (32 bytes); a chunk is kAhead units.
-constexpr int kUnit = 128;
-constexpr int kAhead = 4;
-
-__device__ __forceinline__ void griddep_wait() {
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-}
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
 
 // ---------------------------------------------------------------------------
 // Decode-GEMV over a group of matrices in one persistent launch.
@@ -135,19 +85,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-
 template <int R, int kStages, int kWarps>
 __host__ __device__ constexpr size_t group_smem_ring() {
   return size_t(kWarps) * kStages * (16 * R) * 128;

@@ -32,7 +32,9 @@
 #include <map>
 #include <mutex>
 
+#include "codec.cuh"
 #include "common.cuh"
+#include "gemv_common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -79,36 +81,6 @@ struct TcGroup {
 constexpr size_t kTcSmem = 1024 + size_t(kAStages) * kTcXBytes + size_t(kCStages) * kTcCodeBytes +
                            1024;
 
-template <int C>
-__device__ __forceinline__ uint32_t tc_dec_pair(uint32_t w0, uint32_t w6, uint32_t w12) {
-  constexpr int P = C % 3;
-  const uint32_t src = (C < 3) ? w0 : ((C < 6) ? w6 : w12);
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n"
-      : "=r"(r)
-      : "r"(src), "n"(0x00030003u << (2 * P)), "n"(0x43004300u));
-  return r;
-}
-
-// one 16-code word -> 8 bf16 pairs (decoder order: pair c = positions c, c+8)
-__device__ __forceinline__ void tc_dec_word(uint32_t w, uint32_t* o) {
-  const uint32_t w6 = w >> 6, w12 = w >> 12;
-  o[0] = tc_dec_pair<0>(w, w6, w12);
-  o[1] = tc_dec_pair<1>(w, w6, w12);
-  o[2] = tc_dec_pair<2>(w, w6, w12);
-  o[3] = tc_dec_pair<3>(w, w6, w12);
-  o[4] = tc_dec_pair<4>(w, w6, w12);
-  o[5] = tc_dec_pair<5>(w, w6, w12);
-  o[6] = tc_dec_pair<6>(w, w6, w12);
-  o[7] = tc_dec_pair<7>(w, w6, w12);
-}
-
-__device__ __forceinline__ void griddep_wait() {
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-}
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
 
 __device__ __forceinline__ void tc_fail(const TcGroup& g, volatile int* abort_flag, unsigned site) {
   record_error(g.err, LCVQ_ERR_DEVICE_TIMEOUT, site);
@@ -285,10 +257,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
           const uint4 cw =
               *reinterpret_cast<const uint4*>(crow + (((2 * slot + half) ^ (row & 7)) << 4));
           uint32_t v[32];
-          tc_dec_word(cw.x, v);
-          tc_dec_word(cw.y, v + 8);
-          tc_dec_word(cw.z, v + 16);
-          tc_dec_word(cw.w, v + 24);
+          dec_word8(cw.x, v);
+          dec_word8(cw.y, v + 8);
+          dec_word8(cw.z, v + 16);
+          dec_word8(cw.w, v + 24);
           tmem_st32(tmem + lanes + a * 64 + half * 32, v);
         }
         tmem_st_wait();

@@ -36,6 +36,7 @@
 
 #include <mutex>
 
+#include "codec.cuh"
 #include "common.cuh"
 #include "decode_mma.cuh"
 #include "internal.h"
@@ -105,24 +106,6 @@ __device__ __forceinline__ void tile_coords(int64_t tile, int64_t m_tiles, int64
 __device__ __forceinline__ void fail(const Params& p, volatile int* abort_flag, unsigned site) {
   record_error(p.err, LCVQ_ERR_DEVICE_TIMEOUT, site);
   *abort_flag = 1;
-}
-
-template <int C>
-__device__ __forceinline__ uint32_t dec_pair(uint32_t w0, uint32_t w6, uint32_t w12) {
-  constexpr int P = C % 3;
-  const uint32_t src = (C < 3) ? w0 : ((C < 6) ? w6 : w12);
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(r) : "r"(src), "n"(0x00030003u << (2 * P)), "n"(0x43004300u));
-  return r;
-}
-
-// one 16-code word -> two 16-byte chunks (pairs 0..3, 4..7) in decoder order
-__device__ __forceinline__ void dec_word(uint32_t w, uint4& c0, uint4& c1) {
-  const uint32_t w6 = w >> 6, w12 = w >> 12;
-  c0 = make_uint4(dec_pair<0>(w, w6, w12), dec_pair<1>(w, w6, w12), dec_pair<2>(w, w6, w12),
-                  dec_pair<3>(w, w6, w12));
-  c1 = make_uint4(dec_pair<4>(w, w6, w12), dec_pair<5>(w, w6, w12), dec_pair<6>(w, w6, w12),
-                  dec_pair<7>(w, w6, w12));
 }
 
 __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {

@@ -26,67 +26,11 @@
 // p(c) = c mod 3.
 #include "common.cuh"
 #include "internal.h"
+#include "xform.cuh"
 
 namespace lcvq {
 
 constexpr int kXfThreads = 256;
-
-// One 16-element block of the transform.
-// x16: the block's 16 bf16 activations as two 16-byte words.  sA: A (D x D,
-// row-major, fp32); sBp: B' = B + 3/2 A 1.  Writes the block's X'' in decoder
-// order (o[c] = bf16x2 of positions c and c + 8, each scaled by 4^-(c mod 3))
-// and the block's parts of the per-row constant:
-//   sb   = sum x^T B'           (s')
-//   sxr  = sum bf16(X')         (X'r)
-//   sxpp = sum X''
-template <int D>
-__device__ __forceinline__ void xform_block(const uint4& u0, const uint4& u1,
-                                            const float* __restrict__ sA,
-                                            const float* __restrict__ sBp, uint32_t (&o)[8],
-                                            float& sb, float& sxr, float& sxpp) {
-  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-  float x[16];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    x[2 * q] = bf16_lo(w[q]);
-    x[2 * q + 1] = bf16_hi(w[q]);
-  }
-  float xrd[16];  // bf16(X') as fp32
-  sb = 0.f;
-  sxr = 0.f;
-#pragma unroll
-  for (int v = 0; v < 16 / D; ++v) {
-#pragma unroll
-    for (int j = 0; j < D; ++j) {
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < D; ++i) acc = fmaf(x[v * D + i], sA[i * D + j], acc);
-      xrd[v * D + j] = bf16_to_f32(f32_to_bf16(acc));
-      sxr += xrd[v * D + j];
-    }
-#pragma unroll
-    for (int i = 0; i < D; ++i) sb = fmaf(x[v * D + i], sBp[i], sb);
-  }
-  sxpp = 0.f;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float scale = (c % 3 == 0) ? 1.0f : ((c % 3 == 1) ? 0.25f : 0.0625f);
-    const float lo = xrd[c] * scale;
-    const float hi = xrd[c + 8] * scale;
-    sxpp += lo + hi;
-    o[c] = pack_bf16x2(lo, hi);  // exact: power-of-two scaling of bf16 values
-  }
-}
-
-// B'[i] = B[i] + 3/2 sum_j A[i][j], summed in j order (thread i < D)
-template <int D>
-__device__ __forceinline__ float shifted_offset(const float* __restrict__ A_row, float b) {
-  float rs = 0.f;
-#pragma unroll
-  for (int j = 0; j < D; ++j) rs += A_row[j];
-  return b + 1.5f * rs;
-}
-
 
 // One launch transforms the rows of up to kItems matrices' activations: CTA
 // (m, i) does row m of item i (a single call is a group of one).
@@ -133,29 +77,34 @@ __global__ void __launch_bounds__(kXfThreads)
   const int64_t m = blockIdx.x;
   const uint16_t* xr = X + m * d_in;
   uint16_t* orow = Xpp + m * d_in;
-  double s_b = 0.0, s_xr = 0.0, s_xpp = 0.0;
-  const int64_t nblk = d_in / 16;
-  for (int64_t b = threadIdx.x; b < nblk; b += kXfThreads) {
-    const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
-    const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
-    uint32_t o[8];
-    float sb, sxr, sxpp;
-    xform_block<D>(u0, u1, sA, sBp, o, sb, sxr, sxpp);
-    uint4* dst = reinterpret_cast<uint4*>(orow + 16 * b);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-    s_b += sb;
-    s_xr += sxr;
-    s_xpp += sxpp;
-  }
-  // block reduction in a fixed order
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    s_b += __shfl_down_sync(0xffffffffu, s_b, off);
-    s_xr += __shfl_down_sync(0xffffffffu, s_xr, off);
-    s_xpp += __shfl_down_sync(0xffffffffu, s_xpp, off);
-  }
+  // warp w takes the chunks c = w, w + 8, ... (the classes of the corr sum);
+  // lane l transforms block l of the chunk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  double s_b = 0.0, s_xr = 0.0, s_xpp = 0.0;  // this class's running sums (lane 0)
+  const int64_t nblk = d_in / 16;
+  const int64_t nchunk = ceil_div(d_in, kCorrChunk);
+  for (int64_t c = warp; c < nchunk; c += kCorrClasses) {
+    const int64_t b = c * (kCorrChunk / 16) + lane;
+    float sb = 0.f, sxr = 0.f, sxpp = 0.f;
+    if (b < nblk) {
+      const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
+      const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
+      uint32_t o[8];
+      xform_block<D>(u0, u1, sA, sBp, o, sb, sxr, sxpp);
+      uint4* dst = reinterpret_cast<uint4*>(orow + 16 * b);
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    const double tb = chunk_tree_sum(double(sb));
+    const double txr = chunk_tree_sum(double(sxr));
+    const double txpp = chunk_tree_sum(double(sxpp));
+    if (lane == 0) {
+      s_b += tb;
+      s_xr += txr;
+      s_xpp += txpp;
+    }
+  }
+  static_assert(kXfThreads / 32 == kCorrClasses, "one warp per chunk class");
   if (lane == 0) {
     red[0][warp] = s_b;
     red[1][warp] = s_xr;
@@ -164,7 +113,7 @@ __global__ void __launch_bounds__(kXfThreads)
   __syncthreads();
   if (threadIdx.x == 0) {
     double a = 0.0, b = 0.0, c = 0.0;
-    for (int w = 0; w < kXfThreads / 32; ++w) {
+    for (int w = 0; w < kCorrClasses; ++w) {
       a += red[0][w];
       b += red[1][w];
       c += red[2][w];

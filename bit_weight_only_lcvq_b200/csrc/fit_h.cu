@@ -25,7 +25,8 @@
 //     in the fp32 accumulator (d_out * 9 < 2^24), so S~ is exact.
 //  3. fith_contract_kernel combines C with H in fp64 (exact products of fp32
 //     values) into per-CTA partials of L and R, in a fixed order;
-//     fith_solve_kernel sums the partials in CTA order and solves the
+//     fith_reduce_kernel sums the partials in CTA order; fith_solve_kernel
+//     solves the
 //     d (d+1) x d (d+1) system: Cholesky when every pivot is above 1e-8 of
 //     the largest diagonal entry, otherwise a parallel cyclic Jacobi
 //     eigendecomposition with eigenvalues below 1e-12 of the largest taken as
@@ -87,44 +88,60 @@ __global__ void __launch_bounds__(kPrepThreads) fith_prep_kernel(const float* __
 // ---------------------------------------------------------------- 3a. contraction with H
 // CTA c takes the vector positions g = c, c + G, ...; for each g it streams
 // column chunks of H's rows g d .. g d + d - 1 and of C's rows (g, a) through
-// shared memory.  Thread (i, a) of team tm (NP = d (d+1) threads per team)
-// accumulates L[(i,a), (j,b)] for all (j, b) over the h-blocks h = tm, tm +
-// kTeams, ... of each chunk, and R[(i,a)] over the chunk's k = tm, tm +
-// kTeams, ...; at the end the teams are added in team order into the CTA's
-// partial [L (NP x NP) | R (NP)] (fp64).
-constexpr int kChunkCols = 256;  // columns of H and C per shared-memory chunk
-constexpr int kTeams = 3;
+// shared memory, converted to fp64 once per element.  For every h-block of a
+// chunk with h >= g, L gains the Kronecker product of the H block
+// H[g d + i][h d + j] and the code Gram block S~[(g,a),(h,b)] (half of it for
+// h = g): H and S~ are symmetric, so the (h, g) block adds the transpose of
+// the (g, h) block and the solve forms L as L_half + L_half^T.  A thread owns a
+// register tile of
+// kJT values of j (for one i) times the d + 1 values of b (for one a), so it
+// loads kJT + d + 1 values per kJT (d + 1) fused multiply-adds.  The kTeams
+// teams of a CTA take alternate h-blocks; R[(i,a)] is split over the CTA's
+// threads by k mod parts.  At the end the teams (and the parts of R) are
+// added in a fixed order into the CTA's partial [L (NP x NP) | R (NP)] (fp64).
+constexpr int kChunkCols = 192;  // columns of H and C per shared-memory chunk
+constexpr int kRowPad = 1;       // doubles of padding per shared row: rows 2 banks apart
+constexpr int kTeams = 2;
 
 template <int D>
 struct FitHDims {
   static constexpr int NP = D * (D + 1);
-  static constexpr int kThreads = ((kTeams * NP + 31) / 32) * 32;
-  static constexpr int kCols = kChunkCols;     // a multiple of every d
-  static constexpr int kPart = NP * NP + NP;   // doubles per CTA partial
+  static constexpr int P1 = D + 1;
+  static constexpr int kJT = D < 4 ? D : 4;           // j values per thread tile
+  static constexpr int kTeam = D * (D / kJT) * P1;    // threads per team
+  static constexpr int kThreads = ((kTeams * kTeam + 31) / 32) * 32;
+  static constexpr int kRParts = kThreads / NP;       // threads per R value
+  static constexpr int kCols = kChunkCols;            // a multiple of every d
+  static constexpr int kPart = NP * NP + NP;          // doubles per CTA partial
 };
 
 template <int D>
 __global__ void __launch_bounds__(FitHDims<D>::kThreads) fith_contract_kernel(
     const float* __restrict__ H, const float* __restrict__ C, int64_t K, double* __restrict__ partials) {
   using F = FitHDims<D>;
-  constexpr int NP = F::NP, P1 = D + 1, COLS = F::kCols;
-  // chunk: H rows [D][COLS], S~ rows [D+1][COLS], T~ rows [D+1][COLS] as its
-  // hi and lo parts, and the ones column S~[(g,a),(., d)] = C[row(g,a)][0]
-  __shared__ float sH[D][COLS];
-  __shared__ float sS[P1][COLS];
-  __shared__ float sTh[P1][COLS];
-  __shared__ float sTl[P1][COLS];
-  __shared__ float sOnes[P1];
-  __shared__ double sRed[kTeams][NP + 1];
+  constexpr int NP = F::NP, P1 = F::P1, COLS = F::kCols, JT = F::kJT;
+  __shared__ double sH[D][COLS + kRowPad];
+  __shared__ double sS[P1][COLS + kRowPad];
+  __shared__ double sT[P1][COLS + kRowPad];  // T~ = hi + lo, in fp64
+  __shared__ double sOnes[P1];
+  __shared__ double sRed[kTeams > F::kRParts ? kTeams : F::kRParts][NP + 1];
   const int tid = threadIdx.x;
-  const int tm = tid / NP, me = tid % NP;
-  const bool active = tm < kTeams;
-  const int i = me / P1, a = me % P1;
+  // L tile: team tm, i, j block jb (j = jb JT .. jb JT + JT - 1), a
+  const int tm = tid / F::kTeam, mt = tid % F::kTeam;
+  const bool lact = tm < kTeams;
+  const int a = mt % P1, ij = mt / P1;
+  const int i = ij / (D / JT), j0 = (ij % (D / JT)) * JT;
+  // R: value ro = (i, a), part rp takes the chunk columns rp, rp + kRParts, ...
+  const int ro = tid % NP, rp = tid / NP;
+  const bool ract = rp < F::kRParts;
+  const int ri = ro / P1, ra = ro % P1;
   const int64_t ldc = kOnes + 3 * K;
   const int64_t ng = K / D;
-  double accL[NP];
+  double acc[JT][P1];
 #pragma unroll
-  for (int q = 0; q < NP; ++q) accL[q] = 0.0;
+  for (int x = 0; x < JT; ++x)
+#pragma unroll
+    for (int b = 0; b < P1; ++b) acc[x][b] = 0.0;
   double accR = 0.0;
 
   for (int64_t g = blockIdx.x; g < ng; g += gridDim.x) {
@@ -133,87 +150,139 @@ __global__ void __launch_bounds__(FitHDims<D>::kThreads) fith_contract_kernel(
       return C + (aa < D ? (kOnes + g * D + aa) : 0) * ldc;
     };
     __syncthreads();
-    if (tid < P1) sOnes[tid] = crow(tid)[0];
+    if (tid < P1) sOnes[tid] = static_cast<double>(crow(tid)[0]);
     for (int64_t c0 = 0; c0 < K; c0 += COLS) {
-      const int ncols = static_cast<int>(K - c0 < COLS ? K - c0 : COLS);  // multiple of D
+      const int ncols = static_cast<int>(K - c0 < COLS ? K - c0 : COLS);  // multiple of 64
       __syncthreads();  // the previous chunk is consumed
-      for (int e = tid; e < D * COLS; e += blockDim.x) {
-        const int r = e / COLS, c = e % COLS;
-        sH[r][c] = c < ncols ? H[(g * D + r) * K + c0 + c] : 0.f;
-      }
-      for (int e = tid; e < P1 * COLS; e += blockDim.x) {
-        const int r = e / COLS, c = e % COLS;
-        const float* cr = crow(r);
-        sS[r][c] = c < ncols ? cr[kOnes + c0 + c] : 0.f;
-        sTh[r][c] = c < ncols ? cr[kOnes + K + c0 + c] : 0.f;
-        sTl[r][c] = c < ncols ? cr[kOnes + 2 * K + c0 + c] : 0.f;
+      // 16-byte loads (K, the row pitches and the chunk starts are multiples of 4)
+      constexpr int V = COLS / 4;
+      const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int e = tid; e < (D + 2 * P1) * V; e += blockDim.x) {
+        const int r = e / V, c = (e % V) * 4;
+        double* dst;
+        float4 v = zero4;
+        if (r < D) {
+          if (c < ncols) v = __ldg(reinterpret_cast<const float4*>(H + (g * D + r) * K + c0 + c));
+          dst = &sH[r][c];
+        } else if (r < D + P1) {
+          if (c < ncols) v = __ldcg(reinterpret_cast<const float4*>(crow(r - D) + kOnes + c0 + c));
+          dst = &sS[r - D][c];
+        } else {
+          if (c < ncols) {
+            const float* cr = crow(r - D - P1) + kOnes + K + c0 + c;
+            const float4 hi = __ldcg(reinterpret_cast<const float4*>(cr));
+            const float4 lo = __ldcg(reinterpret_cast<const float4*>(cr + K));
+            dst = &sT[r - D - P1][c];
+            dst[0] = double(hi.x) + double(lo.x);
+            dst[1] = double(hi.y) + double(lo.y);
+            dst[2] = double(hi.z) + double(lo.z);
+            dst[3] = double(hi.w) + double(lo.w);
+            continue;
+          }
+          dst = &sT[r - D - P1][c];
+        }
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
       }
       __syncthreads();
-      if (active) {
-        // L: h-blocks tm, tm + kTeams, ... of the chunk
+      if (lact) {
+        // L: h-blocks tm, tm + kTeams, ... of the chunk with h >= g (the (h, g)
+        // block adds the transpose of the (g, h) block; the diagonal block
+        // counts half, so L = L_half + L_half^T)
+        const int hfirst = static_cast<int>(g - c0 / D);  // chunk's h-block index of h = g
         for (int hb = tm; hb < ncols / D; hb += kTeams) {
-          double hv[D], sv[P1];
+          if (hb < hfirst) continue;
+          const double wgt = hb == hfirst ? 0.5 : 1.0;
+          double hv[JT], sv[P1];
 #pragma unroll
-          for (int j = 0; j < D; ++j) hv[j] = static_cast<double>(sH[i][hb * D + j]);
+          for (int x = 0; x < JT; ++x) hv[x] = wgt * sH[i][hb * D + j0 + x];
 #pragma unroll
-          for (int b = 0; b < D; ++b) sv[b] = static_cast<double>(sS[a][hb * D + b]);
-          sv[D] = static_cast<double>(sOnes[a]);
+          for (int b = 0; b < D; ++b) sv[b] = sS[a][hb * D + b];
+          sv[D] = sOnes[a];
 #pragma unroll
-          for (int j = 0; j < D; ++j)
+          for (int x = 0; x < JT; ++x)
 #pragma unroll
-            for (int b = 0; b < P1; ++b) accL[j * P1 + b] = fma(hv[j], sv[b], accL[j * P1 + b]);
+            for (int b = 0; b < P1; ++b) acc[x][b] = fma(hv[x], sv[b], acc[x][b]);
         }
-        // R: columns tm, tm + kTeams, ... of the chunk
-        for (int c = tm; c < ncols; c += kTeams) {
-          const double hv = static_cast<double>(sH[i][c]);
-          accR = fma(hv, static_cast<double>(sTh[a][c]), accR);
-          accR = fma(hv, static_cast<double>(sTl[a][c]), accR);
+      }
+      if (ract)
+        for (int c = rp; c < ncols; c += F::kRParts) accR = fma(sH[ri][c], sT[ra][c], accR);
+    }
+  }
+  // teams in team order into the CTA partial, one L column (j, b) at a time
+  double* out = partials + int64_t(blockIdx.x) * F::kPart;
+#pragma unroll
+  for (int x = 0; x < JT; ++x)
+#pragma unroll
+    for (int b = 0; b < P1; ++b) {
+      // this thread's value is L[(i,a)][(j0 + x, b)]; threads with the same
+      // (i, a) but another j block hold other columns, so one pass per j block
+      for (int jb = 0; jb < D / JT; ++jb) {
+        __syncthreads();
+        if (lact && (ij % (D / JT)) == jb) sRed[tm][i * P1 + a] = acc[x][b];
+        __syncthreads();
+        if (tid < NP) {
+          double v = 0.0;
+          for (int t2 = 0; t2 < kTeams; ++t2) v += sRed[t2][tid];
+          out[tid * NP + (jb * JT + x) * P1 + b] = v;  // L[(i,a) = tid][(j,b)]
         }
       }
     }
-  }
-  // teams in team order into the CTA partial: one L row (i,a) at a time
-  double* out = partials + int64_t(blockIdx.x) * F::kPart;
-#pragma unroll
-  for (int q = 0; q < NP; ++q) {  // column (j, b) = q of every row
-    __syncthreads();
-    if (active) sRed[tm][me] = accL[q];
-    __syncthreads();
-    if (tid < NP) {
-      double v = 0.0;
-      for (int t = 0; t < kTeams; ++t) v += sRed[t][tid];
-      out[tid * NP + q] = v;  // L[(i,a) = tid][(j,b) = q]
-    }
-  }
   __syncthreads();
-  if (active) sRed[tm][me] = accR;
+  if (ract) sRed[rp][ro] = accR;
   __syncthreads();
   if (tid < NP) {
     double v = 0.0;
-    for (int t = 0; t < kTeams; ++t) v += sRed[t][tid];
+    for (int t2 = 0; t2 < F::kRParts; ++t2) v += sRed[t2][tid];
     out[NP * NP + tid] = v;
   }
 }
 
-// ---------------------------------------------------------------- 3b. solve
-// One CTA.  Sums the partials in CTA order (thread per value), then solves
-// L theta = R in shared memory.
+// ---------------------------------------------------------------- 3b. reduce, solve
+// The partials are summed in CTA order, one thread per value, 8 loads of a
+// thread in flight at a time (a fixed order: bitwise reproducible).
+template <int D>
+__global__ void __launch_bounds__(256) fith_reduce_kernel(const double* __restrict__ partials,
+                                                          int num_parts, double* __restrict__ red) {
+  using F = FitHDims<D>;
+  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  if (v >= F::kPart) return;
+  double acc = 0.0;
+  int c = 0;
+  for (; c + 8 <= num_parts; c += 8) {
+    double x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = __ldcg(partials + int64_t(c + u) * F::kPart + v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += x[u];
+  }
+  for (; c < num_parts; ++c) acc += __ldcg(partials + int64_t(c) * F::kPart + v);
+  red[v] = acc;
+}
+
+// One CTA: L theta = R in shared memory, from the reduced [L | R].
 constexpr int kSolveThreads = 256;
 
+// Cholesky G = L L^T in place (lower triangle) by the whole CTA, one column
+// at a time; then the two triangular solves by warp 0, column by column (lanes
+// take rows).  Returns false, for every thread, on a pivot below kHCholFloor
+// of the largest diagonal entry (G is then partly overwritten).  th (shared)
+// receives theta.
 template <int NP>
-__device__ bool chol_solve_par(double (*G)[NP], double* R, double* th, double* sdiag) {
-  // in place: lower factor in G; returns false on a pivot below the floor
-  const int t = threadIdx.x;
+__device__ bool chol_solve_cta(double (*G)[NP], const double* R, double* th) {
+  const int t = threadIdx.x, lane = t & 31;
   __shared__ int ok;
+  __shared__ double dmax;
   if (t == 0) {
-    double dmax = 0.0;
-    for (int c = 0; c < NP; ++c) dmax = fmax(dmax, G[c][c]);
-    *sdiag = dmax;
-    ok = dmax > 0.0;
+    double m = 0.0;
+    for (int c = 0; c < NP; ++c) m = fmax(m, G[c][c]);
+    dmax = m;
+    ok = m > 0.0;
   }
   __syncthreads();
   if (!ok) return false;
-  const double dmax = *sdiag;
   for (int c = 0; c < NP; ++c) {
     if (t == 0) {
       const double piv = G[c][c];
@@ -228,22 +297,27 @@ __device__ bool chol_solve_par(double (*G)[NP], double* R, double* th, double* s
     // trailing update of the lower triangle: G[r][s] -= L[r][c] L[s][c], c < s <= r
     const int m = NP - c - 1;
     for (int e = t; e < m * m; e += blockDim.x) {
-      const int r = c + 1 + e / m, s = c + 1 + e % m;
-      if (s <= r) G[r][s] -= G[r][c] * G[s][c];
+      const int r = c + 1 + e / m, s2 = c + 1 + e % m;
+      if (s2 <= r) G[r][s2] -= G[r][c] * G[s2][c];
     }
     __syncthreads();
   }
-  if (t == 0) {
-    double y[NP];
-    for (int r = 0; r < NP; ++r) {  // L y = R
-      double v = R[r];
-      for (int k = 0; k < r; ++k) v -= G[r][k] * y[k];
-      y[r] = v / G[r][r];
+  if (t < 32) {
+    for (int r = lane; r < NP; r += 32) th[r] = R[r];
+    __syncwarp();
+    for (int c = 0; c < NP; ++c) {  // L y = R, y in th
+      if (lane == 0) th[c] /= G[c][c];
+      __syncwarp();
+      const double yc = th[c];
+      for (int r = c + 1 + lane; r < NP; r += 32) th[r] -= G[r][c] * yc;
+      __syncwarp();
     }
-    for (int r = NP - 1; r >= 0; --r) {  // L^T theta = y
-      double v = y[r];
-      for (int k = r + 1; k < NP; ++k) v -= G[k][r] * th[k];
-      th[r] = v / G[r][r];
+    for (int c = NP - 1; c >= 0; --c) {  // L^T theta = y, in place
+      if (lane == 0) th[c] /= G[c][c];
+      __syncwarp();
+      const double tc = th[c];
+      for (int r = lane; r < c; r += 32) th[r] -= G[c][r] * tc;
+      __syncwarp();
     }
   }
   __syncthreads();
@@ -344,8 +418,8 @@ __device__ void jacobi_pinv_par(double (*G)[NP], double (*V)[NP], const double* 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kSolveThreads) fith_solve_kernel(const double* __restrict__ partials,
-                                                                   int num_parts, float* __restrict__ A,
+__global__ void __launch_bounds__(kSolveThreads) fith_solve_kernel(const double* __restrict__ red,
+                                                                   float* __restrict__ A,
                                                                    float* __restrict__ B) {
   using F = FitHDims<D>;
   constexpr int NP = F::NP;
@@ -355,36 +429,31 @@ __global__ void __launch_bounds__(kSolveThreads) fith_solve_kernel(const double*
   double (*V)[NP] = G0 + NP;
   double* R = reinterpret_cast<double*>(V + NP);
   double* th = R + NP;
-  double* sdiag = th + NP;
   const int t = threadIdx.x;
   for (int v = t; v < F::kPart; v += blockDim.x) {
-    double acc = 0.0;
-    for (int c = 0; c < num_parts; ++c) acc += partials[int64_t(c) * F::kPart + v];
+    const double acc = red[v];
     if (v < NP * NP) {
-      // symmetrize: the partials hold the full L; average mirrored entries in a
-      // fixed order so both triangles agree bit for bit
-      G[v / NP][v % NP] = acc;
+      G[v / NP][v % NP] = acc;  // L_half
     } else {
       R[v - NP * NP] = acc;
     }
   }
   __syncthreads();
+  // L = L_half + L_half^T (the contraction accumulated the pairs h >= g only)
   for (int e = t; e < NP * NP; e += blockDim.x) {
     const int r = e / NP, c = e % NP;
     if (r < c) {
-      const double s = 0.5 * (G[r][c] + G[c][r]);
+      const double s = G[r][c] + G[c][r];
       G0[r][c] = s;
       G0[c][r] = s;
     } else if (r == c) {
-      G0[r][r] = G[r][r];
+      G0[r][r] = 2.0 * G[r][r];
     }
   }
   __syncthreads();
   for (int e = t; e < NP * NP; e += blockDim.x) G[e / NP][e % NP] = G0[e / NP][e % NP];
   __syncthreads();
-  if (!chol_solve_par<NP>(G, R, th, sdiag)) {
-    jacobi_pinv_par<NP>(G0, V, R, th);
-  }
+  if (!chol_solve_cta<NP>(G, R, th)) jacobi_pinv_par<NP>(G0, V, R, th);
   if (t < D * D) A[t] = static_cast<float>(th[(t / D) * (D + 1) + (t % D)]);
   if (t < D) B[t] = static_cast<float>(th[t * (D + 1) + D]);
 }
@@ -413,6 +482,8 @@ cudaError_t launch_fith_t(const float* W0, const uint8_t* packed, int64_t d_out,
   float* C = reinterpret_cast<float*>(base + q_bytes);
   const size_t c_bytes = (size_t(kOnes + d_in) * ldq * 4 + 255) / 256 * 256;
   double* partials = reinterpret_cast<double*>(base + q_bytes + c_bytes);
+  const int grid = contract_grid(d_in / D);
+  double* red = partials + size_t(grid) * F::kPart;  // the reduced [L | R]
   {
     const int64_t items = d_out * (d_in / 8 + kOnes / 8);
     int64_t grid = ceil_div(items, kPrepThreads);
@@ -424,15 +495,18 @@ cudaError_t launch_fith_t(const float* W0, const uint8_t* packed, int64_t d_out,
   if (cudaError_t e = launch_tc_gram(Q, d_out, kOnes + d_in, ldq, C, err, s, launches);
       e != cudaSuccess)
     return e;
-  const int grid = contract_grid(d_in / D);
   fith_contract_kernel<D><<<grid, F::kThreads, 0, s>>>(H, C, d_in, partials);
+  ++*launches;
+  if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
+  fith_reduce_kernel<D><<<static_cast<unsigned>(ceil_div(F::kPart, 256)), 256, 0, s>>>(partials, grid,
+                                                                                     red);
   ++*launches;
   if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
   auto sk = fith_solve_kernel<D>;
   if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(sk), solve_smem<D>());
       e != cudaSuccess)
     return e;
-  sk<<<1, kSolveThreads, solve_smem<D>(), s>>>(partials, grid, A, B);
+  sk<<<1, kSolveThreads, solve_smem<D>(), s>>>(red, A, B);
   ++*launches;
   return cudaGetLastError();
 }
@@ -444,7 +518,7 @@ size_t fith_scratch_bytes(int64_t d_out, int64_t d_in, int d) {
   const size_t q_bytes = (size_t(d_out) * ldq * 2 + 255) / 256 * 256;
   const size_t c_bytes = (size_t(kOnes + d_in) * ldq * 4 + 255) / 256 * 256;
   const int np = d * (d + 1);
-  const size_t p_bytes = size_t(contract_grid(d_in / (d > 0 ? d : 1))) * size_t(np * np + np) * 8;
+  const size_t p_bytes = (size_t(contract_grid(d_in / (d > 0 ? d : 1))) + 1) * size_t(np * np + np) * 8;
   return q_bytes + c_bytes + p_bytes;
 }
 

@@ -15,12 +15,23 @@ constexpr int kNumSMsB200 = 148;
 // Workspace header: the first 256 bytes of every workspace.
 //   err   - first device-side error code (0 = none), set with atomicCAS
 //   site  - which wait gave up (a small integer naming the wait)
+//   wait_limit - bounded waits give up after this many clock cycles
+//           (0 = kDefaultWaitLimit); a caller may lower it
 struct WsHeader {
   unsigned int err;
   unsigned int site;
-  unsigned int pad[62];
+  long long wait_limit;
+  unsigned int pad[60];
 };
 constexpr size_t kWsHeaderBytes = 256;
+constexpr long long kDefaultWaitLimit = 1LL << 32;  // clock cycles (~2 s)
+
+// the wait limit of the workspace whose header err_word points to
+__device__ __forceinline__ long long wait_limit(const unsigned int* err_word) {
+  if (err_word == nullptr) return kDefaultWaitLimit;
+  const long long v = *reinterpret_cast<const volatile long long*>(err_word + 2);
+  return v > 0 ? v : kDefaultWaitLimit;
+}
 
 __device__ __forceinline__ void record_error(unsigned int* err_word, unsigned int code,
                                              unsigned int site) {

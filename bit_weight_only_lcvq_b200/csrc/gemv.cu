@@ -355,14 +355,14 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
 // chunk c into accumulator c mod 8 in the same unit and MMA order, and ends
 // with the split kernel's fixed-order sum over the 8 accumulators.
 //
-// Every wait is bounded (kWideWaitLimit clock cycles); a warp that gives up
-// records LCVQ_ERR_DEVICE_TIMEOUT in the group's error word and raises the
-// CTA's abort flag, and the others wind down.
+// Every wait is bounded (the workspace's wait limit, default ~2 s); a warp
+// that gives up records LCVQ_ERR_DEVICE_TIMEOUT in the group's error word and
+// raises the CTA's abort flag, the others wind down, and the producer waits
+// for the copies it issued before the CTA exits.
 constexpr int kWideConsumers = 8;
 constexpr int kWideThreads = (kWideConsumers + 1) * 32;
 constexpr int kWideRows = 16 * kWideConsumers;
 constexpr uint32_t kWideXPitch = 1040;    // 1024 X'' bytes per token + 16
-constexpr long long kWideWaitLimit = 1LL << 32;
 
 template <int kItems>
 struct GemvWideGroup {
@@ -411,18 +411,22 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
   __syncthreads();
 
   griddep_wait();  // X'' and corr written by the X-transforms are visible from here
+  const long long lim = wait_limit(grp.err);
+  // the abort flag as one decision per warp: the lanes of a warp go on to
+  // warp-wide instructions together
+  auto warp_abort = [&]() { return __shfl_sync(0xffffffffu, *abort_flag, 0) != 0; };
 
   if (warp == kWideConsumers) {
     // ------------------------------------------------------------ producer
-    int seq = 0, item = 0;
-    for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G) {
+    int seq = 0, item = 0, filled = 0;
+    for (int tile = static_cast<int>(blockIdx.x); tile < T && !warp_abort(); tile += G) {
       while (tile >= grp.item[item].tile_end) ++item;
       const GemvItem& it = grp.item[item];
       const int64_t row0 = int64_t(tile - tile_begin(item)) * kWideRows;
       const int nch = nchunks(it.K);
       for (int c = 0; c < nch; ++c, ++seq) {
         const int s = seq % kStages;
-        if (!sm100::mbar_wait(&empty[s], ((seq / kStages) & 1) ^ 1, kWideWaitLimit)) {
+        if (!__all_sync(0xffffffffu, sm100::mbar_wait(&empty[s], ((seq / kStages) & 1) ^ 1, lim))) {
           if (lane == 0) record_error(grp.err, LCVQ_ERR_DEVICE_TIMEOUT, 50);
           *abort_flag = 1;
           break;
@@ -440,15 +444,23 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
         if (lane < M)
           sm100::bulk_load(st + L::kCodeBytes + lane * kWideXPitch,
                            it.Xpp + int64_t(lane) * it.K + xk, xbytes, &full[s]);
+        ++filled;
       }
     }
     // drain: every stage filled above has been consumed, so its copies landed
-    for (int k = 0; k < kStages && !*abort_flag; ++k, ++seq) {
+    for (int k = 0; k < kStages && !warp_abort(); ++k, ++seq) {
       const int s = seq % kStages;
-      if (!sm100::mbar_wait(&empty[s], ((seq / kStages) & 1) ^ 1, kWideWaitLimit)) {
+      if (!__all_sync(0xffffffffu, sm100::mbar_wait(&empty[s], ((seq / kStages) & 1) ^ 1, lim))) {
         if (lane == 0) record_error(grp.err, LCVQ_ERR_DEVICE_TIMEOUT, 51);
         *abort_flag = 1;
       }
+    }
+    if (warp_abort() && lane == 0) {
+      // gave up: wait for the last kStages fills to land, so no copy writes
+      // shared memory after the CTA exits (the default limit: copies in flight
+      // finish in microseconds)
+      for (int n = filled - 1; n >= 0 && n >= filled - kStages; --n)
+        sm100::mbar_wait(&full[n % kStages], (n / kStages) & 1, kDefaultWaitLimit);
     }
     return;
   }
@@ -470,7 +482,7 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
     xoff[n] = static_cast<uint32_t>((n * 8 + g) * kWideXPitch + 64 * t);
   }
   int seq = 0, item = 0;
-  for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G) {
+  for (int tile = static_cast<int>(blockIdx.x); tile < T && !warp_abort(); tile += G) {
     while (tile >= grp.item[item].tile_end) ++item;
     const GemvItem& it = grp.item[item];
     const int K = it.K;
@@ -489,12 +501,8 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
       for (int v = 0; v < kWideConsumers; ++v) {  // chunk c0 + v -> accumulator v
         const int c = c0 + v;
         if (c >= nch) break;
-        if (*abort_flag) {
-          ok = false;
-          break;
-        }
         const int s = seq % kStages;
-        if (!sm100::mbar_wait(&full[s], (seq / kStages) & 1, kWideWaitLimit)) {
+        if (!__all_sync(0xffffffffu, sm100::mbar_wait(&full[s], (seq / kStages) & 1, lim))) {
           if (lane == 0) record_error(grp.err, LCVQ_ERR_DEVICE_TIMEOUT, 52);
           *abort_flag = 1;
           ok = false;

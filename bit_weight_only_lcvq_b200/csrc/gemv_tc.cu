@@ -23,9 +23,10 @@
 //
 // TMEM columns: kAStages A slots of 64 columns (a k-block: 128 bf16 per row),
 // then two 32-column D buffers (tile i's epilogue overlaps tile i+1's MMAs).
-// Every wait is bounded (kTcWaitLimit cycles); a role that gives up records
-// LCVQ_ERR_DEVICE_TIMEOUT in the group's error word, raises the CTA's abort
-// flag, and the others wind down; the MMA issuer drains its MMAs before the
+// Every wait is bounded (the workspace's wait limit, default ~2 s); a role
+// that gives up records LCVQ_ERR_DEVICE_TIMEOUT in the group's error word,
+// raises the CTA's abort flag, and the others wind down; the producers wait
+// for their copies in flight and the MMA issuer drains its MMAs before the
 // TMEM is released.
 #include <cudaTypedefs.h>
 
@@ -57,7 +58,6 @@ constexpr uint32_t kDCol0 = kAStages * 64;            // first D column
 constexpr int kDecPerQuarter = 4;   // decoder warps per TMEM lane quarter (= kSub)
 constexpr int kDecWarps = 4 * kDecPerQuarter;
 constexpr int kTcThreads = 32 * (3 + kDecWarps + 4);
-constexpr long long kTcWaitLimit = 1LL << 32;
 constexpr int kTcItems = 48;        // matrices per launch (2 tensor maps each)
 
 static_assert(kDCol0 + 2 * kTcTok <= kTmemCols, "TMEM budget");
@@ -140,6 +140,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const long long lim = wait_limit(grp.err);
+  // the abort flag as one decision per warp, for the roles whose lanes go on to
+  // warp-wide instructions together
+  auto warp_abort = [&]() { return __shfl_sync(0xffffffffu, *abort_flag, 0) != 0; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ code producer
@@ -152,7 +156,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
         const int nch = kblocks(item) / kSub;
         for (int ch = 0; ch < nch; ++ch, ++g) {  // g counts chunks here
           const int s = g % kCStages;
-          if (!mbar_wait(&cempty[s], ((g / kCStages) & 1) ^ 1, kTcWaitLimit)) {
+          if (!mbar_wait(&cempty[s], ((g / kCStages) & 1) ^ 1, lim)) {
             tc_fail(grp, abort_flag, 60);
             break;
           }
@@ -161,6 +165,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
                       row0);
         }
       }
+      if (*abort_flag)  // the copies in flight land before the CTA exits
+        for (int n = g - 1; n >= 0 && n >= g - kCStages; --n)
+          mbar_wait(&cfull[n % kCStages], (n / kCStages) & 1, kDefaultWaitLimit);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ X'' producer
@@ -172,7 +179,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
         const int nkb = kblocks(item);
         for (int kb = 0; kb < nkb; ++kb, ++g) {
           const int a = g % kAStages;
-          if (!mbar_wait(&aempty[a], ((g / kAStages) & 1) ^ 1, kTcWaitLimit)) {
+          if (!mbar_wait(&aempty[a], ((g / kAStages) & 1) ^ 1, lim)) {
             tc_fail(grp, abort_flag, 61);
             break;
           }
@@ -182,6 +189,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
                       kb * kTcKB + kTcKB / 2, 0);
         }
       }
+      if (*abort_flag)  // the copies in flight land before the CTA exits
+        for (int n = g - 1; n >= 0 && n >= g - kAStages; --n)
+          mbar_wait(&xfull[n % kAStages], (n / kAStages) & 1, kDefaultWaitLimit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -192,7 +202,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
       for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G, ++local) {
         while (tile >= grp.item[item].tile_end) ++item;
         const int buf = local & 1;
-        if (!mbar_wait(&tempty[buf], ((local >> 1) & 1) ^ 1, kTcWaitLimit)) {
+        if (!mbar_wait(&tempty[buf], ((local >> 1) & 1) ^ 1, lim)) {
           tc_fail(grp, abort_flag, 62);
           break;
         }
@@ -203,7 +213,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
         for (int kb = 0; kb < nkb; ++kb, ++g) {
           const int a = g % kAStages;
           const uint32_t par = (g / kAStages) & 1;
-          if (!mbar_wait(&afull[a], par, kTcWaitLimit) || !mbar_wait(&xfull[a], par, kTcWaitLimit)) {
+          if (!mbar_wait(&afull[a], par, lim) || !mbar_wait(&xfull[a], par, lim)) {
             tc_fail(grp, abort_flag, 63);
             ok = false;
             break;
@@ -225,7 +235,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
       }
       if (issued) {  // no MMA may still run when the TMEM is released
         mma_commit(drain);
-        if (!mbar_wait(drain, 0, kTcWaitLimit)) tc_fail(grp, abort_flag, 64);
+        // the default limit: TMEM may be released only after the running MMAs
+        if (!mbar_wait(drain, 0, kDefaultWaitLimit)) tc_fail(grp, abort_flag, 64);
       }
     }
   } else if (warp < 3 + kDecWarps) {
@@ -234,7 +245,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
     const int slot = (warp - 3) >> 2;       // k-blocks g with g % kDecPerQuarter == slot
     const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
     int g = 0, item = 0;
-    for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G) {
+    for (int tile = static_cast<int>(blockIdx.x); tile < T && !warp_abort(); tile += G) {
       while (tile >= grp.item[item].tile_end) ++item;
       const int nkb = kblocks(item);
       bool ok = true;
@@ -242,8 +253,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
         if (g % kDecPerQuarter != slot) continue;
         const int c = g / kSub;  // code chunk of this k-block (kDecPerQuarter == kSub)
         const int s = c % kCStages, a = g % kAStages;
-        if (!mbar_wait(&cfull[s], (c / kCStages) & 1, kTcWaitLimit) ||
-            !mbar_wait(&aempty[a], ((g / kAStages) & 1) ^ 1, kTcWaitLimit)) {
+        const bool landed = mbar_wait(&cfull[s], (c / kCStages) & 1, lim) &&
+                            mbar_wait(&aempty[a], ((g / kAStages) & 1) ^ 1, lim);
+        if (!__all_sync(0xffffffffu, landed)) {  // one outcome per warp
           tc_fail(grp, abort_flag, 65);
           ok = false;
           break;
@@ -280,11 +292,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
     const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
     const int M = grp.M;
     int item = 0, local = 0;
-    for (int tile = static_cast<int>(blockIdx.x); tile < T && !*abort_flag; tile += G, ++local) {
+    for (int tile = static_cast<int>(blockIdx.x); tile < T && !warp_abort(); tile += G, ++local) {
       while (tile >= grp.item[item].tile_end) ++item;
       const TcItem& it = grp.item[item];
       const int buf = local & 1;
-      if (!mbar_wait(&tfull[buf], (local >> 1) & 1, kTcWaitLimit)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (local >> 1) & 1, lim))) {
         tc_fail(grp, abort_flag, 66);
         break;
       }

@@ -51,6 +51,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe of the phase (no hardware suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Limits below this many clock cycles are polled with test_wait: try_wait may
+// suspend the thread in hardware for longer than such a limit.
+constexpr long long kShortWaitLimit = 1LL << 20;
+
 // Acquire at cluster scope: for barriers that the peer CTA arrives on.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -76,6 +94,13 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 // Waits for the phase of the given parity to complete; gives up after
 // `limit` clock cycles and returns false (the caller records the error).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {
+  if (limit < kShortWaitLimit) {
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity)) {
+      if (clock64() - t0 > limit) return false;
+    }
+    return true;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {

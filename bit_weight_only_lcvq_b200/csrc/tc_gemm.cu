@@ -59,7 +59,6 @@ constexpr int C_BYTES = 4096;         // packed codes of one stage
 // 2048 x 4096 -> 11008 decode form: 1, 2, 3 -> 724, 815, 857 TFLOP/s)
 constexpr int kPairPeerGroup = 3;
 constexpr int kTmemCols = 512;
-constexpr long long kWaitLimit = 1LL << 32;  // clock cycles (~2 s)
 
 enum Kind { kFwdAlg = 0, kFwdDec = 1, kDx = 2, kDw = 3, kGram = 4 };
 
@@ -301,18 +300,24 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const long long lim = wait_limit(p.err);
+  // the abort flag as one decision per warp (lane 0's read), for the roles whose
+  // lanes go on to warp-wide instructions together
+  auto warp_abort = [&]() { return __shfl_sync(0xffffffffu, *abort_flag, 0) != 0; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
+      int64_t issued = 0;
       for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
         int mt, nt;
         tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
         for (int64_t kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1, kWaitLimit)) { fail(p, abort_flag, 1); break; }
+          if (!mbar_wait(&empty[s], ph ^ 1, lim)) { fail(p, abort_flag, 1); break; }
           if (*abort_flag) break;
+          ++issued;
           mbar_arrive_expect_tx(&full[s], C::kStageTx);
           const int kx = static_cast<int>(kb);
           if constexpr (KIND == kFwdAlg || KIND == kFwdDec) {
@@ -331,6 +336,11 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
       }
+      if (*abort_flag) {  // no copy may land in shared memory after the CTA exits
+        // (the default limit: copies in flight finish in microseconds)
+        for (int64_t n = issued - 1; n >= 0 && n >= issued - STAGES; --n)
+          mbar_wait(&full[n % STAGES], static_cast<uint32_t>((n / STAGES) & 1), kDefaultWaitLimit);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -343,13 +353,13 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
       for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++local) {
         const int buf = static_cast<int>(local & 1);
         const uint32_t use = static_cast<uint32_t>(local >> 1);
-        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, kWaitLimit)) { fail(p, abort_flag, 2); break; }
+        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, lim)) { fail(p, abort_flag, 2); break; }
         tc_fence_after();
         const uint32_t dt = tmem + buf * BN;
         bool ok = true;
         for (int64_t kb = 0; kb < kblocks; ++kb) {
           uint64_t* ready = (DW > 0) ? &decd[s] : &full[s];
-          if (!mbar_wait(ready, ph, kWaitLimit)) { fail(p, abort_flag, 3); ok = false; break; }
+          if (!mbar_wait(ready, ph, lim)) { fail(p, abort_flag, 3); ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * A_BYTES);
           const uint32_t b0 = smem_u32(sB + s * B_BYTES);
@@ -370,7 +380,9 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
       }
       if (issued) {  // no MMA may still run when TMEM is released
         mma_commit(drain);
-        if (!mbar_wait(drain, 0, kWaitLimit)) fail(p, abort_flag, 4);
+        // the default limit: running MMAs finish in microseconds, and TMEM may
+        // be released only after them
+        if (!mbar_wait(drain, 0, kDefaultWaitLimit)) fail(p, abort_flag, 4);
       }
     }
   } else if (warp < 2 + DW) {
@@ -378,9 +390,12 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
     const int dt = threadIdx.x - 64;  // 0 .. 32*DW-1
     int s = 0;
     uint32_t ph = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
+    for (int64_t tile = blockIdx.x; tile < tiles && !warp_abort(); tile += gridDim.x) {
       for (int64_t kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&full[s], ph, kWaitLimit)) { fail(p, abort_flag, 5); break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, lim))) {  // one outcome per warp
+          fail(p, abort_flag, 5);
+          break;
+        }
         const uint8_t* cs = sC + s * C_BYTES;
         const uint32_t bs = smem_u32(sB + s * B_BYTES);
         if constexpr (KIND == kFwdAlg) {
@@ -466,12 +481,15 @@ __global__ void __launch_bounds__(Cfg<KIND, DW>::kThreads, 1)
       for (int i = 0; i < D; ++i) pb[i] = 0.f;
     }
     int64_t local = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++local) {
+    for (int64_t tile = blockIdx.x; tile < tiles && !warp_abort(); tile += gridDim.x, ++local) {
       int mt, nt;
-        tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
+      tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
       const int buf = static_cast<int>(local & 1);
       const uint32_t use = static_cast<uint32_t>(local >> 1);
-      if (!mbar_wait(&tfull[buf], use & 1, kWaitLimit)) { fail(p, abort_flag, 6); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1, lim))) {  // one outcome per warp
+        fail(p, abort_flag, 6);
+        break;
+      }
       tc_fence_after();
       const int64_t gm = int64_t(mt) * BM + row;  // D row
       const uint32_t tbase = tmem + buf * BN + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -600,20 +618,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
   cluster_sync();  // barriers of both CTAs initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const long long lim = wait_limit(p.err);
+  auto warp_abort = [&]() { return __shfl_sync(0xffffffffu, *abort_flag, 0) != 0; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
+      int64_t issued = 0;
       for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
         int mt, nt;
         tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
         const int row0 = mt * 2 * BM + static_cast<int>(rank) * BM;  // this CTA's A rows
         const int col0 = nt * BN + static_cast<int>(rank) * (BN / 2);  // this CTA's B rows
         for (int64_t kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1, kWaitLimit)) { fail(p, abort_flag, 11); break; }
+          if (!mbar_wait(&empty[s], ph ^ 1, lim)) { fail(p, abort_flag, 11); break; }
           if (*abort_flag) break;
+          ++issued;
           uint8_t* st = smem + size_t(s) * C::kStage;
           const uint32_t fa0 = mapa_shared(smem_u32(&fullA[s]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&fullA[s], 2 * C::kOperandTx);
@@ -635,6 +657,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
           if (++s == S) { s = 0; ph ^= 1; }
         }
       }
+      if (*abort_flag) {
+        // wait for this CTA's own copies in flight (codes, on its own barrier);
+        // the even CTA also waits for the operand stages, which count both
+        // CTAs' bytes.  The default limit: copies in flight finish quickly.
+        for (int64_t n = issued - 1; n >= 0 && n >= issued - S; --n) {
+          const uint32_t par = static_cast<uint32_t>((n / S) & 1);
+          if (C::kHasCodes) mbar_wait(&fullC[n % S], par, kDefaultWaitLimit);
+          if (rank == 0) mbar_wait(&fullA[n % S], par, kDefaultWaitLimit);
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
@@ -648,19 +680,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
         const int buf = static_cast<int>(local & 1);
         const uint32_t use = static_cast<uint32_t>(local >> 1);
         // the odd CTA's epilogue arrives from the other SM: acquire at cluster scope
-        if (!mbar_wait_cluster(&tempty[buf], (use & 1) ^ 1, kWaitLimit)) { fail(p, abort_flag, 12); break; }
+        if (!mbar_wait_cluster(&tempty[buf], (use & 1) ^ 1, lim)) { fail(p, abort_flag, 12); break; }
         tc_fence_after();
         const uint32_t dt = tmem + buf * BN;
         bool ok = true;
         for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
-          if (!mbar_wait(&fullA[s], ph, kWaitLimit)) { fail(p, abort_flag, 13); ok = false; break; }
+          if (!mbar_wait(&fullA[s], ph, lim)) { fail(p, abort_flag, 13); ok = false; break; }
           if constexpr (C::kHasCodes) {
-            if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 14); ok = false; break; }
+            if (!mbar_wait(&decd[s], ph, lim)) { fail(p, abort_flag, 14); ok = false; break; }
             // the odd CTA's half of B: one cluster-scope wait per group of k blocks
             const int64_t q = it / kPeerGroup;
             if (it % kPeerGroup == 0 &&
                 !mbar_wait_cluster(&decd_peer[q % S], static_cast<uint32_t>((q / S) & 1),
-                                   kWaitLimit)) {
+                                   lim)) {
               fail(p, abort_flag, 18);
               ok = false;
               break;
@@ -686,7 +718,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       }
       if (issued) {
         mma_commit_pair(drain);
-        if (!mbar_wait(drain, 0, kWaitLimit)) fail(p, abort_flag, 15);
+        // the default limit: TMEM may be released only after the running MMAs
+        if (!mbar_wait(drain, 0, kDefaultWaitLimit)) fail(p, abort_flag, 15);
       }
     } else if (rank == 1 && lane == 0 && C::kHasCodes) {
       // odd CTA: forward "B half decoded" to the even CTA, one cluster-scope
@@ -700,7 +733,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
         const bool last_tile = tile + npairs >= tiles;
         for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
-          if (!mbar_wait(&decd[s], ph, kWaitLimit)) { fail(p, abort_flag, 19); break; }
+          if (!mbar_wait(&decd[s], ph, lim)) { fail(p, abort_flag, 19); break; }
           if (it % kPeerGroup == kPeerGroup - 1 || (last_tile && kb + 1 == kblocks))
             mbar_arrive_cluster(mapa_shared(smem_u32(&decd_peer[(it / kPeerGroup) % S]), 0));
           if (++s == S) { s = 0; ph ^= 1; }
@@ -723,13 +756,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
     int s = 0;
     uint32_t ph = 0;
     int64_t it = 0;
-    for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs) {
+    for (int64_t tile = pair; tile < tiles && !warp_abort(); tile += npairs) {
       for (int64_t kb = 0; kb < kblocks; ++kb, ++it) {
         if (it % kGroups != grp) {
           if (++s == S) { s = 0; ph ^= 1; }
           continue;
         }
-        if (!mbar_wait(&fullC[s], ph, kWaitLimit)) { fail(p, abort_flag, 16); break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&fullC[s], ph, lim))) {  // one outcome per warp
+          fail(p, abort_flag, 16);
+          break;
+        }
         uint8_t* st = smem + size_t(s) * C::kStage;
         const uint8_t* cs = st + C::kA + C::kB;
         const uint32_t bs = smem_u32(st + C::kA);
@@ -825,12 +861,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<KIND, DW>::kThr
       for (int i = 0; i < D; ++i) pb[i] = 0.f;
     }
     int64_t local = 0;
-    for (int64_t tile = pair; tile < tiles && !*abort_flag; tile += npairs, ++local) {
+    for (int64_t tile = pair; tile < tiles && !warp_abort(); tile += npairs, ++local) {
       int mt, nt;
       tile_coords(tile, m_tiles, n_tiles, kBand, mt, nt);
       const int buf = static_cast<int>(local & 1);
       const uint32_t use = static_cast<uint32_t>(local >> 1);
-      if (!mbar_wait(&tfull[buf], use & 1, kWaitLimit)) { fail(p, abort_flag, 17); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1, lim))) {  // one outcome per warp
+        fail(p, abort_flag, 17);
+        break;
+      }
       tc_fence_after();
       const int64_t gm = int64_t(mt) * 2 * BM + int64_t(rank) * BM + row;
       const uint32_t tbase = tmem + buf * BN + (static_cast<uint32_t>(quarter * 32) << 16);

@@ -259,6 +259,12 @@ def gemv_static(X: torch.Tensor, packed: torch.Tensor, d_in: int, A: torch.Tenso
     return out
 
 
+def set_wait_limit(workspace: torch.Tensor, cycles: int) -> None:
+    """Writes the workspace header's wait limit (bytes 8..15, int64 clock
+    cycles; 0 = the library's default).  Ordered on the current stream."""
+    workspace[8:16].view(torch.int64).fill_(int(cycles))
+
+
 def check_device_error(workspace: torch.Tensor, stream=None) -> int:
     """Synchronizes the stream and returns the workspace's device error status."""
     return int(lib().lcvq_check_device_error(_ptr(workspace), _stream(stream)))

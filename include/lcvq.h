@@ -39,8 +39,19 @@
  * Errors: arguments are validated before anything is launched; a failing call
  * launches nothing and returns a status.  Launch failures return
  * LCVQ_ERR_CUDA.  Kernels that wait on mbarriers give up after a bounded number
- * of polls and record LCVQ_ERR_DEVICE_TIMEOUT in the workspace's error word,
- * read by lcvq_check_device_error().  Nothing aborts, throws or traps.
+ * of clock cycles and record LCVQ_ERR_DEVICE_TIMEOUT in the workspace's error
+ * word, read by lcvq_check_device_error(); the other roles of the kernel then
+ * wind down, copies in flight land and tensor-core work drains before the
+ * kernel exits, so the next call on the workspace runs normally.  Nothing
+ * aborts, throws or traps.
+ *
+ * Workspace header (its first 256 bytes, zeroed once by the caller):
+ *   bytes 0..3   error word (0, or the first LCVQ_ERR_DEVICE_TIMEOUT)
+ *   bytes 4..7   which wait gave up (a small integer naming the wait)
+ *   bytes 8..15  int64 wait limit in clock cycles of the tensor-core GEMMs and
+ *                the grouped decode-GEMV kernels; 0 (the default) means 2^32
+ *                (about 2 s).  A caller may lower it, e.g. to test its own
+ *                handling of LCVQ_ERR_DEVICE_TIMEOUT.
  *
  * Requirements: a compute capability 10.0 device (sm_100a); otherwise
  * LCVQ_ERR_UNSUPPORTED.  Pointers 16-byte aligned (LCVQ_ERR_ALIGNMENT).
@@ -313,9 +324,9 @@ LCVQ_API lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int
  *   d_in, d) bytes (about 2 d_out d_in * 3 + 12 d_in^2 bytes of scratch),
  *   256-byte aligned, first 256 bytes zeroed once.
  * Shapes: d_in % 64 == 0, d_in <= 65536, d_out <= 2^20; an empty matrix gives
- * A = 0, B = 0.  Launches 4 kernels: the bf16 operand pass, one tcgen05 GEMM
- * of 2 (d_in + 64)(3 d_in + 64) d_out flops, the fp64 contraction with H and
- * the solve. */
+ * A = 0, B = 0.  Launches 5 kernels: the bf16 operand pass, one tcgen05 GEMM
+ * of 2 (d_in + 64)(3 d_in + 64) d_out flops, the fp64 contraction with H, the
+ * fixed-order sum of its partials and the solve. */
 LCVQ_API lcvq_status lcvq_fit_affine_h(const float* W0, const uint8_t* packed, int64_t d_out,
                                        int64_t d_in, int d, const float* H, float* A, float* B,
                                        void* workspace, size_t ws_bytes, void* stream);

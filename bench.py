@@ -472,6 +472,8 @@ def headline(args, D: Dist, pk):
                                             for M in Ms]),
                       traffic_unit="bytes per step (3 launches)",
                       kernel="gemv_group_kernel (decode-GEMV, M=1,4,16 summed)",
+                      launch="lcvq_gemm_xformed back to back; launched on its own, each GEMV "
+                             "waits for the previous launch before it loads codes",
                       per_m_us={str(M): per_m[M] * 1e3 for M in Ms},
                       peak_source=f"{PEAK_SRC} hbm_gbs"),
         e2e=e2e, clocks=ck, gpu_launches=int(launches),

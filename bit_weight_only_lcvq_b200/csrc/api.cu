@@ -300,7 +300,7 @@ lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t*
     e = launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr, s, &launches);
     if (e == cudaSuccess)
       e = launch_gemm_xformed(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), err,
-                              s, &launches);
+                              true, s, &launches);
   } else if (dtype == LCVQ_BF16) {  // decode form on the tensor cores
     e = launch_tc_forward(static_cast<const uint16_t*>(X), false, nullptr, M, packed, d_out, d_in,
                           d, A, B, static_cast<uint16_t*>(Y), err, s, &launches);
@@ -413,8 +413,9 @@ lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64_t M,
     return LCVQ_ERR_ALIGNMENT;
   if (lcvq_status st = check_device(); st != LCVQ_OK) return st;
   int launches = 0;
+  // launched on its own: whatever ran before may have written the codes
   cudaError_t e = launch_gemm_xformed(static_cast<const uint16_t*>(Xpp), corr, M, packed, d_out,
-                                      d_in, static_cast<uint16_t*>(Y), nullptr,
+                                      d_in, static_cast<uint16_t*>(Y), nullptr, false,
                                       static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches);
 }

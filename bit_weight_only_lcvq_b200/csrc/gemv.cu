@@ -16,11 +16,13 @@
 //   * K is cut into chunks of 512 codes; warp w of 8 sums chunks w, w + 8, ...
 //     and the 8 partial sums are added in warp order, so every path gives the
 //     same bits for a matrix;
-//   * programmatic dependent launch: the code loads do not depend on the
-//     X-transform, so they are issued before griddepcontrol.wait and stream
-//     while the prologue runs.  The kernels touch nothing else before the
-//     wait, and the X-transform waits for every earlier kernel before it lets
-//     them launch, so the early reads never race a producer of the codes.
+//   * programmatic dependent launch: launched right after the X-transform of
+//     the same call (early_codes), the split-K kernel issues its code loads
+//     before griddepcontrol.wait, so they stream while the transform runs.
+//     The X-transform lets it launch only after its own wait has returned, so
+//     every kernel that could have written the codes has completed; it touches
+//     nothing else before the wait.  Launched on its own (lcvq_gemm_xformed)
+//     it waits first.
 // gemv_group_kernel (split K, cp.async code rings) serves single matrices and
 // small groups; gemv_wide_kernel (128-row tiles, TMA producer warp) serves
 // large groups; gemv_tc.cu holds the tcgen05 form for 17..32 tokens.
@@ -64,6 +66,7 @@ struct GemvItem {
 template <int kItems>
 struct GemvGroup {
   int count, M;
+  int early_codes;  // launched right after this call's X-transform: codes may load before the wait
   GemvItem item[kItems];
 };
 
@@ -73,18 +76,6 @@ struct GemvGroup {
 // (row & 7) so that the lanes' 8-byte reads of one unit spread over the banks.
 // Copies in flight hold no registers, so every SM keeps kStages - 1 chunks per
 // warp on the way from HBM.
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
 template <int R, int kStages, int kWarps>
 __host__ __device__ constexpr size_t group_smem_ring() {
   return size_t(kWarps) * kStages * (16 * R) * 128;
@@ -199,8 +190,9 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
   for (int j = 0; j < kAhead; ++j)
     coff[j] = static_cast<uint32_t>((((2 * j + (t >> 1)) ^ g) << 4) + ((t & 1) << 3));
 
-  // prologue: the first kStages - 1 chunks (codes only: nothing here depends
-  // on the kernels this one may overlap)
+  // prologue: the first kStages - 1 chunks (codes only), before the wait
+  // when the X-transform of this call precedes the kernel
+  if (!grp.early_codes) griddep_wait();
   Cur cur = seek(Cur{static_cast<int>(blockIdx.x), 0, warp});
   Cur iss = cur;
 #pragma unroll
@@ -210,7 +202,7 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
   }
   Cur nxt = advance(cur);
 
-  griddep_wait();  // X'' and corr written by the X-transform are visible from here
+  if (grp.early_codes) griddep_wait();  // X'' and corr of the X-transform are visible from here
 
   XPos pcur = xpos(cur), pnxt = xpos(nxt);
   uint4 xcur[2][NT][2], xnxt[2][NT][2];
@@ -661,12 +653,13 @@ cudaError_t launch_group(const GemvGroup<kItems>& grp, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
-                        int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s,
-                        int* launches) {
+                        int64_t d_out, int64_t d_in, uint16_t* Y, bool after_xform,
+                        cudaStream_t s, int* launches) {
   // a single matrix is a group of one (the same kernel, so the same bits)
   GemvGroup<1> grp{};
   grp.count = 1;
   grp.M = static_cast<int>(M);
+  grp.early_codes = after_xform ? 1 : 0;
   grp.item[0] = GemvItem{packed, Xpp, corr, Y, static_cast<int>(d_out), static_cast<int>(d_in),
                          static_cast<int>(ceil_div(d_out, group_rows(M)))};
   cudaError_t e = launch_group(grp, s);
@@ -745,6 +738,7 @@ cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaS
     GemvGroup<kMaxGroupItems> grp{};
     grp.count = n;
     grp.M = static_cast<int>(M);
+    grp.early_codes = 1;  // after launch_xform_grouped
     int tiles = 0;
     for (int i = 0; i < n; ++i) {
       const GemvJob& j = jobs[first + i];
@@ -762,8 +756,9 @@ cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaS
 
 cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,
                                 const uint8_t* packed, int64_t d_out, int64_t d_in, uint16_t* Y,
-                                unsigned int* err, cudaStream_t s, int* launches) {
-  if (M <= 32) return launch_gemv(Xpp, corr, M, packed, d_out, d_in, Y, s, launches);
+                                unsigned int* err, bool after_xform, cudaStream_t s,
+                                int* launches) {
+  if (M <= 32) return launch_gemv(Xpp, corr, M, packed, d_out, d_in, Y, after_xform, s, launches);
   return launch_tc_forward(Xpp, true, corr, M, packed, d_out, d_in, 8, nullptr, nullptr, Y, err, s,
                            launches);
 }

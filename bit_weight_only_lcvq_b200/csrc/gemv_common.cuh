@@ -1,7 +1,7 @@
-// Helpers of the decode-GEMV kernels (gemv.cu, gemv_fused.cu, gemv_tc.cu):
+// Helpers of the decode-GEMV kernels (gemv.cu, gemv_tc.cu):
 // the legacy tensor-core MMA they use for few tokens, shared-memory vector
-// loads, programmatic dependent launch controls, and the K chunking of the
-// code stream.
+// loads, cp.async copies, programmatic dependent launch controls, and the K
+// chunking of the code stream.
 #pragma once
 
 #include <stdint.h>
@@ -45,6 +45,21 @@ __device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
+}
+
+// 16-byte global -> shared copy through L2 only (zero-filled when !valid),
+// and its commit / wait groups
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
 }  // namespace lcvq

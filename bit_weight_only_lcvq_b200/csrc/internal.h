@@ -37,8 +37,11 @@ cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, cons
                          int* launches);
 
 // ---- decode-GEMV (bf16, M <= 32) ----
+// after_xform: launched right after launch_xform of the same call on the same
+// stream, so the codes may be read before the kernel's dependency wait
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
-                        int64_t d_out, int64_t d_in, uint16_t* Y, cudaStream_t s, int* launches);
+                        int64_t d_out, int64_t d_in, uint16_t* Y, bool after_xform,
+                        cudaStream_t s, int* launches);
 
 constexpr int kMaxGroupItems = 128;
 
@@ -78,10 +81,12 @@ cudaError_t launch_gemv_tc_grouped(const GemvJob* jobs, int count, int64_t M, un
                                    cudaStream_t s, int* launches);
 
 // integer-code GEMM on X'' (dispatches on M: decode-GEMV for M <= 32, else
-// the tcgen05 GEMM); err may be null (no device error word)
+// the tcgen05 GEMM); err may be null (no device error word); after_xform as
+// for launch_gemv
 cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t M,
                                 const uint8_t* packed, int64_t d_out, int64_t d_in, uint16_t* Y,
-                                unsigned int* err, cudaStream_t s, int* launches);
+                                unsigned int* err, bool after_xform, cudaStream_t s,
+                                int* launches);
 
 // 2D TMA tensor map: `inner` contiguous elements per row, `outer` rows of
 // `row_bytes`; box box_inner x box_outer; 128-byte swizzle or none; zero fill

@@ -87,7 +87,7 @@ extern "C" lcvq_status lcvq_gemv_static(const void* X, int64_t M, const uint8_t*
   cudaError_t e = lcvq::launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr,
                                      s, &launches);
   if (e == cudaSuccess)
-    e = lcvq::launch_gemv(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), s,
+    e = lcvq::launch_gemv(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), true, s,
                           &launches);
   if (e != cudaSuccess) return LCVQ_ERR_CUDA;
   lcvq::set_last_launches(launches);

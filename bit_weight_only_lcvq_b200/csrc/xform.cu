@@ -60,35 +60,47 @@ __global__ void __launch_bounds__(kXfThreads)
   __shared__ float sA[D * D];
   __shared__ float sBp[D];
   __shared__ double red[3][kXfThreads / 32];
-  // Programmatic dependent launch.  The decode-GEMV that follows may launch at
-  // once: before its own wait it only reads packed codes, and the only kernels
-  // that can still be running at that point are this one (waiting below) and
-  // the previous decode-GEMV in its epilogue, neither of which writes codes
-  // (every earlier kernel finished before the previous GEMV passed its wait).
-  // This kernel itself waits for every earlier kernel before it touches
-  // anything (X may be the previous layer's output).
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // Programmatic dependent launch.  This kernel waits for every earlier kernel
+  // before it touches anything (X may be the previous layer's output), and only
+  // then lets the decode-GEMV that follows launch: that GEMV reads packed codes
+  // before its own wait, which is safe because every kernel that could have
+  // written them has completed by the time this wait returns, and this kernel
+  // writes none.
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  if (threadIdx.x < D * D) sA[threadIdx.x] = A[threadIdx.x];
-  if (threadIdx.x < D)
-    sBp[threadIdx.x] = shifted_offset<D>(A + threadIdx.x * D, B[threadIdx.x]);
-  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   const int64_t m = blockIdx.x;
   const uint16_t* xr = X + m * d_in;
   uint16_t* orow = Xpp + m * d_in;
   // warp w takes the chunks c = w, w + 8, ... (the classes of the corr sum);
-  // lane l transforms block l of the chunk
+  // lane l transforms block l of the chunk.  The first chunk's activations
+  // are loaded together with A and B.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  double s_b = 0.0, s_xr = 0.0, s_xpp = 0.0;  // this class's running sums (lane 0)
   const int64_t nblk = d_in / 16;
   const int64_t nchunk = ceil_div(d_in, kCorrChunk);
+  uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+  {
+    const int64_t b = int64_t(warp) * (kCorrChunk / 16) + lane;
+    if (warp < nchunk && b < nblk) {
+      p0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
+      p1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
+    }
+  }
+  if (threadIdx.x < D * D) sA[threadIdx.x] = A[threadIdx.x];
+  if (threadIdx.x < D)
+    sBp[threadIdx.x] = shifted_offset<D>(A + threadIdx.x * D, B[threadIdx.x]);
+  __syncthreads();
+
+  double s_b = 0.0, s_xr = 0.0, s_xpp = 0.0;  // this class's running sums (lane 0)
   for (int64_t c = warp; c < nchunk; c += kCorrClasses) {
     const int64_t b = c * (kCorrChunk / 16) + lane;
     float sb = 0.f, sxr = 0.f, sxpp = 0.f;
     if (b < nblk) {
-      const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
-      const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
+      uint4 u0 = p0, u1 = p1;
+      if (c != warp) {
+        u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
+        u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
+      }
       uint32_t o[8];
       xform_block<D>(u0, u1, sA, sBp, o, sb, sxr, sxpp);
       uint4* dst = reinterpret_cast<uint4*>(orow + 16 * b);

@@ -1,6 +1,5 @@
-// The X-transform of one 16-element block of activations, shared by the
-// X-transform kernel (xform.cu) and the single-launch decode-GEMV
-// (gemv_fused.cu), so that both produce the same bits.  See xform.cu for the
+// The X-transform of one 16-element block of activations (xform.cu), and the
+// fixed order of the corr sum.  See xform.cu for the
 // algebra (the algebraic form of the forward, LC-QAT technical summary,
 // Methodology 3) and the decoder order of X''.
 //

@@ -34,7 +34,11 @@
  * device memory and never synchronizes the stream on the hot path; scratch goes
  * in a caller-provided workspace sized by lcvq_workspace_size().  All calls are
  * asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the legacy
- * default stream).  Outputs are overwritten, never accumulated into.
+ * default stream).  Outputs are overwritten, never accumulated into.  The
+ * decode-GEMV kernels are launched with programmatic dependent launch: a
+ * call's first kernel may become resident while earlier work on the stream
+ * finishes, but it reads no input before that work has completed, so inputs
+ * produced by any earlier kernel or copy on the stream are always seen.
  *
  * Errors: arguments are validated before anything is launched; a failing call
  * launches nothing and returns a status.  Launch failures return

@@ -662,6 +662,71 @@ def test_xform_then_gemm_xformed_equals_gemm(M, d_in, d_out):
     assert_close(f"gemm_xformed M={M}", to_np(Y2), ref, D, TOL_BF16)
 
 
+# ------------------------------ the decode-GEMV against the split calls, over K and d_out shapes
+@pytest.mark.parametrize("M,d_in,d_out,d", [
+    (1, 64, 64, 8),         # one chunk of K (seven empty chunk classes), fewer tiles than CTAs
+    (1, 4672, 16400, 8),    # ten chunks: classes of one and two; more tiles than the grid
+    (8, 14336, 1032, 4),    # 28 chunks, ragged last tile
+    (9, 4096, 264, 2),      # first count of the 32-row tile shape
+    (16, 8256, 520, 1),     # 17 chunks, a 64-position tail
+    (17, 1088, 4104, 8),    # first count of the four-token-tile shape
+    (32, 4096, 1032, 8),
+    (32, 28672, 64, 8),     # 56 chunks, seven per class
+])
+def test_gemm_decode_gemv_equals_split_calls(M, d_in, d_out, d):
+    """lcvq_gemm for M <= 32 (X-transform, then the decode-GEMV reading codes
+    before its dependency wait) gives the bits of lcvq_xform followed by
+    lcvq_gemm_xformed (which waits first), meets the oracle, and writes nothing
+    outside Y."""
+    w, z = _fwd_case(2, M, d_in=d_in, d_out=d_out, d=d)
+    packed = torch.from_numpy(O.pack_codes(z)).to(dev())
+    X = to_dev(w["X"], torch.bfloat16)
+    A, B = torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev())
+    Y1, ybuf = guarded((M, d_out), torch.bfloat16)
+    lcvq.gemm(X, packed, d_in, A, B, d, out=Y1)
+    n1 = lcvq.last_launch_count()
+    xpp, corr = lcvq.xform(X, A, B, d)
+    Y2 = lcvq.gemm_xformed(xpp, corr, packed)
+    torch.cuda.synchronize()
+    assert n1 == 2
+    assert guard_intact(Y1, ybuf)
+    assert torch.equal(Y1, Y2)
+    ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close(f"decode-GEMV M={M} K={d_in}", to_np(Y1), ref, D, TOL_BF16)
+
+
+def test_gemm_decode_gemv_graph_replay():
+    """Back-to-back lcvq_gemm calls with programmatic dependent launch (each
+    X-transform waits for the previous call's GEMV, each GEMV streams its codes
+    during its X-transform), captured in a CUDA graph on one workspace: every
+    replay gives the eager bits."""
+    M, K, N = 4, 4096, 4096
+    cases = []
+    for i in range(3):
+        w, z = _fwd_case(2, M, d_in=K, d_out=N)
+        X = to_dev(w["X"] * (1.0 + i), torch.bfloat16)
+        cases.append((X, torch.from_numpy(O.pack_codes(z)).to(dev()),
+                      torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev())))
+    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, 8), dev())
+    eager = [lcvq.gemm(X, p, K, A, B, 8, workspace=ws) for X, p, A, B in cases]
+    outs = [torch.empty_like(e) for e in eager]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for (X, p, A, B), Y in zip(cases, outs):
+            lcvq.gemm(X, p, K, A, B, 8, out=Y, workspace=ws)
+    for _ in range(2):
+        for Y in outs:
+            Y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for Y, e in zip(outs, eager):
+            assert torch.equal(Y, e)
+    del g
+
+
 def test_gemm_grouped_outputs_are_canaried():
     """Every Y_i of a grouped call (split and wide-tile kernels) stays inside
     its own buffer."""

@@ -61,4 +61,25 @@ __device__ __forceinline__ uint32_t in_mask(float w) { return (w >= 0.0f) & (w <
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// ---- loads of data that an earlier kernel on the stream may have written ----
+// Kernels launched with programmatic dependent launch can become resident
+// before their producer has written, so such data is not constant over the
+// kernel's lifetime and may not be read through the read-only path
+// (ld.global.nc: __ldg, or what the compiler makes of const __restrict__
+// pointers), which can return a line that an earlier kernel left in this SM's
+// L1.  Ordinary global loads issued after griddepcontrol.wait see the
+// producer's writes.  These are volatile so that they stay after that wait.
+__device__ __forceinline__ uint4 ld_global_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float ld_global_f32(const float* p) {
+  float v;
+  asm volatile("ld.global.f32 %0, [%1];\n" : "=f"(v) : "l"(p));
+  return v;
+}
+
 }  // namespace lcvq

@@ -176,8 +176,8 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
       for (int n = 0; n < NT; ++n) {
         if (kok && tokok[n]) {
           const uint4* src = reinterpret_cast<const uint4*>(p.base[n] + j * kUnit + 16 * q);
-          xb[q][n][0] = __ldg(src);
-          xb[q][n][1] = __ldg(src + 1);
+          xb[q][n][0] = ld_global_v4(src);  // written by the X-transform: not the read-only path
+          xb[q][n][1] = ld_global_v4(src + 1);
         } else {
           xb[q][n][0] = make_uint4(0, 0, 0, 0);
           xb[q][n][1] = make_uint4(0, 0, 0, 0);
@@ -323,7 +323,8 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
       float sum = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) sum += part[buf][w][lr][tok];
-      if (grow < it.N) it.Y[int64_t(tok) * it.N + grow] = f32_to_bf16(sum + it.corr[tok]);
+      if (grow < it.N)
+        it.Y[int64_t(tok) * it.N + grow] = f32_to_bf16(sum + ld_global_f32(it.corr + tok));
     }
   }
   cp_async_wait<0>();  // no copy may outlive the CTA (only empty groups remain)
@@ -568,7 +569,8 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
         float sum = 0.f;
 #pragma unroll
         for (int v = 0; v < kWideConsumers; ++v) sum += acc[v][n][e];
-        if (row < it.N && tok < M) it.Y[int64_t(tok) * it.N + row] = f32_to_bf16(sum + it.corr[tok]);
+        if (row < it.N && tok < M)
+          it.Y[int64_t(tok) * it.N + row] = f32_to_bf16(sum + ld_global_f32(it.corr + tok));
       }
   }
   // the last CTA-wide point: consumers are done with every stage

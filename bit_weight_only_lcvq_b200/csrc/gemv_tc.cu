@@ -312,7 +312,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
 #pragma unroll
         for (int tok = 0; tok < kTcTok; ++tok)
           if (tok < M)
-            it.Y[int64_t(tok) * it.N + row] = f32_to_bf16(__uint_as_float(r[tok]) + it.corr[tok]);
+            it.Y[int64_t(tok) * it.N + row] =
+                f32_to_bf16(__uint_as_float(r[tok]) + ld_global_f32(it.corr + tok));
       }
     }
     if (threadIdx.x == 32 * (3 + kDecWarps)) griddep_launch_dependents();

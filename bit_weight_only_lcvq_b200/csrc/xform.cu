@@ -51,13 +51,16 @@ template <int D, int kItems>
 __global__ void __launch_bounds__(kXfThreads)
     xform_kernel(const __grid_constant__ XformGroup<kItems> grp) {
   const XformItem& it = grp.item[blockIdx.y];
-  const uint16_t* __restrict__ X = it.X;
-  const float* __restrict__ A = it.A;
-  const float* __restrict__ B = it.B;
+  // X, A and B may come from the kernel just before this one: read them with
+  // ld_global_*, never through the read-only path
+  const uint16_t* X = it.X;
+  const float* A = it.A;
+  const float* B = it.B;
   uint16_t* __restrict__ Xpp = it.Xpp;
   float* __restrict__ corr = it.corr;
   const int64_t d_in = it.d_in;
   __shared__ float sA[D * D];
+  __shared__ float sB[D];
   __shared__ float sBp[D];
   __shared__ double red[3][kXfThreads / 32];
   // Programmatic dependent launch.  This kernel waits for every earlier kernel
@@ -82,13 +85,14 @@ __global__ void __launch_bounds__(kXfThreads)
   {
     const int64_t b = int64_t(warp) * (kCorrChunk / 16) + lane;
     if (warp < nchunk && b < nblk) {
-      p0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
-      p1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
+      p0 = ld_global_v4(xr + 16 * b);
+      p1 = ld_global_v4(xr + 16 * b + 8);
     }
   }
-  if (threadIdx.x < D * D) sA[threadIdx.x] = A[threadIdx.x];
-  if (threadIdx.x < D)
-    sBp[threadIdx.x] = shifted_offset<D>(A + threadIdx.x * D, B[threadIdx.x]);
+  if (threadIdx.x < D * D) sA[threadIdx.x] = ld_global_f32(A + threadIdx.x);
+  if (threadIdx.x < D) sB[threadIdx.x] = ld_global_f32(B + threadIdx.x);
+  __syncthreads();
+  if (threadIdx.x < D) sBp[threadIdx.x] = shifted_offset<D>(sA + threadIdx.x * D, sB[threadIdx.x]);
   __syncthreads();
 
   double s_b = 0.0, s_xr = 0.0, s_xpp = 0.0;  // this class's running sums (lane 0)
@@ -98,8 +102,8 @@ __global__ void __launch_bounds__(kXfThreads)
     if (b < nblk) {
       uint4 u0 = p0, u1 = p1;
       if (c != warp) {
-        u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
-        u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b) + 1);
+        u0 = ld_global_v4(xr + 16 * b);
+        u1 = ld_global_v4(xr + 16 * b + 8);
       }
       uint32_t o[8];
       xform_block<D>(u0, u1, sA, sBp, o, sb, sxr, sxpp);

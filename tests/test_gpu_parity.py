@@ -695,21 +695,34 @@ def test_gemm_decode_gemv_equals_split_calls(M, d_in, d_out, d):
     assert_close(f"decode-GEMV M={M} K={d_in}", to_np(Y1), ref, D, TOL_BF16)
 
 
-def test_gemm_decode_gemv_graph_replay():
-    """Back-to-back lcvq_gemm calls with programmatic dependent launch (each
-    X-transform waits for the previous call's GEMV, each GEMV streams its codes
-    during its X-transform), captured in a CUDA graph on one workspace: every
-    replay gives the eager bits."""
-    M, K, N = 4, 4096, 4096
+@pytest.mark.parametrize("M", [4, 16])
+def test_gemm_decode_gemv_back_to_back_on_one_workspace(M):
+    """Back-to-back lcvq_gemm calls on one workspace, with programmatic
+    dependent launch (each X-transform waits for the previous call's GEMV and
+    overwrites X'' and corr that GEMV read; each GEMV becomes resident before
+    its X-transform has written): eagerly and replayed from a CUDA graph, every
+    output equals the call run alone on a fresh workspace.  A load of X'' or
+    corr through a path that can return a line an earlier call left in an
+    SM's L1 fails this."""
+    K, N = 4096, 4096
     cases = []
-    for i in range(3):
+    for i in range(4):
         w, z = _fwd_case(2, M, d_in=K, d_out=N)
         X = to_dev(w["X"] * (1.0 + i), torch.bfloat16)
         cases.append((X, torch.from_numpy(O.pack_codes(z)).to(dev()),
                       torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev())))
-    ws = lcvq.new_workspace(lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, 8), dev())
-    eager = [lcvq.gemm(X, p, K, A, B, 8, workspace=ws) for X, p, A, B in cases]
-    outs = [torch.empty_like(e) for e in eager]
+    size = lcvq.workspace_size(lcvq.OP_GEMM, torch.bfloat16, M, N, K, 8)
+    alone = []
+    for X, p, A, B in cases:
+        alone.append(lcvq.gemm(X, p, K, A, B, 8, workspace=lcvq.new_workspace(size, dev())))
+        torch.cuda.synchronize()
+    ws = lcvq.new_workspace(size, dev())
+    for _ in range(3):
+        eager = [lcvq.gemm(X, p, K, A, B, 8, workspace=ws) for X, p, A, B in cases]
+        torch.cuda.synchronize()
+        for Y, r in zip(eager, alone):
+            assert torch.equal(Y, r)
+    outs = [torch.empty_like(r) for r in alone]
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     torch.cuda.synchronize()
@@ -717,13 +730,13 @@ def test_gemm_decode_gemv_graph_replay():
     with torch.cuda.graph(g, stream=s):
         for (X, p, A, B), Y in zip(cases, outs):
             lcvq.gemm(X, p, K, A, B, 8, out=Y, workspace=ws)
-    for _ in range(2):
+    for _ in range(3):
         for Y in outs:
             Y.zero_()
         g.replay()
         torch.cuda.synchronize()
-        for Y, e in zip(outs, eager):
-            assert torch.equal(Y, e)
+        for Y, r in zip(outs, alone):
+            assert torch.equal(Y, r)
     del g
 
 

@@ -89,8 +89,8 @@ GemmWs gemm_ws(lcvq_dtype dtype, int64_t M, int64_t d_in) {
   if (dtype == LCVQ_BF16) {
     w.xpp_off = off;
     off = round_up(off + size_t(M) * size_t(d_in) * 2, 256);
-    w.corr_off = off;
-    off = round_up(off + size_t(M) * 4, 256);
+    w.corr_off = off;  // corr [M], then the int8 path's inv_s [M][8]
+    off = round_up(off + size_t(M) * 36, 256);
   }
   w.total = off;
   return w;
@@ -294,7 +294,18 @@ lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t*
   cudaError_t e = cudaSuccess;
   char* ws = static_cast<char*>(workspace);
   unsigned int* err = reinterpret_cast<unsigned int*>(ws);
-  if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
+  if (dtype == LCVQ_BF16 && M <= kI8MaxM) {
+    // few tokens: the int8 path (X' as two signed byte digits per position,
+    // the integer tensor-core MMA, exact integer sums per chunk class)
+    uint8_t* X8 = reinterpret_cast<uint8_t*>(ws + w.xpp_off);
+    float* corr = reinterpret_cast<float*>(ws + w.corr_off);
+    float* inv_s = corr + M;
+    e = launch_xform_i8(static_cast<const uint16_t*>(X), M, d_in, d, A, B, X8, corr, inv_s, s,
+                        &launches);
+    if (e == cudaSuccess)
+      e = launch_gemv(reinterpret_cast<const uint16_t*>(X8), corr, M, packed, d_out, d_in,
+                      static_cast<uint16_t*>(Y), true, s, &launches, inv_s);
+  } else if (dtype == LCVQ_BF16 && (M <= 32 || form != LCVQ_FORM_DECODE)) {
     uint16_t* Xpp = reinterpret_cast<uint16_t*>(ws + w.xpp_off);
     float* corr = reinterpret_cast<float*>(ws + w.corr_off);
     e = launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr, s, &launches);
@@ -331,7 +342,7 @@ size_t grouped_ws(const lcvq_gemm_item* items, int count, int64_t M, int d,
     if (xpp_off) xpp_off->push_back(off);
     off = round_up(off + size_t(M) * size_t(it.d_in) * 2, 256);
     if (corr_off) corr_off->push_back(off);
-    off = round_up(off + size_t(M) * 4, 256);
+    off = round_up(off + size_t(M) * 36, 256);  // corr [M], then the int8 path's inv_s [M][8]
   }
   return off;
 }
@@ -369,8 +380,9 @@ lcvq_status lcvq_gemm_grouped(const lcvq_gemm_item* items, int count, int64_t M,
     const lcvq_gemm_item& it = items[i];
     uint16_t* Xpp = reinterpret_cast<uint16_t*>(ws + xoff[i]);
     float* corr = reinterpret_cast<float*>(ws + coff[i]);
-    xj[i] = XformJob{static_cast<const uint16_t*>(it.X), it.A, it.B, Xpp, corr, it.d_in};
-    gj[i] = GemvJob{it.packed, Xpp, corr, static_cast<uint16_t*>(it.Y), it.d_out, it.d_in};
+    float* inv_s = M <= kI8MaxM ? corr + M : nullptr;  // set: the int8 path, as lcvq_gemm
+    xj[i] = XformJob{static_cast<const uint16_t*>(it.X), it.A, it.B, Xpp, corr, it.d_in, inv_s};
+    gj[i] = GemvJob{it.packed, Xpp, corr, static_cast<uint16_t*>(it.Y), it.d_out, it.d_in, inv_s};
   }
   int launches = 0;
   // per chunk of matrices: their X-transforms, then their decode-GEMV

@@ -29,6 +29,7 @@
 
 #include <map>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "codec.cuh"
@@ -57,11 +58,12 @@ namespace {
 // decode-GEMV.
 struct GemvItem {
   const uint8_t* packed;  // [N][K/4]
-  const uint16_t* Xpp;    // [M][K] X'' (decoder order)
+  const uint16_t* Xpp;    // [M][K] X'' (decoder order), or the int8 digit planes
   const float* corr;      // [M]
   uint16_t* Y;            // [M][N]
   int N, K;
-  int tile_end;  // tiles of items 0 .. this one
+  int tile_end;         // tiles of items 0 .. this one
+  const float* inv_s;   // [M]: the int8 path's 1 / scale (null on the bf16 path)
 };
 template <int kItems>
 struct GemvGroup {
@@ -85,9 +87,15 @@ __host__ __device__ constexpr size_t group_smem_part() {
   return size_t(2) * kWarps * (16 * R) * (NT * 8 + 1) * sizeof(float);
 }
 
-template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kStages, int kItems>
+// kI8: the int8 path (X as the two digit planes of the int8-digit transform,
+// u8 x s8 m16n8k32 MMAs accumulating exactly in int32): column c of a token
+// tile is token 4 n + c / 2, digit plane c % 2 (hi, lo); otherwise column c is
+// token 8 n + c of the bf16 X''.
+template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kStages, int kItems,
+          bool kI8 = false>
 __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
     gemv_group_kernel(const __grid_constant__ GemvGroup<kItems> grp) {
+  using Acc = typename std::conditional<kI8, int, float>::type;
   constexpr int MP = NT * 8;
   constexpr int ROWS = 16 * R;
   constexpr uint32_t kStageBytes = ROWS * 128;
@@ -147,37 +155,54 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
     cp_async_commit();
   };
   // X'' fragments of unit j of chunk c: word q, token tile n -> two 16-byte halves
-  // X'' of a chunk for this lane: the start of its 32 positions in each token
-  // row, and how many positions of K remain from there (<= 0: none)
+  // X of a chunk for this lane: the byte address of its first position in the
+  // row (bf16: 32 positions of X''; int8: 32 positions of its digit plane) of
+  // each token tile, and how many positions of K remain from there (<= 0: none)
   struct XPos {
-    const uint16_t* base[NT];
+    const unsigned char* base[NT];
     int remt;
   };
   bool tokok[NT];
 #pragma unroll
-  for (int n = 0; n < NT; ++n) tokok[n] = n * 8 + g < M;
+  for (int n = 0; n < NT; ++n) tokok[n] = (kI8 ? n * 4 + (g >> 1) : n * 8 + g) < M;
   auto xpos = [&](const Cur& c) {
     XPos p;
     const bool any = c.tile < T;
     const GemvItem& it = grp.item[any ? c.item : 0];
     const int64_t k0 = int64_t(c.chunk) * (kAhead * kUnit);
     p.remt = any ? static_cast<int>(it.K - k0) - 32 * t : 0;
+    const unsigned char* xb = reinterpret_cast<const unsigned char*>(it.Xpp);
 #pragma unroll
-    for (int n = 0; n < NT; ++n)
-      p.base[n] = it.Xpp + (tokok[n] ? int64_t(n * 8 + g) * it.K : 0) + k0 + 32 * t;
+    for (int n = 0; n < NT; ++n) {
+      if constexpr (kI8) {
+        // chunk c's hi plane at byte 2 k0 of the row, its lo plane n_c bytes on
+        const int64_t nc = it.K - k0 < kAhead * kUnit ? it.K - k0 : kAhead * kUnit;
+        p.base[n] = xb + (tokok[n] ? int64_t(n * 4 + (g >> 1)) * 2 * it.K : 0) + 2 * k0 +
+                    ((g & 1) ? nc : 0) + 32 * t;
+      } else {
+        p.base[n] = xb + 2 * ((tokok[n] ? int64_t(n * 8 + g) * it.K : 0) + k0 + 32 * t);
+      }
+    }
     return p;
   };
-  // X'' fragments of unit j: word q, token tile n -> two 16-byte halves
+  // X fragments of unit j: word q, token tile n -> two 16-byte halves (bf16)
+  // or one 16-byte block of digits (int8)
   auto load_x = [&](const XPos& p, int j, uint4 (&xb)[2][NT][2]) {
     const bool kok = j * kUnit < p.remt;
 #pragma unroll
     for (int q = 0; q < 2; ++q)
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
+        // written by the X-transform: ordinary loads, not the read-only path
         if (kok && tokok[n]) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.base[n] + j * kUnit + 16 * q);
-          xb[q][n][0] = ld_global_v4(src);  // written by the X-transform: not the read-only path
-          xb[q][n][1] = ld_global_v4(src + 1);
+          if constexpr (kI8) {
+            xb[q][n][0] = ld_global_v4(p.base[n] + j * kUnit + 16 * q);
+            xb[q][n][1] = make_uint4(0, 0, 0, 0);
+          } else {
+            const unsigned char* src = p.base[n] + 2 * (j * kUnit + 16 * q);
+            xb[q][n][0] = ld_global_v4(src);
+            xb[q][n][1] = ld_global_v4(src + 16);
+          }
         } else {
           xb[q][n][0] = make_uint4(0, 0, 0, 0);
           xb[q][n][1] = make_uint4(0, 0, 0, 0);
@@ -212,13 +237,13 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
   int eitem = 0;  // item of the tile in the epilogue
   int buf = 0;
   for (int tile = static_cast<int>(blockIdx.x); tile < T; tile += G, buf ^= 1) {
-    float acc[R][NT][4];
+    Acc acc[R][NT][4];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
       for (int n = 0; n < NT; ++n)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[r][n][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[r][n][e] = Acc(0);
 
     while (cur.tile == tile) {  // this warp's chunks of the tile
       cp_async_wait<kStages - 2>();  // this lane's copies of chunk `cur` have landed
@@ -245,6 +270,27 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
 #pragma unroll
             for (int h = 0; h < 2; ++h)
               cw[r][h] = lds_v2(sbase + (r * 16 + g + 8 * h) * 128 + coff[j]);
+          if constexpr (kI8) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {  // word q of each row: 16 codes, 2 k32 tiles
+              uint32_t rp[R][2][4];
+#pragma unroll
+              for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) dec_word_u8(q == 0 ? cw[r][h].x : cw[r][h].y, rp[r][h]);
+#pragma unroll
+              for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                  const uint32_t b0 = word_of(xcur[q][n][0], 2 * mm);
+                  const uint32_t b1 = word_of(xcur[q][n][0], 2 * mm + 1);
+#pragma unroll
+                  for (int r = 0; r < R; ++r)
+                    mma_u8s8_16832(acc[r][n], rp[r][0][2 * mm], rp[r][1][2 * mm],
+                                   rp[r][0][2 * mm + 1], rp[r][1][2 * mm + 1], b0, b1);
+                }
+            }
+          } else {
 #pragma unroll
           for (int q = 0; q < 2; ++q) {  // word q of each row: 16 codes, 4 k16 tiles
             uint32_t w0[R][2], w6[R][2], w12[R][2];
@@ -277,6 +323,7 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
               }
             }
           }
+          }
         }
         if constexpr (kPrefX) {
 #pragma unroll
@@ -306,25 +353,44 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         const int lr = r * 16 + g;
-        const int tk = n * 8 + 2 * t;
-        part[buf][warp][lr][tk] = acc[r][n][0];
-        part[buf][warp][lr][tk + 1] = acc[r][n][1];
-        part[buf][warp][lr + 8][tk] = acc[r][n][2];
-        part[buf][warp][lr + 8][tk + 1] = acc[r][n][3];
+        const int tk = n * 8 + 2 * t;  // int8: token 4 n + t, digit planes hi / lo
+        if constexpr (kI8) {
+          part[buf][warp][lr][tk] = __int_as_float(acc[r][n][0]);
+          part[buf][warp][lr][tk + 1] = __int_as_float(acc[r][n][1]);
+          part[buf][warp][lr + 8][tk] = __int_as_float(acc[r][n][2]);
+          part[buf][warp][lr + 8][tk + 1] = __int_as_float(acc[r][n][3]);
+        } else {
+          part[buf][warp][lr][tk] = acc[r][n][0];
+          part[buf][warp][lr][tk + 1] = acc[r][n][1];
+          part[buf][warp][lr + 8][tk] = acc[r][n][2];
+          part[buf][warp][lr + 8][tk + 1] = acc[r][n][3];
+        }
       }
     __syncthreads();
     while (tile >= grp.item[eitem].tile_end) ++eitem;
     const GemvItem& it = grp.item[eitem];
     const int64_t row0 = int64_t(tile - tile_begin(eitem)) * ROWS;
     // sum the warps' K chunks in warp order, add the per-row constant, store
+    // (int8: each class's exact integer sums scaled by its own 1 / s)
     for (int e = threadIdx.x; e < ROWS * M; e += kWarps * 32) {
       const int lr = e % ROWS, tok = e / ROWS;
       const int64_t grow = row0 + lr;
-      float sum = 0.f;
+      float y;
+      if constexpr (kI8) {  // warp w's chunks are class w: its own scale
+        float sum = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) sum += part[buf][w][lr][tok];
-      if (grow < it.N)
-        it.Y[int64_t(tok) * it.N + grow] = f32_to_bf16(sum + ld_global_f32(it.corr + tok));
+        for (int w = 0; w < kWarps; ++w)
+          sum = i8_add_class(sum, __float_as_int(part[buf][w][lr][2 * tok]),
+                             __float_as_int(part[buf][w][lr][2 * tok + 1]),
+                             ld_global_f32(it.inv_s + tok * kWarps + w));
+        y = sum + ld_global_f32(it.corr + tok);
+      } else {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) sum += part[buf][w][lr][tok];
+        y = sum + ld_global_f32(it.corr + tok);
+      }
+      if (grow < it.N) it.Y[int64_t(tok) * it.N + grow] = f32_to_bf16(y);
     }
   }
   cp_async_wait<0>();  // no copy may outlive the CTA (only empty groups remain)
@@ -374,9 +440,11 @@ struct WideLayout {
   static constexpr size_t kSmem = 1024 + size_t(kBarOff) + 2 * kStages * 8 + 16;  // + alignment
 };
 
-template <int NT, int kStages, int kMinBlocks, int kItems>
+// kI8: the int8 path, as for gemv_group_kernel
+template <int NT, int kStages, int kMinBlocks, int kItems, bool kI8 = false>
 __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
     gemv_wide_kernel(const __grid_constant__ GemvWideGroup<kItems> grp) {
+  using Acc = typename std::conditional<kI8, int, float>::type;
   using L = WideLayout<NT, kStages>;
   extern __shared__ __align__(1024) unsigned char wsm_raw[];
   // SW128 boxes need 1024-byte aligned destinations
@@ -467,12 +535,15 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
 #pragma unroll
   for (int j = 0; j < kAhead; ++j)
     coff[j] = static_cast<uint32_t>(((2 * j + (t >> 1)) ^ g) << 4) + ((t & 1) << 3);
+  // (int8: column g of token tile n is token 4 n + g/2, digit plane g % 2; a
+  // chunk's lo plane starts n_c bytes after its hi plane)
   uint32_t xoff[NT];
   bool tokok[NT];
 #pragma unroll
   for (int n = 0; n < NT; ++n) {
-    tokok[n] = n * 8 + g < M;
-    xoff[n] = static_cast<uint32_t>((n * 8 + g) * kWideXPitch + 64 * t);
+    const int tok = kI8 ? n * 4 + (g >> 1) : n * 8 + g;
+    tokok[n] = tok < M;
+    xoff[n] = static_cast<uint32_t>(tok * kWideXPitch + (kI8 ? 32 * t : 64 * t));
   }
   int seq = 0, item = 0;
   for (int tile = static_cast<int>(blockIdx.x); tile < T && !warp_abort(); tile += G) {
@@ -480,13 +551,13 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
     const GemvItem& it = grp.item[item];
     const int K = it.K;
     const int nch = nchunks(K);
-    float acc[kWideConsumers][NT][4];
+    Acc acc[kWideConsumers][NT][4];
 #pragma unroll
     for (int v = 0; v < kWideConsumers; ++v)
 #pragma unroll
       for (int n = 0; n < NT; ++n)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[v][n][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[v][n][e] = Acc(0);
 
     bool ok = true;
     for (int c0 = 0; c0 < nch && ok; c0 += kWideConsumers) {
@@ -506,6 +577,8 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
         const uint32_t xst = st + L::kCodeBytes;
         const int rem = K - c * (kAhead * kUnit);   // positions of K left from this chunk on
         const int remt = rem - 32 * t;              // ... from this lane's first position on
+        // int8: this lane's digit plane (the lo plane follows the chunk's n_c hi bytes)
+        const uint32_t plane = (kI8 && (g & 1)) ? static_cast<uint32_t>(rem < 512 ? rem : 512) : 0u;
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
           if (j * kUnit >= rem) break;  // warp-uniform: past the end of K
@@ -513,6 +586,25 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
           uint2 cw[2];
           cw[0] = lds_v2(crow + coff[j]);
           cw[1] = lds_v2(crow + 8 * 128 + coff[j]);
+          if constexpr (kI8) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {  // word q of rows g, g + 8: 2 k32 tiles
+              uint4 xq[NT];
+#pragma unroll
+              for (int n = 0; n < NT; ++n)
+                xq[n] = (kok && tokok[n]) ? lds_v4(xst + xoff[n] + plane + j * kUnit + 16 * q)
+                                          : make_uint4(0, 0, 0, 0);
+              uint32_t r0[4], r1[4];
+              dec_word_u8(q == 0 ? cw[0].x : cw[0].y, r0);
+              dec_word_u8(q == 0 ? cw[1].x : cw[1].y, r1);
+#pragma unroll
+              for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+                  mma_u8s8_16832(acc[v][n], r0[2 * mm], r1[2 * mm], r0[2 * mm + 1], r1[2 * mm + 1],
+                                 word_of(xq[n], 2 * mm), word_of(xq[n], 2 * mm + 1));
+            }
+          } else {
           uint4 xb[2][NT][2];
 #pragma unroll
           for (int q = 0; q < 2; ++q)
@@ -550,6 +642,7 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
               }
             }
           }
+          }
         }
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(&empty[s]);
@@ -560,6 +653,23 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
 
     // the split kernel's fixed-order sum over the 8 K partitions, plus corr
     const int64_t row0 = int64_t(tile - tile_begin(item)) * kWideRows + warp * 16;
+    if constexpr (kI8) {  // accumulator v holds class v: the split kernel's class sum
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+          const int64_t row = row0 + g + 8 * rh;
+          const int tok = n * 4 + t;
+          if (row < it.N && tok < M) {
+            float sum = 0.f;
+#pragma unroll
+            for (int v = 0; v < kWideConsumers; ++v)
+              sum = i8_add_class(sum, acc[v][n][2 * rh], acc[v][n][2 * rh + 1],
+                                 ld_global_f32(it.inv_s + tok * kWideConsumers + v));
+            it.Y[int64_t(tok) * it.N + row] = f32_to_bf16(sum + ld_global_f32(it.corr + tok));
+          }
+        }
+    } else {
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -572,6 +682,7 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
         if (row < it.N && tok < M)
           it.Y[int64_t(tok) * it.N + row] = f32_to_bf16(sum + ld_global_f32(it.corr + tok));
       }
+    }
   }
   // the last CTA-wide point: consumers are done with every stage
   griddep_launch_dependents();
@@ -615,9 +726,10 @@ int64_t resident_ctas(const void* kern, int threads, size_t smem) {
   return v;
 }
 
-template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kStages, int kItems>
+template <int NT, int R, int kWarps, bool kPrefX, int kMinBlocks, int kStages, int kItems,
+          bool kI8 = false>
 cudaError_t launch_group_t(const GemvGroup<kItems>& grp, cudaStream_t s) {
-  auto kern = gemv_group_kernel<NT, R, kWarps, kPrefX, kMinBlocks, kStages, kItems>;
+  auto kern = gemv_group_kernel<NT, R, kWarps, kPrefX, kMinBlocks, kStages, kItems, kI8>;
   constexpr size_t smem = group_smem_ring<R, kStages, kWarps>() + group_smem_part<NT, R, kWarps>();
   if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
       e != cudaSuccess)
@@ -647,6 +759,8 @@ int group_rows(int64_t M) { return M <= 8 ? kRowsSmallM : kRowsLargeM; }
 // per SM with room for the X'' prefetch; M <= 32: 32 rows, no prefetch.
 template <int kItems>
 cudaError_t launch_group(const GemvGroup<kItems>& grp, cudaStream_t s) {
+  if (grp.item[0].inv_s != nullptr)  // the int8 path (M <= kI8MaxM: one token tile)
+    return launch_group_t<1, 1, 8, true, 2, LCVQ_GS1, kItems, true>(grp, s);
   if (grp.M <= 8) return launch_group_t<1, 1, 8, true, 2, LCVQ_GS1, kItems>(grp, s);
   if (grp.M <= 16) return launch_group_t<2, 2, 8, true, 1, LCVQ_GS2, kItems>(grp, s);
   return launch_group_t<4, 2, 8, false, 1, LCVQ_GS4, kItems>(grp, s);
@@ -656,14 +770,14 @@ cudaError_t launch_group(const GemvGroup<kItems>& grp, cudaStream_t s) {
 
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
                         int64_t d_out, int64_t d_in, uint16_t* Y, bool after_xform,
-                        cudaStream_t s, int* launches) {
+                        cudaStream_t s, int* launches, const float* inv_s) {
   // a single matrix is a group of one (the same kernel, so the same bits)
   GemvGroup<1> grp{};
   grp.count = 1;
   grp.M = static_cast<int>(M);
   grp.early_codes = after_xform ? 1 : 0;
   grp.item[0] = GemvItem{packed, Xpp, corr, Y, static_cast<int>(d_out), static_cast<int>(d_in),
-                         static_cast<int>(ceil_div(d_out, group_rows(M)))};
+                         static_cast<int>(ceil_div(d_out, group_rows(M))), inv_s};
   cudaError_t e = launch_group(grp, s);
   ++*launches;
   if (e != cudaSuccess) return e;
@@ -671,9 +785,9 @@ cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const
 }
 
 namespace {
-template <int NT, int kStages, int kMinBlocks, int kItems>
+template <int NT, int kStages, int kMinBlocks, int kItems, bool kI8 = false>
 cudaError_t launch_wide_t(const GemvWideGroup<kItems>& grp, cudaStream_t s) {
-  auto kern = gemv_wide_kernel<NT, kStages, kMinBlocks, kItems>;
+  auto kern = gemv_wide_kernel<NT, kStages, kMinBlocks, kItems, kI8>;
   constexpr size_t smem = WideLayout<NT, kStages>::kSmem;
   if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
       e != cudaSuccess)
@@ -720,14 +834,16 @@ cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaS
         const GemvJob& j = jobs[first + i];
         tiles += static_cast<int>(ceil_div(j.d_out, kWideRows));
         grp.item[i] = GemvItem{j.packed, j.Xpp, j.corr, j.Y, static_cast<int>(j.d_out),
-                               static_cast<int>(j.d_in), tiles};
+                               static_cast<int>(j.d_in), tiles, j.inv_s};
         if (!make_tensor_map_2d(&grp.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, j.packed,
                                 uint64_t(j.d_in / 4), uint64_t(j.d_out), uint64_t(j.d_in / 4),
                                 kAhead * 32, kWideRows, true))
           return cudaErrorInvalidValue;
       }
-      cudaError_t e = M <= 8 ? launch_wide_t<1, LCVQ_WS1, 2, kMaxGroupItems>(grp, s)
-                             : launch_wide_t<2, LCVQ_WS2, 1, kMaxGroupItems>(grp, s);
+      cudaError_t e = jobs[0].inv_s != nullptr
+                          ? launch_wide_t<1, LCVQ_WS1, 2, kMaxGroupItems, true>(grp, s)
+                      : M <= 8 ? launch_wide_t<1, LCVQ_WS1, 2, kMaxGroupItems>(grp, s)
+                               : launch_wide_t<2, LCVQ_WS2, 1, kMaxGroupItems>(grp, s);
       ++*launches;
       if (e != cudaSuccess) return e;
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -746,7 +862,7 @@ cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaS
       const GemvJob& j = jobs[first + i];
       tiles += static_cast<int>(ceil_div(j.d_out, rows));
       grp.item[i] = GemvItem{j.packed, j.Xpp, j.corr, j.Y, static_cast<int>(j.d_out),
-                             static_cast<int>(j.d_in), tiles};
+                             static_cast<int>(j.d_in), tiles, j.inv_s};
     }
     cudaError_t e = launch_group(grp, s);
     ++*launches;
@@ -760,7 +876,8 @@ cudaError_t launch_gemm_xformed(const uint16_t* Xpp, const float* corr, int64_t 
                                 const uint8_t* packed, int64_t d_out, int64_t d_in, uint16_t* Y,
                                 unsigned int* err, bool after_xform, cudaStream_t s,
                                 int* launches) {
-  if (M <= 32) return launch_gemv(Xpp, corr, M, packed, d_out, d_in, Y, after_xform, s, launches);
+  if (M <= 32)
+    return launch_gemv(Xpp, corr, M, packed, d_out, d_in, Y, after_xform, s, launches, nullptr);
   return launch_tc_forward(Xpp, true, corr, M, packed, d_out, d_in, 8, nullptr, nullptr, Y, err, s,
                            launches);
 }

@@ -19,6 +19,34 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D += A B for one m16n8k32 tile: A unsigned bytes, B signed bytes, exact
+// int32 accumulate (the int8 path: codes times the digits of X')
+__device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The four u8 registers of one 32-bit word of 2-bit codes for the int8 MMA:
+// register p holds the codes of positions p, p + 4, p + 8, p + 12 (byte i =
+// position 4 i + p), the order of the int8 digit planes of X'.
+__device__ __forceinline__ void dec_word_u8(uint32_t w, uint32_t (&r)[4]) {
+  r[0] = w & 0x03030303u;
+  r[1] = (w >> 2) & 0x03030303u;
+  r[2] = (w >> 4) & 0x03030303u;
+  r[3] = (w >> 6) & 0x03030303u;
+}
+
+// One chunk class's part of Y on the int8 path, added to the running sum of
+// the classes (in class order): the exact integer sums of the codes times the
+// hi and lo digits, (256 hi + lo), scaled by the class's 1 / s (a power of two)
+__device__ __forceinline__ float i8_add_class(float sum, int hi, int lo, float inv_s) {
+  return fmaf(fmaf(256.f, static_cast<float>(hi), static_cast<float>(lo)), inv_s, sum);
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
   return q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
 }

@@ -35,13 +35,23 @@ cudaError_t launch_dge_scale(float* dWp, const float* Wp, int64_t n, float k, cu
 cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
                          const float* B, uint16_t* Xpp, float* corr, cudaStream_t s,
                          int* launches);
+// The int8-digit form for the decode-GEMV's int8 path (M <= kI8MaxM): per row
+// and chunk class r (chunks r, r + 8, ... of 512 positions) a power-of-two
+// scale s, q = rint(X' s) as two signed byte digits per position (X8
+// [M][2 d_in] bytes: per chunk the hi plane, then the lo plane), inv_s[M][8] =
+// 1 / s and corr[M] = s' - 3/2 sum_r (sum of class r's q) / s_r.
+constexpr int64_t kI8MaxM = 4;
+cudaError_t launch_xform_i8(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
+                            const float* B, uint8_t* X8, float* corr, float* inv_s, cudaStream_t s,
+                            int* launches);
 
 // ---- decode-GEMV (bf16, M <= 32) ----
 // after_xform: launched right after launch_xform of the same call on the same
-// stream, so the codes may be read before the kernel's dependency wait
+// stream, so the codes may be read before the kernel's dependency wait.
+// inv_s set: the int8 path on launch_xform_i8's digits (Xpp points at them).
 cudaError_t launch_gemv(const uint16_t* Xpp, const float* corr, int64_t M, const uint8_t* packed,
                         int64_t d_out, int64_t d_in, uint16_t* Y, bool after_xform,
-                        cudaStream_t s, int* launches);
+                        cudaStream_t s, int* launches, const float* inv_s = nullptr);
 
 constexpr int kMaxGroupItems = 128;
 
@@ -52,9 +62,10 @@ struct XformJob {
   const uint16_t* X;
   const float* A;
   const float* B;
-  uint16_t* Xpp;
+  uint16_t* Xpp;  // the int8 digit planes when inv_s is set
   float* corr;
   int64_t d_in;
+  float* inv_s;  // null: bf16 X''; else the int8-digit form (every job of a call alike)
 };
 
 // decode-GEMV over a group of matrices with a common token count M <= 32, in
@@ -64,10 +75,11 @@ struct XformJob {
 // alone; large groups with 17 <= M <= 32 run on the tcgen05 form below.
 struct GemvJob {
   const uint8_t* packed;
-  const uint16_t* Xpp;
+  const uint16_t* Xpp;  // or the int8 digits
   const float* corr;
   uint16_t* Y;
   int64_t d_out, d_in;
+  const float* inv_s;  // set: the int8 path (M <= kI8MaxM; every job of a call alike)
 };
 // err: device error word for the bounded waits of the wide-tile form
 cudaError_t launch_gemv_grouped(const GemvJob* jobs, int count, int64_t M, cudaStream_t s,

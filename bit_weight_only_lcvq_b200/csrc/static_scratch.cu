@@ -24,7 +24,7 @@ constexpr int64_t kStaticMaxM = 32;
 constexpr int64_t kStaticMaxDin = 32768;
 constexpr int64_t kStaticMaxDout = int64_t(1) << 30;  // the same bound as lcvq_gemm
 constexpr size_t kStaticXppBytes = size_t(kStaticMaxM) * size_t(kStaticMaxDin) * 2;  // 2 MiB
-constexpr size_t kStaticScratchBytes = kStaticXppBytes + 256;                        // + corr
+constexpr size_t kStaticScratchBytes = kStaticXppBytes + 256;  // + corr [32], inv_s [<= 4][8]
 
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
@@ -84,11 +84,21 @@ extern "C" lcvq_status lcvq_gemv_static(const void* X, int64_t M, const uint8_t*
   float* corr = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + kStaticXppBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int launches = 0;
-  cudaError_t e = lcvq::launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr,
-                                     s, &launches);
-  if (e == cudaSuccess)
-    e = lcvq::launch_gemv(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), true, s,
-                          &launches);
+  cudaError_t e;
+  if (M <= lcvq::kI8MaxM) {  // the int8 path, as lcvq_gemm takes it
+    float* inv_s = corr + kStaticMaxM;
+    e = lcvq::launch_xform_i8(static_cast<const uint16_t*>(X), M, d_in, d, A, B,
+                              reinterpret_cast<uint8_t*>(Xpp), corr, inv_s, s, &launches);
+    if (e == cudaSuccess)
+      e = lcvq::launch_gemv(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), true, s,
+                            &launches, inv_s);
+  } else {
+    e = lcvq::launch_xform(static_cast<const uint16_t*>(X), M, d_in, d, A, B, Xpp, corr, s,
+                           &launches);
+    if (e == cudaSuccess)
+      e = lcvq::launch_gemv(Xpp, corr, M, packed, d_out, d_in, static_cast<uint16_t*>(Y), true, s,
+                            &launches);
+  }
   if (e != cudaSuccess) return LCVQ_ERR_CUDA;
   lcvq::set_last_launches(launches);
   return LCVQ_OK;

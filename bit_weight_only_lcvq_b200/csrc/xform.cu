@@ -38,8 +38,9 @@ struct XformItem {
   const uint16_t* X;  // [M][d_in] bf16
   const float* A;     // [D*D]
   const float* B;     // [D]
-  uint16_t* Xpp;      // [M][d_in] out
+  uint16_t* Xpp;      // [M][d_in] out (bf16 X'', or the int8 digit planes)
   float* corr;        // [M] out
+  float* inv_s;       // [M] out (int8 digits only: 1 / the row's scale)
   int64_t d_in;
 };
 template <int kItems>
@@ -138,10 +139,184 @@ __global__ void __launch_bounds__(kXfThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// The int8-digit form of X' for few tokens (the decode-GEMV's int8 path).
+//
+// Per row m and chunk class r (the chunks c = r, r + 8, ... of 512 positions,
+// warp r's share), X' = x A (fp32, the same fused multiply-adds as the bf16
+// form) is scaled by a power of two chosen from the class's largest |X'|:
+//     s_{m,r} = 2^k, the largest with max |X'| s <= 32639,
+// rounded to integers q = rint(X' s) (|q| <= 32639) and split into two signed
+// byte digits q = 256 hi + lo with hi = (q + 128) >> 8, lo = q - 256 hi, both in
+// [-128, 127].  The GEMV multiplies the raw codes z (u8) with the digits on the
+// integer tensor-core MMA, exactly: sum_k q_k z_k = 256 sum hi z + sum lo z per
+// class.  Then
+//     Y = sum_k (q_k / s_k) (z_k - 3/2) + s' = sum_r (sum_{k in r} q_k z_k) / s_r + corr,
+//     corr = s' - 3/2 sum_r (sum_{k in r} q_k) / s_r,
+// with s' = sum_g x_g . B' summed in the order of the bf16 form and the q sums
+// exact; inv_s[m][r] = 1/s_{m,r} (exact).  A class with no finite largest
+// |X'| (non-finite activations) gives corr = NaN.
+// Layout per row: 2 d_in bytes; chunk c (512 positions, n_c = min(512,
+// d_in - 512 c) of them) at byte 1024 c holds the hi plane (n_c bytes), then
+// the lo plane (n_c bytes).  Within each 16-position block byte 4 p + i holds
+// position 4 i + p, the order in which the GEMV's decoder extracts codes from
+// a 32-bit code word (shift by 2 p, mask each byte).
+constexpr int kI8Max = 32639;  // 127 * 256 + 127
+
+constexpr int kI8Keep = 4;  // chunks per warp whose X' stays in registers between the passes
+
+template <int D, int kItems>
+__global__ void __launch_bounds__(kXfThreads)
+    xform_i8_kernel(const __grid_constant__ XformGroup<kItems> grp) {
+  const XformItem& it = grp.item[blockIdx.y];
+  // X, A and B may come from the kernel just before this one: ld_global_*
+  const uint16_t* X = it.X;
+  const float* A = it.A;
+  const float* B = it.B;
+  const int64_t d_in = it.d_in;
+  __shared__ float sA[D * D];
+  __shared__ float sB[D];
+  __shared__ float sBp[D];
+  __shared__ double red[2][kXfThreads / 32];
+  // programmatic dependent launch: as xform_kernel
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  const int64_t m = blockIdx.x;
+  const uint16_t* xr = X + m * d_in;
+  uint8_t* orow = reinterpret_cast<uint8_t*>(it.Xpp) + m * 2 * d_in;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nblk = d_in / 16;
+  const int64_t nchunk = ceil_div(d_in, kCorrChunk);
+  // warp w takes the chunks c = w, w + 8, ...; lane l block l of a chunk.  The
+  // activations of the warp's first kI8Keep chunks load together with A and B.
+  auto block_of = [&](int64_t c) { return c * (kCorrChunk / 16) + lane; };
+  uint4 xin[kI8Keep][2];
+#pragma unroll
+  for (int ci = 0; ci < kI8Keep; ++ci) {
+    const int64_t c = warp + int64_t(kCorrClasses) * ci, b = block_of(c);
+    xin[ci][0] = xin[ci][1] = make_uint4(0, 0, 0, 0);
+    if (c < nchunk && b < nblk) {
+      xin[ci][0] = ld_global_v4(xr + 16 * b);
+      xin[ci][1] = ld_global_v4(xr + 16 * b + 8);
+    }
+  }
+  if (threadIdx.x < D * D) sA[threadIdx.x] = ld_global_f32(A + threadIdx.x);
+  if (threadIdx.x < D) sB[threadIdx.x] = ld_global_f32(B + threadIdx.x);
+  __syncthreads();
+  if (threadIdx.x < D) sBp[threadIdx.x] = shifted_offset<D>(sA + threadIdx.x * D, sB[threadIdx.x]);
+  __syncthreads();
+
+  // pass 1: X' (kept in registers for the first kI8Keep chunks) and the
+  // class's largest |X'| (NaN propagates through the comparisons)
+  float xk[kI8Keep][16], sbk[kI8Keep];
+  float mx = 0.f;
+  auto take_max = [&](const float (&xp)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float a = fabsf(xp[e]);
+      mx = (a > mx || a != a) ? a : mx;
+    }
+  };
+#pragma unroll
+  for (int ci = 0; ci < kI8Keep; ++ci) {
+    const int64_t c = warp + int64_t(kCorrClasses) * ci;
+    sbk[ci] = 0.f;
+    if (c < nchunk && block_of(c) < nblk) {
+      xprime_block<D>(xin[ci][0], xin[ci][1], sA, sBp, xk[ci], sbk[ci]);
+      take_max(xk[ci]);
+    }
+  }
+  for (int64_t c = warp + int64_t(kCorrClasses) * kI8Keep; c < nchunk; c += kCorrClasses) {
+    const int64_t b = block_of(c);
+    if (b < nblk) {
+      float xp[16], sb;
+      xprime_block<D>(ld_global_v4(xr + 16 * b), ld_global_v4(xr + 16 * b + 8), sA, sBp, xp, sb);
+      take_max(xp);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, mx, off);
+    mx = (o > mx || o != o) ? o : mx;
+  }
+  // s = 2^k, the largest with mx s <= 32639 (from the exponent bits; k = 0 for
+  // an empty class, sc = 0 marks a non-finite one)
+  int k = 0;
+  const bool finite = mx <= 3.402823466e38f;
+  if (finite && mx > 0.f) {
+    const uint32_t bits = __float_as_uint(mx);
+    const int e = bits >= 0x00800000u ? int(bits >> 23) - 127 : -127;  // subnormal: below 2^-126
+    k = 14 - e;  // mx 2^k in [2^14, 2^15) for a normal mx
+    if (k > 126) k = 126;
+    if (mx * __uint_as_float(uint32_t(k + 127) << 23) > float(kI8Max)) --k;
+  }
+  const float sc = finite ? __uint_as_float(uint32_t(k + 127) << 23) : 0.f;
+  const float inv = __uint_as_float(uint32_t(127 - k) << 23);
+  if (lane == 0) it.inv_s[m * kCorrClasses + warp] = inv;
+
+  // pass 2: digits, and the parts of corr (s' in the order of xform_kernel;
+  // sum q exactly)
+  double s_b = 0.0, s_q = 0.0;  // this class's running sums (lane 0)
+  auto emit = [&](int64_t c, const float (&xp)[16], float sb) {
+    int qsum = 0;
+    if (block_of(c) < nblk) {
+      uint32_t wh[4] = {0, 0, 0, 0}, wl[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int q = sc > 0.f ? __float2int_rn(xp[e] * sc) : 0;
+        const int h = (q + 128) >> 8;
+        const int l = q - h * 256;
+        qsum += q;
+        const int p = e & 3, i = e >> 2;  // position e = 4 i + p -> byte 4 p + i
+        wh[p] |= (uint32_t(h) & 0xFFu) << (8 * i);
+        wl[p] |= (uint32_t(l) & 0xFFu) << (8 * i);
+      }
+      const int64_t nc = d_in - c * kCorrChunk < kCorrChunk ? d_in - c * kCorrChunk : kCorrChunk;
+      uint8_t* dst = orow + c * 2 * kCorrChunk + 16 * lane;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+      *reinterpret_cast<uint4*>(dst + nc) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+    }
+    const double tb = chunk_tree_sum(double(sb));
+    const double tq = chunk_tree_sum(double(qsum));
+    if (lane == 0) {
+      s_b += tb;
+      s_q += tq;
+    }
+  };
+#pragma unroll
+  for (int ci = 0; ci < kI8Keep; ++ci) {
+    const int64_t c = warp + int64_t(kCorrClasses) * ci;
+    if (c < nchunk) emit(c, xk[ci], sbk[ci]);
+  }
+  for (int64_t c = warp + int64_t(kCorrClasses) * kI8Keep; c < nchunk; c += kCorrClasses) {
+    const int64_t b = block_of(c);
+    float xp[16], sb = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) xp[e] = 0.f;
+    if (b < nblk)
+      xprime_block<D>(ld_global_v4(xr + 16 * b), ld_global_v4(xr + 16 * b + 8), sA, sBp, xp, sb);
+    emit(c, xp, sb);
+  }
+  if (lane == 0) {
+    red[0][warp] = s_b;
+    red[1][warp] = finite ? s_q * double(inv) : __longlong_as_double(0x7FF8000000000000LL);  // exact
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // the class parts in class order
+    double a = 0.0, q = 0.0;
+    for (int w = 0; w < kCorrClasses; ++w) {
+      a += red[0][w];
+      q += red[1][w];
+    }
+    it.corr[m] = static_cast<float>(a - 1.5 * q);
+  }
+}
+
 namespace {
 template <int kItems>
 cudaError_t launch_xform_group(const XformGroup<kItems>& grp, int count, int64_t M, int d,
-                               cudaStream_t s) {
+                               bool i8, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(M), static_cast<unsigned>(count), 1);
   cfg.blockDim = dim3(kXfThreads, 1, 1);
@@ -151,6 +326,14 @@ cudaError_t launch_xform_group(const XformGroup<kItems>& grp, int count, int64_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (i8) {
+    switch (d) {
+      case 1: return cudaLaunchKernelEx(&cfg, xform_i8_kernel<1, kItems>, grp);
+      case 2: return cudaLaunchKernelEx(&cfg, xform_i8_kernel<2, kItems>, grp);
+      case 4: return cudaLaunchKernelEx(&cfg, xform_i8_kernel<4, kItems>, grp);
+      default: return cudaLaunchKernelEx(&cfg, xform_i8_kernel<8, kItems>, grp);
+    }
+  }
   switch (d) {
     case 1: return cudaLaunchKernelEx(&cfg, xform_kernel<1, kItems>, grp);
     case 2: return cudaLaunchKernelEx(&cfg, xform_kernel<2, kItems>, grp);
@@ -164,8 +347,19 @@ cudaError_t launch_xform(const uint16_t* X, int64_t M, int64_t d_in, int d, cons
                          const float* B, uint16_t* Xpp, float* corr, cudaStream_t s,
                          int* launches) {
   XformGroup<1> grp{};
-  grp.item[0] = XformItem{X, A, B, Xpp, corr, d_in};
-  cudaError_t e = launch_xform_group(grp, 1, M, d, s);
+  grp.item[0] = XformItem{X, A, B, Xpp, corr, nullptr, d_in};
+  cudaError_t e = launch_xform_group(grp, 1, M, d, false, s);
+  ++*launches;
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_xform_i8(const uint16_t* X, int64_t M, int64_t d_in, int d, const float* A,
+                            const float* B, uint8_t* X8, float* corr, float* inv_s, cudaStream_t s,
+                            int* launches) {
+  XformGroup<1> grp{};
+  grp.item[0] = XformItem{X, A, B, reinterpret_cast<uint16_t*>(X8), corr, inv_s, d_in};
+  cudaError_t e = launch_xform_group(grp, 1, M, d, true, s);
   ++*launches;
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -178,9 +372,9 @@ cudaError_t launch_xform_grouped(const XformJob* jobs, int count, int64_t M, int
     XformGroup<kMaxGroupItems> grp{};
     for (int i = 0; i < n; ++i) {
       const XformJob& j = jobs[first + i];
-      grp.item[i] = XformItem{j.X, j.A, j.B, j.Xpp, j.corr, j.d_in};
+      grp.item[i] = XformItem{j.X, j.A, j.B, j.Xpp, j.corr, j.inv_s, j.d_in};
     }
-    cudaError_t e = launch_xform_group(grp, n, M, d, s);
+    cudaError_t e = launch_xform_group(grp, n, M, d, jobs[first].inv_s != nullptr, s);
     ++*launches;
     if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -16,11 +16,40 @@
 
 namespace lcvq {
 
-// One 16-element block of the transform.
-// x16: the block's 16 bf16 activations as two 16-byte words.  sA: A (D x D,
-// row-major, fp32); sBp: B' = B + 3/2 A 1.  Writes the block's X'' in decoder
-// order (o[c] = bf16x2 of positions c and c + 8, each scaled by 4^-(c mod 3))
-// and the block's parts of the per-row constant:
+// X' of one 16-element block of activations, in fp32: x16 as two 16-byte
+// words of bf16; sA: A (D x D, row-major, fp32); sBp: B' = B + 3/2 A 1.
+//   xp[v d + j] = sum_i x[v d + i] A[i][j]   (fused multiply-adds in i order)
+//   sb          = sum_{v, i} x[v d + i] B'[i]  (s' of the block, in v, i order)
+template <int D>
+__device__ __forceinline__ void xprime_block(const uint4& u0, const uint4& u1,
+                                             const float* __restrict__ sA,
+                                             const float* __restrict__ sBp, float (&xp)[16],
+                                             float& sb) {
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  float x[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    x[2 * q] = bf16_lo(w[q]);
+    x[2 * q + 1] = bf16_hi(w[q]);
+  }
+  sb = 0.f;
+#pragma unroll
+  for (int v = 0; v < 16 / D; ++v) {
+#pragma unroll
+    for (int j = 0; j < D; ++j) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < D; ++i) acc = fmaf(x[v * D + i], sA[i * D + j], acc);
+      xp[v * D + j] = acc;
+    }
+#pragma unroll
+    for (int i = 0; i < D; ++i) sb = fmaf(x[v * D + i], sBp[i], sb);
+  }
+}
+
+// One 16-element block of the bf16 transform.  Writes the block's X'' in
+// decoder order (o[c] = bf16x2 of positions c and c + 8, each scaled by
+// 4^-(c mod 3)) and the block's parts of the per-row constant:
 //   sb   = sum x^T B'           (s')
 //   sxr  = sum bf16(X')         (X'r)
 //   sxpp = sum X''
@@ -29,29 +58,16 @@ __device__ __forceinline__ void xform_block(const uint4& u0, const uint4& u1,
                                             const float* __restrict__ sA,
                                             const float* __restrict__ sBp, uint32_t (&o)[8],
                                             float& sb, float& sxr, float& sxpp) {
-  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-  float x[16];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    x[2 * q] = bf16_lo(w[q]);
-    x[2 * q + 1] = bf16_hi(w[q]);
-  }
-  float xrd[16];  // bf16(X') as fp32
-  sb = 0.f;
+  float xrd[16];  // X', then bf16(X') as fp32
+  xprime_block<D>(u0, u1, sA, sBp, xrd, sb);
   sxr = 0.f;
 #pragma unroll
-  for (int v = 0; v < 16 / D; ++v) {
+  for (int v = 0; v < 16 / D; ++v)
 #pragma unroll
     for (int j = 0; j < D; ++j) {
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < D; ++i) acc = fmaf(x[v * D + i], sA[i * D + j], acc);
-      xrd[v * D + j] = bf16_to_f32(f32_to_bf16(acc));
+      xrd[v * D + j] = bf16_to_f32(f32_to_bf16(xrd[v * D + j]));
       sxr += xrd[v * D + j];
     }
-#pragma unroll
-    for (int i = 0; i < D; ++i) sb = fmaf(x[v * D + i], sBp[i], sb);
-  }
   sxpp = 0.f;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {

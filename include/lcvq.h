@@ -141,6 +141,17 @@ LCVQ_API lcvq_status lcvq_decode(const uint8_t* packed, int64_t d_out, int64_t d
  *   X [M][d_in] in `dtype`; Y [M][d_out] out in `dtype`.
  *   dtype BF16: tensor-core paths (M <= 32: decode-GEMV; larger M: tcgen05
  *   GEMM), fp32 accumulation.  dtype F32: an fp32 CUDA-core path.
+ *   For M <= 4 (bf16) the decode-GEMV takes the int8 path: per token and
+ *   chunk class r (the 512-position chunks r, r + 8, ... of K) X' = x A
+ *   (fp32) is scaled by a power of two s, the largest with max |X'| s <= 32639
+ *   over the class, rounded to q = rint(X' s) and split into two signed byte
+ *   digits q = 256 hi + lo; the codes (u8) times the digits (s8) accumulate
+ *   exactly on the integer tensor cores, each class's sum is scaled by 1/s
+ *   and the classes are added in class order, plus the per-row constant
+ *   s' - 3/2 sum_r (sum q_r) / s_r.  The activations' only rounding is that of
+ *   X' to q: half a step of 1/s, about 2^-16 of the class's largest |X'|
+ *   (bf16's is 2^-9 of each |X'|).  For 5 <= M <= 32 X' is rounded to bf16 (see
+ *   lcvq_xform).
  *   form: see lcvq_form (F32 always uses DECODE).
  *   workspace: >= lcvq_workspace_size(LCVQ_OP_GEMM, ...) bytes, 256-byte aligned.
  * Shapes: d_in % 64 == 0, d_out % 8 == 0, M >= 0, d_in and d_out <= 2^30.
@@ -150,9 +161,10 @@ LCVQ_API lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M,
                       const float* A, const float* B, void* Y, lcvq_form form,
                       void* workspace, size_t ws_bytes, void* stream);
 
-/* The algebraic form in two calls (bf16 only).  lcvq_gemm with
- * LCVQ_FORM_ALGEBRAIC is exactly lcvq_xform followed by lcvq_gemm_xformed; the
- * split lets a caller time or reuse the halves.
+/* The algebraic form in two calls (bf16 only).  For M > 4, lcvq_gemm with
+ * LCVQ_FORM_ALGEBRAIC is exactly lcvq_xform followed by lcvq_gemm_xformed (for
+ * M <= 4 lcvq_gemm takes its int8 path); the split lets a caller time or reuse
+ * the halves.
  *
  * lcvq_xform: X'[m][g d + j] = sum_i X[m][g d + i] A[i][j] is rounded to bf16
  * and stored in the "decoder order" the integer-code GEMM consumes: within each
@@ -179,11 +191,11 @@ LCVQ_API lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64
  * the layer convention); grouping is this library's launch arrangement for
  * many matrices at once (the projections of a layer that read one input, the
  * experts of a layer, or any set of independent decode-time matmuls).  For
- * M <= 16 each Y_i is bit-identical to lcvq_gemm on item i alone.  For
- * 17 <= M <= 32, groups of at least 296 tiles of 128 rows run on the tcgen05
- * tensor cores (decoded weights in tensor memory) and sum in a different fp32
- * order: Y_i then agrees with lcvq_gemm within the forward tolerance, not
- * bitwise.
+ * M <= 16 each Y_i is bit-identical to lcvq_gemm on item i alone (at M <= 4
+ * both take the int8 path described at lcvq_gemm).  For 17 <= M <= 32, groups of at least 296 tiles of 128 rows run on the
+ * tcgen05 tensor cores (decoded weights in tensor memory) and sum in a
+ * different fp32 order: Y_i then agrees with lcvq_gemm within the forward
+ * tolerance, not bitwise.
  *   items  host array of `count` descriptors (read during the call only):
  *          X [M][d_in] bf16, packed [d_out][d_in/4] codes, A [d*d] and B [d]
  *          fp32, Y [M][d_out] bf16 out; every pointer 16-byte aligned.

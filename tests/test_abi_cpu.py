@@ -70,7 +70,9 @@ def test_grouped_gemm_rejects_bad_groups_without_device():
 
     good = items((4096, 4096), (11008, 4096), (4096, 11008))
     need = L.lcvq_workspace_size_grouped(good, 3, 8, 8)
-    per = [256 * -(-(8 * k * 2) // 256) + 256 for _, k in ((0, 4096), (0, 4096), (0, 11008))]
+    # per item: X'' (M d_in bf16), then corr [M] and the int8 path's scales [M][8] (fp32)
+    per = [256 * -(-(8 * k * 2) // 256) + 256 * -(-(8 * 36) // 256)
+           for _, k in ((0, 4096), (0, 4096), (0, 11008))]
     assert need == 256 + sum(per)
     assert L.lcvq_workspace_size_grouped(good, 3, 33, 8) == 0                 # M > 32
     assert L.lcvq_workspace_size_grouped(good, 3, 0, 8) == 0                  # M < 1

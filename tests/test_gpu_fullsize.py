@@ -28,7 +28,9 @@ def test_decode_gemv_full():
     M in {1, 4, 16} bf16; every output element against the oracle, through
     each entry point that computes it (one lcvq_gemm call; the X-transform and
     the integer-code GEMM as two calls, which the benchmark's roofline times;
-    the workspace-free GEMV).  All three give the same bits."""
+    the workspace-free GEMV).  lcvq_gemm and the workspace-free GEMV give the
+    same bits; the two calls give them too for M > 4 (for M <= 4 lcvq_gemm
+    takes the int8 path)."""
     w = synth.workload(2, M=16, with_dy=False)
     packed, _ = lcvq.assign_pack(torch.from_numpy(w["Wp"]).to(dev()), 8, with_mask=False)
     pk = packed.cpu().numpy()
@@ -44,7 +46,9 @@ def test_decode_gemv_full():
         Y3 = lcvq.gemv_static(X, packed, 4096, A, B, 8)
         torch.cuda.synchronize()
         assert_close(f"decode-GEMV M={M}", _bf16_np(Y), ref[:M], Dn[:M], TOL_BF16)
-        assert torch.equal(Y, Y2), f"xform + gemm_xformed differs from lcvq_gemm at M={M}"
+        assert_close(f"split calls M={M}", _bf16_np(Y2), ref[:M], Dn[:M], TOL_BF16)
+        if M > 4:
+            assert torch.equal(Y, Y2), f"xform + gemm_xformed differs from lcvq_gemm at M={M}"
         assert torch.equal(Y, Y3), f"gemv_static differs from lcvq_gemm at M={M}"
 
 
@@ -133,7 +137,8 @@ def test_stack_full():
     the three arrangements the benchmark times: 224 lcvq_gemm calls, one
     lcvq_gemm_grouped per decoder-layer phase, and the whole stack in one
     grouped call.  Every output of every matrix against the oracle; for
-    M <= 16 the three arrangements give the same bits.  As in the benchmark,
+    M <= 16 the three arrangements give the same bits (the int8 path at
+    M = 1).  As in the benchmark,
     each projection shape has one input X, shared by the 32 layers."""
     layers, projs = 32, synth.STACK_PROJS
     mats = [synth.stack_matrix(l, p, 32, with_x=(l == 0)) for l in range(layers)

@@ -336,15 +336,20 @@ def _group_case(shapes, M, seed):
 @pytest.mark.parametrize("M", [1, 5, 16, 32])
 def test_gemm_grouped_bitwise_equals_separate_calls(M):
     """Each Y_i of lcvq_gemm_grouped equals lcvq_gemm on item i alone, bit for
-    bit, for mixed shapes (square, up-, down-projection, ragged)."""
+    bit, for mixed shapes (square, up-, down-projection, ragged); at M = 1 both
+    take the int8 path, and every item also meets the oracle there."""
     shapes = [(4096, 4096), (4096, 11008), (11008, 4096), (1088, 520), (512, 8)]
     jobs, zs, ws = _group_case(shapes, M, 300 + M)
     Ys = lcvq.gemm_grouped(jobs, 8)
     assert lcvq.last_launch_count() == 2
-    for (X, packed, A, B, d_in), Y in zip(jobs, Ys):
+    for i, (job, Y) in enumerate(zip(jobs, Ys)):
+        X, packed, A, B, d_in = job
         Y1 = lcvq.gemm(X, packed, d_in, A, B, 8)
         torch.cuda.synchronize()
         assert torch.equal(Y, Y1)
+        if M <= 4:
+            ref, D = O.forward(ws[i]["X"], zs[i], ws[i]["A"], ws[i]["B"])
+            assert_close(f"grouped int8 item {i} M={M}", to_np(Y), ref, D, TOL_BF16)
     # and the small items against the oracle
     for i in (3, 4):
         ref, D = O.forward(ws[i]["X"], zs[i], ws[i]["A"], ws[i]["B"])
@@ -388,15 +393,17 @@ def test_gemm_grouped_many_items_and_graph_replay():
 def test_gemm_grouped_wide_tiles_bitwise_equal_separate_calls(M):
     """A group large enough for the wide-tile kernel (>= 296 tiles of 128 rows;
     one producer warp streams codes and X'' into a shared-memory ring) gives
-    the split kernel's bits; the group includes a ragged row count and a K
-    that ends inside a chunk."""
+    the split kernel's bits (lcvq_gemm on the item alone; the int8 path for
+    M <= 4); the group includes a ragged row count and a K that ends inside a
+    chunk."""
     shapes = [(4096, 4096)] * 9 + [(1088, 1000), (11008, 4096)]
     jobs, zs, ws = _group_case(shapes, M, 700 + M)
     wsb = lcvq.new_workspace(lcvq.workspace_size_grouped(jobs, M, 8))
     Ys = lcvq.gemm_grouped(jobs, 8, workspace=wsb)
     assert lcvq.last_launch_count() == 2
     assert lcvq.check_device_error(wsb) == 0
-    for i, ((X, packed, A, B, d_in), Y) in enumerate(zip(jobs, Ys)):
+    for i, (job, Y) in enumerate(zip(jobs, Ys)):
+        X, packed, A, B, d_in = job
         Y1 = lcvq.gemm(X, packed, d_in, A, B, 8)
         torch.cuda.synchronize()
         assert torch.equal(Y, Y1), f"item {i}"
@@ -642,9 +649,9 @@ def test_xform_matches_its_definition(M, K, d):
                                           (200, 576, 520)])
 def test_xform_then_gemm_xformed_equals_gemm(M, d_in, d_out):
     """lcvq_gemm with the algebraic form is lcvq_xform followed by
-    lcvq_gemm_xformed: the two calls give lcvq_gemm's bits (decode-GEMV and
-    tensor-core GEMM alike), within the tolerance of the oracle, and write
-    nothing outside their outputs."""
+    lcvq_gemm_xformed: for M > 4 the two calls give lcvq_gemm's bits
+    (decode-GEMV and tensor-core GEMM alike); for M <= 4 lcvq_gemm takes the
+    int8 path and both meet the oracle.  Neither writes outside its output."""
     w, z = _fwd_case(2, M, d_in=d_in, d_out=d_out)
     packed = torch.from_numpy(O.pack_codes(z)).to(dev())
     X = to_dev(w["X"], torch.bfloat16)
@@ -656,9 +663,12 @@ def test_xform_then_gemm_xformed_equals_gemm(M, d_in, d_out):
     lcvq.gemm_xformed(xpp, corr, packed, out=Y2)
     torch.cuda.synchronize()
     assert guard_intact(Y2, ybuf)
-    assert torch.equal(Y1, Y2)
-    assert torch.equal(Ya, Y2)
+    assert torch.equal(Y1, Ya)
     ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    if M > 4:
+        assert torch.equal(Ya, Y2)
+    else:
+        assert_close(f"gemm (int8 path) M={M}", to_np(Ya), ref, D, TOL_BF16)
     assert_close(f"gemm_xformed M={M}", to_np(Y2), ref, D, TOL_BF16)
 
 
@@ -675,9 +685,9 @@ def test_xform_then_gemm_xformed_equals_gemm(M, d_in, d_out):
 ])
 def test_gemm_decode_gemv_equals_split_calls(M, d_in, d_out, d):
     """lcvq_gemm for M <= 32 (X-transform, then the decode-GEMV reading codes
-    before its dependency wait) gives the bits of lcvq_xform followed by
-    lcvq_gemm_xformed (which waits first), meets the oracle, and writes nothing
-    outside Y."""
+    before its dependency wait) meets the oracle and writes nothing outside Y;
+    for M > 4 it gives the bits of lcvq_xform followed by lcvq_gemm_xformed
+    (which waits first); for M <= 4 it takes the int8 path."""
     w, z = _fwd_case(2, M, d_in=d_in, d_out=d_out, d=d)
     packed = torch.from_numpy(O.pack_codes(z)).to(dev())
     X = to_dev(w["X"], torch.bfloat16)
@@ -690,8 +700,10 @@ def test_gemm_decode_gemv_equals_split_calls(M, d_in, d_out, d):
     torch.cuda.synchronize()
     assert n1 == 2
     assert guard_intact(Y1, ybuf)
-    assert torch.equal(Y1, Y2)
+    if M > 4:
+        assert torch.equal(Y1, Y2)
     ref, D = O.forward(w["X"], z, w["A"], w["B"])
+    assert_close(f"split calls M={M} K={d_in}", to_np(Y2), ref, D, TOL_BF16)
     assert_close(f"decode-GEMV M={M} K={d_in}", to_np(Y1), ref, D, TOL_BF16)
 
 
@@ -738,6 +750,74 @@ def test_gemm_decode_gemv_back_to_back_on_one_workspace(M):
         for Y, r in zip(outs, alone):
             assert torch.equal(Y, r)
     del g
+
+
+def _int8_positions(block: np.ndarray) -> np.ndarray:
+    """Digits of 16-byte blocks back to position order (byte 4 p + i holds
+    position 4 i + p)."""
+    b = block.reshape(-1, 4, 4)            # [block][p][i]
+    return b.transpose(0, 2, 1).reshape(-1)  # [block][i][p] -> position 4 i + p
+
+
+@pytest.mark.parametrize("M,K,d", [(1, 1088, 8), (4, 4096, 8), (3, 576, 4), (2, 128, 1),
+                                   (4, 640, 2), (2, 9216, 8)])
+def test_int8_transform_matches_its_definition(M, K, d):
+    """For M <= 4, the int8 path's X-transform writes per row and chunk class r
+    (the chunks r, r + 8, ... of 512 positions) a power-of-two scale s, the
+    largest with max |X'| s <= 32639 over the class, and q = rint(X' s) as two
+    signed byte digits (q = 256 hi + lo, lo in [-128, 127]) per position: per
+    chunk the hi plane, then the lo plane, each 16-position block in the order
+    the GEMV's decoder extracts codes; and corr = s' - 3/2 sum_r (sum q_r) / s_r.
+    Read back from the workspace and checked against that definition in fp64
+    (X' is formed in fp32, so q may sit one step from rint of the fp64 value
+    only where that value is within the fp32 error of a half-integer)."""
+    w, z = _fwd_case(2, M, d_in=K, d_out=64, d=d)
+    packed = torch.from_numpy(O.pack_codes(z)).to(dev())
+    X = to_dev(w["X"], torch.bfloat16)
+    A, B = torch.from_numpy(w["A"]).to(dev()), torch.from_numpy(w["B"]).to(dev())
+    jobs = [(X, packed, A, B, K)]
+    ws = lcvq.new_workspace(lcvq.workspace_size_grouped(jobs, M, d), dev())
+    lcvq.gemm_grouped(jobs, d, workspace=ws)
+    torch.cuda.synchronize()
+    raw = ws.cpu().numpy()   # one item: X8 at 256, then corr [M] and inv_s [M][8]
+    x8 = raw[256:256 + M * 2 * K].reshape(M, 2 * K)
+    coff = (256 + M * K * 2 + 255) // 256 * 256
+    corr = raw[coff:coff + 4 * M].view(np.float32)
+    inv_s = raw[coff + 4 * M:coff + 36 * M].view(np.float32).reshape(M, 8)
+    x = torch.from_numpy(w["X"]).to(torch.bfloat16).double().numpy()
+    A64, B64 = w["A"].astype(np.float64), w["B"].astype(np.float64)
+    xg = x.reshape(M, K // d, d)
+    Xp = np.einsum("mgi,ij->mgj", xg, A64).reshape(M, K)
+    # fp32 fused multiply-adds over d terms: within d 2^-24 of the absolute sum
+    dXp = np.einsum("mgi,ij->mgj", np.abs(xg), np.abs(A64)).reshape(M, K) * (d * 2.0 ** -24 * 1.01)
+    Bp = B64 + 1.5 * A64.sum(axis=1)
+    sp = np.einsum("mgi,i->m", xg, Bp)
+    cls = (np.arange(K) // 512) % 8
+    for m in range(M):
+        hi, lo = [], []
+        for c0 in range(0, K, 512):
+            nc = min(512, K - c0)
+            seg = x8[m, 2 * c0:2 * c0 + 2 * nc].view(np.int8)
+            hi.append(_int8_positions(seg[:nc]))
+            lo.append(_int8_positions(seg[nc:]))
+        hi, lo = np.concatenate(hi).astype(np.int64), np.concatenate(lo).astype(np.int64)
+        q = 256 * hi + lo
+        assert np.all((lo >= -128) & (lo <= 127)) and np.all(np.abs(q) <= 32639)
+        qs = 0.0
+        for r in range(8):
+            s = 1.0 / float(inv_s[m, r])
+            assert s == 2.0 ** np.round(np.log2(s)), "each scale is a power of two"
+            sel = cls == r
+            if not sel.any():
+                assert s == 1.0
+                continue
+            mx = np.abs(Xp[m, sel]).max()
+            assert mx * s <= 32639 * (1 + 1e-6) and mx * 2 * s > 32639 * (1 - 1e-6), "largest s"
+            assert np.all(np.abs(q[sel] - Xp[m, sel] * s) <= 0.5 + dXp[m, sel] * s + 1e-9)
+            qs += q[sel].sum() / s
+        ref = sp[m] - 1.5 * qs
+        scale_c = np.abs(xg[m]).sum() * np.abs(Bp).max() + 1.5 * np.abs(Xp[m]).sum()
+        assert abs(float(corr[m]) - ref) <= 4e-6 * scale_c + 1e-30
 
 
 def test_gemm_grouped_outputs_are_canaried():

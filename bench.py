@@ -58,31 +58,28 @@ def parse():
     return p.parse_args()
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
-# dominant kernel, from one ncu capture of this benchmark's decode-GEMV step,
-# valid only for the kernel source that was captured: keyed by the SHA-1 of
-# the source file.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one decode-GEMV
+# call (its X-transform and its GEMV) per token count, from one ncu capture of
+# this benchmark's step, valid only for the kernel sources that were captured:
+# keyed by the SHA-1 of each source file.
 NCU_TRAFFIC = {
-    # source file -> (sha1 of the file when captured, {token count: bytes per launch})
-    # M = 1 and 4 share one instantiation of the kernel
-    "bit_weight_only_lcvq_b200/csrc/gemv.cu": (
-        "75b5b4bd040af0c1272fbef07a6cd8f3ecdc9ddb", {1: 4242948, 4: 4242948, 16: 4367080}),
+    "sources": {},    # source file -> sha1 of the file when captured
+    "per_call": {},   # token count -> bytes per call
 }
 
 
-def traffic_for(src_rel: str, key):
+def traffic_for(key):
     import hashlib
-    entry = NCU_TRAFFIC.get(src_rel)
-    if entry is None:
+    if not NCU_TRAFFIC["sources"]:
         return None
-    path = os.path.join(ROOT, src_rel)
-    try:
-        h = hashlib.sha1(open(path, "rb").read()).hexdigest()
-    except OSError:
-        return None
-    if h != entry[0]:
-        return None  # the kernel changed since the counters were taken
-    return entry[1].get(key)
+    for src_rel, sha in NCU_TRAFFIC["sources"].items():
+        try:
+            h = hashlib.sha1(open(os.path.join(ROOT, src_rel), "rb").read()).hexdigest()
+        except OSError:
+            return None
+        if h != sha:
+            return None  # a kernel changed since the counters were taken
+    return NCU_TRAFFIC["per_call"].get(key)
 
 
 def peaks():
@@ -376,16 +373,15 @@ def headline(args, D: Dist, pk):
     per_step_bytes = len(Ms) * (N * K // 4)
     value = D.world * args.steps * per_step_bytes / (ms_total * 1e-3) / 1e9
 
-    # dominant kernel alone: decode-GEMV on a pre-transformed X'', per token count
-    xpp, corr = {}, {}
-    for M in Ms:
-        xpp[M], corr[M] = lcvq.xform(X[M], A, B, d)
+    # the decode-GEMV call per token count, back to back (its X-transform and
+    # its GEMV overlap under programmatic dependent launch, so the call, not
+    # one of its two kernels, is what a CUDA event can time)
     per_m = {}
     for M in Ms:
         kc = [0]
 
         def kstep(M=M, kc=kc):
-            lcvq.gemm_xformed(xpp[M], corr[M], copies[kc[0] % R], out=Y[M])
+            lcvq.gemm(X[M], copies[kc[0] % R], K, A, B, d, out=Y[M], workspace=ws[M])
             kc[0] += 1
             return lcvq.last_launch_count()
         n = 4 * R
@@ -396,6 +392,26 @@ def headline(args, D: Dist, pk):
     kern_ms = sum(per_m.values())
     achieved = per_step_bytes / (kern_ms * 1e-3) / 1e9
     hbm = pk["hbm_gbs"]
+
+    # context: the bf16 GEMV kernel alone (lcvq_gemm_xformed on a pre-transformed
+    # X'', back to back; launched on its own it waits before it loads codes)
+    xpp, corr = {}, {}
+    for M in Ms:
+        xpp[M], corr[M] = lcvq.xform(X[M], A, B, d)
+    alone = {}
+    for M in Ms:
+        kc = [0]
+
+        def astep(M=M, kc=kc):
+            lcvq.gemm_xformed(xpp[M], corr[M], copies[kc[0] % R], out=Y[M])
+            kc[0] += 1
+            return lcvq.last_launch_count()
+        n = 4 * R
+        g = StepGraphs(astep, R, n)
+        g.replay()
+        t, _, _ = timed_graphs(D, g)
+        alone[M] = t / n
+    alone_gbs = per_step_bytes / (sum(alone.values()) * 1e-3) / 1e9
 
     # end to end through the public API with pinned host buffers.  Each step's
     # inputs (all token counts) go in with one host-to-device copy and its
@@ -468,13 +484,17 @@ def headline(args, D: Dist, pk):
                 "l2": f"inputs larger than L2: {R} rotated packed-weight copies ({R * 4} MiB)",
                 "parallelism": f"replicas x{D.world}" if D.world > 1 else "single GPU"},
         roofline=dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
-                      traffic=_sum_or_none([traffic_for("bit_weight_only_lcvq_b200/csrc/gemv.cu", M)
-                                            for M in Ms]),
-                      traffic_unit="bytes per step (3 launches)",
-                      kernel="gemv_group_kernel (decode-GEMV, M=1,4,16 summed)",
-                      launch="lcvq_gemm_xformed back to back; launched on its own, each GEMV "
-                             "waits for the previous launch before it loads codes",
+                      traffic=_sum_or_none([traffic_for(M) for M in Ms]),
+                      traffic_unit="bytes per step (3 calls, each an X-transform and a GEMV)",
+                      kernel="decode-GEMV call: X-transform + gemv_group_kernel (int8 path "
+                             "at M = 1, 4; bf16 at M = 16), M = 1, 4, 16 summed",
+                      launch="lcvq_gemm back to back per token count, graph replay, rotated "
+                             "weights",
                       per_m_us={str(M): per_m[M] * 1e3 for M in Ms},
+                      bf16_gemv_alone=dict(per_m_us={str(M): alone[M] * 1e3 for M in Ms},
+                                           achieved=alone_gbs, frac=alone_gbs / hbm,
+                                           note="context: lcvq_gemm_xformed's bf16 GEMV kernel "
+                                                "alone, without its X-transform"),
                       peak_source=f"{PEAK_SRC} hbm_gbs"),
         e2e=e2e, clocks=ck, gpu_launches=int(launches),
     )

@@ -502,9 +502,21 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
                              c * (kAhead * 32), static_cast<int>(row0));
         }
         __syncwarp();
-        if (lane < M)
+        if constexpr (kI8) {
+          // int8 digits: the hi and lo planes (n_c bytes each) of token lane / 2,
+          // the lo plane 16 bytes past the hi plane's end so that the lanes
+          // reading the two planes hit different banks
+          if (lane < 2 * M) {
+            const uint32_t nc = xbytes / 2, pl = static_cast<uint32_t>(lane & 1);
+            const unsigned char* src = reinterpret_cast<const unsigned char*>(it.Xpp) +
+                                       int64_t(lane >> 1) * 2 * it.K + 2 * xk + pl * nc;
+            sm100::bulk_load(st + L::kCodeBytes + (lane >> 1) * kWideXPitch + pl * (nc + 16), src,
+                             nc, &full[s]);
+          }
+        } else if (lane < M) {
           sm100::bulk_load(st + L::kCodeBytes + lane * kWideXPitch,
                            it.Xpp + int64_t(lane) * it.K + xk, xbytes, &full[s]);
+        }
         ++filled;
       }
     }
@@ -577,8 +589,10 @@ __global__ void __launch_bounds__(kWideThreads, kMinBlocks)
         const uint32_t xst = st + L::kCodeBytes;
         const int rem = K - c * (kAhead * kUnit);   // positions of K left from this chunk on
         const int remt = rem - 32 * t;              // ... from this lane's first position on
-        // int8: this lane's digit plane (the lo plane follows the chunk's n_c hi bytes)
-        const uint32_t plane = (kI8 && (g & 1)) ? static_cast<uint32_t>(rem < 512 ? rem : 512) : 0u;
+        // int8: this lane's digit plane (the lo plane starts 16 bytes after the
+        // chunk's n_c hi bytes)
+        const uint32_t plane =
+            (kI8 && (g & 1)) ? static_cast<uint32_t>(rem < 512 ? rem : 512) + 16u : 0u;
 #pragma unroll
         for (int j = 0; j < kAhead; ++j) {
           if (j * kUnit >= rem) break;  // warp-uniform: past the end of K

@@ -33,6 +33,7 @@
 //     zero (the minimum-norm solution), as the diagonal refit does.
 // Every sum runs in a fixed order: the result is bitwise reproducible.
 #include <math.h>
+#include <stddef.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -236,6 +237,183 @@ __global__ void __launch_bounds__(FitHDims<D>::kThreads) fith_contract_kernel(
   if (tid < NP) {
     double v = 0.0;
     for (int t2 = 0; t2 < F::kRParts; ++t2) v += sRed[t2][tid];
+    out[NP * NP + tid] = v;
+  }
+}
+
+// ---------------------------------------------------------------- 3a'. d = 8: tiles and fp64 MMA
+// The same partial [L_half | R] as fith_contract_kernel, for d = 8.  The L sum
+// is a product once reindexed: with U_p = H's block (g, h) (8 x 8, rows i,
+// columns j) and V_p = S~'s block ((g, a), (h, b)) (9 x 9), over the position
+// pairs p = (g, h >= g),
+//     L_half[(i,a),(j,b)] = sum_p w_p U_p[i][j] V_p[a][b],   w = 1/2 if g = h, else 1,
+// a 64 x 81 x #pairs product, run on the fp64 tensor-core MMA (m8n8k4).  CTA
+// c takes the 64 x 64 tiles (gb, hb >= gb) of positions 8 gb .. 8 gb + 7 by
+// 8 hb .. 8 hb + 7 in turn: it stages the tile of H, of the code Gram and of
+// T~ (both T~ tiles (gb rows, hb columns) and (hb rows, gb columns)) in fp64
+// shared memory; warp i accumulates the rows (i, j) of L over the tile's 64
+// pairs (the pairs are the MMA's k), 11 column tiles of 8 over the 81 (a, b).
+// R comes from the same tile, also on the fp64 MMA: warp pl takes position
+// pl of the tile's row block gb against the columns of hb and, by H's
+// symmetry, position pl of hb against the columns of gb (R's rows i are the
+// MMA's 8 rows, its 9 values of a two column tiles, the columns of H its k),
+// so every (row block, column block) of H and T~ is read once; the warps'
+// parts of R are added in warp order at the end.
+constexpr int kC8Tile = 64;               // tile side in elements (8 positions)
+constexpr int kC8Pitch = kC8Tile + 1;     // doubles per shared row: rows 2 banks apart
+constexpr int kC8Threads = 256;           // 8 warps: warp i owns the L rows (i, j)
+struct C8Smem {
+  double U[kC8Tile][kC8Pitch];   // H[64 gb + r][64 hb + c]
+  double S[kC8Tile][kC8Pitch];   // C[64 + 64 gb + r][64 + 64 hb + c]: code Gram S~ (a, b < 8)
+  double T1[kC8Tile][kC8Pitch];  // T~ rows 64 gb + r, columns 64 hb + c (hi + lo)
+  double T2[kC8Tile][kC8Pitch];  // T~ rows 64 hb + r, columns 64 gb + c
+  double Ro[kC8Tile];            // C[0][64 + 64 hb + c]: S~'s ones row over hb
+  double Co[kC8Tile];            // C[64 + 64 gb + r][0]: S~'s ones column over gb
+  double To1[kC8Tile];           // T~ of the ones row over hb columns
+  double To2[kC8Tile];           // ... over gb columns
+  double N;                      // C[0][0]: the number of rows
+  double zero;                   // 0: the padding columns of L's and R's MMAs
+  double Rred[8][72];            // the warps' parts of R
+};
+
+__device__ __forceinline__ void dmma_m8n8k4(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(kC8Threads, 1) fith_contract8_kernel(
+    const float* __restrict__ H, const float* __restrict__ C, int64_t K, double* __restrict__ partials) {
+  constexpr int D = 8, P1 = 9, NP = 72, kNT = 11;  // 11 column tiles of 8 over the 81 (a, b)
+  extern __shared__ __align__(16) unsigned char c8smem[];
+  C8Smem& sm = *reinterpret_cast<C8Smem*>(c8smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t ldc = kOnes + 3 * K;
+  const int nb = static_cast<int>(K / kC8Tile);
+  const int ntiles = nb * (nb + 1) / 2;
+  // L: this lane's MMA coordinates.  A: row j = lane / 4, pair lane % 4 of a
+  // k step; B and D: columns n = 8 nt + lane / 4 and (D) 8 nt + 2 (lane % 4) + e
+  const int i = warp, jrow = lane >> 2, kq = lane & 3;
+  // where column n = 8 nt + lane / 4 of V_p sits, as a double offset in the
+  // shared struct plus strides per gl and hl (branch-free loads):
+  //   a, b < 8: S[8 gl + a][8 hl + b];  b = 8: Co[8 gl + a];  a = 8: Ro[8 hl + b];
+  //   a = b = 8: N;  n >= 81: zero
+  const double* smd = reinterpret_cast<const double*>(c8smem);
+  constexpr int oS = offsetof(C8Smem, S) / 8, oCo = offsetof(C8Smem, Co) / 8;
+  constexpr int oRo = offsetof(C8Smem, Ro) / 8, oN = offsetof(C8Smem, N) / 8;
+  constexpr int oZ = offsetof(C8Smem, zero) / 8;
+  int bo[kNT], bsg[kNT], bsh[kNT];
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) {
+    const int n = nt * 8 + jrow, a = n / P1, b = n % P1;
+    if (n >= P1 * P1) bo[nt] = oZ, bsg[nt] = 0, bsh[nt] = 0;
+    else if (a < D && b < D) bo[nt] = oS + a * kC8Pitch + b, bsg[nt] = D * kC8Pitch, bsh[nt] = D;
+    else if (a < D) bo[nt] = oCo + a, bsg[nt] = D, bsh[nt] = 0;
+    else if (b < D) bo[nt] = oRo + b, bsg[nt] = 0, bsh[nt] = D;
+    else bo[nt] = oN, bsg[nt] = 0, bsh[nt] = 0;
+  }
+  double acc[kNT][2];
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) acc[nt][0] = acc[nt][1] = 0.0;
+  // R: warp pl's MMA: A = H rows (8 pl + i) over 4 columns, B = T~ rows
+  // (8 pl + a) over the same columns (a = 8: the ones row; a > 8: zero)
+  double accR[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+
+  for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    int gb = 0, rem = t;  // tile t of the upper triangle, row by row
+    while (rem >= nb - gb) {
+      rem -= nb - gb;
+      ++gb;
+    }
+    const int hb = gb + rem;
+    const bool diag = gb == hb;
+    __syncthreads();  // the previous tile is consumed
+    const int64_t g0 = int64_t(gb) * kC8Tile, h0 = int64_t(hb) * kC8Tile;
+    for (int e = tid; e < kC8Tile * (kC8Tile / 4); e += kC8Threads) {
+      const int r = e / (kC8Tile / 4), c = (e % (kC8Tile / 4)) * 4;
+      const float4 u = __ldg(reinterpret_cast<const float4*>(H + (g0 + r) * K + h0 + c));
+      const float* crow = C + (kOnes + g0 + r) * ldc;
+      const float4 sv = __ldcg(reinterpret_cast<const float4*>(crow + kOnes + h0 + c));
+      const float4 t1h = __ldcg(reinterpret_cast<const float4*>(crow + kOnes + K + h0 + c));
+      const float4 t1l = __ldcg(reinterpret_cast<const float4*>(crow + kOnes + 2 * K + h0 + c));
+      sm.U[r][c] = u.x, sm.U[r][c + 1] = u.y, sm.U[r][c + 2] = u.z, sm.U[r][c + 3] = u.w;
+      sm.S[r][c] = sv.x, sm.S[r][c + 1] = sv.y, sm.S[r][c + 2] = sv.z, sm.S[r][c + 3] = sv.w;
+      sm.T1[r][c] = double(t1h.x) + double(t1l.x), sm.T1[r][c + 1] = double(t1h.y) + double(t1l.y);
+      sm.T1[r][c + 2] = double(t1h.z) + double(t1l.z), sm.T1[r][c + 3] = double(t1h.w) + double(t1l.w);
+      if (!diag) {
+        const float* crow2 = C + (kOnes + h0 + r) * ldc;
+        const float4 t2h = __ldcg(reinterpret_cast<const float4*>(crow2 + kOnes + K + g0 + c));
+        const float4 t2l = __ldcg(reinterpret_cast<const float4*>(crow2 + kOnes + 2 * K + g0 + c));
+        sm.T2[r][c] = double(t2h.x) + double(t2l.x), sm.T2[r][c + 1] = double(t2h.y) + double(t2l.y);
+        sm.T2[r][c + 2] = double(t2h.z) + double(t2l.z), sm.T2[r][c + 3] = double(t2h.w) + double(t2l.w);
+      }
+    }
+    if (tid < kC8Tile) {
+      sm.Ro[tid] = C[kOnes + h0 + tid];
+      sm.Co[tid] = C[(kOnes + g0 + tid) * ldc];
+      sm.To1[tid] = double(C[kOnes + K + h0 + tid]) + double(C[kOnes + 2 * K + h0 + tid]);
+      sm.To2[tid] = double(C[kOnes + K + g0 + tid]) + double(C[kOnes + 2 * K + g0 + tid]);
+    }
+    if (tid == 0) {
+      sm.N = C[0];
+      sm.zero = 0.0;
+    }
+    __syncthreads();
+
+    // L: the tile's 64 pairs p = 8 gl + hl, four per k step
+#pragma unroll 2
+    for (int ks = 0; ks < 16; ++ks) {
+      const int p = ks * 4 + kq, gl = p >> 3, hl = p & 7;
+      const double w = diag ? (hl > gl ? 1.0 : (hl == gl ? 0.5 : 0.0)) : 1.0;
+      const double av = w * sm.U[gl * D + i][hl * D + jrow];
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+        dmma_m8n8k4(acc[nt], av, smd[bo[nt] + gl * bsg[nt] + hl * bsh[nt]]);
+    }
+    // R, position pl = warp: rows of gb against the columns of hb; off the
+    // diagonal also the rows of hb against the columns of gb
+    // (H[64 hb + 8 pl + i][64 gb + c] = U[c][8 pl + i])
+    {
+      const int pl = warp, ar = jrow;  // B column: a = ar (tile 0), 8 + ar (tile 1)
+#pragma unroll 4
+      for (int c0 = 0; c0 < kC8Tile; c0 += 4) {
+        const int c = c0 + kq;
+        const double av = sm.U[pl * D + jrow][c];
+        dmma_m8n8k4(accR[0], av, sm.T1[pl * D + ar][c]);
+        dmma_m8n8k4(accR[1], av, ar == 0 ? sm.To1[c] : 0.0);
+      }
+      if (!diag) {
+#pragma unroll 4
+        for (int c0 = 0; c0 < kC8Tile; c0 += 4) {
+          const int c = c0 + kq;
+          const double av = sm.U[c][pl * D + jrow];
+          dmma_m8n8k4(accR[0], av, sm.T2[pl * D + ar][c]);
+          dmma_m8n8k4(accR[1], av, ar == 0 ? sm.To2[c] : 0.0);
+        }
+      }
+    }
+  }
+  // the CTA's partial: every L value belongs to one lane of one warp
+  double* out = partials + int64_t(blockIdx.x) * (NP * NP + NP);
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int n = nt * 8 + 2 * kq + e;
+      if (n < P1 * P1) out[(i * P1 + n / P1) * NP + jrow * P1 + n % P1] = acc[nt][e];
+    }
+  // R: lane holds rows i = lane / 4 and columns a = 2 (lane % 4) + e (tile 0)
+  // and 8 + 2 (lane % 4) + e (tile 1: only a = 8 exists)
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    sm.Rred[warp][jrow * P1 + 2 * kq + e] = accR[0][e];
+    if (kq == 0 && e == 0) sm.Rred[warp][jrow * P1 + D] = accR[1][0];
+  }
+  __syncthreads();
+  if (tid < NP) {
+    double v = 0.0;
+    for (int w = 0; w < 8; ++w) v += sm.Rred[w][tid];
     out[NP * NP + tid] = v;
   }
 }
@@ -464,9 +642,19 @@ size_t solve_smem() {
   return size_t(3) * NP * NP * 8 + size_t(2) * NP * 8 + 16;
 }
 
-int contract_grid(int64_t ng) {
-  int64_t g = 2 * kNumSMsB200;
-  if (ng < g) g = ng;
+// CTAs of the contraction: d = 8 takes the (K/64)(K/64 + 1)/2 tiles on one CTA
+// per SM, other d the K/d vector positions on two
+int contract_grid(int64_t d_in, int d) {
+  int64_t g, work;
+  if (d == 8) {
+    const int64_t nb = d_in / kC8Tile;
+    g = kNumSMsB200;
+    work = nb * (nb + 1) / 2;
+  } else {
+    g = 2 * kNumSMsB200;
+    work = d_in / (d > 0 ? d : 1);
+  }
+  if (work < g) g = work;
   return g < 1 ? 1 : static_cast<int>(g);
 }
 
@@ -482,7 +670,7 @@ cudaError_t launch_fith_t(const float* W0, const uint8_t* packed, int64_t d_out,
   float* C = reinterpret_cast<float*>(base + q_bytes);
   const size_t c_bytes = (size_t(kOnes + d_in) * ldq * 4 + 255) / 256 * 256;
   double* partials = reinterpret_cast<double*>(base + q_bytes + c_bytes);
-  const int grid = contract_grid(d_in / D);
+  const int grid = contract_grid(d_in, D);
   double* red = partials + size_t(grid) * F::kPart;  // the reduced [L | R]
   {
     const int64_t items = d_out * (d_in / 8 + kOnes / 8);
@@ -495,7 +683,15 @@ cudaError_t launch_fith_t(const float* W0, const uint8_t* packed, int64_t d_out,
   if (cudaError_t e = launch_tc_gram(Q, d_out, kOnes + d_in, ldq, C, err, s, launches);
       e != cudaSuccess)
     return e;
-  fith_contract_kernel<D><<<grid, F::kThreads, 0, s>>>(H, C, d_in, partials);
+  if constexpr (D == 8) {
+    if (cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fith_contract8_kernel),
+                                             sizeof(C8Smem));
+        e != cudaSuccess)
+      return e;
+    fith_contract8_kernel<<<grid, kC8Threads, sizeof(C8Smem), s>>>(H, C, d_in, partials);
+  } else {
+    fith_contract_kernel<D><<<grid, F::kThreads, 0, s>>>(H, C, d_in, partials);
+  }
   ++*launches;
   if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
   fith_reduce_kernel<D><<<static_cast<unsigned>(ceil_div(F::kPart, 256)), 256, 0, s>>>(partials, grid,
@@ -518,7 +714,7 @@ size_t fith_scratch_bytes(int64_t d_out, int64_t d_in, int d) {
   const size_t q_bytes = (size_t(d_out) * ldq * 2 + 255) / 256 * 256;
   const size_t c_bytes = (size_t(kOnes + d_in) * ldq * 4 + 255) / 256 * 256;
   const int np = d * (d + 1);
-  const size_t p_bytes = (size_t(contract_grid(d_in / (d > 0 ? d : 1))) + 1) * size_t(np * np + np) * 8;
+  const size_t p_bytes = (size_t(contract_grid(d_in, d)) + 1) * size_t(np * np + np) * 8;
   return q_bytes + c_bytes + p_bytes;
 }
 

@@ -450,33 +450,35 @@ constexpr int kSolveThreads = 256;
 // receives theta.
 template <int NP>
 __device__ bool chol_solve_cta(double (*G)[NP], const double* R, double* th) {
-  const int t = threadIdx.x, lane = t & 31;
-  __shared__ int ok;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  constexpr int kW = kSolveThreads / 32;
   __shared__ double dmax;
+  __shared__ double rdiag[NP];  // 1 / L[c][c]
   if (t == 0) {
     double m = 0.0;
     for (int c = 0; c < NP; ++c) m = fmax(m, G[c][c]);
     dmax = m;
-    ok = m > 0.0;
   }
   __syncthreads();
-  if (!ok) return false;
+  const double dm = dmax;
+  if (!(dm > 0.0)) return false;
   for (int c = 0; c < NP; ++c) {
+    // every thread forms the pivot itself: one decision, no barrier for it
+    const double piv = G[c][c];
+    if (!(piv > kHCholFloor * dm)) return false;  // the same for every thread
+    const double lcc = sqrt(piv), rl = 1.0 / lcc;
     if (t == 0) {
-      const double piv = G[c][c];
-      if (!(piv > kHCholFloor * dmax)) ok = 0;
-      else G[c][c] = sqrt(piv);
+      rdiag[c] = rl;
     }
+    __syncthreads();  // every thread has read G[c][c]
+    if (t == 0) G[c][c] = lcc;
+    for (int r = c + 1 + t; r < NP; r += blockDim.x) G[r][c] *= rl;
     __syncthreads();
-    if (!ok) return false;
-    const double lcc = G[c][c];
-    for (int r = c + 1 + t; r < NP; r += blockDim.x) G[r][c] /= lcc;
-    __syncthreads();
-    // trailing update of the lower triangle: G[r][s] -= L[r][c] L[s][c], c < s <= r
-    const int m = NP - c - 1;
-    for (int e = t; e < m * m; e += blockDim.x) {
-      const int r = c + 1 + e / m, s2 = c + 1 + e % m;
-      if (s2 <= r) G[r][s2] -= G[r][c] * G[s2][c];
+    // trailing update of the lower triangle: G[r][s] -= L[r][c] L[s][c], c < s <= r;
+    // warp w takes the rows c + 1 + w, c + 1 + w + 8, ...; lanes the columns
+    for (int r = c + 1 + warp; r < NP; r += kW) {
+      const double lrc = G[r][c];
+      for (int s2 = c + 1 + lane; s2 <= r; s2 += 32) G[r][s2] -= lrc * G[s2][c];
     }
     __syncthreads();
   }
@@ -484,14 +486,14 @@ __device__ bool chol_solve_cta(double (*G)[NP], const double* R, double* th) {
     for (int r = lane; r < NP; r += 32) th[r] = R[r];
     __syncwarp();
     for (int c = 0; c < NP; ++c) {  // L y = R, y in th
-      if (lane == 0) th[c] /= G[c][c];
+      if (lane == 0) th[c] *= rdiag[c];
       __syncwarp();
       const double yc = th[c];
       for (int r = c + 1 + lane; r < NP; r += 32) th[r] -= G[r][c] * yc;
       __syncwarp();
     }
     for (int c = NP - 1; c >= 0; --c) {  // L^T theta = y, in place
-      if (lane == 0) th[c] /= G[c][c];
+      if (lane == 0) th[c] *= rdiag[c];
       __syncwarp();
       const double tc = th[c];
       for (int r = lane; r < c; r += 32) th[r] -= G[c][r] * tc;

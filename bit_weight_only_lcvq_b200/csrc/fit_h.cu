@@ -260,7 +260,9 @@ __global__ void __launch_bounds__(FitHDims<D>::kThreads) fith_contract_kernel(
 // so every (row block, column block) of H and T~ is read once; the warps'
 // parts of R are added in warp order at the end.
 constexpr int kC8Tile = 64;               // tile side in elements (8 positions)
-constexpr int kC8Pitch = kC8Tile + 1;     // doubles per shared row: rows 2 banks apart
+// doubles per shared row, 4 mod 16: fragments that take 8 rows and 4
+// columns (or 8 columns and 4 rows) fill the 16 double slots of the banks twice
+constexpr int kC8Pitch = kC8Tile + 4;
 constexpr int kC8Threads = 256;           // 8 warps: warp i owns the L rows (i, j)
 struct C8Smem {
   double U[kC8Tile][kC8Pitch];   // H[64 gb + r][64 hb + c]
@@ -329,23 +331,23 @@ __global__ void __launch_bounds__(kC8Threads, 1) fith_contract8_kernel(
     const bool diag = gb == hb;
     __syncthreads();  // the previous tile is consumed
     const int64_t g0 = int64_t(gb) * kC8Tile, h0 = int64_t(hb) * kC8Tile;
-    for (int e = tid; e < kC8Tile * (kC8Tile / 4); e += kC8Threads) {
-      const int r = e / (kC8Tile / 4), c = (e % (kC8Tile / 4)) * 4;
-      const float4 u = __ldg(reinterpret_cast<const float4*>(H + (g0 + r) * K + h0 + c));
+    // one element per thread and array: a warp reads 128 contiguous bytes of a
+    // row and writes 32 consecutive doubles (no bank conflicts)
+#pragma unroll 4
+    for (int e = tid; e < kC8Tile * kC8Tile; e += kC8Threads) {
+      const int r = e / kC8Tile, c = e % kC8Tile;
       const float* crow = C + (kOnes + g0 + r) * ldc;
-      const float4 sv = __ldcg(reinterpret_cast<const float4*>(crow + kOnes + h0 + c));
-      const float4 t1h = __ldcg(reinterpret_cast<const float4*>(crow + kOnes + K + h0 + c));
-      const float4 t1l = __ldcg(reinterpret_cast<const float4*>(crow + kOnes + 2 * K + h0 + c));
-      sm.U[r][c] = u.x, sm.U[r][c + 1] = u.y, sm.U[r][c + 2] = u.z, sm.U[r][c + 3] = u.w;
-      sm.S[r][c] = sv.x, sm.S[r][c + 1] = sv.y, sm.S[r][c + 2] = sv.z, sm.S[r][c + 3] = sv.w;
-      sm.T1[r][c] = double(t1h.x) + double(t1l.x), sm.T1[r][c + 1] = double(t1h.y) + double(t1l.y);
-      sm.T1[r][c + 2] = double(t1h.z) + double(t1l.z), sm.T1[r][c + 3] = double(t1h.w) + double(t1l.w);
+      const float u = __ldg(H + (g0 + r) * K + h0 + c);
+      const float sv = __ldcg(crow + kOnes + h0 + c);
+      const float t1h = __ldcg(crow + kOnes + K + h0 + c);
+      const float t1l = __ldcg(crow + kOnes + 2 * K + h0 + c);
+      sm.U[r][c] = u;
+      sm.S[r][c] = sv;
+      sm.T1[r][c] = double(t1h) + double(t1l);
       if (!diag) {
         const float* crow2 = C + (kOnes + h0 + r) * ldc;
-        const float4 t2h = __ldcg(reinterpret_cast<const float4*>(crow2 + kOnes + K + g0 + c));
-        const float4 t2l = __ldcg(reinterpret_cast<const float4*>(crow2 + kOnes + 2 * K + g0 + c));
-        sm.T2[r][c] = double(t2h.x) + double(t2l.x), sm.T2[r][c + 1] = double(t2h.y) + double(t2l.y);
-        sm.T2[r][c + 2] = double(t2h.z) + double(t2l.z), sm.T2[r][c + 3] = double(t2h.w) + double(t2l.w);
+        sm.T2[r][c] = double(__ldcg(crow2 + kOnes + K + g0 + c)) +
+                      double(__ldcg(crow2 + kOnes + 2 * K + g0 + c));
       }
     }
     if (tid < kC8Tile) {

@@ -104,22 +104,29 @@ constexpr int kChunkCols = 192;  // columns of H and C per shared-memory chunk
 constexpr int kRowPad = 1;       // doubles of padding per shared row: rows 2 banks apart
 constexpr int kTeams = 2;
 
+// the system: d (d + 1) unknowns; a CTA's partial is [L (NP x NP) | R (NP)]
 template <int D>
 struct FitHDims {
   static constexpr int NP = D * (D + 1);
+  static constexpr int kPart = NP * NP + NP;  // doubles per CTA partial
+};
+// the CUDA-core contraction's thread layout (d != 8)
+template <int D>
+struct FitHContract {
+  static constexpr int NP = FitHDims<D>::NP;
   static constexpr int P1 = D + 1;
   static constexpr int kJT = D < 4 ? D : 4;           // j values per thread tile
   static constexpr int kTeam = D * (D / kJT) * P1;    // threads per team
   static constexpr int kThreads = ((kTeams * kTeam + 31) / 32) * 32;
   static constexpr int kRParts = kThreads / NP;       // threads per R value
   static constexpr int kCols = kChunkCols;            // a multiple of every d
-  static constexpr int kPart = NP * NP + NP;          // doubles per CTA partial
+  static constexpr int kPart = FitHDims<D>::kPart;
 };
 
 template <int D>
-__global__ void __launch_bounds__(FitHDims<D>::kThreads) fith_contract_kernel(
+__global__ void __launch_bounds__(FitHContract<D>::kThreads) fith_contract_kernel(
     const float* __restrict__ H, const float* __restrict__ C, int64_t K, double* __restrict__ partials) {
-  using F = FitHDims<D>;
+  using F = FitHContract<D>;
   constexpr int NP = F::NP, P1 = F::P1, COLS = F::kCols, JT = F::kJT;
   __shared__ double sH[D][COLS + kRowPad];
   __shared__ double sS[P1][COLS + kRowPad];
@@ -694,7 +701,7 @@ cudaError_t launch_fith_t(const float* W0, const uint8_t* packed, int64_t d_out,
       return e;
     fith_contract8_kernel<<<grid, kC8Threads, sizeof(C8Smem), s>>>(H, C, d_in, partials);
   } else {
-    fith_contract_kernel<D><<<grid, F::kThreads, 0, s>>>(H, C, d_in, partials);
+    fith_contract_kernel<D><<<grid, FitHContract<D>::kThreads, 0, s>>>(H, C, d_in, partials);
   }
   ++*launches;
   if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;

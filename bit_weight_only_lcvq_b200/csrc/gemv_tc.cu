@@ -70,7 +70,7 @@ struct TcItem {
   int tile_end;       // 128-row tiles of items 0 .. this one
 };
 struct TcGroup {
-  CUtensorMap codes[kTcItems];  // [N rows][K/4 bytes], box 32 B x 128 rows
+  CUtensorMap codes[kTcItems];  // [N rows][K/4 bytes], box 128 B x 128 rows
   CUtensorMap xpp[kTcItems];    // [M rows][K] bf16, box 64 x 32, 128-byte swizzle
   int count, M;
   unsigned int* err;
@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem;                                  // kAStages x 8 KB (SW128 boxes)
-  uint8_t* sC = sX + kAStages * kTcXBytes;             // kCStages x 4 KB
+  uint8_t* sC = sX + kAStages * kTcXBytes;             // kCStages x 16 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(sC + kCStages * kTcCodeBytes);
   uint64_t* cfull = bars;                              // codes landed (TMA)
   uint64_t* cempty = cfull + kCStages;                 // codes read (decoders)

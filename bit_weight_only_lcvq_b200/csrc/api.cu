@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "trace.h"
 
 using namespace lcvq;
 
@@ -136,6 +137,7 @@ int lcvq_last_launch_count(void) { return g_last_launches; }
 
 lcvq_status lcvq_assign_pack(const float* Wp, int64_t d_out, int64_t d_in, int d,
                              uint8_t* packed, uint8_t* mask_bits, void* stream) {
+  LCVQ_API_RANGE();
   if (d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
   if (d_in % 8 != 0 || d_in % d != 0) return LCVQ_ERR_INVALID_ARG;
   g_last_launches = 0;
@@ -153,6 +155,7 @@ lcvq_status lcvq_assign_pack(const float* Wp, int64_t d_out, int64_t d_in, int d
 lcvq_status lcvq_decode(const uint8_t* packed, int64_t d_out, int64_t d_in, int d,
                         const float* A, const float* B, void* W, lcvq_dtype w_dtype,
                         void* stream) {
+  LCVQ_API_RANGE();
   if (d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
   if (d_in % 16 != 0) return LCVQ_ERR_INVALID_ARG;
   if (w_dtype != LCVQ_F32 && w_dtype != LCVQ_BF16) return LCVQ_ERR_INVALID_ARG;
@@ -183,6 +186,7 @@ size_t lcvq_workspace_size(lcvq_op op, lcvq_dtype dtype, int64_t M, int64_t d_ou
 lcvq_status lcvq_fit_affine_h(const float* W0, const uint8_t* packed, int64_t d_out, int64_t d_in,
                               int d, const float* H, float* A, float* B, void* workspace,
                               size_t ws_bytes, void* stream) {
+  LCVQ_API_RANGE();
   g_last_launches = 0;
   if (d_out < 0 || d_in < 0 || !valid_d(d) || d_in % 64 != 0) return LCVQ_ERR_INVALID_ARG;
   if (d_in > kMaxFitHDin || d_out > kMaxFitHDout) return LCVQ_ERR_INVALID_ARG;
@@ -204,6 +208,7 @@ lcvq_status lcvq_fit_affine_h(const float* W0, const uint8_t* packed, int64_t d_
 
 lcvq_status lcvq_assign_ldlq(const float* P, const float* U, int64_t d_out, int64_t d_in, int d,
                              uint8_t* packed, void* workspace, size_t ws_bytes, void* stream) {
+  LCVQ_API_RANGE();
   g_last_launches = 0;
   if (d_out < 0 || d_in < 0 || !valid_d(d)) return LCVQ_ERR_INVALID_ARG;
   if (d_in % 64 != 0 || d_in % d != 0 || d_in > kMaxLdlqDim || d_out > kMaxGemmDim)
@@ -224,6 +229,7 @@ lcvq_status lcvq_assign_ldlq(const float* P, const float* U, int64_t d_out, int6
 }
 
 lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, float k, void* stream) {
+  LCVQ_API_RANGE();
   g_last_launches = 0;
   if (n < 0 || n % 4 != 0 || !(k > 0.f) || !std::isfinite(k)) return LCVQ_ERR_INVALID_ARG;
   if (n == 0) return LCVQ_OK;
@@ -238,6 +244,7 @@ lcvq_status lcvq_dge_scale(float* dWp, const float* Wp, int64_t n, float k, void
 lcvq_status lcvq_fit_affine(const float* W0, const uint8_t* packed, int64_t d_out, int64_t d_in,
                             int d, const float* h, float* A, float* B, void* workspace,
                             size_t ws_bytes, void* stream) {
+  LCVQ_API_RANGE();
   g_last_launches = 0;
   if (d_out < 0 || d_in < 0 || !valid_d(d) || d_in % 16 != 0) return LCVQ_ERR_INVALID_ARG;
   if (!A || !B || !workspace) return LCVQ_ERR_INVALID_ARG;
@@ -268,6 +275,7 @@ static lcvq_status validate_gemm_shapes(lcvq_dtype dtype, int64_t M, int64_t d_o
 lcvq_status lcvq_gemm(const void* X, lcvq_dtype dtype, int64_t M, const uint8_t* packed,
                       int64_t d_out, int64_t d_in, int d, const float* A, const float* B,
                       void* Y, lcvq_form form, void* workspace, size_t ws_bytes, void* stream) {
+  LCVQ_API_RANGE();
   if (lcvq_status st = validate_gemm_shapes(dtype, M, d_out, d_in, d); st != LCVQ_OK) return st;
   if (form != LCVQ_FORM_AUTO && form != LCVQ_FORM_DECODE && form != LCVQ_FORM_ALGEBRAIC)
     return LCVQ_ERR_INVALID_ARG;
@@ -357,6 +365,7 @@ size_t lcvq_workspace_size_grouped(const lcvq_gemm_item* items, int count, int64
 
 lcvq_status lcvq_gemm_grouped(const lcvq_gemm_item* items, int count, int64_t M, int d,
                               void* workspace, size_t ws_bytes, void* stream) {
+  LCVQ_API_RANGE();
   g_last_launches = 0;
   std::vector<size_t> xoff, coff;
   const size_t need = grouped_ws(items, count, M, d, &xoff, &coff);
@@ -399,6 +408,7 @@ lcvq_status lcvq_gemm_grouped(const lcvq_gemm_item* items, int count, int64_t M,
 
 lcvq_status lcvq_xform(const void* X, lcvq_dtype dtype, int64_t M, int64_t d_in, int d,
                        const float* A, const float* B, void* Xpp, float* corr, void* stream) {
+  LCVQ_API_RANGE();
   if (lcvq_status st = validate_gemm_shapes(dtype, M, 8, d_in, d); st != LCVQ_OK) return st;
   if (dtype != LCVQ_BF16) return LCVQ_ERR_UNSUPPORTED;
   g_last_launches = 0;
@@ -417,6 +427,7 @@ lcvq_status lcvq_xform(const void* X, lcvq_dtype dtype, int64_t M, int64_t d_in,
 lcvq_status lcvq_gemm_xformed(const void* Xpp, const float* corr, int64_t M,
                               const uint8_t* packed, int64_t d_out, int64_t d_in, void* Y,
                               void* stream) {
+  LCVQ_API_RANGE();
   if (lcvq_status st = validate_gemm_shapes(LCVQ_BF16, M, d_out, d_in, 8); st != LCVQ_OK) return st;
   g_last_launches = 0;
   if (M == 0 || d_out == 0) return LCVQ_OK;
@@ -437,6 +448,7 @@ lcvq_status lcvq_gemm_backward(const void* X, const void* dY, lcvq_dtype dtype, 
                                int64_t d_in, int d, const float* A, const float* B, void* dX,
                                float* dA, float* dB, float* dWp, void* workspace,
                                size_t ws_bytes, void* stream) {
+  LCVQ_API_RANGE();
   if (lcvq_status st = validate_gemm_shapes(dtype, M, d_out, d_in, d); st != LCVQ_OK) return st;
   g_last_launches = 0;
   if (!dA || !dB) return LCVQ_ERR_INVALID_ARG;
@@ -497,6 +509,7 @@ lcvq_status lcvq_gemm_backward(const void* X, const void* dY, lcvq_dtype dtype, 
 }
 
 lcvq_status lcvq_check_device_error(void* workspace, void* stream) {
+  LCVQ_API_RANGE();
   if (!workspace) return LCVQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned int h[2] = {0, 0};

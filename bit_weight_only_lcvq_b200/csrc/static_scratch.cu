@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "trace.h"
 
 namespace {
 
@@ -55,6 +56,7 @@ bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 extern "C" lcvq_status lcvq_gemv_static(const void* X, int64_t M, const uint8_t* packed,
                                         int64_t d_out, int64_t d_in, int d, const float* A,
                                         const float* B, void* Y, void* stream) {
+  LCVQ_API_RANGE();
   lcvq::set_last_launches(0);
   if (M < 0 || d_out < 0 || d_in < 0) return LCVQ_ERR_INVALID_ARG;
   if (!(d == 1 || d == 2 || d == 4 || d == 8)) return LCVQ_ERR_INVALID_ARG;

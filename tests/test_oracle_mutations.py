@@ -7,6 +7,7 @@ mistakes:
 - a flipped sign;
 - a wrong tie or bit order;
 - a lost mask;
+- a normaliser built from signed terms;
 - a dropped intercept or normaliser;
 - missing error feedback;
 - an unreversed factorisation;
@@ -25,6 +26,7 @@ _decode, _assign, _pack = O.decode, O.assign, O.pack_codes
 _backward, _fit, _ldlq = O.backward, O.fit_affine, O.ldlq_assign
 _pack_mask, _dge_d, _ldl, _hess = O.pack_mask, O.dge_derivative, O.ldl_upper, O.code_space_hessian
 _fit_h, _fit_h_normal = O.fit_affine_h, O.fit_affine_h_normal
+_forward = O.forward
 
 
 def _fit_h_block_diagonal(W0, z, d, H):  # the (g, g') coupling of H dropped
@@ -71,6 +73,20 @@ def _transpose_da(o):
     o["dA"] = o["dA"].T.copy()
 
 
+def _signed_dwp_normaliser(o):  # |A| forgotten in D_dWp
+    o["D_dWp"] = o["D_dWp"] * 0 + o["dWp"]
+
+
+def _dwp_with_a_untransposed(X, dY, z, mask, A, B):  # dWp = mask * A G instead of A^T G
+    return _backward(X, dY, z, mask, np.asarray(A).T, B) | {
+        k: v for k, v in _backward(X, dY, z, mask, A, B).items() if k != "dWp"}
+
+
+def _forward_signed_normaliser(X, z, A, B):  # D_Y = |X W~^T| instead of |X| |W~|^T
+    Y, _ = _forward(X, z, A, B)
+    return Y, np.abs(Y)
+
+
 def _backward_no_mask(X, dY, z, mask, A, B):
     return _backward(X, dY, z, np.ones_like(mask, dtype=bool), A, B)
 
@@ -111,6 +127,14 @@ MUTATIONS = [
      [lambda gd: P.test_backward_finite_differences_exact()]),
     ("backward: clamp mask lost", "backward", _backward_no_mask,
      [lambda gd: P.test_backward_dwp_ste_surrogate_finite_differences()]),
+    ("backward: dWp with A where A^T belongs", "backward", _dwp_with_a_untransposed,
+     [lambda gd: P.test_backward_dwp_ste_surrogate_finite_differences()]),
+    ("backward: dWp's normaliser from signed terms", "backward",
+     _backward_with(_signed_dwp_normaliser),
+     [lambda gd: P.test_normalisers_ignore_the_signs_of_the_operands()]),
+    ("forward: normaliser from the signed product", "forward", _forward_signed_normaliser,
+     [lambda gd: P.test_forward_identity_is_integer_code_gemm(),
+      lambda gd: P.test_normalisers_ignore_the_signs_of_the_operands()]),
     ("refit: intercept dropped", "fit_affine", lambda W0, z, d, h=None: (_fit(W0, z, d, h)[0],
                                                                          np.zeros(d)),
      [lambda gd: P.test_fit_affine_recovers_an_exact_affine_map(4)]),

@@ -373,6 +373,49 @@ def test_db_identity_at_any_size():
     assert np.allclose(bw["dB"], ident, rtol=1e-13, atol=1e-13)
 
 
+# ------------------------------------------ the normalisers of the tolerance (R15)
+_NORMS = (("Y", "D_Y"), ("dX", "D_dX"), ("dA", "D_dA"), ("dB", "D_dB"), ("dWp", "D_dWp"))
+
+
+def _all_outputs(X, dY, z, mask, A, B):
+    out = dict(O.backward(X, dY, z, mask, A, B))
+    out["Y"], out["D_Y"] = O.forward(X, z, A, B)
+    return out
+
+
+def test_normalisers_equal_the_outputs_when_no_term_is_negative():
+    """A normaliser is the sum of its output's terms in absolute value; with
+    non-negative X, dY, A and B no term is negative, so each equals its
+    output (codes are non-negative too)."""
+    g = np.random.Generator(np.random.PCG64(91))
+    M, N, K, d = 3, 5, 32, 4
+    X, dY = g.uniform(0, 2, (M, K)), g.uniform(0, 2, (M, N))
+    A, B = g.uniform(0, 1, (d, d)), g.uniform(0, 1, d)
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    out = _all_outputs(X, dY, z, np.ones((N, K), bool), A, B)
+    for v, dn in _NORMS:
+        assert np.allclose(out[dn], out[v], rtol=1e-13, atol=0), v
+
+
+def test_normalisers_ignore_the_signs_of_the_operands():
+    """Flipping the sign of X, of dY, or of the decoded weights (A and B
+    together: W~ -> -W~, a term of Y is x_k w~_k) changes outputs but no
+    normaliser, and every normaliser bounds its output."""
+    g = np.random.Generator(np.random.PCG64(92))
+    M, N, K, d = 3, 5, 32, 4
+    X, dY = g.standard_normal((M, K)), g.standard_normal((M, N))
+    A, B = g.standard_normal((d, d)), g.standard_normal(d)
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    mask = g.random((N, K)) < 0.8
+    base = _all_outputs(X, dY, z, mask, A, B)
+    for v, dn in _NORMS:
+        assert np.all(np.abs(base[v]) <= base[dn] * (1 + 1e-13)), v
+    for flipped in (_all_outputs(-X, dY, z, mask, A, B), _all_outputs(X, -dY, z, mask, A, B),
+                    _all_outputs(X, dY, z, mask, -A, -B)):
+        for _, dn in _NORMS:
+            assert np.allclose(flipped[dn], base[dn], rtol=1e-13, atol=0), dn
+
+
 # ---------------------------------------------------------------- DGE (curve unpinned)
 def test_dge_small_k_limit_is_the_ste_mask():
     """As k -> 0 the DGE factor tends to the STE's clamp mask (1 on [0, 3], 0

@@ -47,6 +47,9 @@ PINS = [
     ("backward finite differences", lambda gd: P.test_backward_finite_differences_exact()),
     ("dWp STE surrogate", lambda gd: P.test_backward_dwp_ste_surrogate_finite_differences()),
     ("dB identity", lambda gd: P.test_db_identity_at_any_size()),
+    ("normalisers = outputs without negative terms",
+     lambda gd: P.test_normalisers_equal_the_outputs_when_no_term_is_negative()),
+    ("normalisers ignore operand signs", lambda gd: P.test_normalisers_ignore_the_signs_of_the_operands()),
 ]
 
 

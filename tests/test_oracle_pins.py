@@ -374,12 +374,14 @@ def test_db_identity_at_any_size():
 
 
 # ------------------------------------------ the normalisers of the tolerance (R15)
-_NORMS = (("Y", "D_Y"), ("dX", "D_dX"), ("dA", "D_dA"), ("dB", "D_dB"), ("dWp", "D_dWp"))
+_NORMS = (("W", "D_W"), ("Y", "D_Y"), ("dX", "D_dX"), ("dA", "D_dA"), ("dB", "D_dB"),
+          ("dWp", "D_dWp"))
 
 
 def _all_outputs(X, dY, z, mask, A, B):
     out = dict(O.backward(X, dY, z, mask, A, B))
     out["Y"], out["D_Y"] = O.forward(X, z, A, B)
+    out["W"], out["D_W"] = O.decode(z, A, B), O.decode_abs(z, A, B)
     return out
 
 

@@ -38,3 +38,41 @@ def test_reference_arm_prints_the_contract_line():
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert line["config"]["workload"].startswith("decode_gemv d_in=4096 d_out=4096 d=8")
+
+
+def _bench_module():
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench
+    return bench
+
+
+def test_ncu_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
+    """roofline.traffic comes from one ncu capture and stands only while every
+    captured source file hashes as it did then."""
+    import hashlib
+    bench = _bench_module()
+    sha = hashlib.sha1(open(os.path.join(ROOT, "bench.py"), "rb").read()).hexdigest()
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"sources": {"bench.py": sha}, "per_call": {1: 123}})
+    assert bench.traffic_for(1) == 123 and bench.traffic_for(4) is None
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"sources": {"bench.py": "0" * 40}, "per_call": {1: 123}})
+    assert bench.traffic_for(1) is None
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"sources": {"no/such/file.cu": sha}, "per_call": {1: 123}})
+    assert bench.traffic_for(1) is None
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"sources": {}, "per_call": {1: 123}})
+    assert bench.traffic_for(1) is None
+
+
+def test_peaks_fall_back_to_the_recipe_values_without_a_measurement(monkeypatch):
+    bench = _bench_module()
+    monkeypatch.setattr(bench, "ROOT", os.path.join(ROOT, "no_such_directory"))
+    p, src = bench.peaks()
+    assert src == "fallback"
+    assert p == {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def test_roofline_fraction_and_sums():
+    bench = _bench_module()
+    r = bench._roof("hbm", 3267.4, 6534.8, "GB/s", traffic=1.0)
+    assert r["frac"] == 3267.4 / 6534.8 and r["bound"] == "hbm" and r["traffic"] == 1.0
+    assert bench._sum_or_none([1, 2, 3]) == 6.0 and bench._sum_or_none([1, None]) is None

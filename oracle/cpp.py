@@ -5,8 +5,8 @@ may use it; the library never does).
 
 The functions take and return numpy arrays with the same names and meanings
 as the numpy oracle's (assign, pack_codes, unpack_codes, pack_mask,
-unpack_mask, decode, forward, backward), so every pin written for one runs on
-the other.  Floating inputs are widened to fp64 (exact for fp32/bf16 values).
+unpack_mask, decode, forward, backward, ldlq_assign), so every pin written for
+one runs on the other.  Floating inputs are widened to fp64 (exact for fp32/bf16 values).
 
 ``build()`` compiles the shared library with g++ (plain C++17, -O2, no
 fast-math, no fused multiply-add contraction); ``lib()`` builds it on first use
@@ -55,7 +55,8 @@ def lib() -> ctypes.CDLL:
         for nm in ("lco_backward_z8", "lco_backward_zf"):
             getattr(L, nm).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _i32, _vp, _vp,
                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32]
-        for f in L.lco_assign, L.lco_pack_codes, L.lco_decode_z8, L.lco_forward_z8:
+        L.lco_ldlq_assign.argtypes = [_vp, _i64, _i64, _vp, _vp, _i32]
+        for f in L.lco_assign, L.lco_pack_codes, L.lco_decode_z8, L.lco_forward_z8, L.lco_ldlq_assign:
             f.restype = None
         _lib = L
     return _lib
@@ -183,3 +184,16 @@ def backward(X, dY, z, mask, A, B, threads: int | None = None):
         _p(out["dA"]), _p(out["D_dA"]), _p(out["dB"]), _p(out["D_dB"]), _p(out["dWp"]),
         _p(out["D_dWp"]), threads or default_threads())
     return out
+
+
+# ---------------------------------------------------------------- H-aware sequential assignment
+def ldlq_assign(P, U, threads: int | None = None):
+    """Codes Z (u8, N x K) of the sequential rule, every row of the targets P
+    (N x K) on its own, elements in increasing k; only the strictly upper
+    triangle of U (K x K) is read."""
+    P, U = _f64(P), _f64(U)
+    n, k = P.shape
+    assert U.shape == (k, k)
+    Z = np.empty((n, k), dtype=np.uint8)
+    lib().lco_ldlq_assign(_p(P), n, k, _p(U), _p(Z), threads or default_threads())
+    return Z

@@ -330,4 +330,30 @@ void lco_backward_zf(const double* X, const double* dY, int64_t M, const double*
   backward_t(X, dY, M, z, mask, N, K, d, A, B, dX, D_dX, dA, D_dA, dB, D_dB, dWp, D_dWp, threads);
 }
 
+// H-aware sequential assignment (decoupleQ page, section 3.3, eq. (8)-(11):
+// fix one element by rounding and clipping, then re-solve the rest of the
+// quadratic objective without the integer constraint and the box -- the error
+// feedback of LDLQ, which the LC-QAT technical summary, Methodology 2, names
+// for the initial codes).  For every row of the code-space targets P [N][K],
+// in increasing j:
+//     t_j = p_j + sum_{i<j} U[i][j] (p_i - z_i),   z_j = clamp(rint(t_j), 0, 3),
+// the sum over i in increasing order.  Only the strictly upper triangle of
+// U [K][K] is read.  Z is u8 [N][K].
+void lco_ldlq_assign(const double* P, int64_t N, int64_t K, const double* U, uint8_t* Z,
+                     int threads) {
+  parallel_rows(N, threads, [=](int64_t a, int64_t b) {
+    std::vector<double> e(static_cast<size_t>(K), 0.0);
+    for (int64_t n = a; n < b; ++n) {
+      const double* p = P + n * K;
+      uint8_t* z = Z + n * K;
+      for (int64_t j = 0; j < K; ++j) {
+        double c = 0.0;
+        for (int64_t i = 0; i < j; ++i) c += U[i * K + j] * e[size_t(i)];
+        z[j] = code_of(p[j] + c);
+        e[size_t(j)] = p[j] - double(z[j]);
+      }
+    }
+  });
+}
+
 }  // extern "C"

@@ -1,8 +1,8 @@
 """Pins for the C++ fp64 oracle (oracle/lcvq_oracle.cpp).
 
 The C++ oracle must pass the same pins as the numpy one: every pin of the
-assign, pack, decode, forward and backward functions runs here with the C++
-functions put in place of the numpy ones.  It must also agree with the numpy
+assign, pack, decode, forward, backward and H-aware assignment functions runs
+here with the C++ functions put in place of the numpy ones.  It must also agree with the numpy
 oracle (an independent restatement of the same definitions) on random ragged
 cases, and give the same bits whatever the thread count.  CPU only.
 """
@@ -15,7 +15,7 @@ from oracle import lcvq_oracle as O
 from tests import test_oracle_pins as P
 
 SUBSTITUTED = ("assign", "pack_codes", "unpack_codes", "pack_mask", "unpack_mask", "decode",
-               "forward", "backward")
+               "forward", "backward", "ldlq_assign")
 
 
 @pytest.fixture
@@ -50,6 +50,17 @@ PINS = [
     ("normalisers = outputs without negative terms",
      lambda gd: P.test_normalisers_equal_the_outputs_when_no_term_is_negative()),
     ("normalisers ignore operand signs", lambda gd: P.test_normalisers_ignore_the_signs_of_the_operands()),
+    ("H-aware: diagonal Hessian is round and clamp",
+     lambda gd: P.test_ldlq_with_a_diagonal_hessian_is_round_and_clamp(gd)),
+    ("H-aware: eq. (11) procedure solved directly",
+     lambda gd: P.test_ldlq_equals_the_eq11_procedure_solved_directly()),
+    ("H-aware: best code by exhaustive search",
+     lambda gd: P.test_ldlq_choice_is_the_best_code_by_exhaustive_search()),
+    ("H-aware: inverse-Cholesky feedback form",
+     lambda gd: P.test_ldlq_equals_the_inverse_cholesky_error_feedback_form()),
+    ("H-aware: targets reproduce the choices", lambda gd: P.test_ldlq_targets_reproduce_the_choices()),
+    ("H-aware: lower objective than rounding",
+     lambda gd: P.test_ldlq_lowers_the_objective_on_a_correlated_hessian()),
 ]
 
 
@@ -107,6 +118,19 @@ def test_cpp_results_do_not_depend_on_the_thread_count():
     b5 = C.backward(X, dY, z, mask, A, B, threads=5)
     for k in b1:
         assert np.array_equal(b1[k], b5[k]), k
+
+
+def test_cpp_h_aware_assignment_equals_numpy_on_exact_inputs_at_any_thread_count():
+    """On a 1/32 grid of targets and a 1/64 grid of factor entries every fp64
+    operation of the rule is exact, so the two oracles' codes agree bit for
+    bit whatever their summation orders; rounding ties are on the grid."""
+    from bit_weight_only_lcvq_b200 import synth
+    g = np.random.Generator(np.random.PCG64(123))
+    P_ = synth.targets_dyadic(37, 192, g)
+    U = synth.strict_upper_dyadic(192, g)
+    Zn = O.ldlq_assign(P_, U)
+    assert np.array_equal(C.ldlq_assign(P_, U, threads=1), Zn)
+    assert np.array_equal(C.ldlq_assign(P_, U, threads=6), Zn)
 
 
 def test_cpp_planted_transpose_is_caught(monkeypatch, golden_dir):

@@ -5,8 +5,8 @@ may use it; the library never does).
 
 The functions take and return numpy arrays with the same names and meanings
 as the numpy oracle's (assign, pack_codes, unpack_codes, pack_mask,
-unpack_mask, decode, forward, backward, ldlq_assign), so every pin written for
-one runs on the other.  Floating inputs are widened to fp64 (exact for fp32/bf16 values).
+unpack_mask, decode, forward, backward, ldlq_assign, fit_affine, fit_affine_h),
+so every pin written for one runs on the other.  Floating inputs are widened to fp64 (exact for fp32/bf16 values).
 
 ``build()`` compiles the shared library with g++ (plain C++17, -O2, no
 fast-math, no fused multiply-add contraction); ``lib()`` builds it on first use
@@ -56,7 +56,10 @@ def lib() -> ctypes.CDLL:
             getattr(L, nm).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _i32, _vp, _vp,
                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32]
         L.lco_ldlq_assign.argtypes = [_vp, _i64, _i64, _vp, _vp, _i32]
-        for f in L.lco_assign, L.lco_pack_codes, L.lco_decode_z8, L.lco_forward_z8, L.lco_ldlq_assign:
+        L.lco_fit_affine.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]
+        L.lco_fit_affine_h.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]
+        for f in (L.lco_assign, L.lco_pack_codes, L.lco_decode_z8, L.lco_forward_z8,
+                  L.lco_ldlq_assign, L.lco_fit_affine, L.lco_fit_affine_h):
             f.restype = None
         _lib = L
     return _lib
@@ -197,3 +200,29 @@ def ldlq_assign(P, U, threads: int | None = None):
     Z = np.empty((n, k), dtype=np.uint8)
     lib().lco_ldlq_assign(_p(P), n, k, _p(U), _p(Z), threads or default_threads())
     return Z
+
+
+# ---------------------------------------------------------------- least-squares refits of (A, B)
+def fit_affine(W0, z, d: int, h=None):
+    """(A, B) minimizing sum_n sum_k h_k (W0[n, k] - W~[n, k])^2 given the codes
+    (h = 1 when None); the minimum-norm solution where a Gram is singular."""
+    W0 = _f64(W0)
+    zz = np.ascontiguousarray(np.asarray(z, dtype=np.uint8))
+    n, k = W0.shape
+    hv = None if h is None else _f64(h)
+    A = np.empty((d, d))
+    B = np.empty(d)
+    lib().lco_fit_affine(_p(W0), _p(zz), n, k, d, None if hv is None else _p(hv), _p(A), _p(B))
+    return A, B
+
+
+def fit_affine_h(W0, z, d: int, H):
+    """(A, B) minimizing sum_n (W~[n] - W0[n])^T H (W~[n] - W0[n]) given the codes."""
+    W0, H = _f64(W0), _f64(H)
+    zz = np.ascontiguousarray(np.asarray(z, dtype=np.uint8))
+    n, k = W0.shape
+    assert H.shape == (k, k)
+    A = np.empty((d, d))
+    B = np.empty(d)
+    lib().lco_fit_affine_h(_p(W0), _p(zz), n, k, d, _p(H), _p(A), _p(B))
+    return A, B

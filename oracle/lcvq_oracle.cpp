@@ -34,6 +34,7 @@
 // increasing order.  Every floating result comes with the normaliser D = the
 // sum of the absolute values of its terms, propagated through each output's
 // own terms (the parity metric is |got - ref| / D).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -240,6 +241,69 @@ void backward_t(const double* X, const double* dY, int64_t M, const Z* z, const 
   }
 }
 
+// Eigen-decomposition of the symmetric n x n matrix S (row-major; destroyed):
+// on return the diagonal of S holds the eigenvalues and the columns of V
+// (row-major) the eigenvectors.  Cyclic Jacobi: every off-diagonal pair (p, q)
+// in turn is zeroed by the plane rotation of the symmetric Schur step (Golub
+// and Van Loan, "Matrix Computations", the cyclic Jacobi method), sweeps until
+// the off-diagonal part is below 1e-30 of the whole (squared norms).
+void jacobi_eigen(std::vector<double>& S, int n, std::vector<double>& V) {
+  V.assign(size_t(n) * size_t(n), 0.0);
+  for (int i = 0; i < n; ++i) V[size_t(i) * n + i] = 1.0;
+  for (int sweep = 0; sweep < 100; ++sweep) {
+    double off = 0.0, all = 0.0;
+    for (int p = 0; p < n; ++p)
+      for (int q = 0; q < n; ++q) {
+        const double v = S[size_t(p) * n + q] * S[size_t(p) * n + q];
+        all += v;
+        if (p != q) off += v;
+      }
+    if (off <= 1e-30 * all) break;
+    for (int p = 0; p < n - 1; ++p)
+      for (int q = p + 1; q < n; ++q) {
+        const double apq = S[size_t(p) * n + q];
+        if (apq == 0.0) continue;
+        const double app = S[size_t(p) * n + p], aqq = S[size_t(q) * n + q];
+        const double tau = (aqq - app) / (2.0 * apq);
+        const double t = (tau >= 0.0 ? 1.0 : -1.0) / (std::fabs(tau) + std::sqrt(1.0 + tau * tau));
+        const double c = 1.0 / std::sqrt(1.0 + t * t), sn = t * c;
+        for (int k = 0; k < n; ++k) {  // S J
+          const double skp = S[size_t(k) * n + p], skq = S[size_t(k) * n + q];
+          S[size_t(k) * n + p] = c * skp - sn * skq;
+          S[size_t(k) * n + q] = sn * skp + c * skq;
+        }
+        for (int k = 0; k < n; ++k) {  // J^T (S J)
+          const double spk = S[size_t(p) * n + k], sqk = S[size_t(q) * n + k];
+          S[size_t(p) * n + k] = c * spk - sn * sqk;
+          S[size_t(q) * n + k] = sn * spk + c * sqk;
+        }
+        for (int k = 0; k < n; ++k) {  // V J
+          const double vkp = V[size_t(k) * n + p], vkq = V[size_t(k) * n + q];
+          V[size_t(k) * n + p] = c * vkp - sn * vkq;
+          V[size_t(k) * n + q] = sn * vkp + c * vkq;
+        }
+      }
+  }
+}
+
+// x = G^+ r for the symmetric n x n G: the eigenvalues at or below rcond of the
+// largest in magnitude count as zero (the minimum-norm least-squares solution)
+constexpr double kPinvRcond = 1e-12;
+void pinv_solve(std::vector<double> G, int n, const double* r, double* x) {
+  std::vector<double> V;
+  jacobi_eigen(G, n, V);
+  double lmax = 0.0;
+  for (int e = 0; e < n; ++e) lmax = std::max(lmax, std::fabs(G[size_t(e) * n + e]));
+  for (int i = 0; i < n; ++i) x[i] = 0.0;
+  for (int e = 0; e < n; ++e) {
+    const double lam = G[size_t(e) * n + e];
+    if (!(std::fabs(lam) > kPinvRcond * lmax)) continue;
+    double vr = 0.0;
+    for (int i = 0; i < n; ++i) vr += V[size_t(i) * n + e] * r[i];
+    for (int i = 0; i < n; ++i) x[i] += V[size_t(i) * n + e] * (vr / lam);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -354,6 +418,89 @@ void lco_ldlq_assign(const double* P, int64_t N, int64_t K, const double* U, uin
       }
     }
   });
+}
+
+// Least-squares refit of (A, B) given the codes (decoupleQ page, eq. (5) with
+// H replaced by its diagonal h, and section 3.3: with the integer part fixed
+// the float part is a quadratic, solved in closed form).  The objective
+// sum_n sum_k h_k (W0[n][k] - W~[n][k])^2 splits over the output coordinate i;
+// with zt = [z_0 .. z_{d-1}, 1] per vector (row n, position g):
+//     G_i = sum_{n,g} h_{g d + i} zt zt^T,   R_i = sum_{n,g} h_{g d + i} W0[n][g d + i] zt,
+// and row i of [A | B] is G_i^+ R_i.  h may be null (h = 1).
+void lco_fit_affine(const double* W0, const uint8_t* z, int64_t N, int64_t K, int d,
+                    const double* h, double* A, double* B) {
+  const int m = d + 1;
+  for (int i = 0; i < d; ++i) {
+    std::vector<double> G(static_cast<size_t>(m * m), 0.0), R(static_cast<size_t>(m), 0.0);
+    std::vector<double> th(static_cast<size_t>(m), 0.0);
+    std::vector<double> zt(static_cast<size_t>(m), 0.0);
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t g = 0; g < K / d; ++g) {
+        const int64_t k = g * d + i;
+        const double hk = h ? h[k] : 1.0;
+        for (int a = 0; a < d; ++a) zt[size_t(a)] = double(z[n * K + g * d + a]);
+        zt[size_t(d)] = 1.0;
+        for (int a = 0; a < m; ++a) {
+          for (int b = 0; b < m; ++b) G[size_t(a) * m + b] += hk * zt[size_t(a)] * zt[size_t(b)];
+          R[size_t(a)] += hk * W0[n * K + k] * zt[size_t(a)];
+        }
+      }
+    pinv_solve(G, m, R.data(), th.data());
+    for (int a = 0; a < d; ++a) A[i * d + a] = th[size_t(a)];
+    B[i] = th[size_t(d)];
+  }
+}
+
+// The same refit under the full K x K input Hessian H (decoupleQ page, eq. (5):
+// the objective sum_n (W~[n] - W0[n])^T H (W~[n] - W0[n]); section 3.3's closed
+// form).  theta = [A | B] enters every decoded element linearly,
+// W~[n][g d + i] = sum_a theta[i][a] zt[n][g][a], so one joint system of
+// d (d + 1) unknowns, index (i, a) -> i (d + 1) + a:
+//     L[(i,a)][(j,b)] = sum_{g,h} H[g d + i][h d + j] S[(g,a)][(h,b)],
+//     R[(i,a)]        = sum_g sum_k H[g d + i][k] T[k][(g,a)],
+// with the code Gram S[(g,a)][(h,b)] = sum_n zt[n][g][a] zt[n][h][b] and
+// T[k][(g,a)] = sum_n W0[n][k] zt[n][g][a] (the sums over n taken first);
+// theta = L^+ R.
+void lco_fit_affine_h(const double* W0, const uint8_t* z, int64_t N, int64_t K, int d,
+                      const double* H, double* A, double* B) {
+  const int m = d + 1, np = d * m;
+  const int64_t ng = K / d, w = ng * m;  // width of S and T: (g, a) pairs
+  std::vector<double> zt(static_cast<size_t>(w), 0.0);
+  std::vector<double> S(size_t(w) * size_t(w), 0.0), T(size_t(K) * size_t(w), 0.0);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < ng; ++g) {
+      for (int a = 0; a < d; ++a) zt[size_t(g * m + a)] = double(z[n * K + g * d + a]);
+      zt[size_t(g * m + d)] = 1.0;
+    }
+    for (int64_t u = 0; u < w; ++u)
+      for (int64_t v = 0; v < w; ++v) S[size_t(u * w + v)] += zt[size_t(u)] * zt[size_t(v)];
+    for (int64_t k = 0; k < K; ++k)
+      for (int64_t u = 0; u < w; ++u) T[size_t(k * w + u)] += W0[n * K + k] * zt[size_t(u)];
+  }
+  std::vector<double> L(static_cast<size_t>(np * np), 0.0), R(static_cast<size_t>(np), 0.0);
+  std::vector<double> th(static_cast<size_t>(np), 0.0);
+  for (int i = 0; i < d; ++i)
+    for (int a = 0; a < m; ++a)
+      for (int j = 0; j < d; ++j)
+        for (int b = 0; b < m; ++b) {
+          double acc = 0.0;
+          for (int64_t g = 0; g < ng; ++g)
+            for (int64_t hh = 0; hh < ng; ++hh)
+              acc += H[(g * d + i) * K + hh * d + j] * S[size_t((g * m + a) * w + hh * m + b)];
+          L[size_t(i * m + a) * np + j * m + b] = acc;
+        }
+  for (int i = 0; i < d; ++i)
+    for (int a = 0; a < m; ++a) {
+      double acc = 0.0;
+      for (int64_t g = 0; g < ng; ++g)
+        for (int64_t k = 0; k < K; ++k) acc += H[(g * d + i) * K + k] * T[size_t(k * w + g * m + a)];
+      R[size_t(i * m + a)] = acc;
+    }
+  pinv_solve(L, np, R.data(), th.data());
+  for (int i = 0; i < d; ++i) {
+    for (int a = 0; a < d; ++a) A[i * d + a] = th[size_t(i * m + a)];
+    B[i] = th[size_t(i * m + d)];
+  }
 }
 
 }  // extern "C"

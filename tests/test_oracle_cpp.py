@@ -1,8 +1,8 @@
 """Pins for the C++ fp64 oracle (oracle/lcvq_oracle.cpp).
 
 The C++ oracle must pass the same pins as the numpy one: every pin of the
-assign, pack, decode, forward, backward and H-aware assignment functions runs
-here with the C++ functions put in place of the numpy ones.  It must also agree with the numpy
+assign, pack, decode, forward, backward, H-aware assignment and (A, B) refit
+functions runs here with the C++ functions put in place of the numpy ones.  It must also agree with the numpy
 oracle (an independent restatement of the same definitions) on random ragged
 cases, and give the same bits whatever the thread count.  CPU only.
 """
@@ -15,7 +15,7 @@ from oracle import lcvq_oracle as O
 from tests import test_oracle_pins as P
 
 SUBSTITUTED = ("assign", "pack_codes", "unpack_codes", "pack_mask", "unpack_mask", "decode",
-               "forward", "backward", "ldlq_assign")
+               "forward", "backward", "ldlq_assign", "fit_affine", "fit_affine_h")
 
 
 @pytest.fixture
@@ -61,6 +61,26 @@ PINS = [
     ("H-aware: targets reproduce the choices", lambda gd: P.test_ldlq_targets_reproduce_the_choices()),
     ("H-aware: lower objective than rounding",
      lambda gd: P.test_ldlq_lowers_the_objective_on_a_correlated_hessian()),
+    ("refit: exact recovery d=1", lambda gd: P.test_fit_affine_recovers_an_exact_affine_map(1)),
+    ("refit: exact recovery d=8", lambda gd: P.test_fit_affine_recovers_an_exact_affine_map(8)),
+    ("refit: stacked-design least squares d=4",
+     lambda gd: P.test_fit_affine_equals_least_squares_on_the_stacked_design(4)),
+    ("refit: scalar case is linear regression",
+     lambda gd: P.test_fit_affine_scalar_case_is_simple_linear_regression()),
+    ("refit: a minimum", lambda gd: P.test_fit_affine_is_a_minimum()),
+    ("refit: singular Gram, minimum norm",
+     lambda gd: P.test_fit_affine_singular_gram_gives_the_minimum_norm_solution()),
+    ("refit: weights scale and mask", lambda gd: P.test_fit_affine_weights_scale_and_mask()),
+    ("full-H refit: exact recovery d=2", lambda gd: P.test_fit_affine_h_recovers_an_exact_affine_map(2)),
+    ("full-H refit: exact recovery d=8", lambda gd: P.test_fit_affine_h_recovers_an_exact_affine_map(8)),
+    ("full-H refit: least squares with H^1/2 d=4",
+     lambda gd: P.test_fit_affine_h_equals_least_squares_with_the_hessian_root(4)),
+    ("full-H refit: diagonal H is the weighted fit d=8",
+     lambda gd: P.test_fit_affine_h_with_a_diagonal_hessian_is_the_weighted_fit(8)),
+    ("full-H refit: a minimum, scale invariant",
+     lambda gd: P.test_fit_affine_h_is_a_minimum_and_scale_invariant()),
+    ("full-H refit: beats the diagonal fit",
+     lambda gd: P.test_fit_affine_h_beats_the_diagonal_fit_on_a_correlated_hessian()),
 ]
 
 
@@ -131,6 +151,24 @@ def test_cpp_h_aware_assignment_equals_numpy_on_exact_inputs_at_any_thread_count
     Zn = O.ldlq_assign(P_, U)
     assert np.array_equal(C.ldlq_assign(P_, U, threads=1), Zn)
     assert np.array_equal(C.ldlq_assign(P_, U, threads=6), Zn)
+
+
+@pytest.mark.parametrize("d", [1, 2, 4, 8])
+def test_cpp_refits_agree_with_numpy(d):
+    """Both refits, random codes and weights, against the numpy oracle (its own
+    einsum contractions and LAPACK pseudo-inverse), to fp64 rounding."""
+    g = np.random.Generator(np.random.PCG64(200 + d))
+    N, K = 29, 16 * d
+    z = g.integers(0, 4, size=(N, K), dtype=np.uint8)
+    W0 = g.standard_normal((N, K))
+    h = g.uniform(0.5, 2.0, K)
+    Xc = g.standard_normal((2 * K, K))
+    H = Xc.T @ Xc / (2 * K) + 0.01 * np.eye(K)
+    for got, ref in ((C.fit_affine(W0, z, d, h), O.fit_affine(W0, z, d, h)),
+                     (C.fit_affine(W0, z, d), O.fit_affine(W0, z, d)),
+                     (C.fit_affine_h(W0, z, d, H), O.fit_affine_h(W0, z, d, H))):
+        for a, b in zip(got, ref):
+            assert np.allclose(a, b, rtol=1e-10, atol=1e-12 * np.max(np.abs(b))), d
 
 
 def test_cpp_planted_transpose_is_caught(monkeypatch, golden_dir):

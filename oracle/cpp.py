@@ -5,8 +5,8 @@ may use it; the library never does).
 
 The functions take and return numpy arrays with the same names and meanings
 as the numpy oracle's (assign, pack_codes, unpack_codes, pack_mask,
-unpack_mask, decode, forward, backward, ldlq_assign, fit_affine, fit_affine_h),
-so every pin written for one runs on the other.  Floating inputs are widened to fp64 (exact for fp32/bf16 values).
+unpack_mask, decode, forward, backward, ldlq_assign, fit_affine, fit_affine_h,
+dge_phi, dge_derivative), so every pin written for one runs on the other.  Floating inputs are widened to fp64 (exact for fp32/bf16 values).
 
 ``build()`` compiles the shared library with g++ (plain C++17, -O2, no
 fast-math, no fused multiply-add contraction); ``lib()`` builds it on first use
@@ -58,6 +58,9 @@ def lib() -> ctypes.CDLL:
         L.lco_ldlq_assign.argtypes = [_vp, _i64, _i64, _vp, _vp, _i32]
         L.lco_fit_affine.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]
         L.lco_fit_affine_h.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]
+        for nm in ("lco_dge_phi", "lco_dge_derivative"):
+            getattr(L, nm).argtypes = [_vp, _i64, ctypes.c_double, _vp]
+            getattr(L, nm).restype = None
         for f in (L.lco_assign, L.lco_pack_codes, L.lco_decode_z8, L.lco_forward_z8,
                   L.lco_ldlq_assign, L.lco_fit_affine, L.lco_fit_affine_h):
             f.restype = None
@@ -226,3 +229,20 @@ def fit_affine_h(W0, z, d: int, H):
     B = np.empty(d)
     lib().lco_fit_affine_h(_p(W0), _p(zz), n, k, d, _p(H), _p(A), _p(B))
     return A, B
+
+
+# ---------------------------------------------------------------- DGE curve (a reading)
+def dge_phi(w, k):
+    """The smooth rounding curve phi_k on [0, 3] (clamped outside)."""
+    x = _f64(w)
+    out = np.empty(x.shape)
+    lib().lco_dge_phi(_p(x), x.size, float(k), _p(out))
+    return out
+
+
+def dge_derivative(Wp, k):
+    """phi_k'(Wp): the factor DGE puts where the STE puts the clamp mask."""
+    x = _f64(Wp)
+    out = np.empty(x.shape)
+    lib().lco_dge_derivative(_p(x), x.size, float(k), _p(out))
+    return out

@@ -420,6 +420,33 @@ void lco_ldlq_assign(const double* P, int64_t N, int64_t K, const double* U, uin
   });
 }
 
+// DGE (the LC-QAT technical summary's gradient estimator: a smooth,
+// differentiable curve through the rounding).  The pages give no curve; the
+// reading taken is the tanh staircase on [0, 3], clamped outside:
+//     phi_k(w) = floor(w) + 1/2 + tanh(k (frac(w) - 1/2)) / (2 tanh(k / 2)),
+// with w = 3 on the last step.  phi_k'(w) = (k / (2 tanh(k / 2))) / cosh^2(k (frac(w) - 1/2))
+// on [0, 3] and 0 outside (and for NaN): the factor DGE puts where the STE
+// puts the clamp mask.
+void lco_dge_phi(const double* w, int64_t n, double k, double* out) {
+  for (int64_t t = 0; t < n; ++t) {
+    const double x = std::min(std::max(w[t], 0.0), kCodeMax);
+    const double fl = std::min(std::floor(x), kCodeMax - 1.0);
+    out[t] = fl + 0.5 + std::tanh(k * (x - fl - 0.5)) / (2.0 * std::tanh(k / 2.0));
+  }
+}
+void lco_dge_derivative(const double* w, int64_t n, double k, double* out) {
+  for (int64_t t = 0; t < n; ++t) {
+    const double x = w[t];
+    if (!(x >= 0.0 && x <= kCodeMax)) {
+      out[t] = 0.0;
+      continue;
+    }
+    const double fl = std::min(std::floor(x), kCodeMax - 1.0);
+    const double c = std::cosh(k * (x - fl - 0.5));
+    out[t] = (k / (2.0 * std::tanh(k / 2.0))) / (c * c);
+  }
+}
+
 // Least-squares refit of (A, B) given the codes (decoupleQ page, eq. (5) with
 // H replaced by its diagonal h, and section 3.3: with the integer part fixed
 // the float part is a quadratic, solved in closed form).  The objective

@@ -1,8 +1,8 @@
 """Pins for the C++ fp64 oracle (oracle/lcvq_oracle.cpp).
 
 The C++ oracle must pass the same pins as the numpy one: every pin of the
-assign, pack, decode, forward, backward, H-aware assignment and (A, B) refit
-functions runs here with the C++ functions put in place of the numpy ones.  It must also agree with the numpy
+assign, pack, decode, forward, backward, DGE, H-aware assignment and (A, B)
+refit functions runs here with the C++ functions put in place of the numpy ones.  It must also agree with the numpy
 oracle (an independent restatement of the same definitions) on random ragged
 cases, and give the same bits whatever the thread count.  CPU only.
 """
@@ -15,7 +15,8 @@ from oracle import lcvq_oracle as O
 from tests import test_oracle_pins as P
 
 SUBSTITUTED = ("assign", "pack_codes", "unpack_codes", "pack_mask", "unpack_mask", "decode",
-               "forward", "backward", "ldlq_assign", "fit_affine", "fit_affine_h")
+               "forward", "backward", "ldlq_assign", "fit_affine", "fit_affine_h", "dge_phi",
+               "dge_derivative")
 
 
 @pytest.fixture
@@ -61,6 +62,10 @@ PINS = [
     ("H-aware: targets reproduce the choices", lambda gd: P.test_ldlq_targets_reproduce_the_choices()),
     ("H-aware: lower objective than rounding",
      lambda gd: P.test_ldlq_lowers_the_objective_on_a_correlated_hessian()),
+    ("DGE: small-k limit is the STE mask", lambda gd: P.test_dge_small_k_limit_is_the_ste_mask()),
+    ("DGE: staircase through the integers",
+     lambda gd: P.test_dge_curve_is_a_staircase_through_the_integers()),
+    ("DGE: backward is STE times the factor", lambda gd: P.test_dge_backward_is_ste_times_the_factor()),
     ("refit: exact recovery d=1", lambda gd: P.test_fit_affine_recovers_an_exact_affine_map(1)),
     ("refit: exact recovery d=8", lambda gd: P.test_fit_affine_recovers_an_exact_affine_map(8)),
     ("refit: stacked-design least squares d=4",
@@ -169,6 +174,14 @@ def test_cpp_refits_agree_with_numpy(d):
                      (C.fit_affine_h(W0, z, d, H), O.fit_affine_h(W0, z, d, H))):
         for a, b in zip(got, ref):
             assert np.allclose(a, b, rtol=1e-10, atol=1e-12 * np.max(np.abs(b))), d
+
+
+def test_cpp_dge_agrees_with_numpy():
+    w = np.concatenate([np.linspace(-1.0, 4.0, 2001), [0.0, 1.0, 2.0, 3.0, np.nan, np.inf, -np.inf]])
+    for k in (1e-3, 0.5, 4.0, 30.0):
+        assert np.allclose(C.dge_derivative(w, k), O.dge_derivative(w, k), rtol=1e-13, atol=0)
+        fin = np.isfinite(w)
+        assert np.allclose(C.dge_phi(w[fin], k), O.dge_phi(w[fin], k), rtol=1e-13, atol=1e-15)
 
 
 def test_cpp_planted_transpose_is_caught(monkeypatch, golden_dir):

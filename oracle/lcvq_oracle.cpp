@@ -17,6 +17,11 @@
 //     rounding straight through (the STE of the gradient-estimator ablation).
 //   * decoupleQ page, eq. (1): the layer is Y = X W~ (W~ stored here as
 //     [d_out][d_in], so Y[m][n] = sum_k X[m][k] W~[n][k]).
+//   * decoupleQ page, eq. (5) and section 3.3: the (A, B) refits for fixed
+//     codes (diagonal and full Hessian); eq. (8)-(11) with LC-QAT's
+//     Methodology 2: the H-aware sequential code assignment.
+//   * LC-QAT page, the gradient estimator DGE: a smooth curve through the
+//     rounding (the curve itself is a reading; see lco_dge_phi).
 //
 // Readings where the pages are silent (the same as the numpy oracle's):
 // round half to even; clamp to [0, 3]; NaN -> 0, +inf -> 3, -inf -> 0; the STE
